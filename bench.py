@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Throughput of one NanoFlow-style serving iteration on B200 (decode tokens/s).
+
+A step is one call of nf_forward_iteration over the whole batch of the workload
+(default: the Llama-3-8B-shaped layer with 512 decode requests, context U[1024,1536],
+plus a 1024-token prefill chunk), with the plan chosen by nf_plan_iteration.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 (launched by torchrun): independent replicas, one per GPU, no collective on the
+data path ("replicas only"); timing is the max over ranks. Rank 0 prints one JSON line.
+--impl reference times the float64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s per B200 (Llama-3-8B shape); % of compute-bound optimum"
+DEFAULT_WORKLOAD = "llama3_8b_layer"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--nano", type=int, default=0, help="force the nano-batch count (0: planner)")
+    ap.add_argument("--sm-attn", type=int, default=0, help="force the attention SM share (0: planner)")
+    ap.add_argument("--template", type=int, default=-1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip e2e / sequential / op-timing passes")
+    ap.add_argument("--cpu-sample", type=int, default=0, help="decode requests in the CPU oracle sample")
+    return ap.parse_args(argv)
+
+
+# --------------------------------------------------------------------------- distributed plumbing
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch
+            import torch.distributed as dist
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if self.pg is None:
+            return x
+        import torch
+        dev = f"cuda:{self.local}" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- work accounting
+
+def iteration_flops(work, batch):
+    """GEMM FLOPs + attention matmul FLOPs of one iteration (compute-bound optimum numerator)."""
+    s = work.shape
+    T, R, C = batch.num_tokens, batch.num_decode, batch.prefill_len
+    H, d, nq, nkv, F = s.hidden, s.head_dim, s.n_q_heads, s.n_kv_heads, s.ffn
+    per_tok = 2 * H * ((nq + 2 * nkv) * d) + 2 * (nq * d) * H
+    if s.n_experts:
+        per_tok += s.top_k * (2 * H * 2 * F + 2 * F * H) + 2 * H * s.n_experts
+    else:
+        per_tok += 2 * H * 2 * F + 2 * F * H
+    gemm = T * per_tok * s.n_layers
+    keys = float(sum(int(c) + 1 for c in batch.ctx_lens))
+    attn = s.n_layers * 4.0 * nq * d * (keys + C * (C + 1) / 2.0)
+    lm = 2.0 * (R + (1 if C else 0)) * H * s.vocab if s.vocab else 0.0
+    return gemm + attn + lm, gemm, attn, lm
+
+
+def op_algorithmic(work, batch, plan, op, nano):
+    """(bound, units per launch) of one op launch: FLOPs for GEMMs, bytes for decode attention."""
+    s = work.shape
+    t0, t1 = plan.tok_begin[nano], plan.tok_end[nano]
+    M = t1 - t0
+    H, d, nq, nkv, F = s.hidden, s.head_dim, s.n_q_heads, s.n_kv_heads, s.ffn
+    if op == "qkv":
+        return "tensor", 2.0 * M * (nq + 2 * nkv) * d * H
+    if op == "o_proj":
+        return "tensor", 2.0 * M * H * nq * d
+    if op == "gate_up":
+        return "tensor", 2.0 * M * 2 * F * H
+    if op == "down":
+        return "tensor", 2.0 * M * H * F
+    if op == "lm_head":
+        return "tensor", 2.0 * (batch.num_decode + (1 if batch.prefill_len else 0)) * H * s.vocab
+    if op == "attention":
+        R = batch.num_decode
+        r0, r1 = min(t0, R), min(t1, R)
+        pages = sum((int(batch.ctx_lens[r]) + 1 + 15) // 16 for r in range(r0, r1))
+        kv = pages * 2 * nkv * 16 * d * 2
+        qo = (r1 - r0) * nq * d * 2 * 2
+        if t1 > R and batch.prefill_len:
+            C = batch.prefill_len
+            kv += ((C + 15) // 16) * 2 * nkv * 16 * d * 2
+        return "hbm", float(kv + qo)
+    return None, 0.0
+
+
+def count_launches(work, plan):
+    s = work.shape
+    R = plan.num_decode
+    per_step = 2 if R > 0 else 1          # decode schedule + residual set-up (or embedding)
+    for j in range(plan.n_nano):
+        t0, t1 = plan.tok_begin[j], plan.tok_end[j]
+        att = (2 if min(t1, R) > min(t0, R) else 0) + (1 if t1 > R and plan.prefill_len else 0)
+        ffn = 6 if s.n_experts else 2      # route+sort, gather, 2 grouped GEMMs, combine
+        if s.n_experts:
+            ffn = 6
+        per_step += s.n_layers * (1 + att + 1 + ffn)
+    if s.vocab:
+        per_step += 3
+    return per_step
+
+
+# --------------------------------------------------------------------------- CPU oracle timing
+
+def cpu_oracle_sample(work, batch, n_requests: int, repeats: int = 1):
+    """Time the float64 oracle on the first n_requests decode rows (inputs pre-generated)."""
+    import numpy as np
+    from oracle.forward import iteration_forward, sub_batch
+    from oracle.run import layer_weights_f64, make_kv
+    from synth import bf16_to_f64
+    from synth import weights as SW
+    s = work.shape
+    sb = sub_batch(batch, list(range(n_requests)), keep_prefill=False)
+    wcache = {l: layer_weights_f64(s, l) for l in range(s.n_layers)}
+    kw = {}
+    if s.vocab:
+        g = SW.global_specs(s)
+        emb = bf16_to_f64(SW.host_rows(g["embed"], sb.tokens))
+        kw = dict(embed_rows=lambda toks: emb, final_norm=bf16_to_f64(SW.host_tensor(g["final_norm"])),
+                  lm_head=bf16_to_f64(SW.host_tensor(g["lm_head"])))
+        x_in = None
+    else:
+        x_in = bf16_to_f64(SW.host_input_rows(s, np.arange(n_requests)))
+    times = []
+    for _ in range(repeats):
+        kv = make_kv(s)
+        for l in range(s.n_layers):   # pre-load the sample's pages (input regeneration is not timed)
+            kv._load(l, sb.page_indices)
+        t = time.perf_counter()
+        iteration_forward(s, sb, lambda l: wcache[l], kv, x_in=x_in, **kw)
+        times.append(time.perf_counter() - t)
+    threads = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        info = [p.get("num_threads") for p in threadpool_info() if p.get("internal_api") == "openblas"]
+        if info:
+            threads = max(info)
+    except Exception:
+        pass
+    return times, threads
+
+
+def run_reference(args, work, dist):
+    if dist.rank != 0:
+        return
+    from synth.workloads import make_batch
+    batch = make_batch(work)
+    n = args.cpu_sample or min(128, batch.num_decode)
+    cpu_oracle_sample(work, batch, n, repeats=max(1, args.warmup))  # warm-up
+    times, threads = cpu_oracle_sample(work, batch, n, repeats=args.steps)
+    tot = sum(times)
+    value = n * len(times) / tot
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "decode tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample_decode_requests": n},
+            "cpu_baseline": {"value": value, "unit": "decode tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{n} of {batch.num_decode} decode requests of {args.workload}, no prefill "
+                                       "chunk, float64 numpy oracle, inputs pre-generated"},
+            "e2e": {"value": value, "unit": "decode tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def run_ours(args, work, dist):
+    import numpy as np
+    import torch
+    import intra_device_overlapped_b200 as nf
+    from intra_device_overlapped_b200.harness import DeviceWorkload
+
+    dev = f"cuda:{dist.local}"
+    torch.cuda.set_device(dev)
+    dw = DeviceWorkload(work, dev, keep_logits=False)
+    b = dw.batch
+    plan = dw.plan(nano=args.nano, sm_attn=args.sm_attn, template=args.template)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(max(args.warmup, 3)):
+        dw.forward(plan, stream)
+    nf.check(dw.sync(), "warm-up")
+
+    # ---- timed region: K iterations back to back, per-op CUDA events on each op's stream
+    nf.check(nf.nf_set_timing(dw.model, True), "timing")
+    clocks = ClockSampler(dist.local)
+    clocks.start()
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        dw.forward(plan, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop()
+    nf.check(dw.sync(), "timed steps")
+    ms_total = dist.max(e0.elapsed_time(e1))
+    st, op_times = nf.nf_get_op_times(dw.model, 1 << 20)
+    nf.check(st, "op times")
+    nf.check(nf.nf_set_timing(dw.model, False), "timing")
+    ms_step = ms_total / args.steps
+    R = b.num_decode
+    value = dist.world * R * args.steps / (ms_total / 1000.0)
+
+    flops, gemm_f, attn_f, lm_f = iteration_flops(work, b)
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = load_peaks()
+    t_opt_ms = flops / (bf16_tf * 1e12) * 1e3
+
+    # per-op averages over the timed region
+    agg = {}
+    for (name, nano, layer, stream_id, grid, us) in op_times:
+        bound, units = op_algorithmic(work, b, plan, name, nano) if nano >= 0 else op_algorithmic(work, b, plan, name, 0)
+        a = agg.setdefault(name, {"launches": 0, "us": 0.0, "units": 0.0, "bound": bound})
+        a["launches"] += 1
+        a["us"] += us
+        a["units"] += units
+    dominant = max(agg, key=lambda k: agg[k]["us"]) if agg else None
+    roofline = None
+    if dominant:
+        a = agg[dominant]
+        avg_us = a["us"] / a["launches"]
+        per_launch = a["units"] / a["launches"]
+        if a["bound"] == "tensor":
+            peak = bf16_tf
+            achieved = per_launch / (avg_us * 1e-6) / 1e12
+            unit = "TFLOP/s"
+        else:
+            peak = hbm_gbs
+            achieved = per_launch / (avg_us * 1e-6) / 1e9
+            unit = "GB/s"
+        roofline = {"kernel": dominant, "bound": a["bound"], "achieved": round(achieved, 1), "peak": peak,
+                    "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
+                    "avg_launch_us": round(avg_us, 2), "launches_per_step": a["launches"] / args.steps,
+                    "peak_source": f"{peak_src} (burst)"}
+    op_summary = {k: {"avg_us": round(v["us"] / v["launches"], 1), "launches": v["launches"],
+                      "share": round(v["us"] / max(sum(x["us"] for x in agg.values()), 1e-9), 3)}
+                  for k, v in agg.items()}
+
+    extras = {}
+    if not args.no_extras:
+        # ---- the same work without overlap: sequential plan, one nano-batch, every SM
+        seq_plan = dw.plan(nano=1, template=0)
+        for _ in range(3):
+            dw.forward(seq_plan, stream)
+        nf.check(nf.nf_set_timing(dw.model, True), "timing")
+        torch.cuda.synchronize(dev)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        nseq = max(3, args.steps // 2)
+        for _ in range(nseq):
+            dw.forward(seq_plan, stream)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        st, seq_ops = nf.nf_get_op_times(dw.model, 1 << 20)
+        nf.nf_set_timing(dw.model, False)
+        seq_ms = s0.elapsed_time(s1) / nseq
+        iso = {}
+        for (name, nano, layer, stream_id, grid, us) in seq_ops:
+            iso[name] = iso.get(name, 0.0) + us / nseq
+        extras["sequential"] = {"ms_per_step": round(seq_ms, 4),
+                                "isolated_op_ms": {k: round(v / 1000, 4) for k, v in iso.items()},
+                                "sum_isolated_gemm_ms": round(sum(v for k, v in iso.items() if k != "attention") / 1000, 4),
+                                "sum_isolated_attention_ms": round(iso.get("attention", 0.0) / 1000, 4)}
+
+        # ---- end to end through the C ABI with host buffers: H2D inputs, D2H result, every step
+        s = work.shape
+        host_in = dw.hidden_in.cpu().pin_memory() if dw.hidden_in is not None else None
+        host_tok = dw.tokens.cpu().pin_memory() if dw.tokens is not None else None
+        host_meta = [t.cpu().pin_memory() for t in (dw.positions, dw.ctx_len, dw.page_indptr, dw.page_indices)]
+        dev_meta = [torch.empty_like(t) for t in (dw.positions, dw.ctx_len, dw.page_indptr, dw.page_indices)]
+        dev_in = torch.empty_like(dw.hidden_in) if dw.hidden_in is not None else None
+        dev_tok = torch.empty_like(dw.tokens) if dw.tokens is not None else None
+        host_out = torch.empty(tuple(dw.hidden_out.shape), dtype=dw.hidden_out.dtype).pin_memory()
+        io = dw.make_io(hidden_in=dev_in)
+        io.positions, io.ctx_len, io.page_indptr, io.page_indices = [t.data_ptr() for t in dev_meta]
+        if dev_tok is not None:
+            io.token_ids = dev_tok.data_ptr()
+        h2d = sum(t.numel() * t.element_size() for t in host_meta)
+        h2d += host_in.numel() * host_in.element_size() if host_in is not None else 0
+        h2d += host_tok.numel() * host_tok.element_size() if host_tok is not None else 0
+        d2h = host_out.numel() * host_out.element_size()
+
+        def e2e_step():
+            for d_, h_ in zip(dev_meta, host_meta):
+                d_.copy_(h_, non_blocking=True)
+            if dev_in is not None:
+                dev_in.copy_(host_in, non_blocking=True)
+            if dev_tok is not None:
+                dev_tok.copy_(host_tok, non_blocking=True)
+            dw.forward(plan, stream, io=io)
+            host_out.copy_(dw.hidden_out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        nf.check(dw.sync(), "e2e steps")
+        e2e_ms = dist.max(t0.elapsed_time(t1))
+        extras["e2e"] = {"value": dist.world * R * args.steps / (e2e_ms / 1000.0), "unit": "decode tokens/s",
+                         "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        n = args.cpu_sample or R
+        times, threads = cpu_oracle_sample(work, b, n, repeats=1)
+        cpu = {"value": n / times[0], "unit": "decode tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} of {R} decode requests of {args.workload}, no prefill chunk, float64 numpy oracle, "
+                         f"inputs pre-generated, {times[0]:.1f} s"}
+
+    line = {"metric": METRIC, "value": value, "unit": "decode tokens/s", "n_gpus": dist.world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded random-init weights, seeded paged KV cache)",
+            "config": {"workload": args.workload, "decode_requests": R, "prefill_len": b.prefill_len,
+                       "tokens": b.num_tokens, "ctx": "uniform [1024,1536]" if args.workload.startswith("llama") else "",
+                       "parallelism": f"replicas x{dist.world}", "plan": plan.describe(),
+                       "l2": "working set (KV cache + weights) > 126 MB L2 on every step; no flush"},
+            "frac_of_compute_optimum": round(t_opt_ms / ms_step, 4),
+            "t_opt_ms": round(t_opt_ms, 4), "iteration_tflop": round(flops / 1e12, 4),
+            "all_tokens_per_s": dist.world * b.num_tokens * args.steps / (ms_total / 1000.0),
+            "ops": op_summary, "roofline": roofline, "cpu_baseline": cpu, "clocks": clk,
+            "gpu_launches": count_launches(work, plan) * args.steps}
+    line.update(extras)
+    if "e2e" not in line:
+        line["e2e"] = None
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dw.close()
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    from synth.workloads import WORKLOADS
+    work = WORKLOADS[args.workload]
+    dist = Dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, work, dist)
+        else:
+            run_ours(args, work, dist)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

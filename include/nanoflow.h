@@ -1,0 +1,291 @@
+/*
+ * nanoflow.h — C ABI of a B200 (sm_100a) implementation of one NanoFlow-style
+ * serving iteration with intra-device overlap.
+ *
+ * What the library computes. One batched serving iteration of a Llama-style
+ * transformer (NanoFlow README "Feasibility": Llama2-70B, Llama3-8B, Mixtral 8x7B)
+ * over a mixed batch: R decode requests (one new token each, attending to their
+ * paged KV cache) followed by one prefill chunk of C tokens. Per layer:
+ * RMSNorm -> QKV projection -> RoPE -> K/V written into the paged cache ->
+ * paged GQA decode attention and causal prefill attention -> output projection
+ * + residual -> RMSNorm -> SwiGLU FFN (or top-k mixture of SwiGLU experts) +
+ * residual; full models add the token embedding, the final norm, the LM head
+ * and greedy argmax.
+ *
+ * How it is scheduled. "Nano-batching" splits the batch into smaller
+ * nano-batches and duplicates each operation per nano-batch so that operations
+ * of different nano-batches no longer depend on one another (arXiv abstract of
+ * "NanoFlow: Towards Optimal Large Language Model Serving Throughput"; README
+ * "Abstract"). A "device-level pipeline with execution unit scheduling" then
+ * runs the compute-bound GEMMs of one nano-batch on one part of the GPU while
+ * the memory-bound attention of another runs on the rest (README
+ * "Introduction" and "Abstract"). The number, size, order and GPU resource
+ * split of the nano-batches are chosen automatically, taking interference into
+ * account (arXiv abstract). Here the split is a set of SMs: GEMM kernels and
+ * attention kernels are persistent and launched with grids that claim disjoint
+ * SM sets on two CUDA streams; nf_plan_iteration picks the plan by exhaustive
+ * search over per-kernel costs.
+ *
+ * Conventions.
+ *  - Every call returns an nf_status; nothing aborts or prints.
+ *  - bf16 tensors are passed as raw 16-bit patterns (void*), row-major.
+ *  - Device pointers are owned by the caller unless stated otherwise; the model
+ *    owns its packed weights and workspace (freed by nf_destroy_model).
+ *  - `stream` arguments are cudaStream_t values passed as void* (NULL = legacy
+ *    default stream). Work is asynchronous on that stream.
+ *  - A model is not thread-safe: one forward at a time per model.
+ *  - Errors detected on the device (page index out of range, token id out of
+ *    range, a wait that timed out) are latched in a device status word and
+ *    returned by nf_sync_status().
+ *  - Token order within an iteration: decode rows first (request order), then
+ *    the prefill chunk. Decode request r has ctx_len[r] cached tokens; its new
+ *    token sits at position ctx_len[r] and its K/V go to that slot. The chunk is
+ *    a fresh prompt at positions 0..C-1.
+ */
+#ifndef NANOFLOW_H
+#define NANOFLOW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NF_OK = 0,
+    NF_ERR_INVALID_ARGUMENT = 1, /* a null pointer, a size out of range, an inconsistent descriptor */
+    NF_ERR_UNSUPPORTED = 2,      /* a shape the kernels do not handle (see nf_init_model) */
+    NF_ERR_OUT_OF_MEMORY = 3,    /* device allocation failed */
+    NF_ERR_CUDA = 4,             /* a CUDA runtime call failed (no device, launch failure, ...) */
+    NF_ERR_DEVICE_TIMEOUT = 5,   /* a device-side wait exceeded its time limit and gave up */
+    NF_ERR_DEVICE_BOUNDS = 6     /* a device-side index check failed; the access was skipped */
+} nf_status;
+
+/* Static description of the string of a status code (never NULL). */
+const char* nf_status_string(int status);
+
+/* ------------------------------------------------------------------ model */
+
+typedef struct nf_model nf_model; /* opaque */
+
+typedef struct {
+    int32_t n_layers;
+    int32_t hidden;       /* H, multiple of 256 */
+    int32_t n_q_heads;    /* nq */
+    int32_t n_kv_heads;   /* nkv; nq % nkv == 0 and nq / nkv <= 16 */
+    int32_t head_dim;     /* d: 64 or 128 */
+    int32_t ffn;          /* F (per expert for MoE), multiple of 128 */
+    int32_t vocab;        /* 0: layer slice (hidden in/out); >0: embedding + final norm + LM head, multiple of 256 */
+    int32_t n_experts;    /* 0: dense SwiGLU FFN; 1..16: mixture of experts */
+    int32_t top_k;        /* experts per token (MoE), 1..n_experts */
+    float rms_eps;        /* RMSNorm epsilon */
+    float rope_theta;     /* RoPE base */
+    int32_t page_size;    /* tokens per KV page; must be 16 */
+    int32_t max_tokens;   /* upper bound on T = R + C per iteration (workspace sizing) */
+    int32_t max_requests; /* upper bound on R */
+    int32_t max_position; /* positions must be < max_position (RoPE table length) */
+} nf_model_config;
+
+/* Validate `cfg`, allocate the model's packed-weight buffers and workspace and
+ * build the RoPE table (angles pos * theta^(-2i/d) in double, stored as fp32).
+ * On success *out owns device memory until nf_destroy_model. Requirements:
+ * (nq + 2 nkv) d, nq d, H and 2F divisible by 256; H divisible by 64. */
+nf_status nf_init_model(const nf_model_config* cfg, nf_model** out);
+
+/* Weights of one layer, canonical Hugging Face layout: device pointers to bf16,
+ * linear weights [out_features x in_features] row-major. The library copies and
+ * repacks them (QKV concatenated, gate/up interleaved per 128-row tile, RMSNorm
+ * gamma folded into the columns of the following projection); the caller may
+ * free its buffers once the stream has passed the copy. */
+typedef struct {
+    const void* attn_norm; /* [H] */
+    const void* wq;        /* [nq*d x H] */
+    const void* wk;        /* [nkv*d x H] */
+    const void* wv;        /* [nkv*d x H] */
+    const void* wo;        /* [H x nq*d] */
+    const void* ffn_norm;  /* [H] */
+    const void* w_gate;    /* [F x H] (dense) */
+    const void* w_up;      /* [F x H] (dense) */
+    const void* w_down;    /* [H x F] (dense) */
+    const void* router;      /* [E x H] (MoE) */
+    const void* router_bias; /* [E] (MoE) */
+    const void* const* expert_gate; /* host array of E device pointers, each [F x H] (MoE) */
+    const void* const* expert_up;   /* host array of E device pointers, each [F x H] (MoE) */
+    const void* const* expert_down; /* host array of E device pointers, each [H x F] (MoE) */
+} nf_layer_weights;
+
+nf_status nf_set_layer_weights(nf_model* m, int32_t layer, const nf_layer_weights* w, void* stream);
+
+/* Embedding, final norm and LM head (models with vocab > 0): device bf16 pointers. */
+typedef struct {
+    const void* embed;      /* [V x H] */
+    const void* final_norm; /* [H] */
+    const void* lm_head;    /* [V x H] */
+} nf_global_weights;
+
+nf_status nf_set_global_weights(nf_model* m, const nf_global_weights* w, void* stream);
+
+void nf_destroy_model(nf_model* m);
+
+/* ------------------------------------------------------------------ plan */
+
+/* Host-side description of the iteration's batch. */
+typedef struct {
+    int32_t num_decode;        /* R >= 0 */
+    int32_t prefill_len;       /* C >= 0 */
+    int32_t prefix_len;        /* must be 0 (fresh prompt) */
+    const int32_t* ctx_len;    /* host [R]: cached tokens per decode request (>= 0) */
+    const int32_t* page_indptr; /* host [R + 2]: CSR offsets of each request's pages (prefill last) */
+    int32_t num_pages;         /* pages in each layer's pool */
+} nf_batch_desc;
+
+#define NF_MAX_NANO 4
+
+typedef struct {
+    int32_t force_nano;     /* 0: search; 1..4: this many nano-batches */
+    int32_t force_sm_attn;  /* 0: search; >0: SMs given to attention kernels (overlapped plans) */
+    int32_t force_template; /* -1: search; else an NF_TEMPLATE_* value */
+    int32_t sm_total;       /* 0: every SM of the device */
+} nf_plan_opts;
+
+enum {
+    NF_TEMPLATE_SEQUENTIAL = 0, /* one nano-batch after another, each op on all SMs (no overlap) */
+    NF_TEMPLATE_PIPELINED = 1,  /* attention of nano-batch j co-runs with the GEMMs of the others */
+};
+
+typedef struct {
+    int32_t n_nano;
+    int32_t tok_begin[NF_MAX_NANO]; /* nano-batch j = tokens [tok_begin[j], tok_end[j]) */
+    int32_t tok_end[NF_MAX_NANO];
+    int32_t nano_order[NF_MAX_NANO]; /* pipeline order of the nano-batches */
+    int32_t order_template;       /* NF_TEMPLATE_* */
+    int32_t sm_attn;              /* SMs claimed by attention kernels while overlapped */
+    int32_t sm_gemm;              /* SMs claimed by GEMM kernels while overlapped */
+    int32_t sm_total;
+    float predicted_us;           /* simulated iteration time of this plan */
+    float predicted_serial_us;    /* simulated time of the same work without overlap */
+    int32_t num_decode, prefill_len, num_tokens; /* copied from the batch */
+    int64_t kv_pages_read;        /* decode + prefill KV pages (all KV heads) read per layer */
+    int64_t decode_items;         /* decode attention work items (sizes the split-KV workspace) */
+} nf_plan;
+
+/* Choose nano-batch count, sizes (token ranges cut at request boundaries, the
+ * prefill chunk whole), op order and SM split minimising the simulated two-stream
+ * makespan over the model's per-kernel cost tables (arXiv abstract: "number,
+ * size, ordering, and GPU resource allocation of nano-batches"). Host only. */
+nf_status nf_plan_iteration(const nf_model* m, const nf_batch_desc* b, const nf_plan_opts* opts, nf_plan* out);
+
+/* The same search for a model configuration without a device or a model handle:
+ * uses the built-in default cost tables and `sm_count` SMs (> 0). Host only. */
+nf_status nf_plan_for_config(const nf_model_config* cfg, int32_t sm_count, const nf_batch_desc* b,
+                             const nf_plan_opts* opts, nf_plan* out);
+
+/* ------------------------------------------------------------------ forward */
+
+/* Per-iteration inputs and outputs, all device pointers owned by the caller. */
+typedef struct {
+    const int32_t* token_ids;    /* [T] (vocab > 0) */
+    const void* hidden_in;       /* [T x H] bf16 (vocab == 0) */
+    const int32_t* positions;    /* [T] */
+    const int32_t* ctx_len;      /* [R] */
+    const int32_t* page_indptr;  /* [R + 2] */
+    const int32_t* page_indices; /* [page_indptr[R+1]] page ids < num_pages */
+    void* const* kv_pools;       /* host array [n_layers]: device [num_pages][2][nkv][16][d] bf16, updated in place */
+    int32_t num_pages;
+    void* hidden_out;            /* [T x H] bf16, nullable */
+    float* hidden_out_f32;       /* [T x H] fp32 residual stream after the last layer, nullable */
+    void* logits;                /* [rows x V] bf16, nullable; rows = R + (C > 0) */
+    int32_t* next_token;         /* [rows], nullable */
+    int32_t* topk_idx;           /* MoE: [n_layers x T x top_k] expert ids, nullable */
+    float* topk_w;               /* MoE: [n_layers x T x top_k] routing weights, nullable */
+    float* router_logits;        /* MoE: [n_layers x T x E] fp32, nullable */
+} nf_iter_io;
+
+/* Run the iteration described by `plan` (made by nf_plan_iteration for the same
+ * batch). GEMMs run on `stream`, attention on a model-owned second stream that
+ * forks from and joins back into `stream`. Asynchronous. */
+nf_status nf_forward_iteration(nf_model* m, const nf_plan* plan, const nf_iter_io* io, void* stream);
+
+/* Wait for the model's streams and return (and clear) the latched device status. */
+nf_status nf_sync_status(nf_model* m);
+
+/* Time each kernel kind of this model at the sizes of `b` and several SM shares,
+ * plus one co-run, and store the results as the planner's cost tables. Runs real
+ * launches on `stream` with the buffers of `io` (the KV pools are rewritten with
+ * the same values a forward would write). */
+nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_iter_io* io, void* stream);
+
+/* Per-CTA placement trace of the last forward (enabled with nf_set_trace):
+ * entries of {kernel id, sm id, start ns, end ns}. Returns the entry count
+ * written (<= capacity), or a negative nf_status. */
+typedef struct {
+    int32_t kernel;   /* NF_KERNEL_* */
+    int32_t smid;
+    uint64_t t_start; /* %globaltimer ns */
+    uint64_t t_end;
+} nf_trace_entry;
+
+enum { NF_KERNEL_GEMM = 1, NF_KERNEL_DECODE_ATTN = 2, NF_KERNEL_PREFILL_ATTN = 3 };
+
+nf_status nf_set_trace(nf_model* m, int32_t enable);
+int64_t nf_get_trace(nf_model* m, nf_trace_entry* out, int64_t capacity);
+
+/* Per-operation CUDA-event timing (enabled with nf_set_timing, which also clears the
+ * record): one entry per operation of every forward since, in issue order, with the duration
+ * between events recorded around it on its own stream (a co-running op on the other
+ * stream is included in the wall time it sees, not excluded). */
+typedef struct {
+    int32_t kind;   /* NF_OP_* */
+    int32_t nano;   /* nano-batch index (-1 for the LM head) */
+    int32_t layer;
+    int32_t stream; /* 0: GEMM stream, 1: attention stream */
+    int32_t grid;   /* CTAs launched (SMs claimed) */
+    float us;
+} nf_op_time;
+
+enum { NF_OP_QKV = 0, NF_OP_ATTN = 1, NF_OP_O = 2, NF_OP_GATE_UP = 3, NF_OP_DOWN = 4, NF_OP_MOE = 5,
+       NF_OP_LM_HEAD = 6 };
+
+nf_status nf_set_timing(nf_model* m, int32_t enable);
+/* Waits for the model's streams; returns the number of entries written (<= capacity) or a negative nf_status. */
+int64_t nf_get_op_times(nf_model* m, nf_op_time* out, int64_t capacity);
+
+/* ------------------------------------------------------------------ single ops
+ * The kernels of the hot path, callable one at a time (tests, calibration,
+ * isolated timing). Same kernels as nf_forward_iteration uses.
+ */
+
+/* C[M x N] (fp32) = A[M x K] * B[N x K]^T with bf16 A, B (device, row-major) on the
+ * tcgen05 tensor cores with TMEM accumulation. M >= 1, N % 256 == 0, K % 64 == 0,
+ * A and B 16-byte aligned. `sm_count` = CTAs of the persistent grid (0 = all SMs). */
+nf_status nf_op_gemm_bf16(const void* A, const void* B, float* C, int32_t M, int32_t N, int32_t K,
+                          int32_t sm_count, void* stream);
+
+/* Paged GQA decode attention of requests [req_begin, req_end) of layer `layer`'s
+ * pool: out[r][h][:] = softmax(q[r][h] K_r^T / sqrt(d)) V_r over the ctx_len[r]+1
+ * keys of request r, K/V of kv head h / (nq / nkv). q and out are [R x nq x d]
+ * bf16 rows of the iteration (decode rows). Uses the model's workspace for the
+ * split-KV partial results. */
+nf_status nf_op_decode_attention(nf_model* m, const void* q, void* out, const nf_iter_io* io, int32_t layer,
+                                 int32_t req_begin, int32_t req_end, int32_t sm_count, void* stream);
+
+/* Causal attention of the prefill chunk (positions 0..C-1) reading its K/V from
+ * the pages of request R (the prefill request) of layer `layer`. q and out are
+ * [C x nq x d] bf16. */
+nf_status nf_op_prefill_attention(nf_model* m, const void* q, void* out, const nf_iter_io* io, int32_t layer,
+                                  int32_t num_decode, int32_t prefill_len, int32_t sm_count, void* stream);
+
+/* Device-wait self test: one CTA waits on a flag in device memory that nothing sets,
+ * with a time limit of `limit_ns`; returns NF_ERR_DEVICE_TIMEOUT (the expected
+ * outcome) after the kernel has given up and exited, or NF_OK if the flag was set. */
+nf_status nf_op_wait_flag_test(int32_t* flag_device, uint64_t limit_ns, void* stream);
+
+/* Library version string. */
+const char* nf_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NANOFLOW_H */

@@ -1,0 +1,783 @@
+// C ABI: model set-up, weight repacking, the two-stream iteration executor, status and
+// trace access, and single-kernel entry points.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "nanoflow.h"
+#include "nf_attention.h"
+#include "nf_internal.h"
+#include "nf_misc.h"
+#include "nf_model.h"
+#include "nf_schedule.h"
+
+using nf::GemmArgs;
+
+namespace {
+
+#define NF_CUDA_TRY(expr)                                    \
+    do {                                                     \
+        cudaError_t _e = (expr);                             \
+        if (_e != cudaSuccess) return NF_ERR_CUDA;           \
+    } while (0)
+
+template <typename T>
+T* dalloc(nf_model* m, size_t count) {
+    void* p = nullptr;
+    if (count == 0) count = 1;
+    if (cudaMalloc(&p, count * sizeof(T)) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    m->allocations.push_back(p);
+    return static_cast<T*>(p);
+}
+
+void dfree(nf_model* m, void* p) {
+    if (p == nullptr) return;
+    auto it = std::find(m->allocations.begin(), m->allocations.end(), p);
+    if (it != m->allocations.end()) m->allocations.erase(it);
+    cudaFree(p);
+}
+
+GemmArgs base_args(const nf_model* m) {
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.n_part = m->n_part;
+    a.inv_dim = 1.0f / (float)m->dims.H;
+    a.eps = m->cfg.rms_eps;
+    a.status = m->status;
+    if (m->trace_on) {
+        a.trace_ctr = m->trace_ctr;
+        a.trace = m->trace;
+        a.trace_cap = m->trace_cap;
+    }
+    return a;
+}
+
+void set_tiles(GemmArgs& a, int M, int N, int K) {
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.m_tiles = (M + nf::kGemmBM - 1) / nf::kGemmBM;
+    a.n_tiles = N / nf::kGemmBN;
+    a.k_blocks = K / nf::kGemmBK;
+}
+
+int gemm_grid(const GemmArgs& a, int grid) {
+    const int tiles = a.m_tiles * a.n_tiles;
+    return std::max(1, std::min(grid, tiles));
+}
+
+bool valid_config(const nf_model_config& c) {
+    if (c.n_layers < 1 || c.hidden <= 0 || c.hidden % 256 != 0) return false;
+    if (c.n_q_heads <= 0 || c.n_kv_heads <= 0 || c.n_q_heads % c.n_kv_heads != 0) return false;
+    if (c.n_q_heads / c.n_kv_heads > 16) return false;
+    if (c.head_dim != 64 && c.head_dim != 128) return false;
+    if (((c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim) % 256 != 0) return false;
+    if ((c.n_q_heads * c.head_dim) % 64 != 0) return false;
+    if (c.ffn <= 0 || c.ffn % 128 != 0) return false;
+    if (c.vocab < 0 || c.vocab % 256 != 0) return false;
+    if (c.n_experts < 0 || c.n_experts > 16) return false;
+    if (c.n_experts > 0 && (c.top_k < 1 || c.top_k > c.n_experts)) return false;
+    if (c.page_size != 16) return false;
+    if (c.max_tokens < 1 || c.max_requests < 0 || c.max_requests > c.max_tokens) return false;
+    if (c.max_position < 1) return false;
+    if (!(c.rms_eps >= 0.f) || !(c.rope_theta > 0.f)) return false;
+    return true;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ status / version
+
+extern "C" const char* nf_status_string(int s) {
+    switch (s) {
+        case NF_OK: return "ok";
+        case NF_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case NF_ERR_UNSUPPORTED: return "unsupported shape";
+        case NF_ERR_OUT_OF_MEMORY: return "out of device memory";
+        case NF_ERR_CUDA: return "CUDA runtime error";
+        case NF_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case NF_ERR_DEVICE_BOUNDS: return "device-side index out of range";
+        default: return "unknown status";
+    }
+}
+
+extern "C" const char* nf_version(void) { return "nanoflow-b200 0.1 (sm_100a)"; }
+
+// ------------------------------------------------------------------ model life cycle
+
+extern "C" void nf_destroy_model(nf_model* m) {
+    if (m == nullptr) return;
+    cudaDeviceSynchronize();
+    for (void* p : m->allocations) cudaFree(p);
+    for (cudaEvent_t e : m->events) cudaEventDestroy(e);
+    for (cudaEvent_t e : m->t_ev) cudaEventDestroy(e);
+    if (m->ev_fork) cudaEventDestroy(m->ev_fork);
+    if (m->ev_join) cudaEventDestroy(m->ev_join);
+    if (m->s_attn) cudaStreamDestroy(m->s_attn);
+    cudaGetLastError();
+    delete m;
+}
+
+extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) {
+    if (cfg == nullptr || out == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    *out = nullptr;
+    if (!valid_config(*cfg)) {
+        const nf_model_config& c = *cfg;
+        const bool structural = c.n_layers >= 1 && c.hidden > 0 && c.n_q_heads > 0 && c.n_kv_heads > 0 &&
+                                c.ffn > 0 && c.max_tokens >= 1 && c.page_size > 0;
+        return structural ? NF_ERR_UNSUPPORTED : NF_ERR_INVALID_ARGUMENT;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return NF_ERR_CUDA; }
+    int major = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (major < 10) return NF_ERR_UNSUPPORTED;
+
+    nf_model* m = new (std::nothrow) nf_model();
+    if (m == nullptr) return NF_ERR_OUT_OF_MEMORY;
+    m->cfg = *cfg;
+    nf::ModelDims& d = m->dims;
+    d.L = cfg->n_layers;
+    d.H = cfg->hidden;
+    d.nq = cfg->n_q_heads;
+    d.nkv = cfg->n_kv_heads;
+    d.d = cfg->head_dim;
+    d.F = cfg->ffn;
+    d.E = cfg->n_experts;
+    d.K = cfg->n_experts > 0 ? cfg->top_k : 1;
+    d.qkv = (d.nq + 2 * d.nkv) * d.d;
+    m->n_part = d.H / 256;
+    m->sm_count = nf::device_sm_count();
+    m->cost = nf::default_cost_model(m->sm_count);
+    m->layers.resize(d.L);
+    m->kv_ptr.assign(d.L, nullptr);
+    m->kv_pages.assign(d.L, 0);
+    m->kv_tm.resize(d.L);
+
+    const size_t T = (size_t)cfg->max_tokens;
+    const size_t TK = T * (size_t)d.K;
+    const size_t act_rows = d.E > 0 ? TK : T;
+    const size_t lm_rows = (size_t)cfg->max_requests + 1;
+    bool ok = true;
+    ok &= (m->resid = dalloc<float>(m, T * d.H)) != nullptr;
+    ok &= (m->xb = dalloc<uint16_t>(m, T * d.H)) != nullptr;
+    ok &= (m->partials = dalloc<float>(m, T * m->n_part)) != nullptr;
+    ok &= (m->q = dalloc<uint16_t>(m, T * d.nq * d.d)) != nullptr;
+    ok &= (m->attn_o = dalloc<uint16_t>(m, T * d.nq * d.d)) != nullptr;
+    ok &= (m->act = dalloc<uint16_t>(m, act_rows * d.F)) != nullptr;
+    ok &= (m->rope_cos = dalloc<float>(m, (size_t)cfg->max_position * d.d / 2)) != nullptr;
+    ok &= (m->rope_sin = dalloc<float>(m, (size_t)cfg->max_position * d.d / 2)) != nullptr;
+    ok &= (m->item_off = dalloc<int>(m, (size_t)cfg->max_requests + 1)) != nullptr;
+    ok &= (m->status = dalloc<int>(m, 1)) != nullptr;
+    m->trace_cap = 65536;
+    ok &= (m->trace_ctr = dalloc<int>(m, 1)) != nullptr;
+    ok &= (m->trace = dalloc<nf_trace_entry>(m, m->trace_cap)) != nullptr;
+    if (cfg->vocab > 0) {
+        ok &= (m->lm_in = dalloc<uint16_t>(m, lm_rows * d.H)) != nullptr;
+        ok &= (m->lm_partials = dalloc<float>(m, lm_rows * m->n_part)) != nullptr;
+        ok &= (m->tile_max = dalloc<float>(m, lm_rows * (cfg->vocab / 256))) != nullptr;
+        ok &= (m->tile_arg = dalloc<int>(m, lm_rows * (cfg->vocab / 256))) != nullptr;
+    }
+    if (d.E > 0) {
+        ok &= (m->moe_logits = dalloc<float>(m, T * d.E)) != nullptr;
+        ok &= (m->moe_idx = dalloc<int>(m, TK)) != nullptr;
+        ok &= (m->moe_w = dalloc<float>(m, TK)) != nullptr;
+        ok &= (m->moe_counts = dalloc<int>(m, (size_t)d.E + 1)) != nullptr;
+        ok &= (m->moe_perm = dalloc<int>(m, TK)) != nullptr;
+        ok &= (m->moe_inv = dalloc<int>(m, TK)) != nullptr;
+        ok &= (m->moe_a = dalloc<uint16_t>(m, TK * d.H)) != nullptr;
+        ok &= (m->moe_part = dalloc<float>(m, TK * m->n_part)) != nullptr;
+        ok &= (m->moe_y = dalloc<float>(m, TK * d.H)) != nullptr;
+    }
+    if (!ok) { nf_destroy_model(m); return NF_ERR_OUT_OF_MEMORY; }
+
+    // RoPE angles pos * theta^(-2i/d) in double, stored as fp32 cos / sin.
+    {
+        const int half = d.d / 2;
+        std::vector<float> c((size_t)cfg->max_position * half), s(c.size());
+        for (int p = 0; p < cfg->max_position; ++p)
+            for (int i = 0; i < half; ++i) {
+                const double ang = (double)p * std::pow((double)cfg->rope_theta, -2.0 * i / d.d);
+                c[(size_t)p * half + i] = (float)std::cos(ang);
+                s[(size_t)p * half + i] = (float)std::sin(ang);
+            }
+        if (cudaMemcpy(m->rope_cos, c.data(), c.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+            cudaMemcpy(m->rope_sin, s.data(), s.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
+            nf_destroy_model(m);
+            return NF_ERR_CUDA;
+        }
+    }
+    if (cudaMemset(m->status, 0, sizeof(int)) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&m->s_attn, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&m->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&m->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+        nf_destroy_model(m);
+        return NF_ERR_CUDA;
+    }
+    ok = nf::make_tmap_bf16_2d(&m->tm_xb, m->xb, T, d.H, nf::kGemmBM) &&
+         nf::make_tmap_bf16_2d(&m->tm_attn_o, m->attn_o, T, (uint64_t)d.nq * d.d, nf::kGemmBM) &&
+         nf::make_tmap_bf16_2d(&m->tm_act, m->act, act_rows, d.F, nf::kGemmBM);
+    if (ok && cfg->vocab > 0) ok = nf::make_tmap_bf16_2d(&m->tm_lm_in, m->lm_in, lm_rows, d.H, nf::kGemmBM);
+    if (ok && d.E > 0) ok = nf::make_tmap_bf16_2d(&m->tm_moe_a, m->moe_a, TK, d.H, nf::kGemmBM);
+    if (!ok) { nf_destroy_model(m); return NF_ERR_CUDA; }
+    *out = m;
+    return NF_OK;
+}
+
+extern "C" nf_status nf_set_layer_weights(nf_model* m, int32_t layer, const nf_layer_weights* w, void* stream) {
+    if (m == nullptr || w == nullptr || layer < 0 || layer >= m->dims.L) return NF_ERR_INVALID_ARGUMENT;
+    const nf::ModelDims& d = m->dims;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo || !w->ffn_norm) return NF_ERR_INVALID_ARGUMENT;
+    if (d.E == 0 && (!w->w_gate || !w->w_up || !w->w_down)) return NF_ERR_INVALID_ARGUMENT;
+    if (d.E > 0 && (!w->router || !w->router_bias || !w->expert_gate || !w->expert_up || !w->expert_down))
+        return NF_ERR_INVALID_ARGUMENT;
+    nf::LayerWeights& L = m->layers[layer];
+    const int E = std::max(d.E, 1);
+    if (!L.loaded) {
+        bool ok = true;
+        ok &= (L.wqkv = dalloc<uint16_t>(m, (size_t)d.qkv * d.H)) != nullptr;
+        ok &= (L.wo = dalloc<uint16_t>(m, (size_t)d.H * d.nq * d.d)) != nullptr;
+        ok &= (L.wgu = dalloc<uint16_t>(m, (size_t)E * 2 * d.F * d.H)) != nullptr;
+        ok &= (L.wd = dalloc<uint16_t>(m, (size_t)E * d.H * d.F)) != nullptr;
+        if (d.E > 0) {
+            ok &= (L.router = dalloc<float>(m, (size_t)d.E * d.H)) != nullptr;
+            ok &= (L.router_bias = dalloc<float>(m, (size_t)d.E)) != nullptr;
+        }
+        if (!ok) return NF_ERR_OUT_OF_MEMORY;
+    }
+    const uint16_t* an = (const uint16_t*)w->attn_norm;
+    const uint16_t* fn = (const uint16_t*)w->ffn_norm;
+    const int qd = d.nq * d.d, kd = d.nkv * d.d;
+    // QKV = [wq; wk; wv] with the attention-norm gamma folded into the columns
+    NF_CUDA_TRY(nf::launch_pack_rows((const uint16_t*)w->wq, L.wqkv, qd, d.H, an, qd, 0, 0, s));
+    NF_CUDA_TRY(nf::launch_pack_rows((const uint16_t*)w->wk, L.wqkv + (size_t)qd * d.H, kd, d.H, an, kd, 0, 0, s));
+    NF_CUDA_TRY(nf::launch_pack_rows((const uint16_t*)w->wv, L.wqkv + (size_t)(qd + kd) * d.H, kd, d.H, an, kd, 0,
+                                     0, s));
+    NF_CUDA_TRY(nf::launch_pack_rows((const uint16_t*)w->wo, L.wo, d.H, qd, nullptr, d.H, 0, 0, s));
+    // gate/up interleaved per 128 rows: rows [256t, 256t+128) = gate [128t, 128t+128), next 128 = up
+    for (int e = 0; e < E; ++e) {
+        const uint16_t* g = (const uint16_t*)(d.E > 0 ? w->expert_gate[e] : w->w_gate);
+        const uint16_t* u = (const uint16_t*)(d.E > 0 ? w->expert_up[e] : w->w_up);
+        const uint16_t* dn = (const uint16_t*)(d.E > 0 ? w->expert_down[e] : w->w_down);
+        if (!g || !u || !dn) return NF_ERR_INVALID_ARGUMENT;
+        uint16_t* gu = L.wgu + (size_t)e * 2 * d.F * d.H;
+        NF_CUDA_TRY(nf::launch_pack_rows(g, gu, d.F, d.H, fn, 128, 256, 0, s));
+        NF_CUDA_TRY(nf::launch_pack_rows(u, gu, d.F, d.H, fn, 128, 256, 128, s));
+        NF_CUDA_TRY(nf::launch_pack_rows(dn, L.wd + (size_t)e * d.H * d.F, d.H, d.F, nullptr, d.H, 0, 0, s));
+    }
+    if (d.E > 0) {
+        NF_CUDA_TRY(nf::launch_widen_scaled((const uint16_t*)w->router, L.router, d.E, d.H, fn, s));
+        NF_CUDA_TRY(nf::launch_widen_scaled((const uint16_t*)w->router_bias, L.router_bias, 1, d.E, nullptr, s));
+    }
+    bool ok = nf::make_tmap_bf16_2d(&L.tm_qkv, L.wqkv, d.qkv, d.H, nf::kGemmBN) &&
+              nf::make_tmap_bf16_2d(&L.tm_o, L.wo, d.H, qd, nf::kGemmBN) &&
+              nf::make_tmap_bf16_2d(&L.tm_gu, L.wgu, (uint64_t)E * 2 * d.F, d.H, nf::kGemmBN) &&
+              nf::make_tmap_bf16_2d(&L.tm_d, L.wd, (uint64_t)E * d.H, d.F, nf::kGemmBN);
+    if (!ok) return NF_ERR_CUDA;
+    L.loaded = true;
+    return NF_OK;
+}
+
+extern "C" nf_status nf_set_global_weights(nf_model* m, const nf_global_weights* w, void* stream) {
+    if (m == nullptr || w == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    if (m->cfg.vocab <= 0) return NF_ERR_INVALID_ARGUMENT;
+    if (!w->embed || !w->final_norm || !w->lm_head) return NF_ERR_INVALID_ARGUMENT;
+    const int V = m->cfg.vocab, H = m->dims.H;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!m->globals_loaded) {
+        if ((m->embed = dalloc<uint16_t>(m, (size_t)V * H)) == nullptr) return NF_ERR_OUT_OF_MEMORY;
+        if ((m->lm_head = dalloc<uint16_t>(m, (size_t)V * H)) == nullptr) return NF_ERR_OUT_OF_MEMORY;
+    }
+    NF_CUDA_TRY(cudaMemcpyAsync(m->embed, w->embed, (size_t)V * H * 2, cudaMemcpyDeviceToDevice, s));
+    NF_CUDA_TRY(nf::launch_pack_rows((const uint16_t*)w->lm_head, m->lm_head, V, H,
+                                     (const uint16_t*)w->final_norm, V, 0, 0, s));
+    if (!nf::make_tmap_bf16_2d(&m->tm_lm, m->lm_head, V, H, nf::kGemmBN)) return NF_ERR_CUDA;
+    m->globals_loaded = true;
+    return NF_OK;
+}
+
+// ------------------------------------------------------------------ executor
+
+namespace {
+
+nf_status ensure_kv_tmap(nf_model* m, int layer, const nf_iter_io* io) {
+    const void* p = io->kv_pools[layer];
+    if (p == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    if (m->kv_ptr[layer] != p || m->kv_pages[layer] != io->num_pages) {
+        if (!nf::make_kv_tmap(&m->kv_tm[layer], p, io->num_pages, m->dims.nkv, m->dims.d)) return NF_ERR_CUDA;
+        m->kv_ptr[layer] = p;
+        m->kv_pages[layer] = io->num_pages;
+    }
+    return NF_OK;
+}
+
+nf_status ensure_part_capacity(nf_model* m, int64_t items) {
+    if (items <= m->part_capacity) return NF_OK;
+    const int64_t cap = std::max<int64_t>(items, 1024);
+    dfree(m, m->part_o);
+    dfree(m, m->part_lse);
+    m->part_o = dalloc<float>(m, (size_t)cap * m->dims.nq / m->dims.nkv * m->dims.d);
+    m->part_lse = dalloc<float>(m, (size_t)cap * m->dims.nq / m->dims.nkv);
+    if (!m->part_o || !m->part_lse) { m->part_capacity = 0; return NF_ERR_OUT_OF_MEMORY; }
+    m->part_capacity = cap;
+    return NF_OK;
+}
+
+nf::DecodeArgs decode_args(const nf_model* m, const nf_iter_io* io, const void* q, void* out, int rb, int re) {
+    nf::DecodeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = (const uint16_t*)q;
+    a.out = (uint16_t*)out;
+    a.part_o = m->part_o;
+    a.part_lse = m->part_lse;
+    a.ctx_len = io->ctx_len;
+    a.page_indptr = io->page_indptr;
+    a.page_indices = io->page_indices;
+    a.item_off = m->item_off;
+    a.req_begin = rb;
+    a.req_end = re;
+    a.nq = m->dims.nq;
+    a.nkv = m->dims.nkv;
+    a.G = m->dims.nq / m->dims.nkv;
+    a.num_pages = io->num_pages;
+    a.split_pages = nf::kDecodeSplitPages;
+    a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m->dims.d));
+    a.merge_smem_pad = 100 * 1024;
+    a.status = m->status;
+    if (m->trace_on) { a.trace_ctr = m->trace_ctr; a.trace = m->trace; a.trace_cap = m->trace_cap; }
+    return a;
+}
+
+nf::PrefillArgs prefill_args(const nf_model* m, const nf_iter_io* io, const void* q, void* out, int R, int C) {
+    nf::PrefillArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = (const uint16_t*)q;
+    a.out = (uint16_t*)out;
+    a.page_indptr = io->page_indptr;
+    a.page_indices = io->page_indices;
+    a.num_decode = R;
+    a.prefill_len = C;
+    a.nq = m->dims.nq;
+    a.nkv = m->dims.nkv;
+    a.G = m->dims.nq / m->dims.nkv;
+    a.num_pages = io->num_pages;
+    a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m->dims.d));
+    a.status = m->status;
+    if (m->trace_on) { a.trace_ctr = m->trace_ctr; a.trace = m->trace; a.trace_cap = m->trace_cap; }
+    return a;
+}
+
+nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::Op& op, int grid,
+                 cudaStream_t s) {
+    const nf::ModelDims& d = m->dims;
+    const int j = op.nano, l = op.layer;
+    const int t0 = p->tok_begin[j], t1 = p->tok_end[j], M = t1 - t0;
+    const int R = p->num_decode, C = p->prefill_len, T = p->num_tokens;
+    if (M <= 0) return NF_OK;
+    nf::LayerWeights& W = m->layers[l];
+    GemmArgs a = base_args(m);
+    a.a_row0 = t0;
+    a.tok0 = t0;
+    switch (op.kind) {
+        case nf::OP_QKV: {
+            set_tiles(a, M, d.qkv, d.H);
+            a.partials = m->partials;
+            a.positions = io->positions;
+            a.rope_cos = m->rope_cos;
+            a.rope_sin = m->rope_sin;
+            a.max_position = m->cfg.max_position;
+            a.q_out = m->q;
+            a.nq = d.nq;
+            a.nkv = d.nkv;
+            a.head_dim = d.d;
+            a.kv_pool = (uint16_t*)io->kv_pools[l];
+            a.num_pages = io->num_pages;
+            a.page_indptr = io->page_indptr;
+            a.page_indices = io->page_indices;
+            a.num_decode = R;
+            NF_CUDA_TRY(nf::launch_gemm(nf::EPI_QKV, m->tm_xb, W.tm_qkv, a, gemm_grid(a, grid), s));
+            return NF_OK;
+        }
+        case nf::OP_ATT: {
+            const int rb = std::min(t0, R), re = std::min(t1, R);
+            if (re > rb) {
+                nf::DecodeArgs da = decode_args(m, io, m->q, m->attn_o, rb, re);
+                NF_CUDA_TRY(nf::launch_decode_attention(m->kv_tm[l], da, d.d, grid, grid, s));
+            }
+            if (t1 > R && C > 0) {
+                nf::PrefillArgs pa = prefill_args(m, io, m->q, m->attn_o, R, C);
+                NF_CUDA_TRY(nf::launch_prefill_attention(m->kv_tm[l], pa, d.d, grid, s));
+            }
+            return NF_OK;
+        }
+        case nf::OP_O: {
+            set_tiles(a, M, d.H, d.nq * d.d);
+            a.resid = m->resid;
+            a.out_bf16 = m->xb;
+            a.ld_bf16 = d.H;
+            a.out_partials = m->partials;
+            NF_CUDA_TRY(nf::launch_gemm(nf::EPI_RESID, m->tm_attn_o, W.tm_o, a, gemm_grid(a, grid), s));
+            return NF_OK;
+        }
+        case nf::OP_GU: {
+            set_tiles(a, M, 2 * d.F, d.H);
+            a.partials = m->partials;
+            a.out_bf16 = m->act;
+            a.ld_bf16 = d.F;
+            NF_CUDA_TRY(nf::launch_gemm(nf::EPI_SWIGLU, m->tm_xb, W.tm_gu, a, gemm_grid(a, grid), s));
+            return NF_OK;
+        }
+        case nf::OP_D: {
+            set_tiles(a, M, d.H, d.F);
+            a.resid = m->resid;
+            a.out_bf16 = m->xb;
+            a.ld_bf16 = d.H;
+            a.out_partials = m->partials;
+            NF_CUDA_TRY(nf::launch_gemm(nf::EPI_RESID, m->tm_act, W.tm_d, a, gemm_grid(a, grid), s));
+            return NF_OK;
+        }
+        case nf::OP_MOE: {
+            nf::MoeArgs ma;
+            std::memset(&ma, 0, sizeof(ma));
+            ma.resid = m->resid;
+            ma.partials = m->partials;
+            ma.router = W.router;
+            ma.router_bias = W.router_bias;
+            ma.tok0 = t0;
+            ma.rows = M;
+            ma.H = d.H;
+            ma.E = d.E;
+            ma.K = d.K;
+            ma.n_part = m->n_part;
+            ma.inv_dim = 1.0f / (float)d.H;
+            ma.eps = m->cfg.rms_eps;
+            ma.logits = m->moe_logits;
+            ma.topk_idx = m->moe_idx;
+            ma.topk_w = m->moe_w;
+            ma.counts = m->moe_counts;
+            ma.perm = m->moe_perm;
+            ma.inv = m->moe_inv;
+            ma.xb = m->xb;
+            ma.a_sorted = m->moe_a;
+            ma.part_sorted = m->moe_part;
+            ma.y_sorted = m->moe_y;
+            ma.resid_out = m->resid;
+            ma.xb_out = m->xb;
+            ma.partials_out = m->partials;
+            if (io->topk_idx) ma.dbg_idx = io->topk_idx + ((size_t)l * T + t0) * d.K;
+            if (io->topk_w) ma.dbg_w = io->topk_w + ((size_t)l * T + t0) * d.K;
+            if (io->router_logits) ma.dbg_logits = io->router_logits + ((size_t)l * T + t0) * d.E;
+            NF_CUDA_TRY(nf::launch_moe_route(ma, grid * 4, s));
+            NF_CUDA_TRY(nf::launch_moe_gather(ma, grid * 4, s));
+            GemmArgs g = base_args(m);
+            set_tiles(g, M * d.K, 2 * d.F, d.H);
+            g.grouped = 1;
+            g.group_offsets = m->moe_counts;
+            g.num_groups = d.E;
+            g.partials = m->moe_part;
+            g.out_bf16 = m->act;
+            g.ld_bf16 = d.F;
+            NF_CUDA_TRY(nf::launch_gemm(nf::EPI_SWIGLU, m->tm_moe_a, W.tm_gu, g, grid, s));
+            GemmArgs g2 = base_args(m);
+            set_tiles(g2, M * d.K, d.H, d.F);
+            g2.grouped = 1;
+            g2.group_offsets = m->moe_counts;
+            g2.num_groups = d.E;
+            g2.out_f32 = m->moe_y;
+            g2.ld_f32 = d.H;
+            NF_CUDA_TRY(nf::launch_gemm(nf::EPI_F32, m->tm_act, W.tm_d, g2, grid, s));
+            NF_CUDA_TRY(nf::launch_moe_combine(ma, grid * 4, s));
+            return NF_OK;
+        }
+    }
+    return NF_ERR_INVALID_ARGUMENT;
+}
+
+nf_status validate_forward(const nf_model* m, const nf_plan* p, const nf_iter_io* io) {
+    if (m == nullptr || p == nullptr || io == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    const int T = p->num_tokens, R = p->num_decode, C = p->prefill_len;
+    if (T <= 0 || T != R + C || R < 0 || C < 0) return NF_ERR_INVALID_ARGUMENT;
+    if (T > m->cfg.max_tokens || R > m->cfg.max_requests) return NF_ERR_INVALID_ARGUMENT;
+    if (p->n_nano < 1 || p->n_nano > NF_MAX_NANO) return NF_ERR_INVALID_ARGUMENT;
+    int expect = 0;
+    for (int j = 0; j < p->n_nano; ++j) {
+        if (p->tok_begin[j] != expect || p->tok_end[j] <= p->tok_begin[j]) return NF_ERR_INVALID_ARGUMENT;
+        if (p->tok_begin[j] > R && p->tok_begin[j] < T) return NF_ERR_INVALID_ARGUMENT;  // chunk stays whole
+        expect = p->tok_end[j];
+    }
+    if (expect != T) return NF_ERR_INVALID_ARGUMENT;
+    bool seen[NF_MAX_NANO] = {false, false, false, false};
+    for (int i = 0; i < p->n_nano; ++i) {
+        const int j = p->nano_order[i];
+        if (j < 0 || j >= p->n_nano || seen[j]) return NF_ERR_INVALID_ARGUMENT;
+        seen[j] = true;
+    }
+    const int S = m->sm_count;
+    if (p->sm_total < 1 || p->sm_total > S) return NF_ERR_INVALID_ARGUMENT;
+    if (p->order_template == NF_TEMPLATE_PIPELINED) {
+        if (p->sm_attn < 1 || p->sm_gemm < 1 || p->sm_attn + p->sm_gemm > p->sm_total) return NF_ERR_INVALID_ARGUMENT;
+    } else if (p->order_template != NF_TEMPLATE_SEQUENTIAL) {
+        return NF_ERR_INVALID_ARGUMENT;
+    }
+    if (!io->positions || !io->page_indptr || !io->page_indices || !io->kv_pools || io->num_pages <= 0)
+        return NF_ERR_INVALID_ARGUMENT;
+    if (R > 0 && !io->ctx_len) return NF_ERR_INVALID_ARGUMENT;
+    if (m->cfg.vocab > 0 && (!io->token_ids || !m->globals_loaded)) return NF_ERR_INVALID_ARGUMENT;
+    if (m->cfg.vocab == 0 && !io->hidden_in) return NF_ERR_INVALID_ARGUMENT;
+    for (int l = 0; l < m->dims.L; ++l)
+        if (!m->layers[l].loaded || io->kv_pools[l] == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    // kv pool coordinates of the TMA maps are 32-bit
+    if ((int64_t)io->num_pages * 2 * m->dims.nkv * 16 >= (int64_t)1 << 31) return NF_ERR_UNSUPPORTED;
+    return NF_OK;
+}
+
+}  // namespace
+
+extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const nf_iter_io* io, void* stream) {
+    nf_status st = validate_forward(m, p, io);
+    if (st != NF_OK) return st;
+    const nf::ModelDims& d = m->dims;
+    const int R = p->num_decode, C = p->prefill_len, T = p->num_tokens;
+    cudaStream_t sg = (cudaStream_t)stream;
+    cudaStream_t sa = m->s_attn;
+    if ((st = ensure_part_capacity(m, std::max<int64_t>(p->decode_items, 1))) != NF_OK) return st;
+    for (int l = 0; l < d.L; ++l)
+        if ((st = ensure_kv_tmap(m, l, io)) != NF_OK) return st;
+
+    const int S = p->sm_total;
+    const bool pipelined = p->order_template == NF_TEMPLATE_PIPELINED;
+    NF_CUDA_TRY(cudaEventRecord(m->ev_fork, sg));
+    NF_CUDA_TRY(cudaStreamWaitEvent(sa, m->ev_fork, 0));
+    if (m->trace_on) NF_CUDA_TRY(cudaMemsetAsync(m->trace_ctr, 0, sizeof(int), sg));
+
+    // prologue: decode work items, residual stream set-up
+    if (R > 0) NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, sg));
+    if (m->cfg.vocab > 0) {
+        NF_CUDA_TRY(nf::launch_embed(io->token_ids, m->embed, T, d.H, m->cfg.vocab, m->resid, m->xb, m->partials,
+                                     m->status, S * 4, sg));
+    } else {
+        NF_CUDA_TRY(nf::launch_prep_hidden((const uint16_t*)io->hidden_in, T, d.H, m->resid, m->xb, m->partials, S * 4,
+                                           sg));
+    }
+
+    int order[NF_MAX_NANO];
+    for (int i = 0; i < p->n_nano; ++i) order[i] = p->nano_order[i];
+    const std::vector<nf::Op> ops = nf::build_ops(p->order_template, p->n_nano, order, d.L, d.E > 0);
+    while (m->events.size() < ops.size()) {
+        cudaEvent_t e;
+        NF_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+        m->events.push_back(e);
+    }
+    // timing entries accumulate over forwards until nf_set_timing is called again
+    const size_t t_base = m->t_ops.size();
+    const size_t n_timed = ops.size() + 1;
+    if (m->timing_on) {
+        while (m->t_ev.size() < 2 * (t_base + n_timed)) {
+            cudaEvent_t e;
+            NF_CUDA_TRY(cudaEventCreate(&e));
+            m->t_ev.push_back(e);
+        }
+    }
+    for (size_t i = 0; i < ops.size(); ++i) {
+        const nf::Op& op = ops[i];
+        cudaStream_t s = op.stream == nf::STREAM_ATTN ? sa : sg;
+        if (op.wait >= 0) NF_CUDA_TRY(cudaStreamWaitEvent(s, m->events[op.wait], 0));
+        int grid = S;
+        if (pipelined) {
+            if (op.stream == nf::STREAM_ATTN) grid = p->sm_attn;
+            else if (!op.full_sm) grid = p->sm_gemm;
+        }
+        const size_t ti = m->t_ops.size();
+        if (m->timing_on) NF_CUDA_TRY(cudaEventRecord(m->t_ev[2 * ti], s));
+        if ((st = run_op(m, p, io, op, grid, s)) != NF_OK) return st;
+        if (m->timing_on) {
+            NF_CUDA_TRY(cudaEventRecord(m->t_ev[2 * ti + 1], s));
+            m->t_ops.push_back(nf_op_time{op.kind, op.nano, op.layer, op.stream, grid, 0.f});
+        }
+        if (op.signal) NF_CUDA_TRY(cudaEventRecord(m->events[i], s));
+    }
+    NF_CUDA_TRY(cudaEventRecord(m->ev_join, sa));
+    NF_CUDA_TRY(cudaStreamWaitEvent(sg, m->ev_join, 0));
+
+    // final norm + LM head + greedy argmax over the decode rows and the chunk's last row
+    if (m->cfg.vocab > 0 && (io->logits || io->next_token)) {
+        const int rows = R + (C > 0 ? 1 : 0);
+        NF_CUDA_TRY(nf::launch_lm_gather(m->xb, m->partials, R, T, rows, d.H, m->lm_in, m->lm_partials, S * 4, sg));
+        const size_t ti = m->t_ops.size();
+        if (m->timing_on) NF_CUDA_TRY(cudaEventRecord(m->t_ev[2 * ti], sg));
+        GemmArgs a = base_args(m);
+        set_tiles(a, rows, m->cfg.vocab, d.H);
+        a.partials = m->lm_partials;
+        a.out_bf16 = (uint16_t*)io->logits;
+        a.ld_bf16 = m->cfg.vocab;
+        a.tile_max = m->tile_max;
+        a.tile_arg = m->tile_arg;
+        NF_CUDA_TRY(nf::launch_gemm(nf::EPI_LMHEAD, m->tm_lm_in, m->tm_lm, a, gemm_grid(a, S), sg));
+        if (io->next_token)
+            NF_CUDA_TRY(nf::launch_argmax_reduce(m->tile_max, m->tile_arg, rows, m->cfg.vocab / 256, io->next_token,
+                                                 S * 4, sg));
+        if (m->timing_on) {
+            NF_CUDA_TRY(cudaEventRecord(m->t_ev[2 * ti + 1], sg));
+            m->t_ops.push_back(nf_op_time{NF_OP_LM_HEAD, -1, d.L, 0, gemm_grid(a, S), 0.f});
+        }
+    }
+    if (io->hidden_out)
+        NF_CUDA_TRY(cudaMemcpyAsync(io->hidden_out, m->xb, (size_t)T * d.H * 2, cudaMemcpyDeviceToDevice, sg));
+    if (io->hidden_out_f32)
+        NF_CUDA_TRY(cudaMemcpyAsync(io->hidden_out_f32, m->resid, (size_t)T * d.H * 4, cudaMemcpyDeviceToDevice, sg));
+    return NF_OK;
+}
+
+extern "C" nf_status nf_sync_status(nf_model* m) {
+    if (m == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    if (cudaStreamSynchronize(m->s_attn) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        cudaGetLastError();
+        return NF_ERR_CUDA;
+    }
+    int h = 0;
+    if (cudaMemcpy(&h, m->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return NF_ERR_CUDA;
+    if (h != 0) cudaMemset(m->status, 0, sizeof(int));
+    return (nf_status)h;
+}
+
+extern "C" nf_status nf_set_trace(nf_model* m, int32_t enable) {
+    if (m == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    m->trace_on = enable != 0;
+    return NF_OK;
+}
+
+extern "C" int64_t nf_get_trace(nf_model* m, nf_trace_entry* out, int64_t capacity) {
+    if (m == nullptr || out == nullptr || capacity < 0) return -(int64_t)NF_ERR_INVALID_ARGUMENT;
+    if (cudaDeviceSynchronize() != cudaSuccess) return -(int64_t)NF_ERR_CUDA;
+    int n = 0;
+    if (cudaMemcpy(&n, m->trace_ctr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return -(int64_t)NF_ERR_CUDA;
+    n = std::min<int64_t>(std::min(n, m->trace_cap), capacity);
+    if (n > 0 && cudaMemcpy(out, m->trace, (size_t)n * sizeof(nf_trace_entry), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return -(int64_t)NF_ERR_CUDA;
+    return n;
+}
+
+extern "C" nf_status nf_set_timing(nf_model* m, int32_t enable) {
+    if (m == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    m->timing_on = enable != 0;
+    m->t_ops.clear();
+    return NF_OK;
+}
+
+extern "C" int64_t nf_get_op_times(nf_model* m, nf_op_time* out, int64_t capacity) {
+    if (m == nullptr || out == nullptr || capacity < 0) return -(int64_t)NF_ERR_INVALID_ARGUMENT;
+    if (cudaStreamSynchronize(m->s_attn) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+        return -(int64_t)NF_ERR_CUDA;
+    const int64_t n = std::min<int64_t>((int64_t)m->t_ops.size(), capacity);
+    for (int64_t i = 0; i < n; ++i) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, m->t_ev[2 * i], m->t_ev[2 * i + 1]) != cudaSuccess) return -(int64_t)NF_ERR_CUDA;
+        out[i] = m->t_ops[i];
+        out[i].us = ms * 1000.f;
+    }
+    return n;
+}
+
+// ------------------------------------------------------------------ single ops
+
+namespace {
+int* g_op_status = nullptr;
+
+nf_status op_status_word(int** out) {
+    if (g_op_status == nullptr) {
+        if (cudaMalloc(&g_op_status, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return NF_ERR_OUT_OF_MEMORY; }
+        if (cudaMemset(g_op_status, 0, sizeof(int)) != cudaSuccess) return NF_ERR_CUDA;
+    }
+    *out = g_op_status;
+    return NF_OK;
+}
+}  // namespace
+
+extern "C" nf_status nf_op_gemm_bf16(const void* A, const void* B, float* C, int32_t M, int32_t N, int32_t K,
+                                     int32_t sm_count, void* stream) {
+    if (!A || !B || !C || M < 1 || N < 256 || N % 256 != 0 || K < 64 || K % 64 != 0) return NF_ERR_INVALID_ARGUMENT;
+    int* status = nullptr;
+    nf_status st = op_status_word(&status);
+    if (st != NF_OK) return st;
+    CUtensorMap ta, tb;
+    if (!nf::make_tmap_bf16_2d(&ta, A, (uint64_t)M, (uint64_t)K, nf::kGemmBM) ||
+        !nf::make_tmap_bf16_2d(&tb, B, (uint64_t)N, (uint64_t)K, nf::kGemmBN))
+        return NF_ERR_INVALID_ARGUMENT;
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    set_tiles(a, M, N, K);
+    a.out_f32 = C;
+    a.ld_f32 = N;
+    a.status = status;
+    int sms = nf::device_sm_count();
+    if (sms <= 0) return NF_ERR_CUDA;
+    const int grid = sm_count > 0 ? std::min(sm_count, sms) : sms;
+    NF_CUDA_TRY(nf::launch_gemm(nf::EPI_F32, ta, tb, a, gemm_grid(a, grid), (cudaStream_t)stream));
+    return NF_OK;
+}
+
+extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* out, const nf_iter_io* io, int32_t layer,
+                                            int32_t req_begin, int32_t req_end, int32_t sm_count, void* stream) {
+    if (!m || !q || !out || !io || !io->ctx_len || !io->page_indptr || !io->page_indices || !io->kv_pools)
+        return NF_ERR_INVALID_ARGUMENT;
+    if (layer < 0 || layer >= m->dims.L || req_begin < 0 || req_end < req_begin || req_end > m->cfg.max_requests)
+        return NF_ERR_INVALID_ARGUMENT;
+    if (req_end == req_begin) return NF_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    nf_status st = ensure_kv_tmap(m, layer, io);
+    if (st != NF_OK) return st;
+    NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, req_end, m->dims.nkv, nf::kDecodeSplitPages, m->item_off, s));
+    int items = 0;
+    NF_CUDA_TRY(cudaMemcpyAsync(&items, m->item_off + req_end, sizeof(int), cudaMemcpyDeviceToHost, s));
+    NF_CUDA_TRY(cudaStreamSynchronize(s));
+    if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
+    const int grid = sm_count > 0 ? std::min(sm_count, m->sm_count) : m->sm_count;
+    nf::DecodeArgs da = decode_args(m, io, q, out, req_begin, req_end);
+    NF_CUDA_TRY(nf::launch_decode_attention(m->kv_tm[layer], da, m->dims.d, grid, grid, s));
+    return NF_OK;
+}
+
+extern "C" nf_status nf_op_prefill_attention(nf_model* m, const void* q, void* out, const nf_iter_io* io,
+                                             int32_t layer, int32_t num_decode, int32_t prefill_len, int32_t sm_count,
+                                             void* stream) {
+    if (!m || !q || !out || !io || !io->page_indptr || !io->page_indices || !io->kv_pools)
+        return NF_ERR_INVALID_ARGUMENT;
+    if (layer < 0 || layer >= m->dims.L || num_decode < 0 || prefill_len < 0) return NF_ERR_INVALID_ARGUMENT;
+    if (prefill_len == 0) return NF_OK;
+    nf_status st = ensure_kv_tmap(m, layer, io);
+    if (st != NF_OK) return st;
+    const int grid = sm_count > 0 ? std::min(sm_count, m->sm_count) : m->sm_count;
+    nf::PrefillArgs pa = prefill_args(m, io, q, out, num_decode, prefill_len);
+    NF_CUDA_TRY(nf::launch_prefill_attention(m->kv_tm[layer], pa, m->dims.d, grid, (cudaStream_t)stream));
+    return NF_OK;
+}
+
+extern "C" nf_status nf_op_wait_flag_test(int32_t* flag_device, uint64_t limit_ns, void* stream) {
+    if (flag_device == nullptr || limit_ns == 0 || limit_ns > 10000000000ull) return NF_ERR_INVALID_ARGUMENT;
+    int* status = nullptr;
+    nf_status st = op_status_word(&status);
+    if (st != NF_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    NF_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
+    NF_CUDA_TRY(nf::launch_wait_flag(flag_device, limit_ns, status, s));
+    int h = 0;
+    NF_CUDA_TRY(cudaMemcpyAsync(&h, status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    NF_CUDA_TRY(cudaStreamSynchronize(s));
+    return (nf_status)h;
+}
+
+extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_iter_io* io, void* stream) {
+    (void)stream;
+    if (m == nullptr || b == nullptr || io == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    return NF_ERR_UNSUPPORTED;
+}

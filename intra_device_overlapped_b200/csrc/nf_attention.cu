@@ -1,0 +1,727 @@
+// Paged-KV attention of the serving iteration: GQA decode attention with split-KV,
+// causal attention of the prefill chunk, and the split-KV merge.
+//
+// Decode attention is the memory-bound operation NanoFlow overlaps with the GEMMs of
+// another nano-batch (README "Introduction"; arXiv abstract). Each decode request r
+// reads ctx_len[r] + 1 keys and values of every KV head from its pages; one page of
+// one KV head is a contiguous 16 x d bf16 block (pool layout
+// [page][K|V][kv_head][16][d]), fetched by TMA (two 128-byte-swizzled 16 x 64 boxes
+// for d = 128) into a 16-stage shared-memory ring by a producer warp. Four consumer
+// warps each take every fourth page of a work item and run q . K^T and P . V on the
+// tensor cores (mma.sync m16n8k16 with the G query heads of a KV head as the rows),
+// with an online softmax in fp32 (exp2, scores pre-scaled by log2(e)/sqrt(d)). The
+// four partial states are merged through shared memory in a fixed order.
+//
+// Work item = (request, KV split, KV head). A request's keys are cut into splits of
+// kDecodeSplitPages pages; the split structure depends only on ctx_len, so results
+// do not depend on how requests are grouped into nano-batches. Items of a launch are
+// dealt to the persistent CTAs in contiguous, equal-count ranges.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "nf_attention.h"
+#include "nf_internal.h"
+#include "nf_ptx.cuh"
+
+namespace nf {
+namespace {
+
+constexpr int DEC_STAGES = 16;
+constexpr int DEC_CONSUMERS = 4;
+constexpr int DEC_THREADS = (DEC_CONSUMERS + 1) * 32;
+constexpr int PRE_STAGES = 4;  // 128 KB for d = 128: one CTA per SM
+constexpr int PRE_THREADS = 5 * 32;
+constexpr int BOX_BYTES = 16 * 128;  // one 16-row x 64-col bf16 box
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Named barrier that also ORs a predicate across the participating threads.
+__device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(threads)
+        : "memory");
+    return r != 0;
+}
+
+// Keep the low / high bf16 of a packed pair.
+__device__ __forceinline__ uint32_t keep_pair(uint32_t v, bool lo, bool hi) {
+    return (lo ? (v & 0xFFFFu) : 0u) | (hi ? (v & 0xFFFF0000u) : 0u);
+}
+
+__device__ __forceinline__ float quad_max(float x) {
+    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
+    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
+    return x;
+}
+__device__ __forceinline__ float quad_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    return x;
+}
+
+// Locate the request of item `it` in item_off[req_begin..req_end] (binary search).
+__device__ __forceinline__ int item_request(const int* item_off, int req_begin, int req_end, int it) {
+    int lo = req_begin, hi = req_end - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (item_off[mid] <= it) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+struct DecItem {
+    int r, split, g, p0, p1, nkeys, nsplit;
+};
+
+__device__ __forceinline__ DecItem dec_item(const DecodeArgs& a, int it) {
+    DecItem d;
+    d.r = item_request(a.item_off, a.req_begin, a.req_end, it);
+    const int local = it - a.item_off[d.r];
+    d.split = local / a.nkv;
+    d.g = local - d.split * a.nkv;
+    d.nkeys = a.ctx_len[d.r] + 1;
+    const int npages = (d.nkeys + 15) >> 4;
+    d.nsplit = (npages + a.split_pages - 1) / a.split_pages;
+    d.p0 = d.split * a.split_pages;
+    d.p1 = min(d.p0 + a.split_pages, npages);
+    return d;
+}
+
+template <int HD>
+__global__ void __launch_bounds__(DEC_THREADS, 1)
+    decode_attention_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ DecodeArgs a) {
+    constexpr int BOXES = HD / 64;
+    constexpr uint32_t KV_BYTES = BOXES * BOX_BYTES;  // one page, one KV head, K or V
+    constexpr uint32_t STAGE_BYTES = 2 * KV_BYTES;
+    constexpr int KSTEPS = HD / 16;
+    constexpr int NT = HD / 8;  // n-tiles of the output
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* mrg_o = reinterpret_cast<float*>(smem + DEC_STAGES * STAGE_BYTES);  // [4][16][HD]
+    float* mrg_m = mrg_o + DEC_CONSUMERS * 16 * HD;                           // [4][16]
+    float* mrg_l = mrg_m + DEC_CONSUMERS * 16;                                // [4][16]
+    uint64_t* full = reinterpret_cast<uint64_t*>(mrg_l + DEC_CONSUMERS * 16);
+    uint64_t* empty = full + DEC_STAGES;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + DEC_STAGES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint64_t t_start = 0;
+    if (threadIdx.x == 0) {
+        t_start = globaltimer_ns();
+        for (int s = 0; s < DEC_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmKV);
+    }
+    __syncthreads();
+
+    const int ib = a.item_off[a.req_begin];
+    const int ie = a.item_off[a.req_end];
+    const int nitems = ie - ib;
+    const int my_b = ib + (int)(((long long)nitems * blockIdx.x) / gridDim.x);
+    const int my_e = ib + (int)(((long long)nitems * (blockIdx.x + 1)) / gridDim.x);
+
+    if (warp == DEC_CONSUMERS) {
+        // ---------------- producer
+        if (lane == 0) {
+            uint32_t seq = 0;
+            bool ok = true;
+            uint32_t outstanding = 0;  // bit s: stage s holds a load the consumers have not released
+            uint32_t parity_bits = 0;  // bit s: parity of that load's phase
+            for (int it = my_b; it < my_e && ok; ++it) {
+                const DecItem d = dec_item(a, it);
+                const int* pt = a.page_indices + a.page_indptr[d.r];
+                for (int pl = d.p0; pl < d.p1; ++pl, ++seq) {
+                    const int stage = (int)(seq % DEC_STAGES);
+                    const uint32_t phase = (seq / DEC_STAGES) & 1u;
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+                    outstanding &= ~(1u << stage);
+                    int page = pt[pl];
+                    if (page < 0 || page >= a.num_pages) { set_status(a.status, NF_ERR_DEVICE_BOUNDS); page = 0; }
+                    uint8_t* st = smem + stage * STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+                    const int rowK = ((page * 2 + 0) * a.nkv + d.g) * 16;
+                    const int rowV = ((page * 2 + 1) * a.nkv + d.g) * 16;
+#pragma unroll
+                    for (int b = 0; b < BOXES; ++b) {
+                        tma_load_2d(st + b * BOX_BYTES, &tmKV, &full[stage], b * 64, rowK);
+                        tma_load_2d(st + KV_BYTES + b * BOX_BYTES, &tmKV, &full[stage], b * 64, rowV);
+                    }
+                    outstanding |= 1u << stage;
+                    parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
+                }
+            }
+            if (!ok) {
+                // let every copy still in flight land before the CTA exits
+                volatile int quiet = 0;
+                for (int st = 0; st < DEC_STAGES; ++st)
+                    if (outstanding & (1u << st)) mbar_wait(&full[st], (parity_bits >> st) & 1u, &quiet, nullptr);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- consumers
+        const int qr = lane >> 2;        // fragment row (query head within the group), +8 for the second half
+        const int qc = (lane & 3) * 2;   // fragment column pair
+        uint32_t seq_base = 0;
+        bool alive = true;
+        for (int it = my_b; it < my_e; ++it) {
+            const DecItem d = dec_item(a, it);
+            const int np = d.p1 - d.p0;
+            // Q fragments of heads g*G .. g*G+G-1 (rows >= G are zero)
+            uint32_t qa[KSTEPS][4];
+            {
+                const uint16_t* q0 = a.q + ((size_t)d.r * a.nq + (size_t)d.g * a.G) * HD;
+                const bool r0 = qr < a.G, r1 = qr + 8 < a.G;
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk) {
+                    const int c = kk * 16 + qc;
+                    qa[kk][0] = r0 ? *reinterpret_cast<const uint32_t*>(q0 + (size_t)qr * HD + c) : 0u;
+                    qa[kk][1] = r1 ? *reinterpret_cast<const uint32_t*>(q0 + (size_t)(qr + 8) * HD + c) : 0u;
+                    qa[kk][2] = r0 ? *reinterpret_cast<const uint32_t*>(q0 + (size_t)qr * HD + c + 8) : 0u;
+                    qa[kk][3] = r1 ? *reinterpret_cast<const uint32_t*>(q0 + (size_t)(qr + 8) * HD + c + 8) : 0u;
+                }
+            }
+            float o[NT][4];
+#pragma unroll
+            for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+            float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+            for (int pl = warp; pl < np && alive; pl += DEC_CONSUMERS) {
+                const uint32_t seq = seq_base + (uint32_t)pl;
+                const int stage = (int)(seq % DEC_STAGES);
+                const uint32_t phase = (seq / DEC_STAGES) & 1u;
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&full[stage], phase, abort_flag, a.status) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) { alive = false; break; }  // still joins this item's barriers below
+                const uint32_t sK = smem_u32(smem + stage * STAGE_BYTES);
+                const uint32_t sV = sK + KV_BYTES;
+                const int key0 = (d.p0 + pl) * 16;
+                const int nvalid = min(16, d.nkeys - key0);  // >= 1
+
+                // S = Q K^T for the page's 16 keys (two n-tiles of 8 keys)
+                float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk) {
+                    const int mi = lane >> 3;
+                    const int key = (mi >> 1) * 8 + (lane & 7);
+                    const int dc = kk * 16 + (mi & 1) * 8;
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4(sK + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64), b0, b1, b2, b3);
+                    mma_16816(s[0], qa[kk], b0, b1);
+                    mma_16816(s[1], qa[kk], b2, b3);
+                }
+                // scale, mask keys beyond the request's length, online softmax
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const bool vis = (j * 8 + qc + e) < nvalid;
+                        s[j][e] = vis ? s[j][e] * a.scale_log2 : -INFINITY;
+                        s[j][2 + e] = vis ? s[j][2 + e] * a.scale_log2 : -INFINITY;
+                        mx0 = fmaxf(mx0, s[j][e]);
+                        mx1 = fmaxf(mx1, s[j][2 + e]);
+                    }
+                }
+                mx0 = quad_max(mx0);
+                mx1 = quad_max(mx1);
+                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                const float c0 = exp2f(m0 - mn0), c1 = exp2f(m1 - mn1);
+                m0 = mn0;
+                m1 = mn1;
+                float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        s[j][e] = exp2f(s[j][e] - mn0);
+                        s[j][2 + e] = exp2f(s[j][2 + e] - mn1);
+                        ps0 += s[j][e];
+                        ps1 += s[j][2 + e];
+                    }
+                }
+                l0 = l0 * c0 + ps0;
+                l1 = l1 * c1 + ps1;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) { o[j][0] *= c0; o[j][1] *= c0; o[j][2] *= c1; o[j][3] *= c1; }
+                uint32_t pa[4];
+                pa[0] = pack_bf16x2(s[0][0], s[0][1]);
+                pa[1] = pack_bf16x2(s[0][2], s[0][3]);
+                pa[2] = pack_bf16x2(s[1][0], s[1][1]);
+                pa[3] = pack_bf16x2(s[1][2], s[1][3]);
+                // O += P V; V rows of keys beyond the request are zeroed in the fragments
+                const int kb = (lane & 3) * 2;
+                const bool k0 = kb < nvalid, k1 = kb + 1 < nvalid, k8 = kb + 8 < nvalid, k9 = kb + 9 < nvalid;
+#pragma unroll
+                for (int j = 0; j < NT; j += 2) {
+                    const int mi = lane >> 3;
+                    const int key = (mi & 1) * 8 + (lane & 7);
+                    const int dc = j * 8 + (mi >> 1) * 8;
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4_trans(sV + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64), b0, b1, b2, b3);
+                    if (nvalid < 16) {
+                        b0 = keep_pair(b0, k0, k1); b1 = keep_pair(b1, k8, k9);
+                        b2 = keep_pair(b2, k0, k1); b3 = keep_pair(b3, k8, k9);
+                    }
+                    mma_16816(o[j], pa, b0, b1);
+                    mma_16816(o[j + 1], pa, b2, b3);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+            }
+            l0 = quad_sum(l0);
+            l1 = quad_sum(l1);
+            // ---- merge the four warps' states (fixed order)
+            float* mo = mrg_o + warp * 16 * HD;
+            const int r0 = qr, r1 = qr + 8;
+            if ((lane & 3) == 0) {
+                mrg_m[warp * 16 + r0] = m0; mrg_l[warp * 16 + r0] = l0;
+                mrg_m[warp * 16 + r1] = m1; mrg_l[warp * 16 + r1] = l1;
+            }
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const int c = j * 8 + qc;
+                if (r0 < a.G) { mo[r0 * HD + c] = o[j][0]; mo[r0 * HD + c + 1] = o[j][1]; }
+                if (r1 < a.G) { mo[r1 * HD + c] = o[j][2]; mo[r1 * HD + c + 1] = o[j][3]; }
+            }
+            named_bar_sync(1, DEC_CONSUMERS * 32);
+            const int total = a.G * HD;
+            const bool single = d.nsplit == 1;
+            for (int e = threadIdx.x; e < total; e += DEC_CONSUMERS * 32) {
+                const int row = e / HD, col = e - row * HD;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < DEC_CONSUMERS; ++w) M = fmaxf(M, mrg_m[w * 16 + row]);
+                float L = 0.f, acc = 0.f;
+#pragma unroll
+                for (int w = 0; w < DEC_CONSUMERS; ++w) {
+                    const float sc = exp2f(mrg_m[w * 16 + row] - M);
+                    L += sc * mrg_l[w * 16 + row];
+                    acc += sc * mrg_o[(w * 16 + row) * HD + col];
+                }
+                const float val = acc / L;
+                const int h = d.g * a.G + row;
+                if (single) {
+                    a.out[((size_t)d.r * a.nq + h) * HD + col] = f2bf(val);
+                } else {
+                    a.part_o[((size_t)it * a.G + row) * HD + col] = val;
+                    if (col == 0) a.part_lse[(size_t)it * a.G + row] = M + log2f(L);
+                }
+            }
+            // every consumer thread leaves together if any warp gave up on a wait
+            if (named_bar_or(1, DEC_CONSUMERS * 32, !alive || *abort_flag)) break;
+            seq_base += (uint32_t)np;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && a.trace != nullptr) {
+        const int i = atomicAdd(a.trace_ctr, 1);
+        if (i < a.trace_cap) {
+            a.trace[i].kernel = NF_KERNEL_DECODE_ATTN;
+            a.trace[i].smid = (int32_t)smid();
+            a.trace[i].t_start = t_start;
+            a.trace[i].t_end = globaltimer_ns();
+        }
+    }
+}
+
+// Split-KV merge: out[r][h] = sum_s 2^(lse_s - LSE) o_s, fixed split order. One warp per (r, h).
+template <int HD>
+__global__ void decode_merge_kernel(const __grid_constant__ DecodeArgs a) {
+    const int warps = (gridDim.x * blockDim.x) >> 5;
+    const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nreq = a.req_end - a.req_begin;
+    for (int w = wid; w < nreq * a.nq; w += warps) {
+        const int r = a.req_begin + w / a.nq;
+        const int h = w % a.nq;
+        const int g = h / a.G, row = h - g * a.G;
+        const int nkeys = a.ctx_len[r] + 1;
+        const int npages = (nkeys + 15) >> 4;
+        const int nsplit = (npages + a.split_pages - 1) / a.split_pages;
+        if (nsplit <= 1) continue;
+        const int base = a.item_off[r];
+        float M = -INFINITY;
+        for (int s = 0; s < nsplit; ++s) M = fmaxf(M, a.part_lse[(size_t)(base + s * a.nkv + g) * a.G + row]);
+        float L = 0.f;
+        float acc[HD / 32];
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) acc[c] = 0.f;
+        for (int s = 0; s < nsplit; ++s) {
+            const int item = base + s * a.nkv + g;
+            const float wgt = exp2f(a.part_lse[(size_t)item * a.G + row] - M);
+            L += wgt;
+            const float* po = a.part_o + ((size_t)item * a.G + row) * HD;
+#pragma unroll
+            for (int c = 0; c < HD / 32; ++c) acc[c] += wgt * po[c * 32 + lane];
+        }
+        uint16_t* dst = a.out + ((size_t)r * a.nq + h) * HD;
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) dst[c * 32 + lane] = f2bf(acc[c] / L);
+    }
+}
+
+// ------------------------------------------------------------------ prefill chunk
+// Work item = (q tile of 64 chunk rows, query head); K/V tiles of 64 keys (4 pages)
+// stream through a 3-stage ring filled by a producer warp; four consumer warps own
+// 16 query rows each. Causal: tile kt is needed by q tile qt iff kt <= qt.
+template <int HD>
+__global__ void __launch_bounds__(PRE_THREADS, 1)
+    prefill_attention_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ PrefillArgs a) {
+    constexpr int BOXES = HD / 64;
+    constexpr uint32_t PAGE_BYTES = BOXES * BOX_BYTES;      // one page of K (or V), one KV head
+    constexpr uint32_t HALF_BYTES = 4 * PAGE_BYTES;          // 64 keys
+    constexpr uint32_t STAGE_BYTES = 2 * HALF_BYTES;
+    constexpr int KSTEPS = HD / 16;
+    constexpr int NT = HD / 8;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + PRE_STAGES * STAGE_BYTES);
+    uint64_t* empty = full + PRE_STAGES;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + PRE_STAGES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint64_t t_start = 0;
+    if (threadIdx.x == 0) {
+        t_start = globaltimer_ns();
+        for (int s = 0; s < PRE_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 4); }
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmKV);
+    }
+    __syncthreads();
+
+    const int C = a.prefill_len;
+    const int nqt = (C + 63) / 64;
+    const int nitems = nqt * a.nq;
+    const int npages = (C + 15) >> 4;
+    const int* pt = a.page_indices + a.page_indptr[a.num_decode];
+
+    if (warp == 4) {
+        if (lane == 0) {
+            uint32_t seq = 0;
+            bool ok = true;
+            uint32_t outstanding = 0, parity_bits = 0;
+            for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+                const int qt = nqt - 1 - it / a.nq;
+                const int h = it % a.nq;
+                const int g = h / a.G;
+                for (int kt = 0; kt <= qt; ++kt, ++seq) {
+                    const int stage = (int)(seq % PRE_STAGES);
+                    const uint32_t phase = (seq / PRE_STAGES) & 1u;
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+                    outstanding &= ~(1u << stage);
+                    uint8_t* st = smem + stage * STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+                    for (int pp = 0; pp < 4; ++pp) {
+                        // pages past the chunk repeat its last page: finite data under masked keys
+                        int pidx = min(kt * 4 + pp, npages - 1);
+                        int page = pt[pidx];
+                        if (page < 0 || page >= a.num_pages) { set_status(a.status, NF_ERR_DEVICE_BOUNDS); page = 0; }
+                        const int rowK = ((page * 2 + 0) * a.nkv + g) * 16;
+                        const int rowV = ((page * 2 + 1) * a.nkv + g) * 16;
+#pragma unroll
+                        for (int b = 0; b < BOXES; ++b) {
+                            tma_load_2d(st + pp * PAGE_BYTES + b * BOX_BYTES, &tmKV, &full[stage], b * 64, rowK);
+                            tma_load_2d(st + HALF_BYTES + pp * PAGE_BYTES + b * BOX_BYTES, &tmKV, &full[stage],
+                                        b * 64, rowV);
+                        }
+                    }
+                    outstanding |= 1u << stage;
+                    parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
+                }
+            }
+            if (!ok) {
+                volatile int quiet = 0;
+                for (int st = 0; st < PRE_STAGES; ++st)
+                    if (outstanding & (1u << st)) mbar_wait(&full[st], (parity_bits >> st) & 1u, &quiet, nullptr);
+            }
+        }
+        __syncwarp();
+    } else {
+        const int qr = lane >> 2, qc = (lane & 3) * 2;
+        uint32_t seq = 0;
+        bool alive = true;
+        for (int it = blockIdx.x; it < nitems && alive; it += gridDim.x) {
+            const int qt = nqt - 1 - it / a.nq;
+            const int h = it % a.nq;
+            const int i0 = qt * 64 + warp * 16 + qr;  // chunk rows of this thread: i0, i0 + 8
+            const int i1 = i0 + 8;
+            uint32_t qa[KSTEPS][4];
+            {
+                const uint16_t* qb = a.q + (size_t)h * HD;
+                const size_t rs = (size_t)a.nq * HD;
+                const bool v0 = i0 < C, v1 = i1 < C;
+                const uint16_t* q0 = qb + (size_t)(a.num_decode + i0) * rs;
+                const uint16_t* q1 = qb + (size_t)(a.num_decode + i1) * rs;
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk) {
+                    const int c = kk * 16 + qc;
+                    qa[kk][0] = v0 ? *reinterpret_cast<const uint32_t*>(q0 + c) : 0u;
+                    qa[kk][1] = v1 ? *reinterpret_cast<const uint32_t*>(q1 + c) : 0u;
+                    qa[kk][2] = v0 ? *reinterpret_cast<const uint32_t*>(q0 + c + 8) : 0u;
+                    qa[kk][3] = v1 ? *reinterpret_cast<const uint32_t*>(q1 + c + 8) : 0u;
+                }
+            }
+            float o[NT][4];
+#pragma unroll
+            for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+            float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+            for (int kt = 0; kt <= qt; ++kt, ++seq) {
+                const int stage = (int)(seq % PRE_STAGES);
+                const uint32_t phase = (seq / PRE_STAGES) & 1u;
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&full[stage], phase, abort_flag, a.status) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) { alive = false; break; }
+                const uint32_t sK = smem_u32(smem + stage * STAGE_BYTES);
+                const uint32_t sV = sK + HALF_BYTES;
+                float s[8][4];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk) {
+#pragma unroll
+                    for (int j = 0; j < 8; j += 2) {
+                        const int mi = lane >> 3;
+                        const int key = (j + (mi >> 1)) * 8 + (lane & 7);
+                        const int dc = kk * 16 + (mi & 1) * 8;
+                        uint32_t b0, b1, b2, b3;
+                        ldmatrix_x4(sK + (key >> 4) * PAGE_BYTES + (dc / 64) * BOX_BYTES + sw128_offset(key & 15, dc % 64),
+                                    b0, b1, b2, b3);
+                        mma_16816(s[j], qa[kk], b0, b1);
+                        mma_16816(s[j + 1], qa[kk], b2, b3);
+                    }
+                }
+                const int kbase = kt * 64;
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int key = kbase + j * 8 + qc + e;
+                        s[j][e] = (key <= i0) ? s[j][e] * a.scale_log2 : -INFINITY;
+                        s[j][2 + e] = (key <= i1) ? s[j][2 + e] * a.scale_log2 : -INFINITY;
+                        mx0 = fmaxf(mx0, s[j][e]);
+                        mx1 = fmaxf(mx1, s[j][2 + e]);
+                    }
+                }
+                mx0 = quad_max(mx0);
+                mx1 = quad_max(mx1);
+                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                // rows whose keys in this tile are all masked keep m = -inf: guard the rescale
+                const float c0 = (mn0 == -INFINITY) ? 1.f : exp2f(m0 - mn0);
+                const float c1 = (mn1 == -INFINITY) ? 1.f : exp2f(m1 - mn1);
+                m0 = mn0;
+                m1 = mn1;
+                float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        s[j][e] = (mn0 == -INFINITY) ? 0.f : exp2f(s[j][e] - mn0);
+                        s[j][2 + e] = (mn1 == -INFINITY) ? 0.f : exp2f(s[j][2 + e] - mn1);
+                        ps0 += s[j][e];
+                        ps1 += s[j][2 + e];
+                    }
+                }
+                l0 = l0 * c0 + ps0;
+                l1 = l1 * c1 + ps1;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) { o[j][0] *= c0; o[j][1] *= c0; o[j][2] *= c1; o[j][3] *= c1; }
+                // keys >= C (only in the last tile) get their V rows zeroed in the fragments
+                const int kb = (lane & 3) * 2;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    uint32_t pa[4];
+                    pa[0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
+                    pa[1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
+                    pa[2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+                    pa[3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+                    const int key0 = kbase + kk * 16;
+                    const bool tail = key0 + 16 > C;
+                    const bool k0 = key0 + kb < C, k1 = key0 + kb + 1 < C;
+                    const bool k8 = key0 + kb + 8 < C, k9 = key0 + kb + 9 < C;
+#pragma unroll
+                    for (int j = 0; j < NT; j += 2) {
+                        const int mi = lane >> 3;
+                        const int key = (mi & 1) * 8 + (lane & 7);
+                        const int dc = j * 8 + (mi >> 1) * 8;
+                        uint32_t b0, b1, b2, b3;
+                        ldmatrix_x4_trans(sV + kk * PAGE_BYTES + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64),
+                                          b0, b1, b2, b3);
+                        if (tail) {
+                            b0 = keep_pair(b0, k0, k1); b1 = keep_pair(b1, k8, k9);
+                            b2 = keep_pair(b2, k0, k1); b3 = keep_pair(b3, k8, k9);
+                        }
+                        mma_16816(o[j], pa, b0, b1);
+                        mma_16816(o[j + 1], pa, b2, b3);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+            }
+            if (!alive) break;
+            l0 = quad_sum(l0);
+            l1 = quad_sum(l1);
+            const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+            const size_t rs = (size_t)a.nq * HD;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const int c = j * 8 + qc;
+                if (i0 < C) {
+                    *reinterpret_cast<uint32_t*>(a.out + (size_t)(a.num_decode + i0) * rs + (size_t)h * HD + c) =
+                        pack_bf16x2(o[j][0] * inv0, o[j][1] * inv0);
+                }
+                if (i1 < C) {
+                    *reinterpret_cast<uint32_t*>(a.out + (size_t)(a.num_decode + i1) * rs + (size_t)h * HD + c) =
+                        pack_bf16x2(o[j][2] * inv1, o[j][3] * inv1);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && a.trace != nullptr) {
+        const int i = atomicAdd(a.trace_ctr, 1);
+        if (i < a.trace_cap) {
+            a.trace[i].kernel = NF_KERNEL_PREFILL_ATTN;
+            a.trace[i].smid = (int32_t)smid();
+            a.trace[i].t_start = t_start;
+            a.trace[i].t_end = globaltimer_ns();
+        }
+    }
+}
+
+// Items per request: nkv * ceil(ceil((ctx+1)/16) / split_pages); exclusive prefix into item_off[0..R].
+__global__ void decode_schedule_kernel(const int* ctx_len, int R, int nkv, int split_pages, int* item_off) {
+    __shared__ int carry;
+    __shared__ int warp_sums[32];
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < R; base += blockDim.x) {
+        const int r = base + threadIdx.x;
+        int v = 0;
+        if (r < R) {
+            const int npages = (ctx_len[r] + 1 + 15) >> 4;
+            v = nkv * ((npages + split_pages - 1) / split_pages);
+        }
+        // block inclusive scan
+        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sums[w] = x;
+        __syncthreads();
+        if (w == 0) {
+            const int nw = blockDim.x >> 5;
+            int s = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, s, o);
+                if (lane >= o) s += y;
+            }
+            if (lane < nw) warp_sums[lane] = s;
+        }
+        __syncthreads();
+        const int incl = x + (w > 0 ? warp_sums[w - 1] : 0);
+        if (r < R) item_off[r] = carry + incl - v;
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry += incl;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) item_off[R] = carry;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace
+
+int decode_smem_bytes(int hd) {
+    const int stage = 2 * (hd / 64) * BOX_BYTES;
+    return DEC_STAGES * stage + DEC_CONSUMERS * 16 * hd * 4 + 2 * DEC_CONSUMERS * 16 * 4 + 2 * DEC_STAGES * 8 + 16 +
+           1024;
+}
+
+int prefill_smem_bytes(int hd) {
+    const int stage = 2 * 4 * (hd / 64) * BOX_BYTES;
+    return PRE_STAGES * stage + 2 * PRE_STAGES * 8 + 16 + 1024;
+}
+
+cudaError_t launch_decode_schedule(const int* ctx_len, int R, int nkv, int split_pages, int* item_off,
+                                   cudaStream_t stream) {
+    decode_schedule_kernel<<<1, 1024, 0, stream>>>(ctx_len, R, nkv, split_pages, item_off);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_attention(const CUtensorMap& tmKV, const DecodeArgs& a, int head_dim, int grid,
+                                    int merge_grid, cudaStream_t stream) {
+    if (grid <= 0 || a.req_end <= a.req_begin) return cudaSuccess;
+    const int smem = decode_smem_bytes(head_dim);
+    cudaError_t e;
+    if (head_dim == 128) {
+        static bool cfg = false;
+        if (!cfg) { if ((e = set_smem(decode_attention_kernel<128>, smem)) != cudaSuccess) return e; cfg = true; }
+        static bool cfg_m = false;
+        if (!cfg_m) { if ((e = set_smem(decode_merge_kernel<128>, a.merge_smem_pad)) != cudaSuccess) return e; cfg_m = true; }
+        decode_attention_kernel<128><<<grid, DEC_THREADS, smem, stream>>>(tmKV, a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        decode_merge_kernel<128><<<merge_grid, 256, a.merge_smem_pad, stream>>>(a);
+    } else if (head_dim == 64) {
+        static bool cfg = false;
+        if (!cfg) { if ((e = set_smem(decode_attention_kernel<64>, smem)) != cudaSuccess) return e; cfg = true; }
+        static bool cfg_m = false;
+        if (!cfg_m) { if ((e = set_smem(decode_merge_kernel<64>, a.merge_smem_pad)) != cudaSuccess) return e; cfg_m = true; }
+        decode_attention_kernel<64><<<grid, DEC_THREADS, smem, stream>>>(tmKV, a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        decode_merge_kernel<64><<<merge_grid, 256, a.merge_smem_pad, stream>>>(a);
+    } else {
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_attention(const CUtensorMap& tmKV, const PrefillArgs& a, int head_dim, int grid,
+                                     cudaStream_t stream) {
+    if (grid <= 0 || a.prefill_len <= 0) return cudaSuccess;
+    const int smem = prefill_smem_bytes(head_dim);
+    cudaError_t e;
+    if (head_dim == 128) {
+        static bool cfg = false;
+        if (!cfg) { if ((e = set_smem(prefill_attention_kernel<128>, smem)) != cudaSuccess) return e; cfg = true; }
+        prefill_attention_kernel<128><<<grid, PRE_THREADS, smem, stream>>>(tmKV, a);
+    } else if (head_dim == 64) {
+        static bool cfg = false;
+        if (!cfg) { if ((e = set_smem(prefill_attention_kernel<64>, smem)) != cudaSuccess) return e; cfg = true; }
+        prefill_attention_kernel<64><<<grid, PRE_THREADS, smem, stream>>>(tmKV, a);
+    } else {
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace nf
+
+namespace nf {
+bool make_kv_tmap(CUtensorMap* map, const void* pool, int num_pages, int nkv, int head_dim) {
+    return make_tmap_bf16_2d(map, pool, (uint64_t)num_pages * 2 * nkv * 16, (uint64_t)head_dim, 16);
+}
+}  // namespace nf

@@ -1,0 +1,65 @@
+// Argument blocks and launchers of the attention kernels.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "nanoflow.h"
+
+namespace nf {
+
+// Decode keys are split into chunks of this many pages (512 keys); the split of a request
+// depends only on its ctx_len.
+constexpr int kDecodeSplitPages = 32;
+
+struct DecodeArgs {
+    const uint16_t* q;   // [rows x nq x d] bf16; decode request r is row r
+    uint16_t* out;       // [rows x nq x d] bf16
+    float* part_o;       // [items x G x d] split partials (normalised)
+    float* part_lse;     // [items x G] log2-sum-exp of each split
+    const int* ctx_len;  // [R]
+    const int* page_indptr;
+    const int* page_indices;
+    const int* item_off;  // [R + 1] first work item of each request
+    int req_begin, req_end;
+    int nq, nkv, G;
+    int num_pages;
+    int split_pages;
+    float scale_log2;     // log2(e) / sqrt(d)
+    int merge_smem_pad;   // dynamic shared memory requested by the merge kernel (SM exclusivity)
+    int* status;
+    int* trace_ctr;
+    nf_trace_entry* trace;
+    int trace_cap;
+};
+
+struct PrefillArgs {
+    const uint16_t* q;   // [rows x nq x d]; chunk row i is row num_decode + i
+    uint16_t* out;
+    const int* page_indptr;
+    const int* page_indices;
+    int num_decode;      // index of the prefill request in the page table
+    int prefill_len;
+    int nq, nkv, G;
+    int num_pages;
+    float scale_log2;
+    int* status;
+    int* trace_ctr;
+    nf_trace_entry* trace;
+    int trace_cap;
+};
+
+int decode_smem_bytes(int head_dim);
+int prefill_smem_bytes(int head_dim);
+
+cudaError_t launch_decode_schedule(const int* ctx_len, int R, int nkv, int split_pages, int* item_off,
+                                   cudaStream_t stream);
+cudaError_t launch_decode_attention(const CUtensorMap& tmKV, const DecodeArgs& a, int head_dim, int grid,
+                                    int merge_grid, cudaStream_t stream);
+cudaError_t launch_prefill_attention(const CUtensorMap& tmKV, const PrefillArgs& a, int head_dim, int grid,
+                                     cudaStream_t stream);
+
+// KV pool as a 2-D tensor [num_pages * 2 * nkv * 16 rows x d cols], 16 x 64 boxes, 128-byte swizzle.
+bool make_kv_tmap(CUtensorMap* map, const void* pool, int num_pages, int nkv, int head_dim);
+
+}  // namespace nf

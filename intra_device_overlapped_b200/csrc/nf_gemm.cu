@@ -1,0 +1,433 @@
+// Persistent bf16 GEMM on the 5th-generation tensor cores (tcgen05 + TMEM), fed by
+// TMA, with the fused epilogues of the serving iteration.
+//
+//   C[M x N] = A[M x K] * B[N x K]^T,  A and B bf16 K-major, fp32 accumulation in TMEM.
+//
+// The iteration's projections (QKV, O, gate/up, down, LM head) are the
+// compute-bound operations that NanoFlow keeps on the critical path while memory-
+// bound attention of another nano-batch runs beside them (README "Introduction").
+// Here each launch claims `grid` SMs: one CTA per SM (the 197 KB shared-memory
+// footprint rules out a second resident CTA of any hot-path kernel), looping over
+// 128 x 256 output tiles with a static stride.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: A box 128x64 and B box 256x64 per k-block into a
+//               4-stage shared-memory ring (128-byte swizzle).
+//   warp 1      TMEM allocator (512 columns = two 256-column accumulators) and the
+//               single thread that issues tcgen05.mma (M=128, N=256, K=16) and
+//               tcgen05.commit.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (thread = output row),
+//               fused math, vectorised global stores. Double-buffered accumulators
+//               let the epilogue of tile i run under the main loop of tile i+1.
+// Every wait is bounded (NF_WAIT_LIMIT_NS); on timeout the CTA records
+// NF_ERR_DEVICE_TIMEOUT, drains its outstanding copies and MMAs, frees TMEM, exits.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "nf_internal.h"
+#include "nf_ptx.cuh"
+
+namespace nf {
+namespace {
+
+constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK, STAGES = kGemmStages;
+constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
+constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr uint32_t IDESC = umma_idesc_bf16_f32(BM, BN);
+
+struct Tile {
+    int a_row;      // TMA row of A
+    int b_row;      // TMA row of B
+    int row_begin;  // launch-row range covered by this tile
+    int row_end;
+    int n_blk;
+};
+
+__device__ __forceinline__ int total_tiles(const GemmArgs& p) {
+    if (!p.grouped) return p.m_tiles * p.n_tiles;
+    int t = 0;
+    for (int g = 0; g < p.num_groups; ++g) {
+        const int rows = p.group_offsets[g + 1] - p.group_offsets[g];
+        t += ((rows + BM - 1) / BM) * p.n_tiles;
+    }
+    return t;
+}
+
+__device__ __forceinline__ Tile tile_at(const GemmArgs& p, int tile) {
+    Tile t;
+    if (!p.grouped) {
+        const int mb = tile % p.m_tiles;
+        t.n_blk = tile / p.m_tiles;
+        t.row_begin = mb * BM;
+        t.row_end = min(p.M, t.row_begin + BM);
+        t.a_row = p.a_row0 + t.row_begin;
+        t.b_row = t.n_blk * BN;
+        return t;
+    }
+    int base = 0;
+    for (int g = 0; g < p.num_groups; ++g) {
+        const int r0 = p.group_offsets[g], r1 = p.group_offsets[g + 1];
+        const int mt = (r1 - r0 + BM - 1) / BM;
+        const int cnt = mt * p.n_tiles;
+        if (tile < base + cnt) {
+            const int local = tile - base;
+            const int mb = local % mt;
+            t.n_blk = local / mt;
+            t.row_begin = r0 + mb * BM;
+            t.row_end = min(r1, t.row_begin + BM);
+            t.a_row = p.a_row0 + t.row_begin;
+            t.b_row = g * p.N + t.n_blk * BN;
+            return t;
+        }
+        base += cnt;
+    }
+    t.n_blk = 0; t.row_begin = 0; t.row_end = 0; t.a_row = 0; t.b_row = 0;
+    return t;
+}
+
+__device__ __forceinline__ float row_scale(const GemmArgs& p, int row) {
+    if (p.partials == nullptr) return 1.0f;
+    const float* pr = p.partials + (size_t)(p.tok0 + row) * p.n_part;
+    float s = 0.f;
+    for (int j = 0; j < p.n_part; ++j) s += pr[j];
+    return rsqrtf(s * p.inv_dim + p.eps);
+}
+
+__device__ __forceinline__ void store_bf16x32(uint16_t* dst, const float* v) {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+        w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+        w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+        w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+        d[q] = w;
+    }
+}
+
+__device__ __forceinline__ void store_f32x32(float* dst, const float* v) {
+    float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+// ------------------------------------------------------------------ epilogues
+// Each is called by all 32 lanes of an epilogue warp (tcgen05.ld is warp-collective);
+// `valid` says whether this lane's row is inside the tile's row range.
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, uint32_t tacc, int row,
+                                              bool valid) {
+    float v[32];
+    const int n0 = t.n_blk * BN;
+    if constexpr (EPI == EPI_F32) {
+        const float rs = valid ? row_scale(p, row) : 1.f;
+        float* dst = p.out_f32 + (size_t)(p.tok0 + row) * p.ld_f32 + n0;
+#pragma unroll 1
+        for (int j = 0; j < BN / 32; ++j) {
+            tmem_ld32(tacc + 32 * j, v);
+            if (valid) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] *= rs;
+                store_f32x32(dst + 32 * j, v);
+            }
+        }
+    } else if constexpr (EPI == EPI_RESID) {
+        const size_t base = (size_t)(p.tok0 + row) * p.N + n0;
+        float ss = 0.f;
+#pragma unroll 1
+        for (int j = 0; j < BN / 32; ++j) {
+            tmem_ld32(tacc + 32 * j, v);
+            if (valid) {
+                float* rp = p.resid + base + 32 * j;
+                const float4* r4 = reinterpret_cast<const float4*>(rp);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 x = r4[q];
+                    v[4 * q + 0] += x.x; v[4 * q + 1] += x.y; v[4 * q + 2] += x.z; v[4 * q + 3] += x.w;
+                }
+#pragma unroll
+                for (int e = 0; e < 32; ++e) ss += v[e] * v[e];
+                store_f32x32(rp, v);
+                store_bf16x32(p.out_bf16 + (size_t)(p.tok0 + row) * p.ld_bf16 + n0 + 32 * j, v);
+                if (p.out_f32) store_f32x32(p.out_f32 + (size_t)(p.tok0 + row) * p.ld_f32 + n0 + 32 * j, v);
+            }
+        }
+        if (valid) p.out_partials[(size_t)(p.tok0 + row) * p.n_tiles + t.n_blk] = ss;
+    } else if constexpr (EPI == EPI_SWIGLU) {
+        const float rs = valid ? row_scale(p, row) : 1.f;
+        float u[32];
+        uint16_t* dst = p.out_bf16 + (size_t)(p.tok0 + row) * p.ld_bf16 + t.n_blk * (BN / 2);
+#pragma unroll 1
+        for (int j = 0; j < BN / 64; ++j) {
+            tmem_ld32(tacc + 32 * j, v);
+            tmem_ld32(tacc + BN / 2 + 32 * j, u);
+            if (valid) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float g = v[e] * rs;
+                    const float up = u[e] * rs;
+                    v[e] = g / (1.0f + __expf(-g)) * up;
+                }
+                store_bf16x32(dst + 32 * j, v);
+            }
+        }
+    } else if constexpr (EPI == EPI_LMHEAD) {
+        const float rs = valid ? row_scale(p, row) : 1.f;
+        float best = -INFINITY;
+        int arg = n0;
+#pragma unroll 1
+        for (int j = 0; j < BN / 32; ++j) {
+            tmem_ld32(tacc + 32 * j, v);
+            if (valid) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    v[e] *= rs;
+                    if (v[e] > best) { best = v[e]; arg = n0 + 32 * j + e; }
+                }
+                if (p.out_bf16) store_bf16x32(p.out_bf16 + (size_t)(p.tok0 + row) * p.ld_bf16 + n0 + 32 * j, v);
+            }
+        }
+        if (valid) {
+            p.tile_max[(size_t)(p.tok0 + row) * p.n_tiles + t.n_blk] = best;
+            p.tile_arg[(size_t)(p.tok0 + row) * p.n_tiles + t.n_blk] = arg;
+        }
+    } else if constexpr (EPI == EPI_QKV) {
+        const int d = p.head_dim, half = d / 2;
+        const int tok = p.tok0 + row;
+        const float rs = valid ? row_scale(p, row) : 1.f;
+        int pos = 0;
+        long long kv_off = -1;  // element offset of this token's K slot for kv head 0
+        bool ok = valid;
+        if (valid) {
+            pos = p.positions[tok];
+            if (pos < 0 || pos >= p.max_position) {
+                set_status(p.status, NF_ERR_DEVICE_BOUNDS);
+                ok = false;
+            } else {
+                const int req = tok < p.num_decode ? tok : p.num_decode;
+                const int idx = p.page_indptr[req] + pos / 16;
+                const int page = (idx < p.page_indptr[req + 1]) ? p.page_indices[idx] : -1;
+                if (page < 0 || page >= p.num_pages) {
+                    set_status(p.status, NF_ERR_DEVICE_BOUNDS);
+                } else {
+                    kv_off = ((long long)page * 2 * p.nkv * 16 + (pos % 16)) * d;
+                }
+            }
+        }
+        float x2[32];
+#pragma unroll 1
+        for (int hc = 0; hc < BN / d; ++hc) {
+            const int head = (n0 + hc * d) / d;
+            const int kind = head < p.nq ? 0 : (head < p.nq + p.nkv ? 1 : 2);
+            uint16_t* dst = nullptr;
+            if (kind == 0) {
+                dst = p.q_out + ((size_t)tok * p.nq + head) * d;
+            } else if (kv_off >= 0) {
+                const int g = kind == 1 ? head - p.nq : head - p.nq - p.nkv;
+                dst = p.kv_pool + kv_off + ((long long)(kind - 1) * p.nkv + g) * 16 * d;
+            }
+#pragma unroll 1
+            for (int j = 0; j < half / 32; ++j) {
+                tmem_ld32(tacc + hc * d + 32 * j, v);
+                tmem_ld32(tacc + hc * d + half + 32 * j, x2);
+                if (ok && dst != nullptr) {
+                    if (kind < 2) {
+                        const float* cs = p.rope_cos + (size_t)pos * half + 32 * j;
+                        const float* sn = p.rope_sin + (size_t)pos * half + 32 * j;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const float a = v[e] * rs, b = x2[e] * rs;
+                            const float c = cs[e], s = sn[e];
+                            v[e] = a * c - b * s;
+                            x2[e] = b * c + a * s;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) { v[e] *= rs; x2[e] *= rs; }
+                    }
+                    store_bf16x32(dst + 32 * j, v);
+                    store_bf16x32(dst + half + 32 * j, x2);
+                }
+            }
+        }
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ GemmArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;   // [2]
+    uint64_t* tempty = tfull + 2;       // [2]
+    uint64_t* drain = tempty + 2;       // [1]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    uint64_t t_start = 0;
+    if (threadIdx.x == 0) {
+        t_start = globaltimer_ns();
+        for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int ntiles = total_tiles(p);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            uint32_t stage = 0, phase = 0;
+            int pending[STAGES];
+            for (int s = 0; s < STAGES; ++s) pending[s] = -1;  // parity of an unconsumed load, -1 = none
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const Tile t = tile_at(p, tile);
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    pending[stage] = -1;
+                    uint8_t* sa = smem + stage * STAGE_BYTES;
+                    uint8_t* sb = sa + A_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+                    tma_load_2d(sa, &tmA, &full[stage], kb * BK, t.a_row);
+                    tma_load_2d(sb, &tmB, &full[stage], kb * BK, t.b_row);
+                    pending[stage] = (int)phase;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok || *abort_flag) {
+                // Let every copy still in flight land before the CTA exits.
+                volatile int quiet = 0;
+                for (int s = 0; s < STAGES; ++s)
+                    if (pending[s] >= 0) mbar_wait(&full[s], (uint32_t)pending[s], &quiet, nullptr);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            uint32_t stage = 0, phase = 0;
+            int local = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++local) {
+                const int acc = local & 1;
+                const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint64_t adesc = umma_desc_sw128(sa);
+                    const uint64_t bdesc = umma_desc_sw128(sa + A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        // advance 16 bf16 = 32 bytes along K inside the 128-byte swizzle atom
+                        umma_bf16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), IDESC,
+                                  (kb | k) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(&empty[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (ok) umma_commit(&tfull[acc]);
+            }
+            // All MMAs issued by this thread have completed once `drain` flips.
+            umma_commit(drain);
+            volatile int quiet = 0;
+            mbar_wait(drain, 0, &quiet, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- epilogue warps 2..5; TMEM lane quarter = warp % 4
+        const int quarter = warp & 3;
+        const int row_in_tile = quarter * 32 + lane;
+        int local = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
+            const int acc = local & 1;
+            const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const Tile t = tile_at(p, tile);
+            const int row = t.row_begin + row_in_tile;
+            const bool valid = row < t.row_end;
+            const uint32_t tacc = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+            epilogue_tile<EPI>(p, t, tacc, row, valid);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+        __syncwarp();
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+    if (threadIdx.x == 0 && p.trace != nullptr) {
+        const int i = atomicAdd(p.trace_ctr, 1);
+        if (i < p.trace_cap) {
+            p.trace[i].kernel = NF_KERNEL_GEMM;
+            p.trace[i].smid = (int32_t)smid();
+            p.trace[i].t_start = t_start;
+            p.trace[i].t_end = globaltimer_ns();
+        }
+    }
+}
+
+template <int EPI>
+cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args, int grid,
+                       cudaStream_t stream) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kGemmSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    gemm_kernel<EPI><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, args);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args, int grid,
+                        cudaStream_t stream) {
+    if (grid <= 0) return cudaSuccess;
+    switch (epi) {
+        case EPI_F32: return launch_one<EPI_F32>(tmA, tmB, args, grid, stream);
+        case EPI_QKV: return launch_one<EPI_QKV>(tmA, tmB, args, grid, stream);
+        case EPI_RESID: return launch_one<EPI_RESID>(tmA, tmB, args, grid, stream);
+        case EPI_SWIGLU: return launch_one<EPI_SWIGLU>(tmA, tmB, args, grid, stream);
+        case EPI_LMHEAD: return launch_one<EPI_LMHEAD>(tmA, tmB, args, grid, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace nf

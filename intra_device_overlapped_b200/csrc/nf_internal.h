@@ -1,0 +1,79 @@
+// Internal interfaces between the C ABI layer and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "nanoflow.h"
+
+namespace nf {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBN = 256;
+constexpr int kGemmBK = 64;
+constexpr int kGemmStages = 4;
+constexpr int kGemmThreads = 192;
+constexpr int kGemmSmemBytes = kGemmStages * (kGemmBM + kGemmBN) * kGemmBK * 2 + 1024 + 256;
+
+enum EpiKind : int {
+    EPI_F32 = 0,     // out_f32 = acc (* rs if partials)
+    EPI_QKV = 1,     // rs, RoPE on q/k heads, q -> q_out, k/v -> paged cache slots
+    EPI_RESID = 2,   // resid += acc; bf16 copy; per-(row, N-tile) sum of squares
+    EPI_SWIGLU = 3,  // rs; silu(gate) * up over interleaved 128-col halves -> bf16
+    EPI_LMHEAD = 4,  // rs; bf16 logits (optional); per-(row, N-tile) max and first argmax
+};
+
+struct GemmArgs {
+    int M;         // rows of the launch (grouped: rows of all groups)
+    int a_row0;    // TMA row coordinate of launch row 0 in A
+    int tok0;      // per-row parameter index of launch row 0
+    int N;         // output columns (grouped: per group)
+    int K;
+    int m_tiles, n_tiles, k_blocks;
+    int grouped;   // 1: rows split by group_offsets, B rows of group g start at g * N
+    const int* group_offsets;  // [num_groups + 1], launch-row offsets (device)
+    int num_groups;
+    // RMSNorm row scale: rs = rsqrt(sum(partials[row][0..n_part)) * inv_dim + eps)
+    const float* partials;
+    int n_part;
+    float inv_dim;
+    float eps;
+    // outputs
+    float* out_f32;
+    int ld_f32;
+    uint16_t* out_bf16;
+    int ld_bf16;
+    float* resid;         // EPI_RESID: [rows x N] fp32 residual, updated in place
+    float* out_partials;  // EPI_RESID: [rows x n_tiles]
+    // EPI_QKV
+    const int* positions;
+    const float* rope_cos;  // [max_position x d/2]
+    const float* rope_sin;
+    int max_position;
+    uint16_t* q_out;        // [rows x nq x d]
+    int nq, nkv, head_dim;
+    uint16_t* kv_pool;      // [num_pages][2][nkv][16][d]
+    int num_pages;
+    const int* page_indptr;
+    const int* page_indices;
+    int num_decode;
+    // EPI_LMHEAD
+    float* tile_max;  // [rows x n_tiles]
+    int* tile_arg;
+    // diagnostics
+    int* status;
+    int* trace_ctr;
+    nf_trace_entry* trace;
+    int trace_cap;
+};
+
+// Encode a 2-D bf16 tensor map over a row-major [rows x cols] matrix with a box of
+// box_rows x 64 columns and 128-byte swizzle. Returns false on failure.
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
+cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args, int grid,
+                        cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace nf

@@ -1,0 +1,91 @@
+// Internal model state behind the opaque nf_model handle.
+#pragma once
+#include <cstdint>
+#include <vector>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "nanoflow.h"
+#include "nf_schedule.h"
+
+namespace nf {
+
+constexpr int kDecodeSplitPagesHost = 32;  // must equal kDecodeSplitPages (nf_attention.h)
+
+struct LayerWeights {
+    uint16_t* wqkv = nullptr;  // [(nq + 2 nkv) d x H], attn-norm gamma folded
+    uint16_t* wo = nullptr;    // [H x nq d]
+    uint16_t* wgu = nullptr;   // dense: [2F x H]; MoE: [E x 2F x H]; gate/up interleaved per 128 rows, gamma folded
+    uint16_t* wd = nullptr;    // dense: [H x F]; MoE: [E x H x F]
+    float* router = nullptr;   // MoE: [E x H] fp32, gamma folded
+    float* router_bias = nullptr;  // MoE: [E]
+    CUtensorMap tm_qkv, tm_o, tm_gu, tm_d;
+    bool loaded = false;
+};
+
+}  // namespace nf
+
+struct nf_model {
+    nf_model_config cfg;
+    nf::ModelDims dims;
+    int sm_count = 0;
+    int n_part = 0;  // H / 256 partial sums of squares per row
+    std::vector<nf::LayerWeights> layers;
+    bool globals_loaded = false;
+    uint16_t* embed = nullptr;    // [V x H]
+    uint16_t* lm_head = nullptr;  // [V x H], final-norm gamma folded
+    CUtensorMap tm_lm;
+
+    // workspace (rows sized by max_tokens; MoE rows by max_tokens * top_k)
+    float* resid = nullptr;       // [T x H] fp32 residual stream
+    uint16_t* xb = nullptr;       // [T x H] bf16 copy: A operand of QKV / gate-up
+    float* partials = nullptr;    // [T x H/256] sums of squares for the next RMSNorm
+    uint16_t* q = nullptr;        // [T x nq d]
+    uint16_t* attn_o = nullptr;   // [T x nq d]
+    uint16_t* act = nullptr;      // [T(*K) x F] SwiGLU output
+    float* rope_cos = nullptr;    // [max_position x d/2]
+    float* rope_sin = nullptr;
+    int* item_off = nullptr;      // [max_requests + 1]
+    float* part_o = nullptr;      // split-KV partials
+    float* part_lse = nullptr;
+    int64_t part_capacity = 0;    // items
+    // LM head
+    uint16_t* lm_in = nullptr;    // [max_requests + 1 x H]
+    float* lm_partials = nullptr;
+    float* tile_max = nullptr;    // [rows x V/256]
+    int* tile_arg = nullptr;
+    // MoE
+    float* moe_logits = nullptr;  // [T x E]
+    int* moe_idx = nullptr;       // [T x K]
+    float* moe_w = nullptr;
+    int* moe_counts = nullptr;    // [E + 1]
+    int* moe_perm = nullptr;      // [T K]
+    int* moe_inv = nullptr;
+    uint16_t* moe_a = nullptr;    // [T K x H]
+    float* moe_part = nullptr;    // [T K x H/256]
+    float* moe_y = nullptr;       // [T K x H]
+    CUtensorMap tm_xb, tm_attn_o, tm_act, tm_lm_in, tm_moe_a;
+
+    int* status = nullptr;        // device status word
+    int* trace_ctr = nullptr;
+    nf_trace_entry* trace = nullptr;
+    int trace_cap = 0;
+    bool trace_on = false;
+
+    cudaStream_t s_attn = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    std::vector<cudaEvent_t> events;
+
+    // KV pool tensor maps, cached per layer by pointer
+    std::vector<const void*> kv_ptr;
+    std::vector<int> kv_pages;
+    std::vector<CUtensorMap> kv_tm;
+
+    // per-op event timing
+    bool timing_on = false;
+    std::vector<cudaEvent_t> t_ev;
+    std::vector<nf_op_time> t_ops;
+
+    nf::CostModel cost;
+    std::vector<void*> allocations;
+};

@@ -1,0 +1,375 @@
+// Planner: nano-batch count, sizes, pipeline order and SM split by exhaustive search
+// over a per-kernel cost model, replacing the external MILP solver of the reference
+// design. NanoFlow "automatically identifies the number, size, ordering, and GPU
+// resource allocation of nano-batches to minimize the execution time, while
+// considering the interference of concurrent operations" (arXiv abstract; README
+// "Abstract": a parameter search algorithm sets up the pipeline).
+//
+// Candidates: n in 1..4 nano-batches; decode rows cut at request boundaries into
+// groups of equal KV bytes; the prefill chunk either its own nano-batch or joined to
+// the last decode group; pipeline order natural or prefill first; SM split for
+// attention in steps of 4; template sequential or pipelined. Each candidate's op list
+// (build_ops) is simulated on two streams; the minimum makespan wins.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "nf_model.h"
+#include "nf_schedule.h"
+
+namespace nf {
+
+std::vector<Op> build_ops(int tmpl, int n, const int* order, int L, bool moe) {
+    std::vector<Op> ops;
+    auto push = [&](int kind, int stream, int j, int l) {
+        Op o{kind, stream, j, l, 0, -1, 0};
+        ops.push_back(o);
+        return (int)ops.size() - 1;
+    };
+    if (tmpl == NF_TEMPLATE_SEQUENTIAL) {
+        for (int l = 0; l < L; ++l)
+            for (int i = 0; i < n; ++i) {
+                const int j = order[i];
+                push(OP_QKV, STREAM_GEMM, j, l);
+                push(OP_ATT, STREAM_GEMM, j, l);
+                push(OP_O, STREAM_GEMM, j, l);
+                if (moe) {
+                    push(OP_MOE, STREAM_GEMM, j, l);
+                } else {
+                    push(OP_GU, STREAM_GEMM, j, l);
+                    push(OP_D, STREAM_GEMM, j, l);
+                }
+            }
+        for (auto& o : ops) o.full_sm = 1;
+        return ops;
+    }
+    // Pipelined: attention of (j, l) on the attention stream right after QKV(j, l);
+    // O(j, l) waits for it; QKV(j, l+1) follows the FFN of (j, l) on the GEMM stream.
+    std::vector<int> qkv_idx((size_t)n * L, -1), att_idx((size_t)n * L, -1);
+    auto issue_qkv = [&](int j, int l) {
+        const int q = push(OP_QKV, STREAM_GEMM, j, l);
+        qkv_idx[(size_t)l * n + j] = q;
+        const int a = push(OP_ATT, STREAM_ATTN, j, l);
+        ops[a].wait = q;
+        ops[q].signal = 1;
+        att_idx[(size_t)l * n + j] = a;
+    };
+    for (int i = 0; i < n; ++i) issue_qkv(order[i], 0);
+    for (int l = 0; l < L; ++l) {
+        for (int i = 0; i < n; ++i) {
+            const int j = order[i];
+            const int o = push(OP_O, STREAM_GEMM, j, l);
+            ops[o].wait = att_idx[(size_t)l * n + j];
+            ops[att_idx[(size_t)l * n + j]].signal = 1;
+            if (moe) {
+                push(OP_MOE, STREAM_GEMM, j, l);
+            } else {
+                push(OP_GU, STREAM_GEMM, j, l);
+                push(OP_D, STREAM_GEMM, j, l);
+            }
+            if (l + 1 < L) issue_qkv(j, l + 1);
+        }
+    }
+    // A GEMM-stream op may take every SM iff it lies in no attention window: ATT(j, l)
+    // can only run between the end of QKV(j, l) and the start of O(j, l).
+    std::vector<int> gpos(ops.size(), -1);
+    int g = 0;
+    for (size_t i = 0; i < ops.size(); ++i)
+        if (ops[i].stream == STREAM_GEMM) gpos[i] = g++;
+    std::vector<int> covered(g + 1, 0);
+    for (size_t i = 0; i < ops.size(); ++i) {
+        if (ops[i].kind != OP_ATT) continue;
+        const int q = ops[i].wait;
+        int o = -1;
+        for (size_t k = i + 1; k < ops.size(); ++k)
+            if (ops[k].wait == (int)i) { o = (int)k; break; }
+        const int lo = gpos[q] + 1, hi = (o >= 0 ? gpos[o] : g);  // G ops in [lo, hi) may overlap
+        for (int x = lo; x < hi; ++x) covered[x] = 1;
+    }
+    for (size_t i = 0; i < ops.size(); ++i)
+        if (ops[i].stream == STREAM_GEMM) ops[i].full_sm = covered[gpos[i]] ? 0 : 1;
+    return ops;
+}
+
+CostModel default_cost_model(int sms) {
+    CostModel c;
+    if (sms <= 0) sms = 148;
+    c.gemm_flops_per_sm = 1.30e15 / 148.0;  // ~78% of the measured cuBLAS bf16 peak
+    c.gemm_tile_us = 0.8;
+    c.gemm_launch_us = 3.0;
+    c.hbm_bw = 6.0e12;
+    c.attn_bw_per_sm = 110e9;
+    c.attn_launch_us = 4.0;
+    c.attn_flops_per_sm = 2.0e12;
+    c.interference = 0.08;
+    c.calibrated = 0;
+    return c;
+}
+
+namespace {
+
+double gemm_us(const CostModel& c, int M, int N, int K, int grid, int64_t weight_bytes) {
+    if (M <= 0) return 0.0;
+    const int64_t tiles = (int64_t)((M + 127) / 128) * (N / 256);
+    const int g = std::max(1, std::min<int>(grid, (int)tiles));
+    const int64_t waves = (tiles + g - 1) / g;
+    const double t_tile = 2.0 * 128 * 256 * (double)K / c.gemm_flops_per_sm * 1e6 + c.gemm_tile_us;
+    const double t_compute = waves * t_tile;
+    const double bw = std::min(c.hbm_bw, g * c.attn_bw_per_sm * 1.2);
+    const double t_mem = (double)weight_bytes / bw * 1e6;
+    return c.gemm_launch_us + std::max(t_compute, t_mem);
+}
+
+}  // namespace
+
+double op_time_us(int kind, int j, const nf_plan& p, const ModelDims& m, const BatchInfo& b, const CostModel& c,
+                  int grid) {
+    const int t0 = p.tok_begin[j], t1 = p.tok_end[j];
+    const int M = t1 - t0;
+    if (M <= 0) return 0.0;
+    switch (kind) {
+        case OP_QKV: return gemm_us(c, M, m.qkv, m.H, grid, (int64_t)m.qkv * m.H * 2);
+        case OP_O: return gemm_us(c, M, m.H, m.nq * m.d, grid, (int64_t)m.H * m.nq * m.d * 2);
+        case OP_GU: return gemm_us(c, M, 2 * m.F, m.H, grid, (int64_t)2 * m.F * m.H * 2);
+        case OP_D: return gemm_us(c, M, m.H, m.F, grid, (int64_t)m.H * m.F * 2);
+        case OP_MOE: {
+            const int rows = M * m.K;
+            const int per = std::max(1, rows / std::max(1, m.E));
+            double t = 0;
+            // E groups of ~rows/E rows; weights of every expert are read once
+            t += gemm_us(c, per, 2 * m.F, m.H, std::max(1, grid / std::max(1, m.E)), (int64_t)2 * m.F * m.H * 2);
+            t += gemm_us(c, per, m.H, m.F, std::max(1, grid / std::max(1, m.E)), (int64_t)m.H * m.F * 2);
+            return t + 20.0;
+        }
+        case OP_ATT: {
+            const int r0 = std::min(t0, b.R), r1 = std::min(t1, b.R);
+            const int64_t bytes = b.req_kv_prefix[r1] - b.req_kv_prefix[r0];
+            double t = 0;
+            if (bytes > 0) {
+                const double bw = std::min(c.hbm_bw, grid * c.attn_bw_per_sm);
+                t += c.attn_launch_us + (double)bytes / bw * 1e6 + 3.0;
+            }
+            if (t1 > b.R && b.C > 0) {
+                const double flops = 4.0 * m.nq * m.d * (double)b.C * (b.C + 1) / 2.0;
+                t += c.attn_launch_us + flops / (grid * c.attn_flops_per_sm) * 1e6;
+            }
+            return t;
+        }
+    }
+    return 0.0;
+}
+
+double simulate_plan(const nf_plan& p, const ModelDims& m, const BatchInfo& b, const CostModel& c,
+                     double* serial_us) {
+    int order[NF_MAX_NANO];
+    for (int i = 0; i < p.n_nano; ++i) order[i] = p.nano_order[i];
+    const std::vector<Op> ops = build_ops(p.order_template, p.n_nano, order, m.L, m.E > 0);
+    const int S = p.sm_total;
+    std::vector<double> dur(ops.size()), beg(ops.size()), end(ops.size());
+    double serial = 0.0;
+    for (size_t i = 0; i < ops.size(); ++i) {
+        const Op& o = ops[i];
+        int grid = S;
+        if (p.order_template == NF_TEMPLATE_PIPELINED && !o.full_sm)
+            grid = (o.stream == STREAM_ATTN) ? p.sm_attn : p.sm_gemm;
+        if (p.order_template == NF_TEMPLATE_PIPELINED && o.kind == OP_ATT) grid = p.sm_attn;
+        dur[i] = op_time_us(o.kind, o.nano, p, m, b, c, grid);
+        serial += op_time_us(o.kind, o.nano, p, m, b, c, S);
+    }
+    if (serial_us) *serial_us = serial;
+    double makespan = 0.0;
+    for (int pass = 0; pass < 2; ++pass) {
+        double free_t[2] = {0.0, 0.0};
+        for (size_t i = 0; i < ops.size(); ++i) {
+            const Op& o = ops[i];
+            double st = free_t[o.stream];
+            if (o.wait >= 0) st = std::max(st, end[o.wait]);
+            beg[i] = st;
+            end[i] = st + dur[i];
+            free_t[o.stream] = end[i];
+        }
+        makespan = std::max(free_t[0], free_t[1]);
+        if (pass == 0 && p.order_template == NF_TEMPLATE_PIPELINED) {
+            // inflate each op by the interference factor times the fraction of it that overlaps the other stream
+            std::vector<std::pair<double, double>> other[2];
+            for (size_t i = 0; i < ops.size(); ++i) other[ops[i].stream].push_back({beg[i], end[i]});
+            for (size_t i = 0; i < ops.size(); ++i) {
+                if (dur[i] <= 0) continue;
+                double ov = 0;
+                for (auto& iv : other[1 - ops[i].stream])
+                    ov += std::max(0.0, std::min(end[i], iv.second) - std::max(beg[i], iv.first));
+                dur[i] *= 1.0 + c.interference * std::min(1.0, ov / dur[i]);
+            }
+        } else {
+            break;
+        }
+    }
+    return makespan;
+}
+
+}  // namespace nf
+
+// ------------------------------------------------------------------ C ABI entry point
+
+namespace {
+
+nf::BatchInfo batch_info(const nf_model* m, const nf_batch_desc* b) {
+    nf::BatchInfo bi;
+    bi.R = b->num_decode;
+    bi.C = b->prefill_len;
+    bi.T = bi.R + bi.C;
+    bi.req_kv_bytes.resize(bi.R);
+    bi.req_kv_prefix.assign(bi.R + 1, 0);
+    const int64_t page_bytes = 2LL * 16 * m->dims.d * 2 * m->dims.nkv;  // K and V of all KV heads
+    for (int r = 0; r < bi.R; ++r) {
+        const int64_t pages = (b->ctx_len[r] + 1 + 15) / 16;
+        bi.req_kv_bytes[r] = pages * page_bytes;
+        bi.req_kv_prefix[r + 1] = bi.req_kv_prefix[r] + bi.req_kv_bytes[r];
+    }
+    return bi;
+}
+
+// Cut decode requests [0, R) into `groups` contiguous ranges of near-equal KV bytes.
+std::vector<int> split_requests(const nf::BatchInfo& bi, int groups) {
+    std::vector<int> cut(groups + 1, 0);
+    cut[groups] = bi.R;
+    const int64_t total = bi.req_kv_prefix[bi.R];
+    for (int g = 1; g < groups; ++g) {
+        const int64_t target = total * g / groups;
+        int r = (int)(std::lower_bound(bi.req_kv_prefix.begin(), bi.req_kv_prefix.end(), target) -
+                      bi.req_kv_prefix.begin());
+        r = std::max(cut[g - 1], std::min(r, bi.R));
+        cut[g] = r;
+    }
+    return cut;
+}
+
+}  // namespace
+
+namespace {
+nf_status plan_impl(const nf_model* m, const nf_batch_desc* b, const nf_plan_opts* opts, nf_plan* out);
+}
+
+extern "C" nf_status nf_plan_iteration(const nf_model* m, const nf_batch_desc* b, const nf_plan_opts* opts,
+                                       nf_plan* out) {
+    return plan_impl(m, b, opts, out);
+}
+
+extern "C" nf_status nf_plan_for_config(const nf_model_config* cfg, int32_t sm_count, const nf_batch_desc* b,
+                                        const nf_plan_opts* opts, nf_plan* out) {
+    if (cfg == nullptr || sm_count <= 0) return NF_ERR_INVALID_ARGUMENT;
+    nf_model m;
+    m.cfg = *cfg;
+    m.dims.L = cfg->n_layers;
+    m.dims.H = cfg->hidden;
+    m.dims.nq = cfg->n_q_heads;
+    m.dims.nkv = cfg->n_kv_heads;
+    m.dims.d = cfg->head_dim;
+    m.dims.F = cfg->ffn;
+    m.dims.E = cfg->n_experts;
+    m.dims.K = cfg->n_experts > 0 ? cfg->top_k : 1;
+    m.dims.qkv = (cfg->n_q_heads + 2 * cfg->n_kv_heads) * cfg->head_dim;
+    m.sm_count = sm_count;
+    m.cost = nf::default_cost_model(sm_count);
+    if (m.dims.nkv <= 0 || m.dims.L <= 0) return NF_ERR_INVALID_ARGUMENT;
+    return plan_impl(&m, b, opts, out);
+}
+
+namespace {
+nf_status plan_impl(const nf_model* m, const nf_batch_desc* b, const nf_plan_opts* opts, nf_plan* out) {
+    if (m == nullptr || b == nullptr || out == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    const int R = b->num_decode, C = b->prefill_len;
+    if (R < 0 || C < 0 || R + C <= 0 || b->prefix_len != 0) return NF_ERR_INVALID_ARGUMENT;
+    if (R + C > m->cfg.max_tokens || R > m->cfg.max_requests) return NF_ERR_INVALID_ARGUMENT;
+    if (R > 0 && (b->ctx_len == nullptr)) return NF_ERR_INVALID_ARGUMENT;
+    if (b->page_indptr == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    // Page-table validation: every request holds enough pages, offsets are monotone.
+    for (int r = 0; r <= R; ++r) {
+        const int keys = r < R ? b->ctx_len[r] + 1 : C;
+        if (r < R && (b->ctx_len[r] < 0 || b->ctx_len[r] + 1 > m->cfg.max_position)) return NF_ERR_INVALID_ARGUMENT;
+        const int have = b->page_indptr[r + 1] - b->page_indptr[r];
+        if (have < 0 || have < (keys + 15) / 16) return NF_ERR_INVALID_ARGUMENT;
+    }
+    if (b->page_indptr[0] != 0 || b->num_pages <= 0) return NF_ERR_INVALID_ARGUMENT;
+
+    nf_plan_opts o;
+    if (opts) o = *opts; else { std::memset(&o, 0, sizeof(o)); o.force_template = -1; }
+    const int S = o.sm_total > 0 ? std::min(o.sm_total, m->sm_count) : m->sm_count;
+    const nf::BatchInfo bi = batch_info(m, b);
+    const nf::CostModel& cm = m->cost;
+
+    nf_plan best;
+    std::memset(&best, 0, sizeof(best));
+    double best_t = 1e30;
+    int n_lo = 1, n_hi = NF_MAX_NANO;
+    if (o.force_nano > 0) n_lo = n_hi = std::min(o.force_nano, NF_MAX_NANO);
+
+    for (int n = n_lo; n <= n_hi; ++n) {
+        for (int prefill_alone = 0; prefill_alone <= 1; ++prefill_alone) {
+            if (prefill_alone && (C == 0 || R == 0 || n < 2)) continue;
+            const int dgroups = prefill_alone ? n - 1 : n;
+            if (dgroups > std::max(R, 1)) continue;
+            if (R == 0 && n > 1) continue;
+            nf_plan p;
+            std::memset(&p, 0, sizeof(p));
+            p.n_nano = n;
+            p.num_decode = R;
+            p.prefill_len = C;
+            p.num_tokens = R + C;
+            p.sm_total = S;
+            const std::vector<int> cut = split_requests(bi, std::max(dgroups, 1));
+            bool degenerate = false;
+            for (int g = 0; g < dgroups; ++g) {
+                p.tok_begin[g] = cut[g];
+                p.tok_end[g] = cut[g + 1];
+                if (p.tok_end[g] <= p.tok_begin[g]) degenerate = true;
+            }
+            if (prefill_alone) {
+                p.tok_begin[n - 1] = R;
+                p.tok_end[n - 1] = R + C;
+            } else {
+                p.tok_end[dgroups - 1] = R + C;
+            }
+            if (degenerate) continue;
+            for (int ord = 0; ord <= 1; ++ord) {
+                if (ord == 1 && !prefill_alone) continue;
+                for (int i = 0; i < n; ++i) p.nano_order[i] = ord == 0 ? i : (i == 0 ? n - 1 : i - 1);
+                for (int tmpl = 0; tmpl <= 1; ++tmpl) {
+                    if (o.force_template >= 0 && tmpl != o.force_template) continue;
+                    if (tmpl == NF_TEMPLATE_PIPELINED && n < 2) continue;
+                    p.order_template = tmpl;
+                    int a_lo = 8, a_hi = S - 8, a_step = 4;
+                    if (tmpl == NF_TEMPLATE_SEQUENTIAL) { a_lo = a_hi = 0; }
+                    if (o.force_sm_attn > 0 && tmpl == NF_TEMPLATE_PIPELINED) a_lo = a_hi = std::min(o.force_sm_attn, S - 4);
+                    for (int sa = a_lo; sa <= a_hi; sa += a_step) {
+                        p.sm_attn = tmpl == NF_TEMPLATE_SEQUENTIAL ? S : sa;
+                        p.sm_gemm = tmpl == NF_TEMPLATE_SEQUENTIAL ? S : S - sa;
+                        double serial = 0;
+                        const double t = nf::simulate_plan(p, m->dims, bi, cm, &serial);
+                        if (t < best_t) {
+                            best_t = t;
+                            best = p;
+                            best.predicted_us = (float)t;
+                            best.predicted_serial_us = (float)serial;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    if (best.n_nano == 0) return NF_ERR_INVALID_ARGUMENT;
+    int64_t pages = 0;
+    for (int r = 0; r < R; ++r) pages += (b->ctx_len[r] + 1 + 15) / 16;
+    pages += (C + 15) / 16;
+    best.kv_pages_read = pages;
+    int64_t items = 0;
+    for (int r = 0; r < R; ++r) {
+        const int np = (b->ctx_len[r] + 1 + 15) / 16;
+        items += (int64_t)m->dims.nkv * ((np + nf::kDecodeSplitPagesHost - 1) / nf::kDecodeSplitPagesHost);
+    }
+    best.decode_items = items;
+    *out = best;
+    return NF_OK;
+}
+}  // namespace

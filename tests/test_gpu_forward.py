@@ -1,0 +1,167 @@
+"""Whole-iteration parity on the GPU: nf_plan_iteration + nf_forward_iteration against the
+float64 oracle, plus the nano-batching invariant (every plan gives bitwise the same result).
+"""
+import numpy as np
+import pytest
+import torch
+
+from synth.workloads import WORKLOADS, TEST_WORKLOADS
+from synth import weights as SW
+import synth
+
+from parity import MAX_ABS, MEAN_REL, errors
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _bits(t):
+    return t.detach().contiguous().view(torch.int16).cpu().numpy()
+
+
+def _run(dw, plan):
+    dw.forward(plan)
+    st = dw.sync()
+    assert st == 0, f"device status {st}"
+    return dw.hidden_out_f32.cpu().numpy().astype(np.float64)
+
+
+def _reset_kv(dw):
+    for layer, pool in enumerate(dw.kv):
+        SW.gpu_fill_kv_pool(dw.shape, layer, pool)
+    torch.cuda.synchronize()
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    from intra_device_overlapped_b200.harness import DeviceWorkload
+    from oracle.run import run_oracle
+    w = TEST_WORKLOADS["tiny_gamma"]
+    dw = DeviceWorkload(w, DEV)
+    b, res, kv = run_oracle(w, batch=dw.batch)
+    yield dw, res, kv
+    dw.close()
+
+
+PLANS = [dict(nano=1, template=0), dict(nano=2, template=1, sm_attn=16), dict(nano=3, template=1, sm_attn=40),
+         dict(nano=4, template=1, sm_attn=64), dict(nano=2, template=0)]
+
+
+@pytest.mark.parametrize("opts", PLANS)
+def test_tiny_iteration_matches_oracle(tiny, opts):
+    dw, res, _ = tiny
+    _reset_kv(dw)
+    plan = dw.plan(**opts)
+    hid = _run(dw, plan)
+    mx, rel = errors(hid, res["hidden"])
+    assert mx <= MAX_ABS and rel <= MEAN_REL, (mx, rel, plan.describe())
+    # bf16 output copy is the rounded fp32 residual
+    hb = dw.hidden_out.float().cpu().numpy()
+    assert np.abs(hb - hid).max() <= np.abs(hid).max() * 2 ** -8
+
+
+def test_tiny_nano_batching_is_bitwise_invariant(tiny):
+    dw, _, _ = tiny
+    outs, kvs = [], []
+    for opts in PLANS + [dict()]:
+        _reset_kv(dw)
+        plan = dw.plan(**opts)
+        _run(dw, plan)
+        outs.append(_bits(dw.hidden_out_f32))
+        kvs.append(_bits(dw.kv[0]))
+    for o, k in zip(outs[1:], kvs[1:]):
+        assert np.array_equal(o, outs[0])
+        assert np.array_equal(k, kvs[0])
+
+
+def test_tiny_kv_slots_written_and_others_untouched(tiny):
+    dw, res, kv_oracle = tiny
+    _reset_kv(dw)
+    _run(dw, dw.plan(nano=2, template=1, sm_attn=20))
+    s, b = dw.shape, dw.batch
+    got = dw.kv[0].float().cpu().numpy()
+    init = synth.bf16_to_f64(SW.host_kv_pool(s, 0, b.num_pages))
+    written = res["layers"][0]["written"]
+    mask = np.zeros(got.shape, dtype=bool)
+    worst = 0.0
+    for t, (page, slot) in written.items():
+        mask[page, :, :, slot, :] = True
+        ref = kv_oracle.pages[(0, page)][:, :, slot, :]
+        worst = max(worst, float(np.abs(got[page, :, :, slot, :] - ref).max()))
+    assert worst <= MAX_ABS, worst
+    assert np.array_equal(got[~mask], init[~mask])          # every other slot bit-identical
+
+
+def test_tiny_iteration_is_idempotent(tiny):
+    dw, _, _ = tiny
+    _reset_kv(dw)
+    plan = dw.plan(nano=2, template=1, sm_attn=24)
+    a = _run(dw, plan).copy()
+    b = _run(dw, plan)          # same K/V rewritten into the same slots
+    assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("name", ["tiny_decode_only", "tiny_prefill_only"])
+def test_degenerate_batches(name):
+    from intra_device_overlapped_b200.harness import DeviceWorkload
+    from oracle.run import run_oracle
+    w = TEST_WORKLOADS[name]
+    dw = DeviceWorkload(w, DEV)
+    try:
+        _, res, _ = run_oracle(w, batch=dw.batch)
+        for opts in (dict(nano=1, template=0), dict()):
+            _reset_kv(dw)
+            hid = _run(dw, dw.plan(**opts))
+            mx, rel = errors(hid, res["hidden"])
+            assert mx <= MAX_ABS and rel <= MEAN_REL, (mx, rel)
+    finally:
+        dw.close()
+
+
+def test_tiny_lm_head_and_argmax():
+    from intra_device_overlapped_b200.harness import DeviceWorkload
+    from oracle.run import run_oracle
+    w = TEST_WORKLOADS["tiny_lm"]
+    dw = DeviceWorkload(w, DEV)
+    try:
+        _, res, _ = run_oracle(w, batch=dw.batch)
+        _run(dw, dw.plan(nano=2, template=1, sm_attn=32))
+        logits = dw.logits.float().cpu().numpy()
+        mx, rel = errors(logits, res["logits"])
+        assert mx <= MAX_ABS and rel <= MEAN_REL, (mx, rel)
+        nxt = dw.next_token.cpu().numpy()
+        ref = res["logits"]
+        for r, tok in enumerate(nxt):
+            top = np.sort(ref[r])[::-1]
+            if top[0] - top[1] > 2 * mx:
+                assert tok == res["next_token"][r]
+            else:  # inside the error margin: the GPU's choice must be a near-maximum
+                assert ref[r, tok] >= top[0] - 2 * mx
+    finally:
+        dw.close()
+
+
+def test_tiny_moe_routing_and_output():
+    from intra_device_overlapped_b200.harness import DeviceWorkload
+    from oracle.run import run_oracle
+    w = TEST_WORKLOADS["tiny_moe"]
+    dw = DeviceWorkload(w, DEV, moe_debug=True)
+    try:
+        _, res, _ = run_oracle(w, batch=dw.batch)
+        hid = _run(dw, dw.plan(nano=2, template=1, sm_attn=24))
+        mx, rel = errors(hid, res["hidden"])
+        assert mx <= MAX_ABS and rel <= MEAN_REL, (mx, rel)
+        for layer in range(w.shape.n_layers):
+            z_gpu = dw.router_logits[layer].cpu().numpy().astype(np.float64)
+            z_ref = res["layers"][layer]["router_logits"]
+            zerr = np.abs(z_gpu - z_ref).max()
+            idx = dw.topk_idx[layer].cpu().numpy()
+            srt = np.sort(z_ref, axis=1)[:, ::-1]
+            for t in range(dw.T):
+                # routing function on the GPU's own logits is exact (top-2, ties to the lower index)
+                own = sorted(range(w.shape.n_experts), key=lambda e: (-z_gpu[t, e], e))[:2]
+                assert idx[t].tolist() == own
+                if srt[t, 1] - srt[t, 2] > 2 * zerr and srt[t, 0] - srt[t, 1] > 2 * zerr:
+                    assert idx[t].tolist() == res["layers"][layer]["topk_idx"][t].tolist()
+    finally:
+        dw.close()
