@@ -174,16 +174,17 @@ def op_algorithmic(work, batch, plan, op, nano):
         return "tensor", 2.0 * M * H * F
     if op == "lm_head":
         return "tensor", 2.0 * (batch.num_decode + (1 if batch.prefill_len else 0)) * H * s.vocab
-    if op == "attention":
+    if op == "decode_attention":
+        # K and V pages of every KV head of the decode requests, plus q in and o out
         R = batch.num_decode
         r0, r1 = min(t0, R), min(t1, R)
         pages = sum((int(batch.ctx_lens[r]) + 1 + 15) // 16 for r in range(r0, r1))
         kv = pages * 2 * nkv * 16 * d * 2
         qo = (r1 - r0) * nq * d * 2 * 2
-        if t1 > R and batch.prefill_len:
-            C = batch.prefill_len
-            kv += ((C + 15) // 16) * 2 * nkv * 16 * d * 2
         return "hbm", float(kv + qo)
+    if op == "prefill_attention":
+        C = batch.prefill_len
+        return "tensor", 4.0 * nq * d * C * (C + 1) / 2.0
     return None, 0.0
 
 
@@ -285,6 +286,7 @@ def run_ours(args, work, dist):
     torch.cuda.set_device(dev)
     dw = DeviceWorkload(work, dev, keep_logits=False)
     b = dw.batch
+    cost = dw.calibrate()
     plan = dw.plan(nano=args.nano, sm_attn=args.sm_attn, template=args.template)
     stream = torch.cuda.current_stream(dev)
 
@@ -370,10 +372,11 @@ def run_ours(args, work, dist):
         iso = {}
         for (name, nano, layer, stream_id, grid, us) in seq_ops:
             iso[name] = iso.get(name, 0.0) + us / nseq
+        att = ("decode_attention", "prefill_attention")
         extras["sequential"] = {"ms_per_step": round(seq_ms, 4),
                                 "isolated_op_ms": {k: round(v / 1000, 4) for k, v in iso.items()},
-                                "sum_isolated_gemm_ms": round(sum(v for k, v in iso.items() if k != "attention") / 1000, 4),
-                                "sum_isolated_attention_ms": round(iso.get("attention", 0.0) / 1000, 4)}
+                                "sum_isolated_gemm_ms": round(sum(v for k, v in iso.items() if k not in att) / 1000, 4),
+                                "sum_isolated_attention_ms": round(sum(iso.get(k, 0.0) for k in att) / 1000, 4)}
 
         # ---- end to end through the C ABI with host buffers: H2D inputs, D2H result, every step
         s = work.shape
@@ -438,7 +441,8 @@ def run_ours(args, work, dist):
             "frac_of_compute_optimum": round(t_opt_ms / ms_step, 4),
             "t_opt_ms": round(t_opt_ms, 4), "iteration_tflop": round(flops / 1e12, 4),
             "all_tokens_per_s": dist.world * b.num_tokens * args.steps / (ms_total / 1000.0),
-            "ops": op_summary, "roofline": roofline, "cpu_baseline": cpu, "clocks": clk,
+            "ops": op_summary, "cost_model": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in cost.items()},
+            "roofline": roofline, "cpu_baseline": cpu, "clocks": clk,
             "gpu_launches": count_launches(work, plan) * args.steps}
     line.update(extras)
     if "e2e" not in line:

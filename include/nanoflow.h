@@ -210,11 +210,27 @@ nf_status nf_forward_iteration(nf_model* m, const nf_plan* plan, const nf_iter_i
 /* Wait for the model's streams and return (and clear) the latched device status. */
 nf_status nf_sync_status(nf_model* m);
 
-/* Time each kernel kind of this model at the sizes of `b` and several SM shares,
- * plus one co-run, and store the results as the planner's cost tables. Runs real
- * launches on `stream` with the buffers of `io` (the KV pools are rewritten with
- * the same values a forward would write). */
+/* Time the model's own kernels at the sizes of `b` on several SM shares, and one
+ * GEMM + decode-attention co-run, and store the fitted rates as the planner's cost
+ * model (synchronous; a few tens of milliseconds). Reads the KV pools of `io`;
+ * writes only the model's workspace. */
 nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_iter_io* io, void* stream);
+
+/* The planner's per-kernel cost model (defaults until nf_calibrate has run). */
+typedef struct {
+    double gemm_flops_per_sm;  /* sustained tensor FLOP/s of one SM in the GEMM main loop */
+    double gemm_tile_us;       /* fixed cost per 128 x 256 output tile */
+    double gemm_launch_us;
+    double hbm_bw;             /* bytes/s the decode attention reaches on every SM */
+    double attn_bw_per_sm;     /* bytes/s one SM of decode attention pulls */
+    double attn_launch_us;
+    double attn_flops_per_sm;  /* prefill attention FLOP/s per SM */
+    double interference;       /* fractional slow-down of a GEMM and an attention kernel co-running */
+    int32_t calibrated;
+} nf_cost_model;
+
+nf_status nf_get_cost_model(const nf_model* m, nf_cost_model* out);
+nf_status nf_set_cost_model(nf_model* m, const nf_cost_model* in);
 
 /* Per-CTA placement trace of the last forward (enabled with nf_set_trace):
  * entries of {kernel id, sm id, start ns, end ns}. Returns the entry count
@@ -244,8 +260,8 @@ typedef struct {
     float us;
 } nf_op_time;
 
-enum { NF_OP_QKV = 0, NF_OP_ATTN = 1, NF_OP_O = 2, NF_OP_GATE_UP = 3, NF_OP_DOWN = 4, NF_OP_MOE = 5,
-       NF_OP_LM_HEAD = 6 };
+enum { NF_OP_QKV = 0, NF_OP_DECODE_ATTN = 1, NF_OP_O = 2, NF_OP_GATE_UP = 3, NF_OP_DOWN = 4, NF_OP_MOE = 5,
+       NF_OP_LM_HEAD = 6, NF_OP_PREFILL_ATTN = 7 };
 
 nf_status nf_set_timing(nf_model* m, int32_t enable);
 /* Waits for the model's streams; returns the number of entries written (<= capacity) or a negative nf_status. */

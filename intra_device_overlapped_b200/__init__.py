@@ -85,7 +85,17 @@ class nf_op_time(ctypes.Structure):
                 ("us", _f32)]
 
 
-NF_OP_NAMES = ("qkv", "attention", "o_proj", "gate_up", "down", "moe", "lm_head")
+NF_OP_NAMES = ("qkv", "decode_attention", "o_proj", "gate_up", "down", "moe", "lm_head", "prefill_attention")
+
+
+class nf_cost_model(ctypes.Structure):
+    _fields_ = [("gemm_flops_per_sm", ctypes.c_double), ("gemm_tile_us", ctypes.c_double),
+                ("gemm_launch_us", ctypes.c_double), ("hbm_bw", ctypes.c_double),
+                ("attn_bw_per_sm", ctypes.c_double), ("attn_launch_us", ctypes.c_double),
+                ("attn_flops_per_sm", ctypes.c_double), ("interference", ctypes.c_double), ("calibrated", _i32)]
+
+    def as_dict(self) -> dict:
+        return {f: getattr(self, f) for f, _ in self._fields_}
 
 
 class nf_trace_entry(ctypes.Structure):
@@ -112,6 +122,8 @@ def _load():
         "nf_forward_iteration": ([_vp, P(nf_plan), P(nf_iter_io), _vp], ctypes.c_int),
         "nf_sync_status": ([_vp], ctypes.c_int),
         "nf_calibrate": ([_vp, P(nf_batch_desc), P(nf_iter_io), _vp], ctypes.c_int),
+        "nf_get_cost_model": ([_vp, P(nf_cost_model)], ctypes.c_int),
+        "nf_set_cost_model": ([_vp, P(nf_cost_model)], ctypes.c_int),
         "nf_set_trace": ([_vp, _i32], ctypes.c_int),
         "nf_set_timing": ([_vp, _i32], ctypes.c_int),
         "nf_get_op_times": ([_vp, P(nf_op_time), _i64], _i64),
@@ -131,6 +143,7 @@ def _load():
 _lib = _load()
 EXPORTED = ("nf_status_string", "nf_version", "nf_init_model", "nf_set_layer_weights", "nf_set_global_weights",
             "nf_destroy_model", "nf_plan_iteration", "nf_plan_for_config", "nf_forward_iteration", "nf_sync_status", "nf_calibrate",
+            "nf_get_cost_model", "nf_set_cost_model",
             "nf_set_trace", "nf_get_trace", "nf_set_timing", "nf_get_op_times", "nf_op_gemm_bf16", "nf_op_decode_attention",
             "nf_op_prefill_attention", "nf_op_wait_flag_test")
 
@@ -200,6 +213,16 @@ def nf_sync_status(model: int) -> int:
 
 def nf_calibrate(model: int, batch: nf_batch_desc, io: nf_iter_io, stream: int = 0) -> int:
     return _lib.nf_calibrate(model, ctypes.byref(batch), ctypes.byref(io), stream)
+
+
+def nf_get_cost_model(model: int):
+    c = nf_cost_model()
+    st = _lib.nf_get_cost_model(model, ctypes.byref(c))
+    return st, c
+
+
+def nf_set_cost_model(model: int, c: nf_cost_model) -> int:
+    return _lib.nf_set_cost_model(model, ctypes.byref(c))
 
 
 def nf_set_trace(model: int, enable: bool) -> int:

@@ -326,9 +326,11 @@ nf_status ensure_part_capacity(nf_model* m, int64_t items) {
     const int64_t cap = std::max<int64_t>(items, 1024);
     dfree(m, m->part_o);
     dfree(m, m->part_lse);
+    dfree(m, m->item_tab);
     m->part_o = dalloc<float>(m, (size_t)cap * m->dims.nq / m->dims.nkv * m->dims.d);
     m->part_lse = dalloc<float>(m, (size_t)cap * m->dims.nq / m->dims.nkv);
-    if (!m->part_o || !m->part_lse) { m->part_capacity = 0; return NF_ERR_OUT_OF_MEMORY; }
+    m->item_tab = dalloc<int4>(m, (size_t)cap);
+    if (!m->part_o || !m->part_lse || !m->item_tab) { m->part_capacity = 0; return NF_ERR_OUT_OF_MEMORY; }
     m->part_capacity = cap;
     return NF_OK;
 }
@@ -344,6 +346,7 @@ nf::DecodeArgs decode_args(const nf_model* m, const nf_iter_io* io, const void* 
     a.page_indptr = io->page_indptr;
     a.page_indices = io->page_indices;
     a.item_off = m->item_off;
+    a.item_tab = m->item_tab;
     a.req_begin = rb;
     a.req_end = re;
     a.nq = m->dims.nq;
@@ -376,6 +379,28 @@ nf::PrefillArgs prefill_args(const nf_model* m, const nf_iter_io* io, const void
     if (m->trace_on) { a.trace_ctr = m->trace_ctr; a.trace = m->trace; a.trace_cap = m->trace_cap; }
     return a;
 }
+
+// Event pair around one launch group when per-op timing is on.
+struct OpTimer {
+    nf_model* m;
+    size_t idx = 0;
+    cudaError_t begin(cudaStream_t s) {
+        if (!m->timing_on) return cudaSuccess;
+        idx = m->t_ops.size();
+        while (m->t_ev.size() < 2 * (idx + 1)) {
+            cudaEvent_t e;
+            cudaError_t err = cudaEventCreate(&e);
+            if (err != cudaSuccess) return err;
+            m->t_ev.push_back(e);
+        }
+        return cudaEventRecord(m->t_ev[2 * idx], s);
+    }
+    cudaError_t end(cudaStream_t s, int kind, int nano, int layer, int stream_id, int grid) {
+        if (!m->timing_on) return cudaSuccess;
+        m->t_ops.push_back(nf_op_time{kind, nano, layer, stream_id, grid, 0.f});
+        return cudaEventRecord(m->t_ev[2 * idx + 1], s);
+    }
+};
 
 nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::Op& op, int grid,
                  cudaStream_t s) {
@@ -410,13 +435,18 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
         }
         case nf::OP_ATT: {
             const int rb = std::min(t0, R), re = std::min(t1, R);
+            OpTimer tm{m};
             if (re > rb) {
                 nf::DecodeArgs da = decode_args(m, io, m->q, m->attn_o, rb, re);
+                NF_CUDA_TRY(tm.begin(s));
                 NF_CUDA_TRY(nf::launch_decode_attention(m->kv_tm[l], da, d.d, grid, grid, s));
+                NF_CUDA_TRY(tm.end(s, NF_OP_DECODE_ATTN, j, l, op.stream, grid));
             }
             if (t1 > R && C > 0) {
                 nf::PrefillArgs pa = prefill_args(m, io, m->q, m->attn_o, R, C);
+                NF_CUDA_TRY(tm.begin(s));
                 NF_CUDA_TRY(nf::launch_prefill_attention(m->kv_tm[l], pa, d.d, grid, s));
+                NF_CUDA_TRY(tm.end(s, NF_OP_PREFILL_ATTN, j, l, op.stream, grid));
             }
             return NF_OK;
         }
@@ -561,7 +591,11 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     if (m->trace_on) NF_CUDA_TRY(cudaMemsetAsync(m->trace_ctr, 0, sizeof(int), sg));
 
     // prologue: decode work items, residual stream set-up
-    if (R > 0) NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, sg));
+    if (R > 0) {
+        NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, sg));
+        NF_CUDA_TRY(nf::launch_decode_items(io->ctx_len, io->page_indptr, R, d.nkv, nf::kDecodeSplitPages,
+                                            m->item_off, m->item_tab, sg));
+    }
     if (m->cfg.vocab > 0) {
         NF_CUDA_TRY(nf::launch_embed(io->token_ids, m->embed, T, d.H, m->cfg.vocab, m->resid, m->xb, m->partials,
                                      m->status, S * 4, sg));
@@ -579,15 +613,6 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
         m->events.push_back(e);
     }
     // timing entries accumulate over forwards until nf_set_timing is called again
-    const size_t t_base = m->t_ops.size();
-    const size_t n_timed = ops.size() + 1;
-    if (m->timing_on) {
-        while (m->t_ev.size() < 2 * (t_base + n_timed)) {
-            cudaEvent_t e;
-            NF_CUDA_TRY(cudaEventCreate(&e));
-            m->t_ev.push_back(e);
-        }
-    }
     for (size_t i = 0; i < ops.size(); ++i) {
         const nf::Op& op = ops[i];
         cudaStream_t s = op.stream == nf::STREAM_ATTN ? sa : sg;
@@ -597,13 +622,11 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
             if (op.stream == nf::STREAM_ATTN) grid = p->sm_attn;
             else if (!op.full_sm) grid = p->sm_gemm;
         }
-        const size_t ti = m->t_ops.size();
-        if (m->timing_on) NF_CUDA_TRY(cudaEventRecord(m->t_ev[2 * ti], s));
+        OpTimer tm{m};
+        const bool self_timed = op.kind == nf::OP_ATT;  // decode / prefill timed separately inside
+        if (!self_timed) NF_CUDA_TRY(tm.begin(s));
         if ((st = run_op(m, p, io, op, grid, s)) != NF_OK) return st;
-        if (m->timing_on) {
-            NF_CUDA_TRY(cudaEventRecord(m->t_ev[2 * ti + 1], s));
-            m->t_ops.push_back(nf_op_time{op.kind, op.nano, op.layer, op.stream, grid, 0.f});
-        }
+        if (!self_timed) NF_CUDA_TRY(tm.end(s, op.kind, op.nano, op.layer, op.stream, grid));
         if (op.signal) NF_CUDA_TRY(cudaEventRecord(m->events[i], s));
     }
     NF_CUDA_TRY(cudaEventRecord(m->ev_join, sa));
@@ -613,8 +636,8 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     if (m->cfg.vocab > 0 && (io->logits || io->next_token)) {
         const int rows = R + (C > 0 ? 1 : 0);
         NF_CUDA_TRY(nf::launch_lm_gather(m->xb, m->partials, R, T, rows, d.H, m->lm_in, m->lm_partials, S * 4, sg));
-        const size_t ti = m->t_ops.size();
-        if (m->timing_on) NF_CUDA_TRY(cudaEventRecord(m->t_ev[2 * ti], sg));
+        OpTimer tm{m};
+        NF_CUDA_TRY(tm.begin(sg));
         GemmArgs a = base_args(m);
         set_tiles(a, rows, m->cfg.vocab, d.H);
         a.partials = m->lm_partials;
@@ -626,10 +649,7 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
         if (io->next_token)
             NF_CUDA_TRY(nf::launch_argmax_reduce(m->tile_max, m->tile_arg, rows, m->cfg.vocab / 256, io->next_token,
                                                  S * 4, sg));
-        if (m->timing_on) {
-            NF_CUDA_TRY(cudaEventRecord(m->t_ev[2 * ti + 1], sg));
-            m->t_ops.push_back(nf_op_time{NF_OP_LM_HEAD, -1, d.L, 0, gemm_grid(a, S), 0.f});
-        }
+        NF_CUDA_TRY(tm.end(sg, NF_OP_LM_HEAD, -1, d.L, 0, gemm_grid(a, S)));
     }
     if (io->hidden_out)
         NF_CUDA_TRY(cudaMemcpyAsync(io->hidden_out, m->xb, (size_t)T * d.H * 2, cudaMemcpyDeviceToDevice, sg));
@@ -741,6 +761,8 @@ extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* ou
     NF_CUDA_TRY(cudaMemcpyAsync(&items, m->item_off + req_end, sizeof(int), cudaMemcpyDeviceToHost, s));
     NF_CUDA_TRY(cudaStreamSynchronize(s));
     if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
+    NF_CUDA_TRY(nf::launch_decode_items(io->ctx_len, io->page_indptr, req_end, m->dims.nkv, nf::kDecodeSplitPages,
+                                        m->item_off, m->item_tab, s));
     const int grid = sm_count > 0 ? std::min(sm_count, m->sm_count) : m->sm_count;
     nf::DecodeArgs da = decode_args(m, io, q, out, req_begin, req_end);
     NF_CUDA_TRY(nf::launch_decode_attention(m->kv_tm[layer], da, m->dims.d, grid, grid, s));
@@ -776,8 +798,160 @@ extern "C" nf_status nf_op_wait_flag_test(int32_t* flag_device, uint64_t limit_n
     return (nf_status)h;
 }
 
+namespace {
+
+// Mean time (us) of `reps` runs of fn on stream s, after one warm-up run.
+template <typename F>
+nf_status time_us(cudaStream_t s, int reps, F fn, double* out) {
+    cudaEvent_t a, b;
+    if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return NF_ERR_CUDA;
+    nf_status st = fn();
+    if (st == NF_OK && cudaEventRecord(a, s) != cudaSuccess) st = NF_ERR_CUDA;
+    for (int i = 0; i < reps && st == NF_OK; ++i) st = fn();
+    if (st == NF_OK && cudaEventRecord(b, s) != cudaSuccess) st = NF_ERR_CUDA;
+    float ms = 0.f;
+    if (st == NF_OK && (cudaEventSynchronize(b) != cudaSuccess || cudaEventElapsedTime(&ms, a, b) != cudaSuccess))
+        st = NF_ERR_CUDA;
+    cudaEventDestroy(a);
+    cudaEventDestroy(b);
+    *out = ms * 1000.0 / reps;
+    return st;
+}
+
+}  // namespace
+
 extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_iter_io* io, void* stream) {
-    (void)stream;
     if (m == nullptr || b == nullptr || io == nullptr) return NF_ERR_INVALID_ARGUMENT;
-    return NF_ERR_UNSUPPORTED;
+    const nf::ModelDims& d = m->dims;
+    const int R = b->num_decode, C = b->prefill_len, T = R + C;
+    if (T <= 0 || T > m->cfg.max_tokens || R > m->cfg.max_requests) return NF_ERR_INVALID_ARGUMENT;
+    if (!m->layers[0].loaded || io->kv_pools == nullptr || io->kv_pools[0] == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    if (R > 0 && (io->ctx_len == nullptr || b->ctx_len == nullptr)) return NF_ERR_INVALID_ARGUMENT;
+    cudaStream_t sg = (cudaStream_t)stream, sa = m->s_attn;
+    nf_status st = ensure_kv_tmap(m, 0, io);
+    if (st != NF_OK) return st;
+    const int S = m->sm_count;
+    nf::CostModel c = m->cost;
+
+    // (a) GEMM: the gate/up projection over all T rows on all SMs and on half of them
+    nf::LayerWeights& W = m->layers[0];
+    auto gemm = [&](int grid, cudaStream_t s) -> nf_status {
+        GemmArgs a = base_args(m);
+        set_tiles(a, T, 2 * d.F, d.H);
+        a.partials = m->partials;
+        a.out_bf16 = m->act;
+        a.ld_bf16 = d.F;
+        if (d.E > 0) {  // dense-shaped timing on the first expert's slice
+            a.m_tiles = (T + nf::kGemmBM - 1) / nf::kGemmBM;
+        }
+        return nf::launch_gemm(nf::EPI_SWIGLU, m->tm_xb, W.tm_gu, a, gemm_grid(a, grid), s) == cudaSuccess
+                   ? NF_OK : NF_ERR_CUDA;
+    };
+    NF_CUDA_TRY(cudaMemsetAsync(m->partials, 0, (size_t)T * m->n_part * sizeof(float), sg));
+    const int64_t tiles = (int64_t)((T + 127) / 128) * (2 * d.F / 256);
+    const double tile_flops = 2.0 * 128 * 256 * d.H;
+    double t_full = 0, t_half = 0;
+    if ((st = time_us(sg, 5, [&] { return gemm(S, sg); }, &t_full)) != NF_OK) return st;
+    const int half = std::max(8, S / 2);
+    if ((st = time_us(sg, 5, [&] { return gemm(half, sg); }, &t_half)) != NF_OK) return st;
+    {
+        const double w_full = (double)((tiles + S - 1) / S), w_half = (double)((tiles + half - 1) / half);
+        // t = launch + waves * (tile_flops / rate + tile_us): two equations, two unknowns (launch fixed)
+        const double per_tile_full = std::max(1e-3, (t_full - c.gemm_launch_us) / w_full);
+        const double per_tile_half = std::max(1e-3, (t_half - c.gemm_launch_us) / w_half);
+        const double per_tile = 0.5 * (per_tile_full + per_tile_half);
+        c.gemm_flops_per_sm = tile_flops / ((per_tile - c.gemm_tile_us) * 1e-6);
+    }
+
+    // (b) decode attention over every decode request at several SM shares
+    double bw_small = 0, bw_full = 0;
+    int64_t kv_bytes = 0;
+    for (int r = 0; r < R; ++r) kv_bytes += (int64_t)((b->ctx_len[r] + 1 + 15) / 16) * 2 * 16 * d.d * 2 * d.nkv;
+    if (R > 0) {
+        int64_t items = 0;
+        for (int r = 0; r < R; ++r) {
+            const int np = (b->ctx_len[r] + 1 + 15) / 16;
+            items += (int64_t)d.nkv * ((np + nf::kDecodeSplitPages - 1) / nf::kDecodeSplitPages);
+        }
+        if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
+        NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, sg));
+        NF_CUDA_TRY(nf::launch_decode_items(io->ctx_len, io->page_indptr, R, d.nkv, nf::kDecodeSplitPages,
+                                            m->item_off, m->item_tab, sg));
+        NF_CUDA_TRY(cudaMemsetAsync(m->q, 0, (size_t)R * d.nq * d.d * 2, sg));
+        auto dec = [&](int grid, cudaStream_t s) -> nf_status {
+            nf::DecodeArgs da = decode_args(m, io, m->q, m->attn_o, 0, R);
+            return nf::launch_decode_attention(m->kv_tm[0], da, d.d, grid, grid, s) == cudaSuccess ? NF_OK
+                                                                                                  : NF_ERR_CUDA;
+        };
+        const int small = std::max(4, S / 8);
+        double t_small = 0, t_all = 0;
+        if ((st = time_us(sg, 3, [&] { return dec(small, sg); }, &t_small)) != NF_OK) return st;
+        if ((st = time_us(sg, 3, [&] { return dec(S, sg); }, &t_all)) != NF_OK) return st;
+        bw_small = kv_bytes / ((t_small - c.attn_launch_us) * 1e-6) / small;
+        bw_full = kv_bytes / ((t_all - c.attn_launch_us) * 1e-6);
+        c.attn_bw_per_sm = bw_small;
+        c.hbm_bw = bw_full;
+
+        // (d) co-run: decode attention on a quarter of the SMs beside the GEMM on the rest
+        const int sa_n = std::max(8, S / 4), sg_n = S - sa_n;
+        double t_g = 0, t_a = 0;
+        if ((st = time_us(sg, 3, [&] { return gemm(sg_n, sg); }, &t_g)) != NF_OK) return st;
+        if ((st = time_us(sg, 2, [&] { return dec(sa_n, sg); }, &t_a)) != NF_OK) return st;
+        // run both, the attention stream repeating while the GEMMs run
+        cudaEvent_t e0, e1, e2, e3;
+        cudaEventCreate(&e0); cudaEventCreate(&e1); cudaEventCreate(&e2); cudaEventCreate(&e3);
+        NF_CUDA_TRY(cudaEventRecord(e0, sg));
+        NF_CUDA_TRY(cudaStreamWaitEvent(sa, e0, 0));
+        NF_CUDA_TRY(cudaEventRecord(e2, sa));
+        if ((st = dec(sa_n, sa)) != NF_OK) return st;
+        NF_CUDA_TRY(cudaEventRecord(e3, sa));
+        const int reps = std::max(1, (int)(t_a / std::max(1.0, t_g)));
+        for (int i = 0; i < reps && st == NF_OK; ++i) st = gemm(sg_n, sg);
+        NF_CUDA_TRY(cudaEventRecord(e1, sg));
+        NF_CUDA_TRY(cudaStreamWaitEvent(sg, e3, 0));
+        NF_CUDA_TRY(cudaStreamSynchronize(sg));
+        float ms_g = 0, ms_a = 0;
+        cudaEventElapsedTime(&ms_g, e0, e1);
+        cudaEventElapsedTime(&ms_a, e2, e3);
+        cudaEventDestroy(e0); cudaEventDestroy(e1); cudaEventDestroy(e2); cudaEventDestroy(e3);
+        if (st != NF_OK) return st;
+        const double slow_g = ms_g * 1000.0 / (reps * t_g), slow_a = ms_a * 1000.0 / t_a;
+        c.interference = std::max(0.0, std::min(1.0, 0.5 * (slow_g + slow_a) - 1.0));
+    }
+
+    // (c) prefill attention at a quarter of the SMs
+    if (C > 0) {
+        const int q = std::max(8, S / 4);
+        double t_p = 0;
+        auto pre = [&]() -> nf_status {
+            nf::PrefillArgs pa = prefill_args(m, io, m->q, m->attn_o, R, C);
+            return nf::launch_prefill_attention(m->kv_tm[0], pa, d.d, q, sg) == cudaSuccess ? NF_OK : NF_ERR_CUDA;
+        };
+        if ((st = time_us(sg, 3, pre, &t_p)) != NF_OK) return st;
+        const double flops = 4.0 * d.nq * d.d * (double)C * (C + 1) / 2.0;
+        c.attn_flops_per_sm = flops / ((t_p - c.attn_launch_us) * 1e-6) / q;
+    }
+    NF_CUDA_TRY(cudaStreamSynchronize(sg));
+    c.calibrated = 1;
+    m->cost = c;
+    return NF_OK;
+}
+
+extern "C" nf_status nf_get_cost_model(const nf_model* m, nf_cost_model* out) {
+    if (m == nullptr || out == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    const nf::CostModel& c = m->cost;
+    *out = nf_cost_model{c.gemm_flops_per_sm, c.gemm_tile_us, c.gemm_launch_us, c.hbm_bw, c.attn_bw_per_sm,
+                         c.attn_launch_us, c.attn_flops_per_sm, c.interference, c.calibrated};
+    return NF_OK;
+}
+
+extern "C" nf_status nf_set_cost_model(nf_model* m, const nf_cost_model* in) {
+    if (m == nullptr || in == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    if (!(in->gemm_flops_per_sm > 0) || !(in->hbm_bw > 0) || !(in->attn_bw_per_sm > 0) ||
+        !(in->attn_flops_per_sm > 0) || in->interference < 0)
+        return NF_ERR_INVALID_ARGUMENT;
+    m->cost = nf::CostModel{in->gemm_flops_per_sm, in->gemm_tile_us, in->gemm_launch_us, in->hbm_bw,
+                            in->attn_bw_per_sm, in->attn_launch_us, in->attn_flops_per_sm, in->interference,
+                            in->calibrated};
+    return NF_OK;
 }

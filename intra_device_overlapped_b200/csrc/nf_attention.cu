@@ -27,30 +27,11 @@
 namespace nf {
 namespace {
 
-constexpr int DEC_STAGES = 16;
-constexpr int DEC_CONSUMERS = 4;
-constexpr int DEC_THREADS = (DEC_CONSUMERS + 1) * 32;
+constexpr int DEC_WARPS = 6;  // independent streaming warps per CTA
+__host__ __device__ constexpr int dec_wstages(int hd) { return hd == 128 ? 4 : 8; }  // 32 KB in flight per warp
 constexpr int PRE_STAGES = 4;  // 128 KB for d = 128: one CTA per SM
 constexpr int PRE_THREADS = 5 * 32;
 constexpr int BOX_BYTES = 16 * 128;  // one 16-row x 64-col bf16 box
-
-__device__ __forceinline__ void named_bar_sync(int id, int threads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-// Named barrier that also ORs a predicate across the participating threads.
-__device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(threads)
-        : "memory");
-    return r != 0;
-}
 
 // Keep the low / high bf16 of a packed pair.
 __device__ __forceinline__ uint32_t keep_pair(uint32_t v, bool lo, bool hi) {
@@ -68,58 +49,77 @@ __device__ __forceinline__ float quad_sum(float x) {
     return x;
 }
 
-// Locate the request of item `it` in item_off[req_begin..req_end] (binary search).
-__device__ __forceinline__ int item_request(const int* item_off, int req_begin, int req_end, int it) {
-    int lo = req_begin, hi = req_end - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (item_off[mid] <= it) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
-
-struct DecItem {
-    int r, split, g, p0, p1, nkeys, nsplit;
+// Work-item table entry (built by decode_schedule_kernel):
+//   x = request r, y = g | split << 8 | nsplit << 20, z = index in page_indices of the item's
+//   first page, w = keys of the request (ctx_len + 1).
+struct DecMeta {
+    int r, g, split, nsplit, base, nkeys, np;
 };
 
-__device__ __forceinline__ DecItem dec_item(const DecodeArgs& a, int it) {
-    DecItem d;
-    d.r = item_request(a.item_off, a.req_begin, a.req_end, it);
-    const int local = it - a.item_off[d.r];
-    d.split = local / a.nkv;
-    d.g = local - d.split * a.nkv;
-    d.nkeys = a.ctx_len[d.r] + 1;
-    const int npages = (d.nkeys + 15) >> 4;
-    d.nsplit = (npages + a.split_pages - 1) / a.split_pages;
-    d.p0 = d.split * a.split_pages;
-    d.p1 = min(d.p0 + a.split_pages, npages);
-    return d;
+__device__ __forceinline__ DecMeta unpack_meta(int4 v, int split_pages) {
+    DecMeta m;
+    m.r = v.x;
+    m.g = v.y & 0xFF;
+    m.split = (v.y >> 8) & 0xFFF;
+    m.nsplit = (v.y >> 20) & 0xFFF;
+    m.base = v.z;
+    m.nkeys = v.w;
+    const int npages = (m.nkeys + 15) >> 4;
+    m.np = v.x < 0 ? 0 : min(split_pages, npages - m.split * split_pages);
+    return m;
 }
 
+template <int KSTEPS>
+__device__ __forceinline__ void load_q_frags(const DecodeArgs& a, const DecMeta& m, int qr, int qc, int hd,
+                                             uint32_t (&qa)[KSTEPS][4]) {
+    const bool r0 = m.r >= 0 && qr < a.G, r1 = m.r >= 0 && qr + 8 < a.G;
+    const uint16_t* q0 = a.q + ((size_t)(m.r < 0 ? 0 : m.r) * a.nq + (size_t)m.g * a.G) * hd;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+        const int c = kk * 16 + qc;
+        qa[kk][0] = r0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + (size_t)qr * hd + c)) : 0u;
+        qa[kk][1] = r1 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + (size_t)(qr + 8) * hd + c)) : 0u;
+        qa[kk][2] = r0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + (size_t)qr * hd + c + 8)) : 0u;
+        qa[kk][3] = r1 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + (size_t)(qr + 8) * hd + c + 8)) : 0u;
+    }
+}
+
+__device__ __forceinline__ int load_page_ids(const DecodeArgs& a, const DecMeta& m, int lane) {
+    int pg = 0;
+    if (lane < m.np) {
+        pg = __ldg(a.page_indices + m.base + lane);
+        if (pg < 0 || pg >= a.num_pages) {
+            set_status(a.status, NF_ERR_DEVICE_BOUNDS);
+            pg = 0;
+        }
+    }
+    return pg;
+}
+
+// Each warp is an independent streaming pipeline: it owns NSTW ring stages (one page of
+// one KV head, K and V, per stage), issues its own TMA loads (lane 0) and processes work
+// items my_b + w, my_b + w + DEC_WARPS, ... Its page stream runs across item boundaries;
+// the next item's table entry, page list and Q fragments are loaded while the current item
+// streams, so no global-load latency sits between pages or between items.
 template <int HD>
-__global__ void __launch_bounds__(DEC_THREADS, 1)
+__global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     decode_attention_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ DecodeArgs a) {
     constexpr int BOXES = HD / 64;
     constexpr uint32_t KV_BYTES = BOXES * BOX_BYTES;  // one page, one KV head, K or V
     constexpr uint32_t STAGE_BYTES = 2 * KV_BYTES;
+    constexpr int NSTW = dec_wstages(HD);
     constexpr int KSTEPS = HD / 16;
-    constexpr int NT = HD / 8;  // n-tiles of the output
+    constexpr int NT = HD / 8;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* mrg_o = reinterpret_cast<float*>(smem + DEC_STAGES * STAGE_BYTES);  // [4][16][HD]
-    float* mrg_m = mrg_o + DEC_CONSUMERS * 16 * HD;                           // [4][16]
-    float* mrg_l = mrg_m + DEC_CONSUMERS * 16;                                // [4][16]
-    uint64_t* full = reinterpret_cast<uint64_t*>(mrg_l + DEC_CONSUMERS * 16);
-    uint64_t* empty = full + DEC_STAGES;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + DEC_STAGES);
+    uint64_t* full_all = reinterpret_cast<uint64_t*>(smem + DEC_WARPS * NSTW * STAGE_BYTES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint64_t t_start = 0;
     if (threadIdx.x == 0) {
         t_start = globaltimer_ns();
-        for (int s = 0; s < DEC_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        *abort_flag = 0;
+        for (int s = 0; s < DEC_WARPS * NSTW; ++s) mbar_init(&full_all[s], 1);
         fence_mbar_init();
         tma_prefetch_desc(&tmKV);
     }
@@ -131,200 +131,205 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     const int my_b = ib + (int)(((long long)nitems * blockIdx.x) / gridDim.x);
     const int my_e = ib + (int)(((long long)nitems * (blockIdx.x + 1)) / gridDim.x);
 
-    if (warp == DEC_CONSUMERS) {
-        // ---------------- producer
-        if (lane == 0) {
-            uint32_t seq = 0;
-            bool ok = true;
-            uint32_t outstanding = 0;  // bit s: stage s holds a load the consumers have not released
-            uint32_t parity_bits = 0;  // bit s: parity of that load's phase
-            for (int it = my_b; it < my_e && ok; ++it) {
-                const DecItem d = dec_item(a, it);
-                const int* pt = a.page_indices + a.page_indptr[d.r];
-                for (int pl = d.p0; pl < d.p1; ++pl, ++seq) {
-                    const int stage = (int)(seq % DEC_STAGES);
-                    const uint32_t phase = (seq / DEC_STAGES) & 1u;
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
-                    outstanding &= ~(1u << stage);
-                    int page = pt[pl];
-                    if (page < 0 || page >= a.num_pages) { set_status(a.status, NF_ERR_DEVICE_BOUNDS); page = 0; }
-                    uint8_t* st = smem + stage * STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-                    const int rowK = ((page * 2 + 0) * a.nkv + d.g) * 16;
-                    const int rowV = ((page * 2 + 1) * a.nkv + d.g) * 16;
+    uint8_t* wsm = smem + warp * NSTW * STAGE_BYTES;
+    uint64_t* full = full_all + warp * NSTW;
+    const uint32_t wsm_u32 = smem_u32(wsm);
+    const int qr = lane >> 2, qc = (lane & 3) * 2;
+    const int4* tab = reinterpret_cast<const int4*>(a.item_tab);
+    const int4 none = make_int4(-1, 0, 0, 0);
+
+    int it = my_b + warp;
+    DecMeta cur = unpack_meta(it < my_e ? __ldg(tab + it) : none, a.split_pages);
+    DecMeta nxt = unpack_meta(it + DEC_WARPS < my_e ? __ldg(tab + it + DEC_WARPS) : none, a.split_pages);
+    int4 tab_nn = it + 2 * DEC_WARPS < my_e ? __ldg(tab + it + 2 * DEC_WARPS) : none;
+    uint32_t q_cur[KSTEPS][4], q_nxt[KSTEPS][4];
+    load_q_frags<KSTEPS>(a, cur, qr, qc, HD, q_cur);
+    int pages_cur = load_page_ids(a, cur, lane);
+    int pages_nxt = load_page_ids(a, nxt, lane);
+
+    // issue cursor over the warp's page stream: src 0 = current item, 1 = next item, 2 = wait
+    int iss_src = cur.np > 0 ? 0 : 2, iss_k = 0;
+    uint32_t issued = 0, consumed = 0;
+    volatile int quiet = 0;
+    bool alive = true;
+
+#define NF_DEC_TOP_UP()                                                                              \
+    while (issued - consumed < (uint32_t)NSTW && iss_src < 2) {                                      \
+        const DecMeta& im = iss_src == 0 ? cur : nxt;                                                \
+        const int pg = __shfl_sync(0xffffffffu, iss_src == 0 ? pages_cur : pages_nxt, iss_k);        \
+        if (lane == 0) {                                                                             \
+            const int st = (int)(issued % NSTW);                                                     \
+            uint8_t* dst = wsm + st * STAGE_BYTES;                                                   \
+            fence_proxy_async_smem();                                                                \
+            mbar_arrive_expect_tx(&full[st], STAGE_BYTES);                                           \
+            const int rowK = ((pg * 2 + 0) * a.nkv + im.g) * 16;                                     \
+            const int rowV = ((pg * 2 + 1) * a.nkv + im.g) * 16;                                     \
+            _Pragma("unroll") for (int b = 0; b < BOXES; ++b) {                                      \
+                tma_load_2d(dst + b * BOX_BYTES, &tmKV, &full[st], b * 64, rowK);                    \
+                tma_load_2d(dst + KV_BYTES + b * BOX_BYTES, &tmKV, &full[st], b * 64, rowV);         \
+            }                                                                                        \
+        }                                                                                            \
+        ++issued;                                                                                    \
+        if (++iss_k == im.np) {                                                                      \
+            iss_k = 0;                                                                               \
+            iss_src = (iss_src == 0 && nxt.np > 0) ? 1 : 2;                                          \
+        }                                                                                            \
+    }
+
+    NF_DEC_TOP_UP();
+    while (cur.np > 0 && alive) {
+        // prefetch two items ahead: Q fragments of the next item (its table entry and page list
+        // are already in registers), table entry of the one after
+        load_q_frags<KSTEPS>(a, nxt, qr, qc, HD, q_nxt);
+
+        float o[NT][4];
 #pragma unroll
-                    for (int b = 0; b < BOXES; ++b) {
-                        tma_load_2d(st + b * BOX_BYTES, &tmKV, &full[stage], b * 64, rowK);
-                        tma_load_2d(st + KV_BYTES + b * BOX_BYTES, &tmKV, &full[stage], b * 64, rowV);
-                    }
-                    outstanding |= 1u << stage;
-                    parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
+        for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+        for (int p = 0; p < cur.np; ++p) {
+            const int st = (int)(consumed % NSTW);
+            const uint32_t phase = (consumed / NSTW) & 1u;
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&full[st], phase, &quiet, a.status) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) { alive = false; break; }
+            const uint32_t sK = wsm_u32 + st * STAGE_BYTES;
+            const uint32_t sV = sK + KV_BYTES;
+            const int key0 = (cur.split * a.split_pages + p) * 16;
+            const int nvalid = min(16, cur.nkeys - key0);
+
+            float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+                const int mi = lane >> 3;
+                const int key = (mi >> 1) * 8 + (lane & 7);
+                const int dc = kk * 16 + (mi & 1) * 8;
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(sK + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64), b0, b1, b2, b3);
+                mma_16816(s[0], q_cur[kk], b0, b1);
+                mma_16816(s[1], q_cur[kk], b2, b3);
+            }
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const bool vis = (j * 8 + qc + e) < nvalid;
+                    s[j][e] = vis ? s[j][e] * a.scale_log2 : -INFINITY;
+                    s[j][2 + e] = vis ? s[j][2 + e] * a.scale_log2 : -INFINITY;
+                    mx0 = fmaxf(mx0, s[j][e]);
+                    mx1 = fmaxf(mx1, s[j][2 + e]);
                 }
             }
-            if (!ok) {
-                // let every copy still in flight land before the CTA exits
-                volatile int quiet = 0;
-                for (int st = 0; st < DEC_STAGES; ++st)
-                    if (outstanding & (1u << st)) mbar_wait(&full[st], (parity_bits >> st) & 1u, &quiet, nullptr);
+            mx0 = quad_max(mx0);
+            mx1 = quad_max(mx1);
+            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+            const float c0 = exp2f(m0 - mn0), c1 = exp2f(m1 - mn1);
+            m0 = mn0;
+            m1 = mn1;
+            float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    s[j][e] = exp2f(s[j][e] - mn0);
+                    s[j][2 + e] = exp2f(s[j][2 + e] - mn1);
+                    ps0 += s[j][e];
+                    ps1 += s[j][2 + e];
+                }
             }
+            l0 = l0 * c0 + ps0;
+            l1 = l1 * c1 + ps1;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) { o[j][0] *= c0; o[j][1] *= c0; o[j][2] *= c1; o[j][3] *= c1; }
+            uint32_t pa[4];
+            pa[0] = pack_bf16x2(s[0][0], s[0][1]);
+            pa[1] = pack_bf16x2(s[0][2], s[0][3]);
+            pa[2] = pack_bf16x2(s[1][0], s[1][1]);
+            pa[3] = pack_bf16x2(s[1][2], s[1][3]);
+            const int kb = (lane & 3) * 2;
+            const bool k0 = kb < nvalid, k1 = kb + 1 < nvalid, k8 = kb + 8 < nvalid, k9 = kb + 9 < nvalid;
+#pragma unroll
+            for (int j = 0; j < NT; j += 2) {
+                const int mi = lane >> 3;
+                const int key = (mi & 1) * 8 + (lane & 7);
+                const int dc = j * 8 + (mi >> 1) * 8;
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4_trans(sV + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64), b0, b1, b2, b3);
+                if (nvalid < 16) {  // V rows of keys past the request are zeroed
+                    b0 = keep_pair(b0, k0, k1); b1 = keep_pair(b1, k8, k9);
+                    b2 = keep_pair(b2, k0, k1); b3 = keep_pair(b3, k8, k9);
+                }
+                mma_16816(o[j], pa, b0, b1);
+                mma_16816(o[j + 1], pa, b2, b3);
+            }
+            __syncwarp();
+            ++consumed;
+            NF_DEC_TOP_UP();
         }
-        __syncwarp();
-    } else {
-        // ---------------- consumers
-        const int qr = lane >> 2;        // fragment row (query head within the group), +8 for the second half
-        const int qc = (lane & 3) * 2;   // fragment column pair
-        uint32_t seq_base = 0;
-        bool alive = true;
-        for (int it = my_b; it < my_e; ++it) {
-            const DecItem d = dec_item(a, it);
-            const int np = d.p1 - d.p0;
-            // Q fragments of heads g*G .. g*G+G-1 (rows >= G are zero)
-            uint32_t qa[KSTEPS][4];
-            {
-                const uint16_t* q0 = a.q + ((size_t)d.r * a.nq + (size_t)d.g * a.G) * HD;
-                const bool r0 = qr < a.G, r1 = qr + 8 < a.G;
-#pragma unroll
-                for (int kk = 0; kk < KSTEPS; ++kk) {
-                    const int c = kk * 16 + qc;
-                    qa[kk][0] = r0 ? *reinterpret_cast<const uint32_t*>(q0 + (size_t)qr * HD + c) : 0u;
-                    qa[kk][1] = r1 ? *reinterpret_cast<const uint32_t*>(q0 + (size_t)(qr + 8) * HD + c) : 0u;
-                    qa[kk][2] = r0 ? *reinterpret_cast<const uint32_t*>(q0 + (size_t)qr * HD + c + 8) : 0u;
-                    qa[kk][3] = r1 ? *reinterpret_cast<const uint32_t*>(q0 + (size_t)(qr + 8) * HD + c + 8) : 0u;
-                }
-            }
-            float o[NT][4];
-#pragma unroll
-            for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-            float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-
-            for (int pl = warp; pl < np && alive; pl += DEC_CONSUMERS) {
-                const uint32_t seq = seq_base + (uint32_t)pl;
-                const int stage = (int)(seq % DEC_STAGES);
-                const uint32_t phase = (seq / DEC_STAGES) & 1u;
-                int ok = 1;
-                if (lane == 0) ok = mbar_wait(&full[stage], phase, abort_flag, a.status) ? 1 : 0;
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) { alive = false; break; }  // still joins this item's barriers below
-                const uint32_t sK = smem_u32(smem + stage * STAGE_BYTES);
-                const uint32_t sV = sK + KV_BYTES;
-                const int key0 = (d.p0 + pl) * 16;
-                const int nvalid = min(16, d.nkeys - key0);  // >= 1
-
-                // S = Q K^T for the page's 16 keys (two n-tiles of 8 keys)
-                float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-                for (int kk = 0; kk < KSTEPS; ++kk) {
-                    const int mi = lane >> 3;
-                    const int key = (mi >> 1) * 8 + (lane & 7);
-                    const int dc = kk * 16 + (mi & 1) * 8;
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4(sK + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64), b0, b1, b2, b3);
-                    mma_16816(s[0], qa[kk], b0, b1);
-                    mma_16816(s[1], qa[kk], b2, b3);
-                }
-                // scale, mask keys beyond the request's length, online softmax
-                float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const bool vis = (j * 8 + qc + e) < nvalid;
-                        s[j][e] = vis ? s[j][e] * a.scale_log2 : -INFINITY;
-                        s[j][2 + e] = vis ? s[j][2 + e] * a.scale_log2 : -INFINITY;
-                        mx0 = fmaxf(mx0, s[j][e]);
-                        mx1 = fmaxf(mx1, s[j][2 + e]);
-                    }
-                }
-                mx0 = quad_max(mx0);
-                mx1 = quad_max(mx1);
-                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-                const float c0 = exp2f(m0 - mn0), c1 = exp2f(m1 - mn1);
-                m0 = mn0;
-                m1 = mn1;
-                float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        s[j][e] = exp2f(s[j][e] - mn0);
-                        s[j][2 + e] = exp2f(s[j][2 + e] - mn1);
-                        ps0 += s[j][e];
-                        ps1 += s[j][2 + e];
-                    }
-                }
-                l0 = l0 * c0 + ps0;
-                l1 = l1 * c1 + ps1;
-#pragma unroll
-                for (int j = 0; j < NT; ++j) { o[j][0] *= c0; o[j][1] *= c0; o[j][2] *= c1; o[j][3] *= c1; }
-                uint32_t pa[4];
-                pa[0] = pack_bf16x2(s[0][0], s[0][1]);
-                pa[1] = pack_bf16x2(s[0][2], s[0][3]);
-                pa[2] = pack_bf16x2(s[1][0], s[1][1]);
-                pa[3] = pack_bf16x2(s[1][2], s[1][3]);
-                // O += P V; V rows of keys beyond the request are zeroed in the fragments
-                const int kb = (lane & 3) * 2;
-                const bool k0 = kb < nvalid, k1 = kb + 1 < nvalid, k8 = kb + 8 < nvalid, k9 = kb + 9 < nvalid;
-#pragma unroll
-                for (int j = 0; j < NT; j += 2) {
-                    const int mi = lane >> 3;
-                    const int key = (mi & 1) * 8 + (lane & 7);
-                    const int dc = j * 8 + (mi >> 1) * 8;
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4_trans(sV + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64), b0, b1, b2, b3);
-                    if (nvalid < 16) {
-                        b0 = keep_pair(b0, k0, k1); b1 = keep_pair(b1, k8, k9);
-                        b2 = keep_pair(b2, k0, k1); b3 = keep_pair(b3, k8, k9);
-                    }
-                    mma_16816(o[j], pa, b0, b1);
-                    mma_16816(o[j + 1], pa, b2, b3);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[stage]);
-            }
-            l0 = quad_sum(l0);
-            l1 = quad_sum(l1);
-            // ---- merge the four warps' states (fixed order)
-            float* mo = mrg_o + warp * 16 * HD;
-            const int r0 = qr, r1 = qr + 8;
-            if ((lane & 3) == 0) {
-                mrg_m[warp * 16 + r0] = m0; mrg_l[warp * 16 + r0] = l0;
-                mrg_m[warp * 16 + r1] = m1; mrg_l[warp * 16 + r1] = l1;
-            }
+        if (!alive) break;
+        // ---- item output: final (single split) or a split partial for the merge kernel
+        l0 = quad_sum(l0);
+        l1 = quad_sum(l1);
+        const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+        const int h0 = cur.g * a.G + qr, h1 = h0 + 8;
+        const int item = it;
+        if (cur.nsplit == 1) {
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
                 const int c = j * 8 + qc;
-                if (r0 < a.G) { mo[r0 * HD + c] = o[j][0]; mo[r0 * HD + c + 1] = o[j][1]; }
-                if (r1 < a.G) { mo[r1 * HD + c] = o[j][2]; mo[r1 * HD + c + 1] = o[j][3]; }
+                if (qr < a.G)
+                    *reinterpret_cast<uint32_t*>(a.out + ((size_t)cur.r * a.nq + h0) * HD + c) =
+                        pack_bf16x2(o[j][0] * inv0, o[j][1] * inv0);
+                if (qr + 8 < a.G)
+                    *reinterpret_cast<uint32_t*>(a.out + ((size_t)cur.r * a.nq + h1) * HD + c) =
+                        pack_bf16x2(o[j][2] * inv1, o[j][3] * inv1);
             }
-            named_bar_sync(1, DEC_CONSUMERS * 32);
-            const int total = a.G * HD;
-            const bool single = d.nsplit == 1;
-            for (int e = threadIdx.x; e < total; e += DEC_CONSUMERS * 32) {
-                const int row = e / HD, col = e - row * HD;
-                float M = -INFINITY;
+        } else {
 #pragma unroll
-                for (int w = 0; w < DEC_CONSUMERS; ++w) M = fmaxf(M, mrg_m[w * 16 + row]);
-                float L = 0.f, acc = 0.f;
-#pragma unroll
-                for (int w = 0; w < DEC_CONSUMERS; ++w) {
-                    const float sc = exp2f(mrg_m[w * 16 + row] - M);
-                    L += sc * mrg_l[w * 16 + row];
-                    acc += sc * mrg_o[(w * 16 + row) * HD + col];
-                }
-                const float val = acc / L;
-                const int h = d.g * a.G + row;
-                if (single) {
-                    a.out[((size_t)d.r * a.nq + h) * HD + col] = f2bf(val);
-                } else {
-                    a.part_o[((size_t)it * a.G + row) * HD + col] = val;
-                    if (col == 0) a.part_lse[(size_t)it * a.G + row] = M + log2f(L);
-                }
+            for (int j = 0; j < NT; ++j) {
+                const int c = j * 8 + qc;
+                if (qr < a.G)
+                    *reinterpret_cast<float2*>(a.part_o + ((size_t)item * a.G + qr) * HD + c) =
+                        make_float2(o[j][0] * inv0, o[j][1] * inv0);
+                if (qr + 8 < a.G)
+                    *reinterpret_cast<float2*>(a.part_o + ((size_t)item * a.G + qr + 8) * HD + c) =
+                        make_float2(o[j][2] * inv1, o[j][3] * inv1);
             }
-            // every consumer thread leaves together if any warp gave up on a wait
-            if (named_bar_or(1, DEC_CONSUMERS * 32, !alive || *abort_flag)) break;
-            seq_base += (uint32_t)np;
+            if ((lane & 3) == 0) {
+                if (qr < a.G) a.part_lse[(size_t)item * a.G + qr] = m0 + log2f(l0);
+                if (qr + 8 < a.G) a.part_lse[(size_t)item * a.G + qr + 8] = m1 + log2f(l1);
+            }
         }
+        // ---- rotate: next item becomes current
+        it += DEC_WARPS;
+        cur = nxt;
+        pages_cur = pages_nxt;
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+            q_cur[kk][0] = q_nxt[kk][0]; q_cur[kk][1] = q_nxt[kk][1];
+            q_cur[kk][2] = q_nxt[kk][2]; q_cur[kk][3] = q_nxt[kk][3];
+        }
+        nxt = unpack_meta(tab_nn, a.split_pages);
+        pages_nxt = load_page_ids(a, nxt, lane);
+        tab_nn = it + 2 * DEC_WARPS < my_e ? __ldg(tab + it + 2 * DEC_WARPS) : none;
+        // the cursor was on the old next item (now current) or had issued all of it
+        if (iss_src == 1) {
+            iss_src = 0;
+        } else {
+            iss_src = nxt.np > 0 ? 1 : 2;
+            iss_k = 0;
+        }
+        NF_DEC_TOP_UP();
     }
+#undef NF_DEC_TOP_UP
+    if (!alive && lane == 0) {
+        // let this warp's copies still in flight land before the CTA exits
+        for (uint32_t sq = consumed; sq < issued; ++sq)
+            mbar_wait(&full[sq % NSTW], (sq / NSTW) & 1u, &quiet, nullptr);
+    }
+    __syncwarp();
     __syncthreads();
     if (threadIdx.x == 0 && a.trace != nullptr) {
         const int i = atomicAdd(a.trace_ctr, 1);
@@ -648,6 +653,21 @@ __global__ void decode_schedule_kernel(const int* ctx_len, int R, int nkv, int s
     if (threadIdx.x == 0) item_off[R] = carry;
 }
 
+// Work-item table: items of request r are item_off[r] + split * nkv + g.
+__global__ void decode_items_kernel(const int* ctx_len, const int* page_indptr, int R, int nkv, int split_pages,
+                                    const int* item_off, int4* tab) {
+    for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < R; r += gridDim.x * blockDim.x) {
+        const int nkeys = ctx_len[r] + 1;
+        const int npages = (nkeys + 15) >> 4;
+        const int nsplit = (npages + split_pages - 1) / split_pages;
+        const int base = item_off[r];
+        const int pbase = page_indptr[r];
+        for (int sp = 0; sp < nsplit; ++sp)
+            for (int g = 0; g < nkv; ++g)
+                tab[base + sp * nkv + g] = make_int4(r, g | (sp << 8) | (nsplit << 20), pbase + sp * split_pages, nkeys);
+    }
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -657,8 +677,7 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 int decode_smem_bytes(int hd) {
     const int stage = 2 * (hd / 64) * BOX_BYTES;
-    return DEC_STAGES * stage + DEC_CONSUMERS * 16 * hd * 4 + 2 * DEC_CONSUMERS * 16 * 4 + 2 * DEC_STAGES * 8 + 16 +
-           1024;
+    return DEC_WARPS * dec_wstages(hd) * (stage + 8) + 1024;
 }
 
 int prefill_smem_bytes(int hd) {
@@ -672,6 +691,15 @@ cudaError_t launch_decode_schedule(const int* ctx_len, int R, int nkv, int split
     return cudaGetLastError();
 }
 
+cudaError_t launch_decode_items(const int* ctx_len, const int* page_indptr, int R, int nkv, int split_pages,
+                                const int* item_off, void* item_tab, cudaStream_t stream) {
+    const int grid = (R + 255) / 256;
+    if (grid <= 0) return cudaSuccess;
+    decode_items_kernel<<<grid, 256, 0, stream>>>(ctx_len, page_indptr, R, nkv, split_pages, item_off,
+                                                 reinterpret_cast<int4*>(item_tab));
+    return cudaGetLastError();
+}
+
 cudaError_t launch_decode_attention(const CUtensorMap& tmKV, const DecodeArgs& a, int head_dim, int grid,
                                     int merge_grid, cudaStream_t stream) {
     if (grid <= 0 || a.req_end <= a.req_begin) return cudaSuccess;
@@ -682,7 +710,7 @@ cudaError_t launch_decode_attention(const CUtensorMap& tmKV, const DecodeArgs& a
         if (!cfg) { if ((e = set_smem(decode_attention_kernel<128>, smem)) != cudaSuccess) return e; cfg = true; }
         static bool cfg_m = false;
         if (!cfg_m) { if ((e = set_smem(decode_merge_kernel<128>, a.merge_smem_pad)) != cudaSuccess) return e; cfg_m = true; }
-        decode_attention_kernel<128><<<grid, DEC_THREADS, smem, stream>>>(tmKV, a);
+        decode_attention_kernel<128><<<grid, DEC_WARPS * 32, smem, stream>>>(tmKV, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         decode_merge_kernel<128><<<merge_grid, 256, a.merge_smem_pad, stream>>>(a);
     } else if (head_dim == 64) {
@@ -690,7 +718,7 @@ cudaError_t launch_decode_attention(const CUtensorMap& tmKV, const DecodeArgs& a
         if (!cfg) { if ((e = set_smem(decode_attention_kernel<64>, smem)) != cudaSuccess) return e; cfg = true; }
         static bool cfg_m = false;
         if (!cfg_m) { if ((e = set_smem(decode_merge_kernel<64>, a.merge_smem_pad)) != cudaSuccess) return e; cfg_m = true; }
-        decode_attention_kernel<64><<<grid, DEC_THREADS, smem, stream>>>(tmKV, a);
+        decode_attention_kernel<64><<<grid, DEC_WARPS * 32, smem, stream>>>(tmKV, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         decode_merge_kernel<64><<<merge_grid, 256, a.merge_smem_pad, stream>>>(a);
     } else {

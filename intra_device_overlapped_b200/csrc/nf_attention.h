@@ -21,6 +21,7 @@ struct DecodeArgs {
     const int* page_indptr;
     const int* page_indices;
     const int* item_off;  // [R + 1] first work item of each request
+    const void* item_tab; // [items] int4 work-item table (decode_items_kernel)
     int req_begin, req_end;
     int nq, nkv, G;
     int num_pages;
@@ -54,6 +55,8 @@ int prefill_smem_bytes(int head_dim);
 
 cudaError_t launch_decode_schedule(const int* ctx_len, int R, int nkv, int split_pages, int* item_off,
                                    cudaStream_t stream);
+cudaError_t launch_decode_items(const int* ctx_len, const int* page_indptr, int R, int nkv, int split_pages,
+                                const int* item_off, void* item_tab, cudaStream_t stream);
 cudaError_t launch_decode_attention(const CUtensorMap& tmKV, const DecodeArgs& a, int head_dim, int grid,
                                     int merge_grid, cudaStream_t stream);
 cudaError_t launch_prefill_attention(const CUtensorMap& tmKV, const PrefillArgs& a, int head_dim, int grid,

@@ -48,6 +48,7 @@ struct nf_model {
     int* item_off = nullptr;      // [max_requests + 1]
     float* part_o = nullptr;      // split-KV partials
     float* part_lse = nullptr;
+    void* item_tab = nullptr;     // [part_capacity] int4 decode work items
     int64_t part_capacity = 0;    // items
     // LM head
     uint16_t* lm_in = nullptr;    // [max_requests + 1 x H]

@@ -319,11 +319,9 @@ nf_status plan_impl(const nf_model* m, const nf_batch_desc* b, const nf_plan_opt
             p.num_tokens = R + C;
             p.sm_total = S;
             const std::vector<int> cut = split_requests(bi, std::max(dgroups, 1));
-            bool degenerate = false;
             for (int g = 0; g < dgroups; ++g) {
                 p.tok_begin[g] = cut[g];
                 p.tok_end[g] = cut[g + 1];
-                if (p.tok_end[g] <= p.tok_begin[g]) degenerate = true;
             }
             if (prefill_alone) {
                 p.tok_begin[n - 1] = R;
@@ -331,6 +329,9 @@ nf_status plan_impl(const nf_model* m, const nf_batch_desc* b, const nf_plan_opt
             } else {
                 p.tok_end[dgroups - 1] = R + C;
             }
+            bool degenerate = false;
+            for (int j = 0; j < n; ++j)
+                if (p.tok_end[j] <= p.tok_begin[j]) degenerate = true;
             if (degenerate) continue;
             for (int ord = 0; ord <= 1; ++ord) {
                 if (ord == 1 && !prefill_alone) continue;

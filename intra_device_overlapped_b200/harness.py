@@ -17,7 +17,7 @@ import synth
 from synth import weights as SW
 from synth.workloads import Workload, make_batch
 
-from . import (NF_OK, check, nf_batch_desc, nf_destroy_model, nf_forward_iteration, nf_global_weights,
+from . import (NF_OK, check, nf_calibrate, nf_get_cost_model, nf_batch_desc, nf_destroy_model, nf_forward_iteration, nf_global_weights,
                nf_init_model, nf_iter_io, nf_layer_weights, nf_model_config, nf_plan_iteration, nf_plan_opts,
                nf_set_global_weights, nf_set_layer_weights, nf_sync_status, nf_set_trace, nf_get_trace)
 
@@ -171,6 +171,14 @@ class DeviceWorkload:
     def forward(self, plan, stream: Optional[torch.cuda.Stream] = None, io: Optional[nf_iter_io] = None) -> None:
         s = stream.cuda_stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
         check(nf_forward_iteration(self.model, plan, io if io is not None else self.io, s), "nf_forward_iteration")
+
+    def calibrate(self, stream: Optional[torch.cuda.Stream] = None) -> dict:
+        """Time the model's kernels on this batch and install the fitted cost model for planning."""
+        s = stream.cuda_stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        check(nf_calibrate(self.model, self.desc, self.io, s), "nf_calibrate")
+        st, c = nf_get_cost_model(self.model)
+        check(st, "nf_get_cost_model")
+        return c.as_dict()
 
     def sync(self) -> int:
         return nf_sync_status(self.model)
