@@ -73,7 +73,7 @@ typedef struct {
     int32_t n_layers;
     int32_t hidden;       /* H, multiple of 256 */
     int32_t n_q_heads;    /* nq */
-    int32_t n_kv_heads;   /* nkv; nq % nkv == 0 and nq / nkv <= 16 */
+    int32_t n_kv_heads;   /* nkv; nq % nkv == 0 and nq / nkv <= 8 */
     int32_t head_dim;     /* d: 64 or 128 */
     int32_t ffn;          /* F (per expert for MoE), multiple of 128 */
     int32_t vocab;        /* 0: layer slice (hidden in/out); >0: embedding + final norm + LM head, multiple of 256 */

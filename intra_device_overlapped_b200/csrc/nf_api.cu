@@ -78,7 +78,7 @@ int gemm_grid(const GemmArgs& a, int grid) {
 bool valid_config(const nf_model_config& c) {
     if (c.n_layers < 1 || c.hidden <= 0 || c.hidden % 256 != 0) return false;
     if (c.n_q_heads <= 0 || c.n_kv_heads <= 0 || c.n_q_heads % c.n_kv_heads != 0) return false;
-    if (c.n_q_heads / c.n_kv_heads > 16) return false;
+    if (c.n_q_heads / c.n_kv_heads > 8) return false;  // decode attention packs a KV head's queries in 8 columns
     if (c.head_dim != 64 && c.head_dim != 128) return false;
     if (((c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim) % 256 != 0) return false;
     if ((c.n_q_heads * c.head_dim) % 64 != 0) return false;

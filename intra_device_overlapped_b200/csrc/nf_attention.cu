@@ -27,8 +27,8 @@
 namespace nf {
 namespace {
 
-constexpr int DEC_WARPS = 6;  // independent streaming warps per CTA
-__host__ __device__ constexpr int dec_wstages(int hd) { return hd == 128 ? 4 : 8; }  // 32 KB in flight per warp
+constexpr int DEC_WARPS = 8;  // independent streaming warps per CTA
+__host__ __device__ constexpr int dec_wstages(int hd) { return hd == 128 ? 3 : 6; }  // 24 KB in flight per warp
 constexpr int PRE_STAGES = 4;  // 128 KB for d = 128: one CTA per SM
 constexpr int PRE_THREADS = 5 * 32;
 constexpr int BOX_BYTES = 16 * 128;  // one 16-row x 64-col bf16 box
@@ -69,18 +69,18 @@ __device__ __forceinline__ DecMeta unpack_meta(int4 v, int split_pages) {
     return m;
 }
 
+// Q of the item's G heads as the B operand (k = d, n = 8 heads; heads >= G are zero):
+// b0 = Q[head lane/4][d = 16 kk + 2 (lane%4) + {0,1}], b1 = the same at d + 8.
 template <int KSTEPS>
-__device__ __forceinline__ void load_q_frags(const DecodeArgs& a, const DecMeta& m, int qr, int qc, int hd,
-                                             uint32_t (&qa)[KSTEPS][4]) {
-    const bool r0 = m.r >= 0 && qr < a.G, r1 = m.r >= 0 && qr + 8 < a.G;
-    const uint16_t* q0 = a.q + ((size_t)(m.r < 0 ? 0 : m.r) * a.nq + (size_t)m.g * a.G) * hd;
+__device__ __forceinline__ void load_q_frags(const DecodeArgs& a, const DecMeta& m, int lane, int hd,
+                                             uint32_t (&qb)[KSTEPS][2]) {
+    const int h = lane >> 2, c0 = (lane & 3) * 2;
+    const bool ok = m.r >= 0 && h < a.G;
+    const uint16_t* q0 = a.q + ((size_t)(m.r < 0 ? 0 : m.r) * a.nq + (size_t)m.g * a.G + (ok ? h : 0)) * hd;
 #pragma unroll
     for (int kk = 0; kk < KSTEPS; ++kk) {
-        const int c = kk * 16 + qc;
-        qa[kk][0] = r0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + (size_t)qr * hd + c)) : 0u;
-        qa[kk][1] = r1 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + (size_t)(qr + 8) * hd + c)) : 0u;
-        qa[kk][2] = r0 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + (size_t)qr * hd + c + 8)) : 0u;
-        qa[kk][3] = r1 ? __ldg(reinterpret_cast<const unsigned int*>(q0 + (size_t)(qr + 8) * hd + c + 8)) : 0u;
+        qb[kk][0] = ok ? __ldg(reinterpret_cast<const unsigned int*>(q0 + kk * 16 + c0)) : 0u;
+        qb[kk][1] = ok ? __ldg(reinterpret_cast<const unsigned int*>(q0 + kk * 16 + 8 + c0)) : 0u;
     }
 }
 
@@ -96,11 +96,31 @@ __device__ __forceinline__ int load_page_ids(const DecodeArgs& a, const DecMeta&
     return pg;
 }
 
+// max / sum over the 8 lanes that share lane % 4 (the 16 keys of a page, per head column)
+__device__ __forceinline__ float col_max(float x) {
+    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
+    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+    return x;
+}
+__device__ __forceinline__ float col_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    x += __shfl_xor_sync(0xffffffffu, x, 8);
+    x += __shfl_xor_sync(0xffffffffu, x, 16);
+    return x;
+}
+
 // Each warp is an independent streaming pipeline: it owns NSTW ring stages (one page of
 // one KV head, K and V, per stage), issues its own TMA loads (lane 0) and processes work
 // items my_b + w, my_b + w + DEC_WARPS, ... Its page stream runs across item boundaries;
 // the next item's table entry, page list and Q fragments are loaded while the current item
 // streams, so no global-load latency sits between pages or between items.
+//
+// Per page (16 keys) the warp computes S^T = K Q^T (m16n8k16: keys as rows, the G query
+// heads of the KV head as the 8 columns), an online softmax per head column, and
+// O^T += V^T P^T (d as rows). P^T is turned from accumulator layout into operand layout
+// with movmatrix. The running maximum is only moved when a page's maximum exceeds it by
+// more than 2^8 (exponents stay <= 256), which skips most accumulator rescales.
 template <int HD>
 __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     decode_attention_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ DecodeArgs a) {
@@ -109,7 +129,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     constexpr uint32_t STAGE_BYTES = 2 * KV_BYTES;
     constexpr int NSTW = dec_wstages(HD);
     constexpr int KSTEPS = HD / 16;
-    constexpr int NT = HD / 8;
+    constexpr int MT = HD / 16;  // m-tiles of O^T
+    constexpr float LAZY = 8.0f;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -134,7 +155,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     uint8_t* wsm = smem + warp * NSTW * STAGE_BYTES;
     uint64_t* full = full_all + warp * NSTW;
     const uint32_t wsm_u32 = smem_u32(wsm);
-    const int qr = lane >> 2, qc = (lane & 3) * 2;
+    const int kr = lane >> 2;            // key row of the S^T fragment (and +8)
+    const int hc = (lane & 3) * 2;       // head column pair of the S^T fragment
     const int4* tab = reinterpret_cast<const int4*>(a.item_tab);
     const int4 none = make_int4(-1, 0, 0, 0);
 
@@ -142,8 +164,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     DecMeta cur = unpack_meta(it < my_e ? __ldg(tab + it) : none, a.split_pages);
     DecMeta nxt = unpack_meta(it + DEC_WARPS < my_e ? __ldg(tab + it + DEC_WARPS) : none, a.split_pages);
     int4 tab_nn = it + 2 * DEC_WARPS < my_e ? __ldg(tab + it + 2 * DEC_WARPS) : none;
-    uint32_t q_cur[KSTEPS][4], q_nxt[KSTEPS][4];
-    load_q_frags<KSTEPS>(a, cur, qr, qc, HD, q_cur);
+    uint32_t q_cur[KSTEPS][2], q_nxt[KSTEPS][2];
+    load_q_frags<KSTEPS>(a, cur, lane, HD, q_cur);
     int pages_cur = load_page_ids(a, cur, lane);
     int pages_nxt = load_page_ids(a, nxt, lane);
 
@@ -178,14 +200,12 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
 
     NF_DEC_TOP_UP();
     while (cur.np > 0 && alive) {
-        // prefetch two items ahead: Q fragments of the next item (its table entry and page list
-        // are already in registers), table entry of the one after
-        load_q_frags<KSTEPS>(a, nxt, qr, qc, HD, q_nxt);
+        load_q_frags<KSTEPS>(a, nxt, lane, HD, q_nxt);  // prefetch for the next item
 
-        float o[NT][4];
+        float o[MT][4];
 #pragma unroll
-        for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;  // heads hc, hc + 1
 
         for (int p = 0; p < cur.np; ++p) {
             const int st = (int)(consumed % NSTW);
@@ -199,70 +219,64 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             const int key0 = (cur.split * a.split_pages + p) * 16;
             const int nvalid = min(16, cur.nkeys - key0);
 
-            float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int kk = 0; kk < KSTEPS; ++kk) {
-                const int mi = lane >> 3;
-                const int key = (mi >> 1) * 8 + (lane & 7);
-                const int dc = kk * 16 + (mi & 1) * 8;
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4(sK + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64), b0, b1, b2, b3);
-                mma_16816(s[0], q_cur[kk], b0, b1);
-                mma_16816(s[1], q_cur[kk], b2, b3);
-            }
-            float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const bool vis = (j * 8 + qc + e) < nvalid;
-                    s[j][e] = vis ? s[j][e] * a.scale_log2 : -INFINITY;
-                    s[j][2 + e] = vis ? s[j][2 + e] * a.scale_log2 : -INFINITY;
-                    mx0 = fmaxf(mx0, s[j][e]);
-                    mx1 = fmaxf(mx1, s[j][2 + e]);
-                }
-            }
-            mx0 = quad_max(mx0);
-            mx1 = quad_max(mx1);
-            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-            const float c0 = exp2f(m0 - mn0), c1 = exp2f(m1 - mn1);
-            m0 = mn0;
-            m1 = mn1;
-            float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    s[j][e] = exp2f(s[j][e] - mn0);
-                    s[j][2 + e] = exp2f(s[j][2 + e] - mn1);
-                    ps0 += s[j][e];
-                    ps1 += s[j][2 + e];
-                }
-            }
-            l0 = l0 * c0 + ps0;
-            l1 = l1 * c1 + ps1;
-#pragma unroll
-            for (int j = 0; j < NT; ++j) { o[j][0] *= c0; o[j][1] *= c0; o[j][2] *= c1; o[j][3] *= c1; }
-            uint32_t pa[4];
-            pa[0] = pack_bf16x2(s[0][0], s[0][1]);
-            pa[1] = pack_bf16x2(s[0][2], s[0][3]);
-            pa[2] = pack_bf16x2(s[1][0], s[1][1]);
-            pa[3] = pack_bf16x2(s[1][2], s[1][3]);
-            const int kb = (lane & 3) * 2;
-            const bool k0 = kb < nvalid, k1 = kb + 1 < nvalid, k8 = kb + 8 < nvalid, k9 = kb + 9 < nvalid;
-#pragma unroll
-            for (int j = 0; j < NT; j += 2) {
+            // S^T[16 keys x 8 heads] = K Q^T
+            float s[4] = {0.f, 0.f, 0.f, 0.f};
+            {
                 const int mi = lane >> 3;
                 const int key = (mi & 1) * 8 + (lane & 7);
-                const int dc = j * 8 + (mi >> 1) * 8;
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4_trans(sV + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64), b0, b1, b2, b3);
-                if (nvalid < 16) {  // V rows of keys past the request are zeroed
-                    b0 = keep_pair(b0, k0, k1); b1 = keep_pair(b1, k8, k9);
-                    b2 = keep_pair(b2, k0, k1); b3 = keep_pair(b3, k8, k9);
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk) {
+                    const int dc = kk * 16 + (mi >> 1) * 8;
+                    uint32_t ka[4];
+                    ldmatrix_x4(sK + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64), ka[0], ka[1], ka[2], ka[3]);
+                    mma_16816(s, ka, q_cur[kk][0], q_cur[kk][1]);
                 }
-                mma_16816(o[j], pa, b0, b1);
-                mma_16816(o[j + 1], pa, b2, b3);
+            }
+            const bool v0 = kr < nvalid, v8 = kr + 8 < nvalid;
+            s[0] = v0 ? s[0] * a.scale_log2 : -INFINITY;   // key kr, head hc
+            s[1] = v0 ? s[1] * a.scale_log2 : -INFINITY;   // key kr, head hc + 1
+            s[2] = v8 ? s[2] * a.scale_log2 : -INFINITY;   // key kr + 8, head hc
+            s[3] = v8 ? s[3] * a.scale_log2 : -INFINITY;   // key kr + 8, head hc + 1
+            const float xA = col_max(fmaxf(s[0], s[2]));
+            const float xB = col_max(fmaxf(s[1], s[3]));
+            if (__any_sync(0xffffffffu, xA > mA + LAZY || xB > mB + LAZY)) {
+                const float nA = fmaxf(mA, xA), nB = fmaxf(mB, xB);
+                const float cA = exp2f(mA - nA), cB = exp2f(mB - nB);
+                mA = nA;
+                mB = nB;
+                lA *= cA;
+                lB *= cB;
+#pragma unroll
+                for (int i = 0; i < MT; ++i) { o[i][0] *= cA; o[i][1] *= cB; o[i][2] *= cA; o[i][3] *= cB; }
+            }
+            s[0] = exp2f(s[0] - mA);
+            s[1] = exp2f(s[1] - mB);
+            s[2] = exp2f(s[2] - mA);
+            s[3] = exp2f(s[3] - mB);
+            lA += s[0] + s[2];
+            lB += s[1] + s[3];
+            // P^T as the B operand (k = keys, n = heads)
+            const uint32_t pb0 = movmatrix_trans(pack_bf16x2(s[0], s[1]));
+            const uint32_t pb1 = movmatrix_trans(pack_bf16x2(s[2], s[3]));
+
+            // O^T[d x 8 heads] += V^T P^T; V rows of keys past the request are zeroed
+            const int kb = (lane & 3) * 2;
+            const bool k0 = kb < nvalid, k1 = kb + 1 < nvalid, k8 = kb + 8 < nvalid, k9 = kb + 9 < nvalid;
+            {
+                const int mi = lane >> 3;
+                const int key = (mi >> 1) * 8 + (lane & 7);
+#pragma unroll
+                for (int i = 0; i < MT; ++i) {
+                    const int dc = i * 16 + (mi & 1) * 8;
+                    uint32_t va[4];
+                    ldmatrix_x4_trans(sV + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64), va[0], va[1], va[2],
+                                      va[3]);
+                    if (nvalid < 16) {
+                        va[0] = keep_pair(va[0], k0, k1); va[1] = keep_pair(va[1], k0, k1);
+                        va[2] = keep_pair(va[2], k8, k9); va[3] = keep_pair(va[3], k8, k9);
+                    }
+                    mma_16816(o[i], va, pb0, pb1);
+                }
             }
             __syncwarp();
             ++consumed;
@@ -270,36 +284,30 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
         }
         if (!alive) break;
         // ---- item output: final (single split) or a split partial for the merge kernel
-        l0 = quad_sum(l0);
-        l1 = quad_sum(l1);
-        const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-        const int h0 = cur.g * a.G + qr, h1 = h0 + 8;
-        const int item = it;
+        lA = col_sum(lA);
+        lB = col_sum(lB);
+        const float iA = 1.f / lA, iB = 1.f / lB;
+        const bool okA = hc < a.G, okB = hc + 1 < a.G;
+        const size_t hA = (size_t)cur.g * a.G + hc;
         if (cur.nsplit == 1) {
+            uint16_t* ob = a.out + (size_t)cur.r * a.nq * HD;
 #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                const int c = j * 8 + qc;
-                if (qr < a.G)
-                    *reinterpret_cast<uint32_t*>(a.out + ((size_t)cur.r * a.nq + h0) * HD + c) =
-                        pack_bf16x2(o[j][0] * inv0, o[j][1] * inv0);
-                if (qr + 8 < a.G)
-                    *reinterpret_cast<uint32_t*>(a.out + ((size_t)cur.r * a.nq + h1) * HD + c) =
-                        pack_bf16x2(o[j][2] * inv1, o[j][3] * inv1);
+            for (int i = 0; i < MT; ++i) {
+                const int d0 = i * 16 + kr;
+                if (okA) { ob[hA * HD + d0] = f2bf(o[i][0] * iA); ob[hA * HD + d0 + 8] = f2bf(o[i][2] * iA); }
+                if (okB) { ob[(hA + 1) * HD + d0] = f2bf(o[i][1] * iB); ob[(hA + 1) * HD + d0 + 8] = f2bf(o[i][3] * iB); }
             }
         } else {
+            float* po = a.part_o + (size_t)it * a.G * HD;
 #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                const int c = j * 8 + qc;
-                if (qr < a.G)
-                    *reinterpret_cast<float2*>(a.part_o + ((size_t)item * a.G + qr) * HD + c) =
-                        make_float2(o[j][0] * inv0, o[j][1] * inv0);
-                if (qr + 8 < a.G)
-                    *reinterpret_cast<float2*>(a.part_o + ((size_t)item * a.G + qr + 8) * HD + c) =
-                        make_float2(o[j][2] * inv1, o[j][3] * inv1);
+            for (int i = 0; i < MT; ++i) {
+                const int d0 = i * 16 + kr;
+                if (okA) { po[(size_t)hc * HD + d0] = o[i][0] * iA; po[(size_t)hc * HD + d0 + 8] = o[i][2] * iA; }
+                if (okB) { po[(size_t)(hc + 1) * HD + d0] = o[i][1] * iB; po[(size_t)(hc + 1) * HD + d0 + 8] = o[i][3] * iB; }
             }
-            if ((lane & 3) == 0) {
-                if (qr < a.G) a.part_lse[(size_t)item * a.G + qr] = m0 + log2f(l0);
-                if (qr + 8 < a.G) a.part_lse[(size_t)item * a.G + qr + 8] = m1 + log2f(l1);
+            if (kr == 0) {
+                if (okA) a.part_lse[(size_t)it * a.G + hc] = mA + log2f(lA);
+                if (okB) a.part_lse[(size_t)it * a.G + hc + 1] = mB + log2f(lB);
             }
         }
         // ---- rotate: next item becomes current
@@ -307,10 +315,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
         cur = nxt;
         pages_cur = pages_nxt;
 #pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk) {
-            q_cur[kk][0] = q_nxt[kk][0]; q_cur[kk][1] = q_nxt[kk][1];
-            q_cur[kk][2] = q_nxt[kk][2]; q_cur[kk][3] = q_nxt[kk][3];
-        }
+        for (int kk = 0; kk < KSTEPS; ++kk) { q_cur[kk][0] = q_nxt[kk][0]; q_cur[kk][1] = q_nxt[kk][1]; }
         nxt = unpack_meta(tab_nn, a.split_pages);
         pages_nxt = load_page_ids(a, nxt, lane);
         tab_nn = it + 2 * DEC_WARPS < my_e ? __ldg(tab + it + 2 * DEC_WARPS) : none;
