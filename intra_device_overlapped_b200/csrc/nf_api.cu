@@ -177,6 +177,7 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) {
     ok &= (m->rope_cos = dalloc<float>(m, (size_t)cfg->max_position * d.d / 2)) != nullptr;
     ok &= (m->rope_sin = dalloc<float>(m, (size_t)cfg->max_position * d.d / 2)) != nullptr;
     ok &= (m->item_off = dalloc<int>(m, (size_t)cfg->max_requests + 1)) != nullptr;
+    ok &= (m->merge_cnt = dalloc<int>(m, ((size_t)cfg->max_requests + 1) * d.nkv)) != nullptr;
     ok &= (m->status = dalloc<int>(m, 1)) != nullptr;
     m->trace_cap = 65536;
     ok &= (m->trace_ctr = dalloc<int>(m, 1)) != nullptr;
@@ -355,7 +356,7 @@ nf::DecodeArgs decode_args(const nf_model* m, const nf_iter_io* io, const void* 
     a.num_pages = io->num_pages;
     a.split_pages = nf::kDecodeSplitPages;
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m->dims.d));
-    a.merge_smem_pad = 100 * 1024;
+    a.merge_cnt = m->merge_cnt;
     a.status = m->status;
     if (m->trace_on) { a.trace_ctr = m->trace_ctr; a.trace = m->trace; a.trace_cap = m->trace_cap; }
     return a;
@@ -439,7 +440,7 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
             if (re > rb) {
                 nf::DecodeArgs da = decode_args(m, io, m->q, m->attn_o, rb, re);
                 NF_CUDA_TRY(tm.begin(s));
-                NF_CUDA_TRY(nf::launch_decode_attention(m->kv_tm[l], da, d.d, grid, grid, s));
+                NF_CUDA_TRY(nf::launch_decode_attention(m->kv_tm[l], da, d.d, grid, s));
                 NF_CUDA_TRY(tm.end(s, NF_OP_DECODE_ATTN, j, l, op.stream, grid));
             }
             if (t1 > R && C > 0) {
@@ -594,7 +595,7 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     if (R > 0) {
         NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, sg));
         NF_CUDA_TRY(nf::launch_decode_items(io->ctx_len, io->page_indptr, R, d.nkv, nf::kDecodeSplitPages,
-                                            m->item_off, m->item_tab, sg));
+                                            m->item_off, m->item_tab, m->merge_cnt, sg));
     }
     if (m->cfg.vocab > 0) {
         NF_CUDA_TRY(nf::launch_embed(io->token_ids, m->embed, T, d.H, m->cfg.vocab, m->resid, m->xb, m->partials,
@@ -762,10 +763,10 @@ extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* ou
     NF_CUDA_TRY(cudaStreamSynchronize(s));
     if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
     NF_CUDA_TRY(nf::launch_decode_items(io->ctx_len, io->page_indptr, req_end, m->dims.nkv, nf::kDecodeSplitPages,
-                                        m->item_off, m->item_tab, s));
+                                        m->item_off, m->item_tab, m->merge_cnt, s));
     const int grid = sm_count > 0 ? std::min(sm_count, m->sm_count) : m->sm_count;
     nf::DecodeArgs da = decode_args(m, io, q, out, req_begin, req_end);
-    NF_CUDA_TRY(nf::launch_decode_attention(m->kv_tm[layer], da, m->dims.d, grid, grid, s));
+    NF_CUDA_TRY(nf::launch_decode_attention(m->kv_tm[layer], da, m->dims.d, grid, s));
     return NF_OK;
 }
 
@@ -876,11 +877,11 @@ extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_
         if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
         NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, sg));
         NF_CUDA_TRY(nf::launch_decode_items(io->ctx_len, io->page_indptr, R, d.nkv, nf::kDecodeSplitPages,
-                                            m->item_off, m->item_tab, sg));
+                                            m->item_off, m->item_tab, m->merge_cnt, sg));
         NF_CUDA_TRY(cudaMemsetAsync(m->q, 0, (size_t)R * d.nq * d.d * 2, sg));
         auto dec = [&](int grid, cudaStream_t s) -> nf_status {
             nf::DecodeArgs da = decode_args(m, io, m->q, m->attn_o, 0, R);
-            return nf::launch_decode_attention(m->kv_tm[0], da, d.d, grid, grid, s) == cudaSuccess ? NF_OK
+            return nf::launch_decode_attention(m->kv_tm[0], da, d.d, grid, s) == cudaSuccess ? NF_OK
                                                                                                   : NF_ERR_CUDA;
         };
         const int small = std::max(4, S / 8);

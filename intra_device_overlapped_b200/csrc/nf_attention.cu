@@ -219,8 +219,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             const int key0 = (cur.split * a.split_pages + p) * 16;
             const int nvalid = min(16, cur.nkeys - key0);
 
-            // S^T[16 keys x 8 heads] = K Q^T
-            float s[4] = {0.f, 0.f, 0.f, 0.f};
+            // S^T[16 keys x 8 heads] = K Q^T, even and odd k-steps in two independent chains
+            float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
             {
                 const int mi = lane >> 3;
                 const int key = (mi & 1) * 8 + (lane & 7);
@@ -229,17 +229,18 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
                     const int dc = kk * 16 + (mi >> 1) * 8;
                     uint32_t ka[4];
                     ldmatrix_x4(sK + (dc / 64) * BOX_BYTES + sw128_offset(key, dc % 64), ka[0], ka[1], ka[2], ka[3]);
-                    mma_16816(s, ka, q_cur[kk][0], q_cur[kk][1]);
+                    mma_16816((kk & 1) ? s2 : s, ka, q_cur[kk][0], q_cur[kk][1]);
                 }
             }
             const bool v0 = kr < nvalid, v8 = kr + 8 < nvalid;
-            s[0] = v0 ? s[0] * a.scale_log2 : -INFINITY;   // key kr, head hc
-            s[1] = v0 ? s[1] * a.scale_log2 : -INFINITY;   // key kr, head hc + 1
-            s[2] = v8 ? s[2] * a.scale_log2 : -INFINITY;   // key kr + 8, head hc
-            s[3] = v8 ? s[3] * a.scale_log2 : -INFINITY;   // key kr + 8, head hc + 1
-            const float xA = col_max(fmaxf(s[0], s[2]));
-            const float xB = col_max(fmaxf(s[1], s[3]));
-            if (__any_sync(0xffffffffu, xA > mA + LAZY || xB > mB + LAZY)) {
+            s[0] = v0 ? (s[0] + s2[0]) * a.scale_log2 : -INFINITY;   // key kr, head hc
+            s[1] = v0 ? (s[1] + s2[1]) * a.scale_log2 : -INFINITY;   // key kr, head hc + 1
+            s[2] = v8 ? (s[2] + s2[2]) * a.scale_log2 : -INFINITY;   // key kr + 8, head hc
+            s[3] = v8 ? (s[3] + s2[3]) * a.scale_log2 : -INFINITY;   // key kr + 8, head hc + 1
+            // the running maximum moves only if some score exceeds it by more than LAZY
+            const float tA = fmaxf(s[0], s[2]), tB = fmaxf(s[1], s[3]);
+            if (__any_sync(0xffffffffu, tA > mA + LAZY || tB > mB + LAZY)) {
+                const float xA = col_max(tA), xB = col_max(tB);
                 const float nA = fmaxf(mA, xA), nB = fmaxf(mB, xB);
                 const float cA = exp2f(mA - nA), cB = exp2f(mB - nB);
                 mA = nA;
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             }
             __syncwarp();
             ++consumed;
-            NF_DEC_TOP_UP();
+            NF_DEC_TOP_UP();  // refills the stage just released (at most one page)
         }
         if (!alive) break;
         // ---- item output: final (single split) or a split partial for the merge kernel
@@ -308,6 +309,33 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             if (kr == 0) {
                 if (okA) a.part_lse[(size_t)it * a.G + hc] = mA + log2f(lA);
                 if (okB) a.part_lse[(size_t)it * a.G + hc + 1] = mB + log2f(lB);
+            }
+            // The warp that writes the last split of (r, g) merges all splits in split order.
+            // Each launch adds exactly nsplit arrivals per (r, g), so counters need no reset
+            // between the layers of an iteration.
+            __threadfence();
+            __syncwarp();
+            int last = 0;
+            if (lane == 0)
+                last = (atomicAdd(a.merge_cnt + (size_t)cur.r * a.nkv + cur.g, 1) + 1) % cur.nsplit == 0;
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) {
+                __threadfence();
+                const int base = it - cur.split * a.nkv;  // item of split 0
+                for (int e = lane; e < a.G * HD; e += 32) {
+                    const int row = e / HD, col = e - row * HD;
+                    float M = -INFINITY;
+                    for (int sp = 0; sp < cur.nsplit; ++sp)
+                        M = fmaxf(M, __ldcg(a.part_lse + (size_t)(base + sp * a.nkv) * a.G + row));
+                    float L = 0.f, acc = 0.f;
+                    for (int sp = 0; sp < cur.nsplit; ++sp) {
+                        const size_t itm = (size_t)(base + sp * a.nkv);
+                        const float w = exp2f(__ldcg(a.part_lse + itm * a.G + row) - M);
+                        L += w;
+                        acc += w * __ldcg(a.part_o + (itm * a.G + row) * HD + col);
+                    }
+                    a.out[((size_t)cur.r * a.nq + (size_t)cur.g * a.G + row) * HD + col] = f2bf(acc / L);
+                }
             }
         }
         // ---- rotate: next item becomes current
@@ -344,42 +372,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             a.trace[i].t_start = t_start;
             a.trace[i].t_end = globaltimer_ns();
         }
-    }
-}
-
-// Split-KV merge: out[r][h] = sum_s 2^(lse_s - LSE) o_s, fixed split order. One warp per (r, h).
-template <int HD>
-__global__ void decode_merge_kernel(const __grid_constant__ DecodeArgs a) {
-    const int warps = (gridDim.x * blockDim.x) >> 5;
-    const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    const int nreq = a.req_end - a.req_begin;
-    for (int w = wid; w < nreq * a.nq; w += warps) {
-        const int r = a.req_begin + w / a.nq;
-        const int h = w % a.nq;
-        const int g = h / a.G, row = h - g * a.G;
-        const int nkeys = a.ctx_len[r] + 1;
-        const int npages = (nkeys + 15) >> 4;
-        const int nsplit = (npages + a.split_pages - 1) / a.split_pages;
-        if (nsplit <= 1) continue;
-        const int base = a.item_off[r];
-        float M = -INFINITY;
-        for (int s = 0; s < nsplit; ++s) M = fmaxf(M, a.part_lse[(size_t)(base + s * a.nkv + g) * a.G + row]);
-        float L = 0.f;
-        float acc[HD / 32];
-#pragma unroll
-        for (int c = 0; c < HD / 32; ++c) acc[c] = 0.f;
-        for (int s = 0; s < nsplit; ++s) {
-            const int item = base + s * a.nkv + g;
-            const float wgt = exp2f(a.part_lse[(size_t)item * a.G + row] - M);
-            L += wgt;
-            const float* po = a.part_o + ((size_t)item * a.G + row) * HD;
-#pragma unroll
-            for (int c = 0; c < HD / 32; ++c) acc[c] += wgt * po[c * 32 + lane];
-        }
-        uint16_t* dst = a.out + ((size_t)r * a.nq + h) * HD;
-#pragma unroll
-        for (int c = 0; c < HD / 32; ++c) dst[c * 32 + lane] = f2bf(acc[c] / L);
     }
 }
 
@@ -660,7 +652,7 @@ __global__ void decode_schedule_kernel(const int* ctx_len, int R, int nkv, int s
 
 // Work-item table: items of request r are item_off[r] + split * nkv + g.
 __global__ void decode_items_kernel(const int* ctx_len, const int* page_indptr, int R, int nkv, int split_pages,
-                                    const int* item_off, int4* tab) {
+                                    const int* item_off, int4* tab, int* merge_cnt) {
     for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < R; r += gridDim.x * blockDim.x) {
         const int nkeys = ctx_len[r] + 1;
         const int npages = (nkeys + 15) >> 4;
@@ -670,6 +662,7 @@ __global__ void decode_items_kernel(const int* ctx_len, const int* page_indptr, 
         for (int sp = 0; sp < nsplit; ++sp)
             for (int g = 0; g < nkv; ++g)
                 tab[base + sp * nkv + g] = make_int4(r, g | (sp << 8) | (nsplit << 20), pbase + sp * split_pages, nkeys);
+        for (int g = 0; g < nkv; ++g) merge_cnt[(size_t)r * nkv + g] = 0;
     }
 }
 
@@ -697,35 +690,27 @@ cudaError_t launch_decode_schedule(const int* ctx_len, int R, int nkv, int split
 }
 
 cudaError_t launch_decode_items(const int* ctx_len, const int* page_indptr, int R, int nkv, int split_pages,
-                                const int* item_off, void* item_tab, cudaStream_t stream) {
+                                const int* item_off, void* item_tab, int* merge_cnt, cudaStream_t stream) {
     const int grid = (R + 255) / 256;
     if (grid <= 0) return cudaSuccess;
     decode_items_kernel<<<grid, 256, 0, stream>>>(ctx_len, page_indptr, R, nkv, split_pages, item_off,
-                                                 reinterpret_cast<int4*>(item_tab));
+                                                 reinterpret_cast<int4*>(item_tab), merge_cnt);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode_attention(const CUtensorMap& tmKV, const DecodeArgs& a, int head_dim, int grid,
-                                    int merge_grid, cudaStream_t stream) {
+                                    cudaStream_t stream) {
     if (grid <= 0 || a.req_end <= a.req_begin) return cudaSuccess;
     const int smem = decode_smem_bytes(head_dim);
     cudaError_t e;
     if (head_dim == 128) {
         static bool cfg = false;
         if (!cfg) { if ((e = set_smem(decode_attention_kernel<128>, smem)) != cudaSuccess) return e; cfg = true; }
-        static bool cfg_m = false;
-        if (!cfg_m) { if ((e = set_smem(decode_merge_kernel<128>, a.merge_smem_pad)) != cudaSuccess) return e; cfg_m = true; }
         decode_attention_kernel<128><<<grid, DEC_WARPS * 32, smem, stream>>>(tmKV, a);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        decode_merge_kernel<128><<<merge_grid, 256, a.merge_smem_pad, stream>>>(a);
     } else if (head_dim == 64) {
         static bool cfg = false;
         if (!cfg) { if ((e = set_smem(decode_attention_kernel<64>, smem)) != cudaSuccess) return e; cfg = true; }
-        static bool cfg_m = false;
-        if (!cfg_m) { if ((e = set_smem(decode_merge_kernel<64>, a.merge_smem_pad)) != cudaSuccess) return e; cfg_m = true; }
         decode_attention_kernel<64><<<grid, DEC_WARPS * 32, smem, stream>>>(tmKV, a);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        decode_merge_kernel<64><<<merge_grid, 256, a.merge_smem_pad, stream>>>(a);
     } else {
         return cudaErrorInvalidValue;
     }

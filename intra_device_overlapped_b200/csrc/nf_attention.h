@@ -27,7 +27,7 @@ struct DecodeArgs {
     int num_pages;
     int split_pages;
     float scale_log2;     // log2(e) / sqrt(d)
-    int merge_smem_pad;   // dynamic shared memory requested by the merge kernel (SM exclusivity)
+    int* merge_cnt;       // [R x nkv] split arrival counters (zeroed by decode_items_kernel)
     int* status;
     int* trace_ctr;
     nf_trace_entry* trace;
@@ -56,9 +56,9 @@ int prefill_smem_bytes(int head_dim);
 cudaError_t launch_decode_schedule(const int* ctx_len, int R, int nkv, int split_pages, int* item_off,
                                    cudaStream_t stream);
 cudaError_t launch_decode_items(const int* ctx_len, const int* page_indptr, int R, int nkv, int split_pages,
-                                const int* item_off, void* item_tab, cudaStream_t stream);
+                                const int* item_off, void* item_tab, int* merge_cnt, cudaStream_t stream);
 cudaError_t launch_decode_attention(const CUtensorMap& tmKV, const DecodeArgs& a, int head_dim, int grid,
-                                    int merge_grid, cudaStream_t stream);
+                                    cudaStream_t stream);
 cudaError_t launch_prefill_attention(const CUtensorMap& tmKV, const PrefillArgs& a, int head_dim, int grid,
                                      cudaStream_t stream);
 

@@ -46,6 +46,7 @@ struct nf_model {
     float* rope_cos = nullptr;    // [max_position x d/2]
     float* rope_sin = nullptr;
     int* item_off = nullptr;      // [max_requests + 1]
+    int* merge_cnt = nullptr;     // [max_requests x nkv] split-KV arrival counters
     float* part_o = nullptr;      // split-KV partials
     float* part_lse = nullptr;
     void* item_tab = nullptr;     // [part_capacity] int4 decode work items
