@@ -150,15 +150,17 @@ typedef struct {
 } nf_plan_opts;
 
 enum {
-    NF_TEMPLATE_SEQUENTIAL = 0, /* one nano-batch after another, each op on all SMs (no overlap) */
-    NF_TEMPLATE_PIPELINED = 1,  /* attention of nano-batch j co-runs with the GEMMs of the others */
+    NF_TEMPLATE_SEQUENTIAL = 0,       /* one nano-batch after another, each op on all SMs (no overlap) */
+    NF_TEMPLATE_PIPELINED = 1,        /* attention of nano-batch j co-runs with the GEMMs of the others */
+    NF_TEMPLATE_PREFILL_ON_GEMM = 2,  /* as PIPELINED, but the compute-bound prefill attention runs on the
+                                         GEMM stream and SMs; only decode attention co-runs */
 };
 
 typedef struct {
     int32_t n_nano;
     int32_t tok_begin[NF_MAX_NANO]; /* nano-batch j = tokens [tok_begin[j], tok_end[j]) */
     int32_t tok_end[NF_MAX_NANO];
-    int32_t nano_order[NF_MAX_NANO]; /* pipeline order of the nano-batches */
+    int32_t nano_order[NF_MAX_NANO]; /* pipeline order of the nano-batches (O / FFN phase) */
     int32_t order_template;       /* NF_TEMPLATE_* */
     int32_t sm_attn;              /* SMs claimed by attention kernels while overlapped */
     int32_t sm_gemm;              /* SMs claimed by GEMM kernels while overlapped */

@@ -25,6 +25,7 @@ NF_ERR_DEVICE_BOUNDS = 6
 NF_MAX_NANO = 4
 NF_TEMPLATE_SEQUENTIAL = 0
 NF_TEMPLATE_PIPELINED = 1
+NF_TEMPLATE_PREFILL_ON_GEMM = 2
 NF_KERNEL_GEMM, NF_KERNEL_DECODE_ATTN, NF_KERNEL_PREFILL_ATTN = 1, 2, 3
 
 _i32, _i64, _u64, _f32, _vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_float, ctypes.c_void_p
@@ -68,7 +69,7 @@ class nf_plan(ctypes.Structure):
         n = self.n_nano
         return {"n_nano": n, "tokens": [(self.tok_begin[j], self.tok_end[j]) for j in range(n)],
                 "order": [self.nano_order[i] for i in range(n)],
-                "template": ["sequential", "pipelined"][self.order_template],
+                "template": ["sequential", "pipelined", "prefill_on_gemm"][self.order_template],
                 "sm_attn": self.sm_attn, "sm_gemm": self.sm_gemm, "sm_total": self.sm_total,
                 "predicted_us": round(self.predicted_us, 1), "predicted_serial_us": round(self.predicted_serial_us, 1)}
 

@@ -434,20 +434,18 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
             NF_CUDA_TRY(nf::launch_gemm(nf::EPI_QKV, m->tm_xb, W.tm_qkv, a, gemm_grid(a, grid), s));
             return NF_OK;
         }
-        case nf::OP_ATT: {
+        case nf::OP_DATT: {
             const int rb = std::min(t0, R), re = std::min(t1, R);
-            OpTimer tm{m};
             if (re > rb) {
                 nf::DecodeArgs da = decode_args(m, io, m->q, m->attn_o, rb, re);
-                NF_CUDA_TRY(tm.begin(s));
                 NF_CUDA_TRY(nf::launch_decode_attention(m->kv_tm[l], da, d.d, grid, s));
-                NF_CUDA_TRY(tm.end(s, NF_OP_DECODE_ATTN, j, l, op.stream, grid));
             }
+            return NF_OK;
+        }
+        case nf::OP_PATT: {
             if (t1 > R && C > 0) {
                 nf::PrefillArgs pa = prefill_args(m, io, m->q, m->attn_o, R, C);
-                NF_CUDA_TRY(tm.begin(s));
                 NF_CUDA_TRY(nf::launch_prefill_attention(m->kv_tm[l], pa, d.d, grid, s));
-                NF_CUDA_TRY(tm.end(s, NF_OP_PREFILL_ATTN, j, l, op.stream, grid));
             }
             return NF_OK;
         }
@@ -555,7 +553,7 @@ nf_status validate_forward(const nf_model* m, const nf_plan* p, const nf_iter_io
     }
     const int S = m->sm_count;
     if (p->sm_total < 1 || p->sm_total > S) return NF_ERR_INVALID_ARGUMENT;
-    if (p->order_template == NF_TEMPLATE_PIPELINED) {
+    if (p->order_template == NF_TEMPLATE_PIPELINED || p->order_template == NF_TEMPLATE_PREFILL_ON_GEMM) {
         if (p->sm_attn < 1 || p->sm_gemm < 1 || p->sm_attn + p->sm_gemm > p->sm_total) return NF_ERR_INVALID_ARGUMENT;
     } else if (p->order_template != NF_TEMPLATE_SEQUENTIAL) {
         return NF_ERR_INVALID_ARGUMENT;
@@ -586,7 +584,6 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
         if ((st = ensure_kv_tmap(m, l, io)) != NF_OK) return st;
 
     const int S = p->sm_total;
-    const bool pipelined = p->order_template == NF_TEMPLATE_PIPELINED;
     NF_CUDA_TRY(cudaEventRecord(m->ev_fork, sg));
     NF_CUDA_TRY(cudaStreamWaitEvent(sa, m->ev_fork, 0));
     if (m->trace_on) NF_CUDA_TRY(cudaMemsetAsync(m->trace_ctr, 0, sizeof(int), sg));
@@ -607,27 +604,27 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
 
     int order[NF_MAX_NANO];
     for (int i = 0; i < p->n_nano; ++i) order[i] = p->nano_order[i];
-    const std::vector<nf::Op> ops = nf::build_ops(p->order_template, p->n_nano, order, d.L, d.E > 0);
+    bool has_dec[NF_MAX_NANO], has_pre[NF_MAX_NANO];
+    nf::nano_content(*p, has_dec, has_pre);
+    const std::vector<nf::Op> ops =
+        nf::build_ops(p->order_template, p->n_nano, order, d.L, d.E > 0, has_dec, has_pre);
     while (m->events.size() < ops.size()) {
         cudaEvent_t e;
         NF_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
         m->events.push_back(e);
     }
     // timing entries accumulate over forwards until nf_set_timing is called again
+    static const int kTimingKind[] = {NF_OP_QKV, NF_OP_DECODE_ATTN, NF_OP_O, NF_OP_GATE_UP, NF_OP_DOWN, NF_OP_MOE,
+                                      NF_OP_PREFILL_ATTN};
     for (size_t i = 0; i < ops.size(); ++i) {
         const nf::Op& op = ops[i];
         cudaStream_t s = op.stream == nf::STREAM_ATTN ? sa : sg;
         if (op.wait >= 0) NF_CUDA_TRY(cudaStreamWaitEvent(s, m->events[op.wait], 0));
-        int grid = S;
-        if (pipelined) {
-            if (op.stream == nf::STREAM_ATTN) grid = p->sm_attn;
-            else if (!op.full_sm) grid = p->sm_gemm;
-        }
+        const int grid = nf::op_grid(*p, op);
         OpTimer tm{m};
-        const bool self_timed = op.kind == nf::OP_ATT;  // decode / prefill timed separately inside
-        if (!self_timed) NF_CUDA_TRY(tm.begin(s));
+        NF_CUDA_TRY(tm.begin(s));
         if ((st = run_op(m, p, io, op, grid, s)) != NF_OK) return st;
-        if (!self_timed) NF_CUDA_TRY(tm.end(s, op.kind, op.nano, op.layer, op.stream, grid));
+        NF_CUDA_TRY(tm.end(s, kTimingKind[op.kind], op.nano, op.layer, op.stream, grid));
         if (op.signal) NF_CUDA_TRY(cudaEventRecord(m->events[i], s));
     }
     NF_CUDA_TRY(cudaEventRecord(m->ev_join, sa));

@@ -20,70 +20,97 @@
 
 namespace nf {
 
-std::vector<Op> build_ops(int tmpl, int n, const int* order, int L, bool moe) {
+void nano_content(const nf_plan& p, bool* has_dec, bool* has_pre) {
+    for (int j = 0; j < p.n_nano; ++j) {
+        has_dec[j] = p.tok_begin[j] < p.num_decode;
+        has_pre[j] = p.tok_end[j] > p.num_decode && p.prefill_len > 0;
+    }
+}
+
+std::vector<Op> build_ops(int tmpl, int n, const int* order, int L, bool moe, const bool* has_dec,
+                          const bool* has_pre) {
     std::vector<Op> ops;
     auto push = [&](int kind, int stream, int j, int l) {
         Op o{kind, stream, j, l, 0, -1, 0};
         ops.push_back(o);
         return (int)ops.size() - 1;
     };
+    auto push_ffn = [&](int j, int l) {
+        if (moe) {
+            push(OP_MOE, STREAM_GEMM, j, l);
+        } else {
+            push(OP_GU, STREAM_GEMM, j, l);
+            push(OP_D, STREAM_GEMM, j, l);
+        }
+    };
     if (tmpl == NF_TEMPLATE_SEQUENTIAL) {
         for (int l = 0; l < L; ++l)
             for (int i = 0; i < n; ++i) {
                 const int j = order[i];
                 push(OP_QKV, STREAM_GEMM, j, l);
-                push(OP_ATT, STREAM_GEMM, j, l);
+                if (has_dec[j]) push(OP_DATT, STREAM_GEMM, j, l);
+                if (has_pre[j]) push(OP_PATT, STREAM_GEMM, j, l);
                 push(OP_O, STREAM_GEMM, j, l);
-                if (moe) {
-                    push(OP_MOE, STREAM_GEMM, j, l);
-                } else {
-                    push(OP_GU, STREAM_GEMM, j, l);
-                    push(OP_D, STREAM_GEMM, j, l);
-                }
+                push_ffn(j, l);
             }
         for (auto& o : ops) o.full_sm = 1;
         return ops;
     }
-    // Pipelined: attention of (j, l) on the attention stream right after QKV(j, l);
-    // O(j, l) waits for it; QKV(j, l+1) follows the FFN of (j, l) on the GEMM stream.
-    std::vector<int> qkv_idx((size_t)n * L, -1), att_idx((size_t)n * L, -1);
+    // Pipelined: decode attention of (j, l) on the attention stream right after QKV(j, l);
+    // prefill attention on the attention stream too, or (NF_TEMPLATE_PREFILL_ON_GEMM) on the
+    // GEMM stream right before O(j, l). O(j, l) waits for the attention-stream ops of (j, l);
+    // QKV(j, l+1) follows the FFN of (j, l) on the GEMM stream.
+    const bool pre_on_gemm = tmpl == NF_TEMPLATE_PREFILL_ON_GEMM;
+    std::vector<int> last_a((size_t)n * L, -1);
     auto issue_qkv = [&](int j, int l) {
         const int q = push(OP_QKV, STREAM_GEMM, j, l);
-        qkv_idx[(size_t)l * n + j] = q;
-        const int a = push(OP_ATT, STREAM_ATTN, j, l);
-        ops[a].wait = q;
-        ops[q].signal = 1;
-        att_idx[(size_t)l * n + j] = a;
+        int prev = q;
+        if (has_dec[j]) {
+            const int a = push(OP_DATT, STREAM_ATTN, j, l);
+            ops[a].wait = q;
+            ops[q].signal = 1;
+            prev = a;
+            last_a[(size_t)l * n + j] = a;
+        }
+        if (has_pre[j] && !pre_on_gemm) {
+            const int a = push(OP_PATT, STREAM_ATTN, j, l);
+            if (prev == q) { ops[a].wait = q; ops[q].signal = 1; }
+            last_a[(size_t)l * n + j] = a;
+        }
     };
-    for (int i = 0; i < n; ++i) issue_qkv(order[i], 0);
+    // first layer: nano-batches with attention-stream work get their QKV first
+    for (int pass = 0; pass < 2; ++pass)
+        for (int i = 0; i < n; ++i) {
+            const int j = order[i];
+            const bool a_work = has_dec[j] || (has_pre[j] && !pre_on_gemm);
+            if ((pass == 0) == a_work) issue_qkv(j, 0);
+        }
     for (int l = 0; l < L; ++l) {
         for (int i = 0; i < n; ++i) {
             const int j = order[i];
+            if (has_pre[j] && pre_on_gemm) push(OP_PATT, STREAM_GEMM, j, l);
             const int o = push(OP_O, STREAM_GEMM, j, l);
-            ops[o].wait = att_idx[(size_t)l * n + j];
-            ops[att_idx[(size_t)l * n + j]].signal = 1;
-            if (moe) {
-                push(OP_MOE, STREAM_GEMM, j, l);
-            } else {
-                push(OP_GU, STREAM_GEMM, j, l);
-                push(OP_D, STREAM_GEMM, j, l);
-            }
+            const int a = last_a[(size_t)l * n + j];
+            if (a >= 0) { ops[o].wait = a; ops[a].signal = 1; }
+            push_ffn(j, l);
             if (l + 1 < L) issue_qkv(j, l + 1);
         }
     }
-    // A GEMM-stream op may take every SM iff it lies in no attention window: ATT(j, l)
-    // can only run between the end of QKV(j, l) and the start of O(j, l).
+    // A GEMM-stream op may take every SM iff it lies in no attention window: an
+    // attention-stream op can only run between the end of its QKV and the start of its O.
     std::vector<int> gpos(ops.size(), -1);
     int g = 0;
     for (size_t i = 0; i < ops.size(); ++i)
         if (ops[i].stream == STREAM_GEMM) gpos[i] = g++;
     std::vector<int> covered(g + 1, 0);
     for (size_t i = 0; i < ops.size(); ++i) {
-        if (ops[i].kind != OP_ATT) continue;
-        const int q = ops[i].wait;
+        if (ops[i].stream != STREAM_ATTN) continue;
+        int q = -1;  // QKV of the same (j, l)
+        for (int k = (int)i - 1; k >= 0; --k)
+            if (ops[k].kind == OP_QKV && ops[k].nano == ops[i].nano && ops[k].layer == ops[i].layer) { q = k; break; }
         int o = -1;
         for (size_t k = i + 1; k < ops.size(); ++k)
-            if (ops[k].wait == (int)i) { o = (int)k; break; }
+            if (ops[k].kind == OP_O && ops[k].nano == ops[i].nano && ops[k].layer == ops[i].layer) { o = (int)k; break; }
         const int lo = gpos[q] + 1, hi = (o >= 0 ? gpos[o] : g);  // G ops in [lo, hi) may overlap
         for (int x = lo; x < hi; ++x) covered[x] = 1;
     }
@@ -123,6 +150,12 @@ double gemm_us(const CostModel& c, int M, int N, int K, int grid, int64_t weight
 
 }  // namespace
 
+int op_grid(const nf_plan& p, const Op& o) {
+    if (p.order_template == NF_TEMPLATE_SEQUENTIAL) return p.sm_total;
+    if (o.stream == STREAM_ATTN) return p.sm_attn;
+    return o.full_sm ? p.sm_total : p.sm_gemm;
+}
+
 double op_time_us(int kind, int j, const nf_plan& p, const ModelDims& m, const BatchInfo& b, const CostModel& c,
                   int grid) {
     const int t0 = p.tok_begin[j], t1 = p.tok_end[j];
@@ -142,19 +175,17 @@ double op_time_us(int kind, int j, const nf_plan& p, const ModelDims& m, const B
             t += gemm_us(c, per, m.H, m.F, std::max(1, grid / std::max(1, m.E)), (int64_t)m.H * m.F * 2);
             return t + 20.0;
         }
-        case OP_ATT: {
+        case OP_DATT: {
             const int r0 = std::min(t0, b.R), r1 = std::min(t1, b.R);
             const int64_t bytes = b.req_kv_prefix[r1] - b.req_kv_prefix[r0];
-            double t = 0;
-            if (bytes > 0) {
-                const double bw = std::min(c.hbm_bw, grid * c.attn_bw_per_sm);
-                t += c.attn_launch_us + (double)bytes / bw * 1e6 + 3.0;
-            }
-            if (t1 > b.R && b.C > 0) {
-                const double flops = 4.0 * m.nq * m.d * (double)b.C * (b.C + 1) / 2.0;
-                t += c.attn_launch_us + flops / (grid * c.attn_flops_per_sm) * 1e6;
-            }
-            return t;
+            if (bytes <= 0) return 0.0;
+            const double bw = std::min(c.hbm_bw, grid * c.attn_bw_per_sm);
+            return c.attn_launch_us + (double)bytes / bw * 1e6;
+        }
+        case OP_PATT: {
+            if (!(t1 > b.R && b.C > 0)) return 0.0;
+            const double flops = 4.0 * m.nq * m.d * (double)b.C * (b.C + 1) / 2.0;
+            return c.attn_launch_us + flops / (grid * c.attn_flops_per_sm) * 1e6;
         }
     }
     return 0.0;
@@ -164,16 +195,16 @@ double simulate_plan(const nf_plan& p, const ModelDims& m, const BatchInfo& b, c
                      double* serial_us) {
     int order[NF_MAX_NANO];
     for (int i = 0; i < p.n_nano; ++i) order[i] = p.nano_order[i];
-    const std::vector<Op> ops = build_ops(p.order_template, p.n_nano, order, m.L, m.E > 0);
+    bool has_dec[NF_MAX_NANO], has_pre[NF_MAX_NANO];
+    nano_content(p, has_dec, has_pre);
+    const std::vector<Op> ops = build_ops(p.order_template, p.n_nano, order, m.L, m.E > 0, has_dec, has_pre);
     const int S = p.sm_total;
+    const bool pipelined = p.order_template != NF_TEMPLATE_SEQUENTIAL;
     std::vector<double> dur(ops.size()), beg(ops.size()), end(ops.size());
     double serial = 0.0;
     for (size_t i = 0; i < ops.size(); ++i) {
         const Op& o = ops[i];
-        int grid = S;
-        if (p.order_template == NF_TEMPLATE_PIPELINED && !o.full_sm)
-            grid = (o.stream == STREAM_ATTN) ? p.sm_attn : p.sm_gemm;
-        if (p.order_template == NF_TEMPLATE_PIPELINED && o.kind == OP_ATT) grid = p.sm_attn;
+        const int grid = op_grid(p, o);
         dur[i] = op_time_us(o.kind, o.nano, p, m, b, c, grid);
         serial += op_time_us(o.kind, o.nano, p, m, b, c, S);
     }
@@ -190,7 +221,7 @@ double simulate_plan(const nf_plan& p, const ModelDims& m, const BatchInfo& b, c
             free_t[o.stream] = end[i];
         }
         makespan = std::max(free_t[0], free_t[1]);
-        if (pass == 0 && p.order_template == NF_TEMPLATE_PIPELINED) {
+        if (pass == 0 && pipelined) {
             // inflate each op by the interference factor times the fraction of it that overlaps the other stream
             std::vector<std::pair<double, double>> other[2];
             for (size_t i = 0; i < ops.size(); ++i) other[ops[i].stream].push_back({beg[i], end[i]});
@@ -333,16 +364,20 @@ nf_status plan_impl(const nf_model* m, const nf_batch_desc* b, const nf_plan_opt
             for (int j = 0; j < n; ++j)
                 if (p.tok_end[j] <= p.tok_begin[j]) degenerate = true;
             if (degenerate) continue;
-            for (int ord = 0; ord <= 1; ++ord) {
-                if (ord == 1 && !prefill_alone) continue;
-                for (int i = 0; i < n; ++i) p.nano_order[i] = ord == 0 ? i : (i == 0 ? n - 1 : i - 1);
-                for (int tmpl = 0; tmpl <= 1; ++tmpl) {
+            int perm[NF_MAX_NANO];
+            for (int i = 0; i < n; ++i) perm[i] = i;
+            do {
+                for (int i = 0; i < n; ++i) p.nano_order[i] = perm[i];
+                for (int tmpl = 0; tmpl <= 2; ++tmpl) {
                     if (o.force_template >= 0 && tmpl != o.force_template) continue;
-                    if (tmpl == NF_TEMPLATE_PIPELINED && n < 2) continue;
+                    if (tmpl != NF_TEMPLATE_SEQUENTIAL && n < 2) continue;
+                    if (tmpl == NF_TEMPLATE_PREFILL_ON_GEMM && C == 0) continue;
+                    if (tmpl == NF_TEMPLATE_SEQUENTIAL && perm[0] != 0) continue;  // order is irrelevant
                     p.order_template = tmpl;
                     int a_lo = 8, a_hi = S - 8, a_step = 4;
                     if (tmpl == NF_TEMPLATE_SEQUENTIAL) { a_lo = a_hi = 0; }
-                    if (o.force_sm_attn > 0 && tmpl == NF_TEMPLATE_PIPELINED) a_lo = a_hi = std::min(o.force_sm_attn, S - 4);
+                    if (o.force_sm_attn > 0 && tmpl != NF_TEMPLATE_SEQUENTIAL)
+                        a_lo = a_hi = std::min(o.force_sm_attn, S - 4);
                     for (int sa = a_lo; sa <= a_hi; sa += a_step) {
                         p.sm_attn = tmpl == NF_TEMPLATE_SEQUENTIAL ? S : sa;
                         p.sm_gemm = tmpl == NF_TEMPLATE_SEQUENTIAL ? S : S - sa;
@@ -356,7 +391,7 @@ nf_status plan_impl(const nf_model* m, const nf_batch_desc* b, const nf_plan_opt
                         }
                     }
                 }
-            }
+            } while (std::next_permutation(perm, perm + n));
         }
     }
     if (best.n_nano == 0) return NF_ERR_INVALID_ARGUMENT;

@@ -8,7 +8,7 @@
 
 namespace nf {
 
-enum OpKind : int { OP_QKV = 0, OP_ATT = 1, OP_O = 2, OP_GU = 3, OP_D = 4, OP_MOE = 5 };
+enum OpKind : int { OP_QKV = 0, OP_DATT = 1, OP_O = 2, OP_GU = 3, OP_D = 4, OP_MOE = 5, OP_PATT = 6 };
 enum StreamId : int { STREAM_GEMM = 0, STREAM_ATTN = 1 };
 
 struct Op {
@@ -22,8 +22,13 @@ struct Op {
 };
 
 // Issue order of every operation of the iteration (excluding the prologue and the LM head).
-// `order` lists the nano-batches in pipeline order.
-std::vector<Op> build_ops(int tmpl, int n_nano, const int* order, int n_layers, bool moe);
+// `order` lists the nano-batches in pipeline order; has_dec[j] / has_pre[j] say whether
+// nano-batch j holds decode rows / the prefill chunk.
+std::vector<Op> build_ops(int tmpl, int n_nano, const int* order, int n_layers, bool moe, const bool* has_dec,
+                          const bool* has_pre);
+
+// has_dec / has_pre of every nano-batch of a plan
+void nano_content(const nf_plan& p, bool* has_dec, bool* has_pre);
 
 // Per-kernel cost model used by the planner (microseconds, bytes, FLOPs).
 struct CostModel {
@@ -53,6 +58,8 @@ struct BatchInfo {
 // Simulated makespan (us) of a plan; also returns the no-overlap time.
 double simulate_plan(const nf_plan& p, const ModelDims& m, const BatchInfo& b, const CostModel& c,
                      double* serial_us);
+
+int op_grid(const nf_plan& p, const Op& o);
 
 double op_time_us(int kind, int nano, const nf_plan& p, const ModelDims& m, const BatchInfo& b, const CostModel& c,
                   int grid);
