@@ -228,6 +228,7 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) {
          nf::make_tmap_bf16_2d(&m->tm_attn_o, m->attn_o, T, (uint64_t)d.nq * d.d, nf::kGemmBM) &&
          nf::make_tmap_bf16_2d(&m->tm_act, m->act, act_rows, d.F, nf::kGemmBM);
     if (ok && cfg->vocab > 0) ok = nf::make_tmap_bf16_2d(&m->tm_lm_in, m->lm_in, lm_rows, d.H, nf::kGemmBM);
+    if (ok && d.d == 128) ok = nf::make_tmap_bf16_2d(&m->tm_q, m->q, T * d.nq, d.d, 16);
     if (ok && d.E > 0) ok = nf::make_tmap_bf16_2d(&m->tm_moe_a, m->moe_a, TK, d.H, nf::kGemmBM);
     if (!ok) { nf_destroy_model(m); return NF_ERR_CUDA; }
     *out = m;
@@ -403,6 +404,26 @@ struct OpTimer {
     }
 };
 
+// Work-item tables of the decode attention for requests [0, R): tensor-core kernel (d = 128)
+// streams whole requests in 128-key chunks; the warp-level kernel (d = 64) uses split items.
+cudaError_t decode_prologue(nf_model* m, const nf_iter_io* io, int R, cudaStream_t s) {
+    if (R <= 0) return cudaSuccess;
+    const nf::ModelDims& d = m->dims;
+    if (d.d == 128)
+        return nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeTcChunkPages, m->item_off, s);
+    cudaError_t e = nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, s);
+    if (e != cudaSuccess) return e;
+    return nf::launch_decode_items(io->ctx_len, io->page_indptr, R, d.nkv, nf::kDecodeSplitPages, m->item_off,
+                                   m->item_tab, m->merge_cnt, s);
+}
+
+cudaError_t launch_decode(nf_model* m, const nf_iter_io* io, const CUtensorMap& tmq, const void* q, void* out,
+                          int layer, int rb, int re, int grid, cudaStream_t s) {
+    nf::DecodeArgs da = decode_args(m, io, q, out, rb, re);
+    if (m->dims.d == 128) return nf::launch_decode_attention_tc(m->kv_tm[layer], tmq, da, grid, s);
+    return nf::launch_decode_attention(m->kv_tm[layer], da, m->dims.d, grid, s);
+}
+
 nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::Op& op, int grid,
                  cudaStream_t s) {
     const nf::ModelDims& d = m->dims;
@@ -436,10 +457,7 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
         }
         case nf::OP_DATT: {
             const int rb = std::min(t0, R), re = std::min(t1, R);
-            if (re > rb) {
-                nf::DecodeArgs da = decode_args(m, io, m->q, m->attn_o, rb, re);
-                NF_CUDA_TRY(nf::launch_decode_attention(m->kv_tm[l], da, d.d, grid, s));
-            }
+            if (re > rb) NF_CUDA_TRY(launch_decode(m, io, m->tm_q, m->q, m->attn_o, l, rb, re, grid, s));
             return NF_OK;
         }
         case nf::OP_PATT: {
@@ -589,11 +607,7 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     if (m->trace_on) NF_CUDA_TRY(cudaMemsetAsync(m->trace_ctr, 0, sizeof(int), sg));
 
     // prologue: decode work items, residual stream set-up
-    if (R > 0) {
-        NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, sg));
-        NF_CUDA_TRY(nf::launch_decode_items(io->ctx_len, io->page_indptr, R, d.nkv, nf::kDecodeSplitPages,
-                                            m->item_off, m->item_tab, m->merge_cnt, sg));
-    }
+    NF_CUDA_TRY(decode_prologue(m, io, R, sg));
     if (m->cfg.vocab > 0) {
         NF_CUDA_TRY(nf::launch_embed(io->token_ids, m->embed, T, d.H, m->cfg.vocab, m->resid, m->xb, m->partials,
                                      m->status, S * 4, sg));
@@ -754,16 +768,21 @@ extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* ou
     cudaStream_t s = (cudaStream_t)stream;
     nf_status st = ensure_kv_tmap(m, layer, io);
     if (st != NF_OK) return st;
-    NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, req_end, m->dims.nkv, nf::kDecodeSplitPages, m->item_off, s));
-    int items = 0;
-    NF_CUDA_TRY(cudaMemcpyAsync(&items, m->item_off + req_end, sizeof(int), cudaMemcpyDeviceToHost, s));
-    NF_CUDA_TRY(cudaStreamSynchronize(s));
-    if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
-    NF_CUDA_TRY(nf::launch_decode_items(io->ctx_len, io->page_indptr, req_end, m->dims.nkv, nf::kDecodeSplitPages,
-                                        m->item_off, m->item_tab, m->merge_cnt, s));
+    if (m->dims.d != 128) {
+        NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, req_end, m->dims.nkv, nf::kDecodeSplitPages, m->item_off,
+                                               s));
+        int items = 0;
+        NF_CUDA_TRY(cudaMemcpyAsync(&items, m->item_off + req_end, sizeof(int), cudaMemcpyDeviceToHost, s));
+        NF_CUDA_TRY(cudaStreamSynchronize(s));
+        if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
+    }
+    NF_CUDA_TRY(decode_prologue(m, io, req_end, s));
+    CUtensorMap tmq;
+    if (m->dims.d == 128 &&
+        !nf::make_tmap_bf16_2d(&tmq, q, (uint64_t)req_end * m->dims.nq, m->dims.d, 16))
+        return NF_ERR_INVALID_ARGUMENT;
     const int grid = sm_count > 0 ? std::min(sm_count, m->sm_count) : m->sm_count;
-    nf::DecodeArgs da = decode_args(m, io, q, out, req_begin, req_end);
-    NF_CUDA_TRY(nf::launch_decode_attention(m->kv_tm[layer], da, m->dims.d, grid, s));
+    NF_CUDA_TRY(launch_decode(m, io, tmq, q, out, layer, req_begin, req_end, grid, s));
     return NF_OK;
 }
 
@@ -872,14 +891,11 @@ extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_
             items += (int64_t)d.nkv * ((np + nf::kDecodeSplitPages - 1) / nf::kDecodeSplitPages);
         }
         if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
-        NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, sg));
-        NF_CUDA_TRY(nf::launch_decode_items(io->ctx_len, io->page_indptr, R, d.nkv, nf::kDecodeSplitPages,
-                                            m->item_off, m->item_tab, m->merge_cnt, sg));
+        NF_CUDA_TRY(decode_prologue(m, io, R, sg));
         NF_CUDA_TRY(cudaMemsetAsync(m->q, 0, (size_t)R * d.nq * d.d * 2, sg));
         auto dec = [&](int grid, cudaStream_t s) -> nf_status {
-            nf::DecodeArgs da = decode_args(m, io, m->q, m->attn_o, 0, R);
-            return nf::launch_decode_attention(m->kv_tm[0], da, d.d, grid, s) == cudaSuccess ? NF_OK
-                                                                                                  : NF_ERR_CUDA;
+            return launch_decode(m, io, m->tm_q, m->q, m->attn_o, 0, 0, R, grid, s) == cudaSuccess ? NF_OK
+                                                                                                   : NF_ERR_CUDA;
         };
         const int small = std::max(4, S / 8);
         double t_small = 0, t_all = 0;

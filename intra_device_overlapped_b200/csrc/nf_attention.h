@@ -62,6 +62,13 @@ cudaError_t launch_decode_attention(const CUtensorMap& tmKV, const DecodeArgs& a
 cudaError_t launch_prefill_attention(const CUtensorMap& tmKV, const PrefillArgs& a, int head_dim, int grid,
                                      cudaStream_t stream);
 
+// Tensor-core (tcgen05) decode attention for head dim 128; a.item_off holds, per request,
+// the prefix of nkv * ceil((ctx_len + 1) / 128) (decode_schedule with split_pages = 8).
+constexpr int kDecodeTcChunkPages = 8;
+int decode_tc_smem_bytes();
+cudaError_t launch_decode_attention_tc(const CUtensorMap& tmKV, const CUtensorMap& tmQ, const DecodeArgs& a,
+                                       int grid, cudaStream_t stream);
+
 // KV pool as a 2-D tensor [num_pages * 2 * nkv * 16 rows x d cols], 16 x 64 boxes, 128-byte swizzle.
 bool make_kv_tmap(CUtensorMap* map, const void* pool, int num_pages, int nkv, int head_dim);
 

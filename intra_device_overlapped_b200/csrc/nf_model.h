@@ -67,6 +67,7 @@ struct nf_model {
     float* moe_part = nullptr;    // [T K x H/256]
     float* moe_y = nullptr;       // [T K x H]
     CUtensorMap tm_xb, tm_attn_o, tm_act, tm_lm_in, tm_moe_a;
+    CUtensorMap tm_q;             // q as [T * nq rows x d], 16-row boxes (decode attention Q loads)
 
     int* status = nullptr;        // device status word
     int* trace_ctr = nullptr;
