@@ -420,6 +420,7 @@ cudaError_t decode_prologue(nf_model* m, const nf_iter_io* io, int R, cudaStream
 cudaError_t launch_decode(nf_model* m, const nf_iter_io* io, const CUtensorMap& tmq, const void* q, void* out,
                           int layer, int rb, int re, int grid, cudaStream_t s) {
     nf::DecodeArgs da = decode_args(m, io, q, out, rb, re);
+    da.kv_pool = (const uint16_t*)io->kv_pools[layer];
     if (m->dims.d == 128) return nf::launch_decode_attention_tc(m->kv_tm[layer], tmq, da, grid, s);
     return nf::launch_decode_attention(m->kv_tm[layer], da, m->dims.d, grid, s);
 }

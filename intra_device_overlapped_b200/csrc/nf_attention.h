@@ -22,6 +22,7 @@ struct DecodeArgs {
     const int* page_indices;
     const int* item_off;  // [R + 1] first work item of each request
     const void* item_tab; // [items] int4 work-item table (decode_items_kernel)
+    const uint16_t* kv_pool;  // layer's pool (L2 prefetch addresses)
     int req_begin, req_end;
     int nq, nkv, G;
     int num_pages;
