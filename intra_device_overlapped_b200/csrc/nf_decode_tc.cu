@@ -33,9 +33,9 @@ constexpr uint32_t REGION = 16384;          // 128 rows x 128 B
 constexpr uint32_t KV_STAGE = 4 * REGION;   // K halves, then V halves
 constexpr uint32_t QP_BYTES = 4096;         // 16 rows x 256 B as two 2 KB regions
 constexpr int MAX_ITEM_PAGES = 1024;        // page list of one request held in shared memory
-constexpr int PREFETCH_CHUNKS = 4;          // L2 bulk prefetch runs this many chunks ahead of the TMA loads
 constexpr uint32_t TMEM_COLS = 64;
-constexpr int THREADS = 192;                // warp 0 TMA, warp 1 MMA + TMEM, warps 2..5 softmax
+constexpr int LOADERS = 4;                  // warps 6..9: K/V page loads (cp.async)
+constexpr int THREADS = (6 + LOADERS) * 32; // warp 0 Q loads (TMA), warp 1 MMA + TMEM, warps 2..5 softmax
 constexpr uint32_t IDESC_S = umma_idesc_bf16_f32(128, 16);
 constexpr uint32_t IDESC_PV = umma_idesc_bf16_f32_amn(128, 16);
 constexpr float LAZY = 8.0f;
@@ -43,7 +43,7 @@ constexpr float LAZY = 8.0f;
 constexpr uint32_t OFF_Q = NS * KV_STAGE;
 constexpr uint32_t OFF_P = OFF_Q + 2 * QP_BYTES;
 constexpr uint32_t OFF_PAGES = OFF_P + 2 * QP_BYTES;
-constexpr uint32_t OFF_RED = OFF_PAGES + 2 * MAX_ITEM_PAGES * 4;
+constexpr uint32_t OFF_RED = OFF_PAGES + MAX_ITEM_PAGES * 4;
 constexpr uint32_t OFF_BAR = OFF_RED + 4 * 16 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 24 * 8 + 16 + 1024;
 
@@ -98,7 +98,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                                const __grid_constant__ DecodeArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    int* pages_sm = reinterpret_cast<int*>(smem + OFF_PAGES);
     float* red = reinterpret_cast<float*>(smem + OFF_RED);  // [4 warps][16]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint64_t* kv_full = bars;            // [NS]
@@ -118,7 +117,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t t_start = 0;
     if (threadIdx.x == 0) {
         t_start = globaltimer_ns();
-        for (int i = 0; i < NS; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+        for (int i = 0; i < NS; ++i) { mbar_init(&kv_full[i], LOADERS * 32); mbar_init(&kv_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1);
             mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 4);
@@ -147,98 +146,73 @@ __global__ void __launch_bounds__(THREADS, 1)
     const long long hi = W0 + W * (blockIdx.x + 1) / gridDim.x;
 
     if (warp == 0) {
-        // ---------------- TMA producer. Two cursors walk the CTA's chunk sequence: the
-        // prefetch cursor (page lists staged in shared memory, K and V page blocks prefetched
-        // into L2) runs PREFETCH_CHUNKS ahead of the TMA cursor (loads into the ring), and at
-        // most one item ahead, so item k's page list sits in buffer k & 1 for both.
-        ItemIter tit, pit;
-        iter_init(tit, a, lo, hi);
-        pit = tit;
-        uint32_t cs = 0, tni = 0, tc = 0;     // TMA cursor: chunk seq, item seq, chunk in item
-        uint32_t pcs = 0, pni = 0, pc = 0;    // prefetch cursor
-        bool ok = true;
-        const size_t blk = (size_t)16 * 128;  // elements of one page block of one KV head
-        auto stage_list = [&](const ItemIter& x, uint32_t seq) {
-            int* buf = pages_sm + (seq & 1u) * MAX_ITEM_PAGES;
-            const int npages = (x.nkeys + 15) >> 4;
-            const int base = a.page_indptr[x.r];
-            for (int j = lane; j < npages && j < MAX_ITEM_PAGES; j += 32) {
-                int pg = a.page_indices[base + j];
-                if (pg < 0 || pg >= a.num_pages) { set_status(a.status, NF_ERR_DEVICE_BOUNDS); pg = 0; }
-                buf[j] = pg;
-            }
-            __syncwarp();
-        };
-        if (pit.valid) stage_list(pit, 0);
-        while (tit.valid && ok) {
-            // ---- prefetch cursor: keep PREFETCH_CHUNKS chunks ahead
-            while (pit.valid && pcs < cs + PREFETCH_CHUNKS) {
-                if (pc == (uint32_t)pit.nch) {          // this item is prefetched: move to the next one
-                    if (pni > tni) break;               // never two items ahead of the TMA cursor
-                    iter_next(pit, a, hi);
-                    ++pni;
-                    pc = 0;
-                    if (!pit.valid) break;
-                    stage_list(pit, pni);
-                    continue;
-                }
-                const int* buf = pages_sm + (pni & 1u) * MAX_ITEM_PAGES;
-                const int npages = (pit.nkeys + 15) >> 4;
-                const int j0 = 8 * (int)pc, np = min(8, npages - j0);
-                if (lane < 2 * np) {
-                    const int pg = buf[min(j0 + (lane >> 1), MAX_ITEM_PAGES - 1)];
-                    const uint16_t* src = a.kv_pool + (((size_t)pg * 2 + (lane & 1)) * a.nkv + pit.g) * blk;
-                    prefetch_l2_bulk(src, (uint32_t)(blk * 2));
-                }
-                ++pcs;
-                ++pc;
-            }
-            // ---- TMA cursor: one chunk into the ring
-            if (tc == 0) {
-                const uint32_t qb = tni & 1u;
-                if (!wait_bcast(&q_empty[qb], ((tni >> 1) & 1u) ^ 1u, abort_flag, a.status, lane)) { ok = false; break; }
-                if (lane == 0) {
-                    uint8_t* qd = smem + OFF_Q + qb * QP_BYTES;
-                    mbar_arrive_expect_tx(&q_full[qb], QP_BYTES);
-                    const int y = tit.r * a.nq + tit.g * a.G;
-                    tma_load_2d(qd, &tmQ, &q_full[qb], 0, y);
-                    tma_load_2d(qd + 2048, &tmQ, &q_full[qb], 64, y);
-                }
-            }
-            const int st = (int)(cs % NS);
-            if (!wait_bcast(&kv_empty[st], ((cs / NS) & 1u) ^ 1u, abort_flag, a.status, lane)) { ok = false; break; }
+        // ---------------- Q loads: the 16 query rows starting at head g * G of request r (TMA)
+        ItemIter it;
+        iter_init(it, a, lo, hi);
+        uint32_t ni = 0;
+        for (; it.valid; iter_next(it, a, hi), ++ni) {
+            const uint32_t qb = ni & 1u;
+            if (!wait_bcast(&q_empty[qb], ((ni >> 1) & 1u) ^ 1u, abort_flag, a.status, lane)) break;
             if (lane == 0) {
-                const int* buf = pages_sm + (tni & 1u) * MAX_ITEM_PAGES;
-                const int npages = (tit.nkeys + 15) >> 4;
-                const int np = min(8, npages - 8 * (int)tc);
-                uint8_t* kd = smem + st * KV_STAGE;
-                uint8_t* vd = kd + 2 * REGION;
-                mbar_arrive_expect_tx(&kv_full[st], (uint32_t)np * 4u * 2048u);
-                for (int j = 0; j < np; ++j) {
-                    const int pg = buf[min(8 * (int)tc + j, MAX_ITEM_PAGES - 1)];
-                    const int yk = ((pg * 2 + 0) * a.nkv + tit.g) * 16;
-                    const int yv = ((pg * 2 + 1) * a.nkv + tit.g) * 16;
-                    tma_load_2d(kd + j * 2048, &tmKV, &kv_full[st], 0, yk);
-                    tma_load_2d(kd + REGION + j * 2048, &tmKV, &kv_full[st], 64, yk);
-                    tma_load_2d(vd + j * 2048, &tmKV, &kv_full[st], 0, yv);
-                    tma_load_2d(vd + REGION + j * 2048, &tmKV, &kv_full[st], 64, yv);
-                }
-            }
-            __syncwarp();
-            ++cs;
-            if (++tc == (uint32_t)tit.nch) {
-                tc = 0;
-                iter_next(tit, a, hi);
-                ++tni;  // the prefetch cursor is on this item or the next: its page list is staged
+                uint8_t* qd = smem + OFF_Q + qb * QP_BYTES;
+                mbar_arrive_expect_tx(&q_full[qb], QP_BYTES);
+                const int y = it.r * a.nq + it.g * a.G;
+                tma_load_2d(qd, &tmQ, &q_full[qb], 0, y);
+                tma_load_2d(qd + 2048, &tmQ, &q_full[qb], 64, y);
             }
         }
-        if (!ok && lane == 0) {
-            // let the copies still in flight land before the CTA exits
+        if (lane == 0) {  // the last Q copy must land before the CTA exits
             volatile int quiet = 0;
-            for (uint32_t x = cs > (uint32_t)NS ? cs - NS : 0u; x < cs; ++x)
-                mbar_wait(&kv_full[x % NS], (x / NS) & 1u, &quiet, nullptr);
-            mbar_wait(&q_full[tni & 1u], (tni >> 1) & 1u, &quiet, nullptr);
+            if (ni > 0) mbar_wait(&q_full[(ni - 1) & 1u], ((ni - 1) >> 1) & 1u, &quiet, nullptr);
         }
+        __syncwarp();
+    } else if (warp >= 6) {
+        // ---------------- K/V loader warps: each chunk is 8 pages x (K, V) blocks of 4 KB
+        // (16 keys x 256 B, contiguous in the pool); consecutive threads copy consecutive 16 B
+        // of a block into its 128-byte-swizzled place. Keys past the request are zero-filled.
+        // Each loader thread arrives (no-increment) on the stage barrier when its copies land.
+        const int t = threadIdx.x - 6 * 32;              // 0 .. 127
+        ItemIter it;
+        iter_init(it, a, lo, hi);
+        uint32_t cs = 0;
+        bool ok = true;
+        const char* pool = reinterpret_cast<const char*>(a.kv_pool);
+        for (; it.valid && ok; iter_next(it, a, hi)) {
+            const int npages = (it.nkeys + 15) >> 4;
+            const int base = a.page_indptr[it.r];
+            for (int c = 0; c < it.nch && ok; ++c, ++cs) {
+                const int st = (int)(cs % NS);
+                if (!wait_bcast(&kv_empty[st], ((cs / NS) & 1u) ^ 1u, abort_flag, a.status, lane)) { ok = false; break; }
+                const uint32_t sdst = sbase + st * KV_STAGE;
+                const int np = min(8, npages - 8 * c);
+                // this thread's page ids for the chunk: block index (i*128 + t) >> 8 = 2 j + isv
+                int pgs[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    int pg = 0;
+                    if (j < np) {
+                        pg = __ldg(a.page_indices + base + 8 * c + j);
+                        if (pg < 0 || pg >= a.num_pages) { set_status(a.status, NF_ERR_DEVICE_BOUNDS); pg = 0; }
+                    }
+                    pgs[j] = pg;
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    // 16-byte chunk i * 128 + t of the stage: block (i >> 1) = 2 j + isv, chunk b in the block
+                    const int j = i >> 2, isv = (i >> 1) & 1;
+                    const int b = (i & 1) * 128 + t;
+                    const int kr = b >> 4, cc = b & 15;
+                    const bool valid = j < np && (8 * c + j) * 16 + kr < it.nkeys;
+                    const char* src = pool + ((((size_t)pgs[j] * 2 + isv) * a.nkv + it.g) * 16 + kr) * 256 + cc * 16;
+                    const uint32_t dst = sdst + isv * 2 * REGION + (cc >> 3) * REGION + j * 2048 + kr * 128 +
+                                         ((((cc & 7) ^ (kr & 7))) << 4);
+                    cp_async_16(dst, valid ? (const void*)src : (const void*)pool, valid ? 16u : 0u);
+                }
+                cp_async_arrive_noinc(&kv_full[st]);
+            }
+        }
+        // let this thread's copies land before the CTA exits
+        asm volatile("cp.async.wait_all;" ::: "memory");
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer
@@ -273,6 +247,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t st = cs % NS, sb = cs & 1u;
                     if (!mbar_wait(&kv_full[st], (cs / NS) & 1u, abort_flag, a.status)) { ok = false; break; }
                     if (!mbar_wait(&s_free[sb], ((cs >> 1) & 1u) ^ 1u, abort_flag, a.status)) { ok = false; break; }
+                    fence_proxy_async_smem();  // cp.async data -> tensor-core reads
                     tc_fence_after();
                     const uint32_t kbase = sbase + st * KV_STAGE;
 #pragma unroll
@@ -375,15 +350,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                             lp[h] += p;
                             *reinterpret_cast<__nv_bfloat16*>(pbuf + sw128_offset(h, jl & 63)) = __float2bfloat16_rn(p);
                         }
-                    }
-                    if (!valid) {
-                        // V row of a key past the request: zero it so that 0 * garbage cannot occur
-                        uint8_t* vrow = smem + (cs % NS) * KV_STAGE + 2 * REGION + (jl >> 4) * 2048 + (jl & 15) * 128;
-#pragma unroll
-                        for (int b = 0; b < 2; ++b)
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                reinterpret_cast<uint4*>(vrow + b * REGION)[i] = make_uint4(0u, 0u, 0u, 0u);
                     }
                 }
                 fence_proxy_async_smem();
