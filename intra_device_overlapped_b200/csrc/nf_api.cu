@@ -159,9 +159,7 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) {
     m->sm_count = nf::device_sm_count();
     m->cost = nf::default_cost_model(m->sm_count);
     m->layers.resize(d.L);
-    m->kv_ptr.assign(d.L, nullptr);
-    m->kv_pages.assign(d.L, 0);
-    m->kv_tm.resize(d.L);
+    m->decode_tc = nf::decode_tc_supported(d.nq, d.nkv, d.d);
 
     const size_t T = (size_t)cfg->max_tokens;
     const size_t TK = T * (size_t)d.K;
@@ -228,7 +226,7 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) {
          nf::make_tmap_bf16_2d(&m->tm_attn_o, m->attn_o, T, (uint64_t)d.nq * d.d, nf::kGemmBM) &&
          nf::make_tmap_bf16_2d(&m->tm_act, m->act, act_rows, d.F, nf::kGemmBM);
     if (ok && cfg->vocab > 0) ok = nf::make_tmap_bf16_2d(&m->tm_lm_in, m->lm_in, lm_rows, d.H, nf::kGemmBM);
-    if (ok && d.d == 128) ok = nf::make_tmap_bf16_2d(&m->tm_q, m->q, T * d.nq, d.d, 16);
+    if (ok && m->decode_tc) ok = nf::make_tmap_bf16_2d(&m->tm_q, m->q, T * d.nq, d.d, (uint32_t)d.nq);
     if (ok && d.E > 0) ok = nf::make_tmap_bf16_2d(&m->tm_moe_a, m->moe_a, TK, d.H, nf::kGemmBM);
     if (!ok) { nf_destroy_model(m); return NF_ERR_CUDA; }
     *out = m;
@@ -312,14 +310,10 @@ extern "C" nf_status nf_set_global_weights(nf_model* m, const nf_global_weights*
 
 namespace {
 
-nf_status ensure_kv_tmap(nf_model* m, int layer, const nf_iter_io* io) {
+nf_status check_pool(const nf_model* m, int layer, const nf_iter_io* io) {
     const void* p = io->kv_pools[layer];
-    if (p == nullptr) return NF_ERR_INVALID_ARGUMENT;
-    if (m->kv_ptr[layer] != p || m->kv_pages[layer] != io->num_pages) {
-        if (!nf::make_kv_tmap(&m->kv_tm[layer], p, io->num_pages, m->dims.nkv, m->dims.d)) return NF_ERR_CUDA;
-        m->kv_ptr[layer] = p;
-        m->kv_pages[layer] = io->num_pages;
-    }
+    if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) != 0) return NF_ERR_INVALID_ARGUMENT;
+    (void)m;
     return NF_OK;
 }
 
@@ -409,8 +403,7 @@ struct OpTimer {
 cudaError_t decode_prologue(nf_model* m, const nf_iter_io* io, int R, cudaStream_t s) {
     if (R <= 0) return cudaSuccess;
     const nf::ModelDims& d = m->dims;
-    if (d.d == 128)
-        return nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeTcChunkPages, m->item_off, s);
+    if (m->decode_tc) return nf::launch_decode_schedule(io->ctx_len, R, 1, 1, m->item_off, s);
     cudaError_t e = nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, s);
     if (e != cudaSuccess) return e;
     return nf::launch_decode_items(io->ctx_len, io->page_indptr, R, d.nkv, nf::kDecodeSplitPages, m->item_off,
@@ -421,8 +414,8 @@ cudaError_t launch_decode(nf_model* m, const nf_iter_io* io, const CUtensorMap& 
                           int layer, int rb, int re, int grid, cudaStream_t s) {
     nf::DecodeArgs da = decode_args(m, io, q, out, rb, re);
     da.kv_pool = (const uint16_t*)io->kv_pools[layer];
-    if (m->dims.d == 128) return nf::launch_decode_attention_tc(m->kv_tm[layer], tmq, da, grid, s);
-    return nf::launch_decode_attention(m->kv_tm[layer], da, m->dims.d, grid, s);
+    if (m->decode_tc) return nf::launch_decode_attention_tc(tmq, da, grid, s);
+    return nf::launch_decode_attention(da, m->dims.d, grid, s);
 }
 
 nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::Op& op, int grid,
@@ -464,7 +457,8 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
         case nf::OP_PATT: {
             if (t1 > R && C > 0) {
                 nf::PrefillArgs pa = prefill_args(m, io, m->q, m->attn_o, R, C);
-                NF_CUDA_TRY(nf::launch_prefill_attention(m->kv_tm[l], pa, d.d, grid, s));
+                pa.kv_pool = (const uint16_t*)io->kv_pools[l];
+                NF_CUDA_TRY(nf::launch_prefill_attention(pa, d.d, grid, s));
             }
             return NF_OK;
         }
@@ -600,7 +594,7 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     cudaStream_t sa = m->s_attn;
     if ((st = ensure_part_capacity(m, std::max<int64_t>(p->decode_items, 1))) != NF_OK) return st;
     for (int l = 0; l < d.L; ++l)
-        if ((st = ensure_kv_tmap(m, l, io)) != NF_OK) return st;
+        if ((st = check_pool(m, l, io)) != NF_OK) return st;
 
     const int S = p->sm_total;
     NF_CUDA_TRY(cudaEventRecord(m->ev_fork, sg));
@@ -767,9 +761,9 @@ extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* ou
         return NF_ERR_INVALID_ARGUMENT;
     if (req_end == req_begin) return NF_OK;
     cudaStream_t s = (cudaStream_t)stream;
-    nf_status st = ensure_kv_tmap(m, layer, io);
+    nf_status st = check_pool(m, layer, io);
     if (st != NF_OK) return st;
-    if (m->dims.d != 128) {
+    if (!m->decode_tc) {
         NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, req_end, m->dims.nkv, nf::kDecodeSplitPages, m->item_off,
                                                s));
         int items = 0;
@@ -779,8 +773,9 @@ extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* ou
     }
     NF_CUDA_TRY(decode_prologue(m, io, req_end, s));
     CUtensorMap tmq;
-    if (m->dims.d == 128 &&
-        !nf::make_tmap_bf16_2d(&tmq, q, (uint64_t)req_end * m->dims.nq, m->dims.d, 16))
+    std::memset(&tmq, 0, sizeof(tmq));
+    if (m->decode_tc &&
+        !nf::make_tmap_bf16_2d(&tmq, q, (uint64_t)req_end * m->dims.nq, m->dims.d, (uint32_t)m->dims.nq))
         return NF_ERR_INVALID_ARGUMENT;
     const int grid = sm_count > 0 ? std::min(sm_count, m->sm_count) : m->sm_count;
     NF_CUDA_TRY(launch_decode(m, io, tmq, q, out, layer, req_begin, req_end, grid, s));
@@ -794,11 +789,12 @@ extern "C" nf_status nf_op_prefill_attention(nf_model* m, const void* q, void* o
         return NF_ERR_INVALID_ARGUMENT;
     if (layer < 0 || layer >= m->dims.L || num_decode < 0 || prefill_len < 0) return NF_ERR_INVALID_ARGUMENT;
     if (prefill_len == 0) return NF_OK;
-    nf_status st = ensure_kv_tmap(m, layer, io);
+    nf_status st = check_pool(m, layer, io);
     if (st != NF_OK) return st;
     const int grid = sm_count > 0 ? std::min(sm_count, m->sm_count) : m->sm_count;
     nf::PrefillArgs pa = prefill_args(m, io, q, out, num_decode, prefill_len);
-    NF_CUDA_TRY(nf::launch_prefill_attention(m->kv_tm[layer], pa, m->dims.d, grid, (cudaStream_t)stream));
+    pa.kv_pool = (const uint16_t*)io->kv_pools[layer];
+    NF_CUDA_TRY(nf::launch_prefill_attention(pa, m->dims.d, grid, (cudaStream_t)stream));
     return NF_OK;
 }
 
@@ -846,7 +842,7 @@ extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_
     if (!m->layers[0].loaded || io->kv_pools == nullptr || io->kv_pools[0] == nullptr) return NF_ERR_INVALID_ARGUMENT;
     if (R > 0 && (io->ctx_len == nullptr || b->ctx_len == nullptr)) return NF_ERR_INVALID_ARGUMENT;
     cudaStream_t sg = (cudaStream_t)stream, sa = m->s_attn;
-    nf_status st = ensure_kv_tmap(m, 0, io);
+    nf_status st = check_pool(m, 0, io);
     if (st != NF_OK) return st;
     const int S = m->sm_count;
     nf::CostModel c = m->cost;
@@ -940,7 +936,8 @@ extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_
         double t_p = 0;
         auto pre = [&]() -> nf_status {
             nf::PrefillArgs pa = prefill_args(m, io, m->q, m->attn_o, R, C);
-            return nf::launch_prefill_attention(m->kv_tm[0], pa, d.d, q, sg) == cudaSuccess ? NF_OK : NF_ERR_CUDA;
+            pa.kv_pool = (const uint16_t*)io->kv_pools[0];
+            return nf::launch_prefill_attention(pa, d.d, q, sg) == cudaSuccess ? NF_OK : NF_ERR_CUDA;
         };
         if ((st = time_us(sg, 3, pre, &t_p)) != NF_OK) return st;
         const double flops = 4.0 * d.nq * d.d * (double)C * (C + 1) / 2.0;

@@ -123,7 +123,7 @@ __device__ __forceinline__ float col_sum(float x) {
 // more than 2^8 (exponents stay <= 256), which skips most accumulator rescales.
 template <int HD>
 __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
-    decode_attention_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ DecodeArgs a) {
+    decode_attention_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr int BOXES = HD / 64;
     constexpr uint32_t KV_BYTES = BOXES * BOX_BYTES;  // one page, one KV head, K or V
     constexpr uint32_t STAGE_BYTES = 2 * KV_BYTES;
@@ -142,7 +142,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
         t_start = globaltimer_ns();
         for (int s = 0; s < DEC_WARPS * NSTW; ++s) mbar_init(&full_all[s], 1);
         fence_mbar_init();
-        tma_prefetch_desc(&tmKV);
     }
     __syncthreads();
 
@@ -184,11 +183,12 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             uint8_t* dst = wsm + st * STAGE_BYTES;                                                   \
             fence_proxy_async_smem();                                                                \
             mbar_arrive_expect_tx(&full[st], STAGE_BYTES);                                           \
-            const int rowK = ((pg * 2 + 0) * a.nkv + im.g) * 16;                                     \
-            const int rowV = ((pg * 2 + 1) * a.nkv + im.g) * 16;                                     \
+            const char* pgb = reinterpret_cast<const char*>(a.kv_pool) + (size_t)pg * 2 * a.nkv * 16 * HD * 2; \
             _Pragma("unroll") for (int b = 0; b < BOXES; ++b) {                                      \
-                tma_load_2d(dst + b * BOX_BYTES, &tmKV, &full[st], b * 64, rowK);                    \
-                tma_load_2d(dst + KV_BYTES + b * BOX_BYTES, &tmKV, &full[st], b * 64, rowV);         \
+                bulk_load(dst + b * BOX_BYTES, pgb + ((size_t)(0 * BOXES + b) * a.nkv + im.g) * BOX_BYTES, \
+                          BOX_BYTES, &full[st]);                                                     \
+                bulk_load(dst + KV_BYTES + b * BOX_BYTES,                                            \
+                          pgb + ((size_t)(1 * BOXES + b) * a.nkv + im.g) * BOX_BYTES, BOX_BYTES, &full[st]); \
             }                                                                                        \
         }                                                                                            \
         ++issued;                                                                                    \
@@ -381,7 +381,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
 // 16 query rows each. Causal: tile kt is needed by q tile qt iff kt <= qt.
 template <int HD>
 __global__ void __launch_bounds__(PRE_THREADS, 1)
-    prefill_attention_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ PrefillArgs a) {
+    prefill_attention_kernel(const __grid_constant__ PrefillArgs a) {
     constexpr int BOXES = HD / 64;
     constexpr uint32_t PAGE_BYTES = BOXES * BOX_BYTES;      // one page of K (or V), one KV head
     constexpr uint32_t HALF_BYTES = 4 * PAGE_BYTES;          // 64 keys
@@ -402,7 +402,6 @@ __global__ void __launch_bounds__(PRE_THREADS, 1)
         for (int s = 0; s < PRE_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 4); }
         *abort_flag = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tmKV);
     }
     __syncthreads();
 
@@ -433,13 +432,13 @@ __global__ void __launch_bounds__(PRE_THREADS, 1)
                         int pidx = min(kt * 4 + pp, npages - 1);
                         int page = pt[pidx];
                         if (page < 0 || page >= a.num_pages) { set_status(a.status, NF_ERR_DEVICE_BOUNDS); page = 0; }
-                        const int rowK = ((page * 2 + 0) * a.nkv + g) * 16;
-                        const int rowV = ((page * 2 + 1) * a.nkv + g) * 16;
+                        const char* pgb = reinterpret_cast<const char*>(a.kv_pool) + (size_t)page * 2 * a.nkv * 16 * HD * 2;
 #pragma unroll
                         for (int b = 0; b < BOXES; ++b) {
-                            tma_load_2d(st + pp * PAGE_BYTES + b * BOX_BYTES, &tmKV, &full[stage], b * 64, rowK);
-                            tma_load_2d(st + HALF_BYTES + pp * PAGE_BYTES + b * BOX_BYTES, &tmKV, &full[stage],
-                                        b * 64, rowV);
+                            bulk_load(st + pp * PAGE_BYTES + b * BOX_BYTES,
+                                      pgb + ((size_t)(0 * BOXES + b) * a.nkv + g) * BOX_BYTES, BOX_BYTES, &full[stage]);
+                            bulk_load(st + HALF_BYTES + pp * PAGE_BYTES + b * BOX_BYTES,
+                                      pgb + ((size_t)(1 * BOXES + b) * a.nkv + g) * BOX_BYTES, BOX_BYTES, &full[stage]);
                         }
                     }
                     outstanding |= 1u << stage;
@@ -698,38 +697,36 @@ cudaError_t launch_decode_items(const int* ctx_len, const int* page_indptr, int 
     return cudaGetLastError();
 }
 
-cudaError_t launch_decode_attention(const CUtensorMap& tmKV, const DecodeArgs& a, int head_dim, int grid,
-                                    cudaStream_t stream) {
+cudaError_t launch_decode_attention(const DecodeArgs& a, int head_dim, int grid, cudaStream_t stream) {
     if (grid <= 0 || a.req_end <= a.req_begin) return cudaSuccess;
     const int smem = decode_smem_bytes(head_dim);
     cudaError_t e;
     if (head_dim == 128) {
         static bool cfg = false;
         if (!cfg) { if ((e = set_smem(decode_attention_kernel<128>, smem)) != cudaSuccess) return e; cfg = true; }
-        decode_attention_kernel<128><<<grid, DEC_WARPS * 32, smem, stream>>>(tmKV, a);
+        decode_attention_kernel<128><<<grid, DEC_WARPS * 32, smem, stream>>>(a);
     } else if (head_dim == 64) {
         static bool cfg = false;
         if (!cfg) { if ((e = set_smem(decode_attention_kernel<64>, smem)) != cudaSuccess) return e; cfg = true; }
-        decode_attention_kernel<64><<<grid, DEC_WARPS * 32, smem, stream>>>(tmKV, a);
+        decode_attention_kernel<64><<<grid, DEC_WARPS * 32, smem, stream>>>(a);
     } else {
         return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_attention(const CUtensorMap& tmKV, const PrefillArgs& a, int head_dim, int grid,
-                                     cudaStream_t stream) {
+cudaError_t launch_prefill_attention(const PrefillArgs& a, int head_dim, int grid, cudaStream_t stream) {
     if (grid <= 0 || a.prefill_len <= 0) return cudaSuccess;
     const int smem = prefill_smem_bytes(head_dim);
     cudaError_t e;
     if (head_dim == 128) {
         static bool cfg = false;
         if (!cfg) { if ((e = set_smem(prefill_attention_kernel<128>, smem)) != cudaSuccess) return e; cfg = true; }
-        prefill_attention_kernel<128><<<grid, PRE_THREADS, smem, stream>>>(tmKV, a);
+        prefill_attention_kernel<128><<<grid, PRE_THREADS, smem, stream>>>(a);
     } else if (head_dim == 64) {
         static bool cfg = false;
         if (!cfg) { if ((e = set_smem(prefill_attention_kernel<64>, smem)) != cudaSuccess) return e; cfg = true; }
-        prefill_attention_kernel<64><<<grid, PRE_THREADS, smem, stream>>>(tmKV, a);
+        prefill_attention_kernel<64><<<grid, PRE_THREADS, smem, stream>>>(a);
     } else {
         return cudaErrorInvalidValue;
     }
@@ -738,8 +735,3 @@ cudaError_t launch_prefill_attention(const CUtensorMap& tmKV, const PrefillArgs&
 
 }  // namespace nf
 
-namespace nf {
-bool make_kv_tmap(CUtensorMap* map, const void* pool, int num_pages, int nkv, int head_dim) {
-    return make_tmap_bf16_2d(map, pool, (uint64_t)num_pages * 2 * nkv * 16, (uint64_t)head_dim, 16);
-}
-}  // namespace nf

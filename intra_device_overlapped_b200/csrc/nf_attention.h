@@ -22,7 +22,7 @@ struct DecodeArgs {
     const int* page_indices;
     const int* item_off;  // [R + 1] first work item of each request
     const void* item_tab; // [items] int4 work-item table (decode_items_kernel)
-    const uint16_t* kv_pool;  // layer's pool (L2 prefetch addresses)
+    const uint16_t* kv_pool;  // the layer's pool, physical page layout (see store_kv_row32 / nanoflow.h)
     int req_begin, req_end;
     int nq, nkv, G;
     int num_pages;
@@ -38,6 +38,7 @@ struct DecodeArgs {
 struct PrefillArgs {
     const uint16_t* q;   // [rows x nq x d]; chunk row i is row num_decode + i
     uint16_t* out;
+    const uint16_t* kv_pool;
     const int* page_indptr;
     const int* page_indices;
     int num_decode;      // index of the prefill request in the page table
@@ -58,19 +59,14 @@ cudaError_t launch_decode_schedule(const int* ctx_len, int R, int nkv, int split
                                    cudaStream_t stream);
 cudaError_t launch_decode_items(const int* ctx_len, const int* page_indptr, int R, int nkv, int split_pages,
                                 const int* item_off, void* item_tab, int* merge_cnt, cudaStream_t stream);
-cudaError_t launch_decode_attention(const CUtensorMap& tmKV, const DecodeArgs& a, int head_dim, int grid,
-                                    cudaStream_t stream);
-cudaError_t launch_prefill_attention(const CUtensorMap& tmKV, const PrefillArgs& a, int head_dim, int grid,
-                                     cudaStream_t stream);
+cudaError_t launch_decode_attention(const DecodeArgs& a, int head_dim, int grid, cudaStream_t stream);
+cudaError_t launch_prefill_attention(const PrefillArgs& a, int head_dim, int grid, cudaStream_t stream);
 
-// Tensor-core (tcgen05) decode attention for head dim 128; a.item_off holds, per request,
-// the prefix of nkv * ceil((ctx_len + 1) / 128) (decode_schedule with split_pages = 8).
-constexpr int kDecodeTcChunkPages = 8;
-int decode_tc_smem_bytes();
-cudaError_t launch_decode_attention_tc(const CUtensorMap& tmKV, const CUtensorMap& tmQ, const DecodeArgs& a,
-                                       int grid, cudaStream_t stream);
-
-// KV pool as a 2-D tensor [num_pages * 2 * nkv * 16 rows x d cols], 16 x 64 boxes, 128-byte swizzle.
-bool make_kv_tmap(CUtensorMap* map, const void* pool, int num_pages, int nkv, int head_dim);
+// Tensor-core (tcgen05) decode attention for 8 KV heads of dim 128 and 32 or 64 query heads:
+// one request (all heads) per work item, one 64 KB page per pipeline stage. a.item_off holds
+// the per-request prefix of page counts (decode_schedule with nkv = 1, split_pages = 1); tmQ
+// maps q as [rows * nq x d] with boxes of nq rows.
+bool decode_tc_supported(int nq, int nkv, int head_dim);
+cudaError_t launch_decode_attention_tc(const CUtensorMap& tmQ, const DecodeArgs& a, int grid, cudaStream_t stream);
 
 }  // namespace nf

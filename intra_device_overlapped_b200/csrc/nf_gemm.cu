@@ -115,6 +115,25 @@ __device__ __forceinline__ void store_f32x32(float* dst, const float* v) {
     for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
+// 32 consecutive columns [c0, c0 + 32) of row `slot` of (K|V = kv, head g) in a page of the
+// physical KV layout: [K|V][64-column half][head][16 rows][8 chunks of 16 B], logical chunk c
+// of row r stored at chunk c ^ (r & 7). c0 is a multiple of 32, so the columns stay in one half.
+__device__ __forceinline__ void store_kv_row32(uint16_t* page, int kv, int g, int nkv, int d, int slot, int c0,
+                                               const float* v) {
+    const int halves = d / 64;
+    uint16_t* rowp = page + (((size_t)kv * halves + (c0 >> 6)) * nkv + g) * 16 * 64 + (size_t)slot * 64;
+    const int chunk0 = (c0 & 63) >> 3;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+        w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+        w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+        w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+        *reinterpret_cast<uint4*>(rowp + (((chunk0 + q) ^ (slot & 7)) << 3)) = w;
+    }
+}
+
 // ------------------------------------------------------------------ epilogues
 // Each is called by all 32 lanes of an epilogue warp (tcgen05.ld is warp-collective);
 // `valid` says whether this lane's row is inside the tile's row range.
@@ -201,7 +220,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, 
         const int tok = p.tok0 + row;
         const float rs = valid ? row_scale(p, row) : 1.f;
         int pos = 0;
-        long long kv_off = -1;  // element offset of this token's K slot for kv head 0
+        long long page_base = -1;  // element offset of this token's page in the pool
         bool ok = valid;
         if (valid) {
             pos = p.positions[tok];
@@ -215,43 +234,43 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, 
                 if (page < 0 || page >= p.num_pages) {
                     set_status(p.status, NF_ERR_DEVICE_BOUNDS);
                 } else {
-                    kv_off = ((long long)page * 2 * p.nkv * 16 + (pos % 16)) * d;
+                    page_base = (long long)page * 2 * p.nkv * 16 * d;
                 }
             }
         }
+        const int slot = pos & 15;
         float x2[32];
 #pragma unroll 1
         for (int hc = 0; hc < BN / d; ++hc) {
             const int head = (n0 + hc * d) / d;
             const int kind = head < p.nq ? 0 : (head < p.nq + p.nkv ? 1 : 2);
-            uint16_t* dst = nullptr;
-            if (kind == 0) {
-                dst = p.q_out + ((size_t)tok * p.nq + head) * d;
-            } else if (kv_off >= 0) {
-                const int g = kind == 1 ? head - p.nq : head - p.nq - p.nkv;
-                dst = p.kv_pool + kv_off + ((long long)(kind - 1) * p.nkv + g) * 16 * d;
-            }
+            const int g = kind == 1 ? head - p.nq : head - p.nq - p.nkv;
 #pragma unroll 1
             for (int j = 0; j < half / 32; ++j) {
                 tmem_ld32(tacc + hc * d + 32 * j, v);
                 tmem_ld32(tacc + hc * d + half + 32 * j, x2);
-                if (ok && dst != nullptr) {
-                    if (kind < 2) {
-                        const float* cs = p.rope_cos + (size_t)pos * half + 32 * j;
-                        const float* sn = p.rope_sin + (size_t)pos * half + 32 * j;
+                if (!ok || (kind != 0 && page_base < 0)) continue;
+                if (kind < 2) {
+                    const float* cs = p.rope_cos + (size_t)pos * half + 32 * j;
+                    const float* sn = p.rope_sin + (size_t)pos * half + 32 * j;
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const float a = v[e] * rs, b = x2[e] * rs;
-                            const float c = cs[e], s = sn[e];
-                            v[e] = a * c - b * s;
-                            x2[e] = b * c + a * s;
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) { v[e] *= rs; x2[e] *= rs; }
+                    for (int e = 0; e < 32; ++e) {
+                        const float a = v[e] * rs, b = x2[e] * rs;
+                        const float c = cs[e], s = sn[e];
+                        v[e] = a * c - b * s;
+                        x2[e] = b * c + a * s;
                     }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) { v[e] *= rs; x2[e] *= rs; }
+                }
+                if (kind == 0) {
+                    uint16_t* dst = p.q_out + ((size_t)tok * p.nq + head) * d;
                     store_bf16x32(dst + 32 * j, v);
                     store_bf16x32(dst + half + 32 * j, x2);
+                } else {
+                    store_kv_row32(p.kv_pool + page_base, kind - 1, g, p.nkv, d, slot, 32 * j, v);
+                    store_kv_row32(p.kv_pool + page_base, kind - 1, g, p.nkv, d, slot, half + 32 * j, x2);
                 }
             }
         }

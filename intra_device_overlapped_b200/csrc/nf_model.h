@@ -67,7 +67,8 @@ struct nf_model {
     float* moe_part = nullptr;    // [T K x H/256]
     float* moe_y = nullptr;       // [T K x H]
     CUtensorMap tm_xb, tm_attn_o, tm_act, tm_lm_in, tm_moe_a;
-    CUtensorMap tm_q;             // q as [T * nq rows x d], 16-row boxes (decode attention Q loads)
+    CUtensorMap tm_q;             // q as [T * nq rows x d], nq-row boxes (tensor-core decode attention Q loads)
+    bool decode_tc = false;       // the tensor-core decode kernel handles this model's head shape
 
     int* status = nullptr;        // device status word
     int* trace_ctr = nullptr;
@@ -79,10 +80,6 @@ struct nf_model {
     cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
     std::vector<cudaEvent_t> events;
 
-    // KV pool tensor maps, cached per layer by pointer
-    std::vector<const void*> kv_ptr;
-    std::vector<int> kv_pages;
-    std::vector<CUtensorMap> kv_tm;
 
     // per-op event timing
     bool timing_on = false;

@@ -58,9 +58,8 @@ class DeviceWorkload:
         st, self.model = nf_init_model(cfg)
         check(st, "nf_init_model")
         self._load_weights()
-        # paged KV pools, one per layer
-        self.kv = [_empty_bf16((b.num_pages, 2, s.n_kv_heads, s.page_size, s.head_dim), self.device)
-                   for _ in range(s.n_layers)]
+        # paged KV pools, one per layer (physical page images, see synth.weights.kv_phys_to_logical)
+        self.kv = [_empty_bf16((b.num_pages, SW.kv_page_elems(s)), self.device) for _ in range(s.n_layers)]
         for layer, pool in enumerate(self.kv):
             SW.gpu_fill_kv_pool(s, layer, pool)
         self._kv_ptrs = (_vp * s.n_layers)(*[p.data_ptr() for p in self.kv])
@@ -201,6 +200,11 @@ class DeviceWorkload:
             self.close()
         except Exception:
             pass
+
+
+def kv_logical(dw: "DeviceWorkload", layer: int) -> np.ndarray:
+    """Host copy of a layer's pool as bf16 bit patterns in the logical view [pages, 2, nkv, P, d]."""
+    return SW.kv_phys_to_logical(bf16_bits(dw.kv[layer]), dw.shape)
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:

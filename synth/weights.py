@@ -5,9 +5,11 @@ Every tensor is an element-indexed stream of the generator in ``synth_cpu.c``
 bf16 value on both, so the oracle can regenerate any slice of an input that the
 device filled in HBM.
 
-Layouts are the canonical ones the library's C ABI accepts: linear weights are
-[out_features x in_features] row-major, norms are [hidden], the paged KV pool of
-one layer is [num_pages][2 (K, V)][n_kv_heads][page_size][head_dim].
+Layouts are the ones the library's C ABI accepts: linear weights are
+[out_features x in_features] row-major, norms are [hidden]. The paged KV pool of one
+layer holds, per page, the physical image described by ``kv_phys_to_logical``; the
+generator fills the physical pool element by element, and the host helpers below hand
+the oracle the logical view [pages, 2 (K, V), n_kv_heads, page_size, head_dim].
 """
 from __future__ import annotations
 
@@ -84,17 +86,37 @@ def kv_page_elems(s: ModelShape) -> int:
     return 2 * s.n_kv_heads * s.page_size * s.head_dim
 
 
+def kv_phys_to_logical(phys: np.ndarray, s: ModelShape) -> np.ndarray:
+    """Logical view [n, 2, nkv, 16, d] of physical page images [n, page elements].
+
+    Physical order within a page: K|V, then 64-column half of the head dimension, then KV
+    head, then the 16 rows (tokens), then eight 16-byte chunks of 8 elements, where logical
+    chunk c of row r is stored at chunk position c XOR (r mod 8). Each (K|V, half, head)
+    block is thus the 2 KB image of a 16 x 64 tile in 128-byte-swizzled form, and all heads
+    of a half are one contiguous region.
+    """
+    n = phys.shape[0]
+    nkv, d, P = s.n_kv_heads, s.head_dim, s.page_size
+    h2 = d // 64
+    a = np.asarray(phys).reshape(n, 2, h2, nkv, P, 8, 8)
+    rows = np.arange(P)[:, None]
+    src = np.arange(8)[None, :] ^ (rows & 7)
+    a = a[:, :, :, :, rows, src, :]                       # [n, 2, h2, nkv, P, 8, 8], logical chunks
+    return a.transpose(0, 1, 3, 4, 2, 5, 6).reshape(n, 2, nkv, P, d)
+
+
 def host_kv_pool(s: ModelShape, layer: int, num_pages: int) -> np.ndarray:
+    """Initial contents of a whole pool, logical view [num_pages, 2, nkv, P, d]."""
     n = num_pages * kv_page_elems(s)
-    return normal_bf16(SEED_KV, layer, n).reshape(num_pages, 2, s.n_kv_heads, s.page_size, s.head_dim)
+    return kv_phys_to_logical(normal_bf16(SEED_KV, layer, n).reshape(num_pages, -1), s)
 
 
 def host_kv_pages(s: ModelShape, layer: int, pages: np.ndarray) -> np.ndarray:
-    """Initial contents of the listed pages of one layer's pool, [len(pages), 2, nkv, P, d]."""
+    """Initial contents of the listed pages of one layer's pool, logical view [len(pages), 2, nkv, P, d]."""
     pe = kv_page_elems(s)
     starts = np.asarray(pages, dtype=np.uint64) * np.uint64(pe)
     out = ranges_normal_bf16(SEED_KV, layer, starts, pe)
-    return out.reshape(len(pages), 2, s.n_kv_heads, s.page_size, s.head_dim)
+    return kv_phys_to_logical(out, s)
 
 
 def host_input_hidden(s: ModelShape, num_tokens: int) -> np.ndarray:

@@ -148,5 +148,8 @@ TEST_WORKLOADS = {
     "tiny_moe": Workload(replace(TINY, n_layers=2, n_experts=4, top_k=2, norm_sigma=0.1), 8, 16, 64,
                          prefill_len=32),
     "tiny_decode_only": Workload(TINY, 6, 1, 40, prefill_len=0),
+    # 8 KV heads of dim 128 with 32 query heads: the head shape of the Llama-3-8B / Mixtral layers
+    "small_gqa8": Workload(ModelShape("small_gqa8", 2, 1024, 32, 8, 128, 1024, rope_theta=500000.0,
+                                      norm_sigma=0.1), 24, 1, 300, prefill_len=70),
     "tiny_prefill_only": Workload(TINY, 0, prefill_len=45),
 }

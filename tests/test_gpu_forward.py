@@ -79,8 +79,9 @@ def test_tiny_kv_slots_written_and_others_untouched(tiny):
     dw, res, kv_oracle = tiny
     _reset_kv(dw)
     _run(dw, dw.plan(nano=2, template=1, sm_attn=20))
+    from intra_device_overlapped_b200.harness import kv_logical
     s, b = dw.shape, dw.batch
-    got = dw.kv[0].float().cpu().numpy()
+    got = synth.bf16_to_f64(kv_logical(dw, 0))
     init = synth.bf16_to_f64(SW.host_kv_pool(s, 0, b.num_pages))
     written = res["layers"][0]["written"]
     mask = np.zeros(got.shape, dtype=bool)
@@ -164,5 +165,27 @@ def test_tiny_moe_routing_and_output():
                 assert idx[t].tolist() == own
                 if srt[t, 1] - srt[t, 2] > 2 * zerr and srt[t, 0] - srt[t, 1] > 2 * zerr:
                     assert idx[t].tolist() == res["layers"][layer]["topk_idx"][t].tolist()
+    finally:
+        dw.close()
+
+
+def test_gqa8_iteration_matches_oracle_and_is_invariant():
+    """Head shape of the Llama-3-8B layer (32 query / 8 KV heads of 128): tensor-core decode path."""
+    from intra_device_overlapped_b200.harness import DeviceWorkload
+    from oracle.run import run_oracle
+    w = TEST_WORKLOADS["small_gqa8"]
+    dw = DeviceWorkload(w, DEV)
+    try:
+        _, res, _ = run_oracle(w, batch=dw.batch)
+        outs = []
+        for opts in (dict(nano=1, template=0), dict(nano=2, template=1, sm_attn=20),
+                     dict(nano=3, template=2, sm_attn=36), dict()):
+            _reset_kv(dw)
+            hid = _run(dw, dw.plan(**opts))
+            mx, rel = errors(hid, res["hidden"])
+            assert mx <= MAX_ABS and rel <= MEAN_REL, (mx, rel, opts)
+            outs.append(_bits(dw.hidden_out_f32))
+        for o in outs[1:]:
+            assert np.array_equal(o, outs[0])
     finally:
         dw.close()

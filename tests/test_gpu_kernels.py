@@ -88,6 +88,9 @@ ATT_SHAPES = {
     "d64": Workload(ModelShape("attn64", 1, 256, 4, 2, 64, 512), 9, 0, 70, prefill_len=45),
     # G = 8 (Llama-2-70B head grouping)
     "g8": Workload(ModelShape("attn_g8", 1, 2048, 16, 2, 128, 512), 5, 300, 600, prefill_len=17),
+    # 8 KV heads x 128, 32 / 64 query heads: the tensor-core decode kernel (whole pages, all heads)
+    "tc32": Workload(ModelShape("attn_tc32", 1, 1024, 32, 8, 128, 512), 40, 0, 700, prefill_len=100),
+    "tc64": Workload(ModelShape("attn_tc64", 1, 1024, 64, 8, 128, 512), 13, 200, 1100, prefill_len=33),
 }
 
 

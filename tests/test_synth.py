@@ -100,6 +100,22 @@ def test_kv_pages_match_pool():
     assert np.array_equal(sel[0], pool[11]) and np.array_equal(sel[1], pool[3])
 
 
+@pytest.mark.parametrize("d,nkv", [(64, 2), (128, 8)])
+def test_kv_physical_layout_is_a_permutation_with_the_documented_formula(d, nkv):
+    from synth.workloads import ModelShape
+    s = ModelShape("t", 1, 256, nkv, nkv, d, 128)
+    pe = W.kv_page_elems(s)
+    phys = np.arange(2 * pe, dtype=np.int64).reshape(2, pe)
+    logical = W.kv_phys_to_logical(phys, s)
+    assert sorted(logical.ravel().tolist()) == list(range(2 * pe))
+    rng = np.random.default_rng(0)
+    for _ in range(200):
+        n, kv, h, r, c = (rng.integers(2), rng.integers(2), rng.integers(nkv), rng.integers(16), rng.integers(d))
+        off = (kv * (d // 64) * nkv * 16 * 64 + (c // 64) * nkv * 16 * 64 + (h * 16 + r) * 64
+               + (((c % 64) // 8) ^ (r % 8)) * 8 + c % 8)
+        assert logical[n, kv, h, r, c] == n * pe + off
+
+
 def test_weight_rows_match_full_tensor():
     s = TEST_WORKLOADS["tiny_lm"].shape
     spec = W.global_specs(s)["embed"]
