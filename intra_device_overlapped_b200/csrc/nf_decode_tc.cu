@@ -33,25 +33,42 @@ namespace {
 
 constexpr int ROWS = 128;                   // 8 KV heads x 16 keys of one page
 constexpr uint32_t PAGE_BYTES = 65536;      // K and V of all heads of one page
+constexpr uint32_t HALF_PAGE = 32768;       // K (or V) of all heads of one page
 constexpr uint32_t REGION = 16384;          // one 64-column half of K or V: 128 rows x 128 B
 constexpr float LAZY = 8.0f;
 
 template <int NQ>
 struct TcCfg {
-    static constexpr int NS = NQ <= 32 ? 3 : 2;           // page stages
+    static constexpr int NSK = 3;                         // K stages (released after Q K^T)
+    static constexpr int NSV = NQ <= 32 ? 3 : 2;          // V stages (released after P V)
+    static constexpr int NSB = 3;                         // S^T buffers in TMEM
+    static constexpr int LOOK = NSB - 1;                  // S is issued this many pages ahead of P V
+    static constexpr int NPB = 3;                         // P buffers: the softmax of page c reuses the
+                                                          // buffer of page c - 3, whose P V precedes S(c)
     static constexpr uint32_t QB = NQ * 256;              // Q: two halves of NQ rows x 128 B
     static constexpr uint32_t PB = NQ * 256;              // P buffer: two key halves of NQ rows x 128 B
-    static constexpr uint32_t OFF_Q = NS * PAGE_BYTES;
+    static constexpr uint32_t OFF_V = NSK * HALF_PAGE;
+    static constexpr uint32_t OFF_Q = OFF_V + NSV * HALF_PAGE;
     static constexpr uint32_t OFF_P = OFF_Q + QB;
-    static constexpr uint32_t OFF_CF = OFF_P + 2 * PB;    // float[NQ] rescale factors / row sums
+    static constexpr uint32_t OFF_CF = OFF_P + NPB * PB;  // float[NQ] rescale factors / row sums
     static constexpr uint32_t OFF_BAR = OFF_CF + NQ * 4;
     static constexpr uint32_t SMEM = OFF_BAR + 32 * 8 + 1024;
-    static constexpr uint32_t TMEM_COLS = NQ <= 32 ? 128 : 256;  // S[2] + O^T: 3 NQ columns
+    static constexpr uint32_t O_COL = NSB * NQ;           // O^T accumulator after the S^T buffers
+    static constexpr uint32_t TMEM_COLS = (NSB + 1) * NQ <= 128 ? 128 : 256;
     static constexpr uint32_t IDESC_S = umma_idesc_bf16_f32(128, NQ);
     static constexpr uint32_t IDESC_PV = umma_idesc_bf16_f32_amn(128, NQ);
+    static_assert(SMEM <= 232448, "shared memory");
+    // a K stage is free once the S^T of its page completes (s_full), a V stage once its P V
+    // completes (pv_done): the loaders wait on those barriers directly
+    static_assert(NSK == NSB && NSV <= NPB, "stage / buffer counts");
+    static_assert((NSB + 1) * NQ <= 256, "tensor memory");
+    static_assert(NSK + NSV + 2 + 2 * NSB + 2 * NPB + 2 + 1 <= 32,
+                  "barrier slots (+1 for the TMEM slot and abort flag)");
 };
 
-constexpr int THREADS = 192;  // warp 0 loads (Q by TMA, pages by bulk copy), warp 1 MMA + TMEM, warps 2..5 softmax
+// warp 0 loads Q (TMA) and K halves of pages, warp 1 issues MMAs and owns TMEM, warps 2..5 softmax,
+// warp 6 loads V halves of pages (bulk copies)
+constexpr int THREADS = 224;
 
 // Walks the CTA's requests whose first page index (in the page-prefix work space) is in [lo, hi).
 struct ReqIter {
@@ -86,8 +103,44 @@ __device__ __forceinline__ void req_next(ReqIter& it, const DecodeArgs& a, long 
     it.valid = it.r < a.req_end && it.w < hi;
 }
 
+// Position in the CTA's page sequence: page j of request it.r, cs-th page overall, ni-th request.
+struct PageCursor {
+    ReqIter it;
+    int j;
+    uint32_t cs, ni;
+    bool valid;
+};
+
+__device__ __forceinline__ void cursor_init(PageCursor& x, const DecodeArgs& a, long long lo, long long hi) {
+    req_init(x.it, a, lo, hi);
+    x.j = 0;
+    x.cs = 0;
+    x.ni = 0;
+    x.valid = x.it.valid;
+}
+
+__device__ __forceinline__ void cursor_next(PageCursor& x, const DecodeArgs& a, long long hi) {
+    ++x.cs;
+    if (++x.j == x.it.npages) {
+        req_next(x.it, a, hi);
+        x.j = 0;
+        ++x.ni;
+        x.valid = x.it.valid;
+    }
+}
+
+// Non-blocking: has the phase of `bar` with this parity completed? (uniform across the warp)
+__device__ __forceinline__ bool test_bcast(uint64_t* bar, uint32_t parity, int lane) {
+    int ok = 0;
+    if (lane == 0) ok = mbar_try_wait(smem_u32(bar), parity) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 __device__ __forceinline__ bool wait_bcast(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
                                            int lane) {
+    // fast path: every lane tests the (usually already completed) phase; a completed phase stays
+    // completed until this warp moves on, so the lanes agree once all have seen it
+    if (__all_sync(0xffffffffu, mbar_test_wait(smem_u32(bar), parity))) return true;
     int ok = 1;
     if (lane == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
@@ -97,21 +150,21 @@ template <int NQ>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ DecodeArgs a) {
     using C = TcCfg<NQ>;
-    constexpr int NS = C::NS;
+    constexpr int NSK = C::NSK, NSV = C::NSV, NSB = C::NSB, NPB = C::NPB;
     constexpr int G = NQ / 8;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* cfs = reinterpret_cast<float*>(smem + C::OFF_CF);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    uint64_t* kv_full = bars;            // [NS]
-    uint64_t* kv_empty = bars + NS;      // [NS]
-    uint64_t* q_full = bars + 2 * NS;    // [1]
-    uint64_t* q_empty = q_full + 1;      // [1]
-    uint64_t* s_full = q_empty + 1;      // [2]
-    uint64_t* s_free = s_full + 2;       // [2]
-    uint64_t* p_full = s_free + 2;       // [2]
-    uint64_t* pv_done = p_full + 2;      // [2]
-    uint64_t* o_free = pv_done + 2;      // [1]
+    uint64_t* k_full = bars;                   // [NSK]
+    uint64_t* v_full = k_full + NSK;           // [NSV]
+    uint64_t* q_full = v_full + NSV;           // [1]
+    uint64_t* q_empty = q_full + 1;            // [1]
+    uint64_t* s_full = q_empty + 1;            // [NSB]
+    uint64_t* s_free = s_full + NSB;           // [NSB]
+    uint64_t* p_full = s_free + NSB;           // [NPB]
+    uint64_t* pv_done = p_full + NPB;          // [NPB]
+    uint64_t* o_free = pv_done + NPB;          // [1]
     uint64_t* drain = o_free + 1;        // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -119,17 +172,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint64_t t_start = 0;
     // P buffers start at zero: only the block-diagonal entries are ever written
-    for (uint32_t i = threadIdx.x; i < 2 * C::PB / 16; i += THREADS)
+    for (uint32_t i = threadIdx.x; i < NPB * C::PB / 16; i += THREADS)
         reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
     if (threadIdx.x == 0) {
         t_start = globaltimer_ns();
-        for (int i = 0; i < NS; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+        for (int i = 0; i < NSK; ++i) mbar_init(&k_full[i], 1);
+        for (int i = 0; i < NSV; ++i) mbar_init(&v_full[i], 1);
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 4);
-            mbar_init(&p_full[i], 4); mbar_init(&pv_done[i], 1);
-        }
+        for (int i = 0; i < NPB; ++i) { mbar_init(&p_full[i], 4); mbar_init(&pv_done[i], 1); }
+        for (int i = 0; i < NSB; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 4); }
         mbar_init(o_free, 4);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -152,23 +204,29 @@ __global__ void __launch_bounds__(THREADS, 1)
     const long long lo = W0 + W * blockIdx.x / gridDim.x;
     const long long hi = W0 + W * (blockIdx.x + 1) / gridDim.x;
 
-    if (warp == 0) {
-        // ---------------- loader warp: Q of the request (TMA, two 64-column halves of NQ rows),
-        // then each page with one 64 KB bulk copy. Page ids are read 32 at a time (one per lane)
-        // and handed to lane 0 with shuffles.
+    if (warp == 0 || warp == 6) {
+        // ---------------- loader warps: warp 0 streams Q of each request (TMA, two 64-column
+        // halves of NQ rows) and the K half of each page, warp 6 the V half; one 32 KB bulk copy
+        // per half page. Page ids are read 32 at a time (one per lane) and handed to lane 0.
+        const bool is_k = warp == 0;
+        const int nstage = is_k ? NSK : NSV;
+        uint64_t* full = is_k ? k_full : v_full;
+        uint8_t* ring = smem + (is_k ? 0u : C::OFF_V);
         ReqIter it;
         req_init(it, a, lo, hi);
         uint32_t cs = 0, ni = 0;
         bool ok = true;
-        const char* pool = reinterpret_cast<const char*>(a.kv_pool);
+        const char* pool = reinterpret_cast<const char*>(a.kv_pool) + (is_k ? 0 : HALF_PAGE);
         for (; it.valid && ok; req_next(it, a, hi), ++ni) {
             const int base = a.page_indptr[it.r];
-            if (!wait_bcast(q_empty, (ni & 1u) ^ 1u, abort_flag, a.status, lane)) { ok = false; break; }
-            if (lane == 0) {
-                uint8_t* qd = smem + C::OFF_Q;
-                mbar_arrive_expect_tx(q_full, C::QB);
-                tma_load_2d(qd, &tmQ, q_full, 0, it.r * NQ);
-                tma_load_2d(qd + NQ * 128, &tmQ, q_full, 64, it.r * NQ);
+            if (is_k) {
+                if (!wait_bcast(q_empty, (ni & 1u) ^ 1u, abort_flag, a.status, lane)) { ok = false; break; }
+                if (lane == 0) {
+                    uint8_t* qd = smem + C::OFF_Q;
+                    mbar_arrive_expect_tx(q_full, C::QB);
+                    tma_load_2d(qd, &tmQ, q_full, 0, it.r * NQ);
+                    tma_load_2d(qd + NQ * 128, &tmQ, q_full, 64, it.r * NQ);
+                }
             }
             int ids = 0;
             for (int j = 0; j < it.npages; ++j, ++cs) {
@@ -178,69 +236,97 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (ids < 0 || ids >= a.num_pages) { set_status(a.status, NF_ERR_DEVICE_BOUNDS); ids = 0; }
                 }
                 const int pg = __shfl_sync(0xffffffffu, ids, j & 31);
-                const int st = (int)(cs % NS);
-                if (!wait_bcast(&kv_empty[st], ((cs / NS) & 1u) ^ 1u, abort_flag, a.status, lane)) { ok = false; break; }
+                const int st = (int)(cs % nstage);
+                // the stage's previous page (cs - nstage) must be consumed: its S^T (K) or P V (V)
+                if (cs >= (uint32_t)nstage) {
+                    const uint32_t prev = cs - nstage;
+                    uint64_t* done = is_k ? &s_full[prev % NSB] : &pv_done[prev % NPB];
+                    const uint32_t par = is_k ? (prev / NSB) & 1u : (prev / NPB) & 1u;
+                    if (!wait_bcast(done, par, abort_flag, a.status, lane)) { ok = false; break; }
+                }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&kv_full[st], PAGE_BYTES);
-                    bulk_load(smem + st * PAGE_BYTES, pool + (size_t)pg * PAGE_BYTES, PAGE_BYTES, &kv_full[st]);
+                    mbar_arrive_expect_tx(&full[st], HALF_PAGE);
+                    bulk_load(ring + st * HALF_PAGE, pool + (size_t)pg * PAGE_BYTES, HALF_PAGE, &full[st]);
                 }
             }
         }
         if (lane == 0) {
             // let the copies still in flight land before the CTA exits
             volatile int quiet = 0;
-            for (uint32_t x = cs > (uint32_t)NS ? cs - NS : 0u; x < cs; ++x)
-                mbar_wait(&kv_full[x % NS], (x / NS) & 1u, &quiet, nullptr);
-            if (ni > 0) mbar_wait(q_full, (ni - 1) & 1u, &quiet, nullptr);
+            for (uint32_t x = cs > (uint32_t)nstage ? cs - nstage : 0u; x < cs; ++x)
+                mbar_wait(&full[x % nstage], (x / nstage) & 1u, &quiet, nullptr);
+            if (is_k && ni > 0) mbar_wait(q_full, (ni - 1) & 1u, &quiet, nullptr);
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer
-        if (lane == 0) {
-            ReqIter it;
-            req_init(it, a, lo, hi);
-            uint32_t cs = 0, ni = 0;
-            bool ok = true;
-            const uint32_t qbase = sbase + C::OFF_Q;
-            auto issue_pv = [&](uint32_t x, bool first) -> bool {
-                const uint32_t pb = x & 1u;
-                if (!mbar_wait(&p_full[pb], (x >> 1) & 1u, abort_flag, a.status)) return false;
-                if (first && !mbar_wait(o_free, (ni & 1u) ^ 1u, abort_flag, a.status)) return false;
-                tc_fence_after();
-                const uint32_t vbase = sbase + (x % NS) * PAGE_BYTES + 2 * REGION;
-                const uint32_t pbase = sbase + C::OFF_P + pb * C::PB;
+        // ---------------- MMA issuer. The whole warp follows the page cursors and one elected lane
+        // issues; descriptors are built once and offset by constants, so the issue loop holds little
+        // besides the MMAs (16 per page, whose issue rate bounds this kernel). The scores S^T of page
+        // cs + LOOK are issued before P V of page cs, so the tensor core has work while the softmax
+        // warps handle page cs.
+        PageCursor sc, pc;
+        cursor_init(sc, a, lo, hi);
+        cursor_init(pc, a, lo, hi);
+        bool ok = true;
+        const uint64_t kd0 = umma_desc_sw128(sbase);
+        const uint64_t qd0 = umma_desc_sw128(sbase + C::OFF_Q);
+        const uint64_t vd0 = umma_desc_sw128_mn(sbase + C::OFF_V, REGION, 1024);
+        const uint64_t pd0 = umma_desc_sw128(sbase + C::OFF_P);
+        auto issue_s = [&](const PageCursor& x) -> bool {
+            const uint32_t st = x.cs % NSK, sb = x.cs % NSB;
+            if (x.j == 0 && !wait_bcast(q_full, x.ni & 1u, abort_flag, a.status, lane)) return false;
+            if (!wait_bcast(&k_full[st], (x.cs / NSK) & 1u, abort_flag, a.status, lane)) return false;
+            if (!wait_bcast(&s_free[sb], ((x.cs / NSB) & 1u) ^ 1u, abort_flag, a.status, lane)) return false;
+            tc_fence_after();
+            const uint64_t ad = kd0 + ((st * HALF_PAGE) >> 4);
+            const uint64_t bd = qd0;
+            const uint32_t d = tmem + sb * NQ;
+            if (elect_one()) {
+                umma_bf16_c<false>(d, ad, bd, C::IDESC_S);
 #pragma unroll
-                for (int kk = 0; kk < ROWS / 16; ++kk) {
-                    const uint64_t ad = umma_desc_sw128_mn(vbase + kk * 2048, REGION, 1024);
-                    const uint64_t bd = umma_desc_sw128(pbase + (kk >> 2) * (NQ * 128) + (kk & 3) * 32);
-                    umma_bf16(tmem + 2 * NQ, ad, bd, C::IDESC_PV, (first && kk == 0) ? 0u : 1u);
-                }
-                umma_commit(&pv_done[pb]);
-                umma_commit(&kv_empty[x % NS]);
-                return true;
-            };
-            for (; it.valid && ok; req_next(it, a, hi), ++ni) {
-                if (!mbar_wait(q_full, ni & 1u, abort_flag, a.status)) { ok = false; break; }
-                for (int c = 0; c < it.npages; ++c, ++cs) {
-                    const uint32_t st = cs % NS, sb = cs & 1u;
-                    if (!mbar_wait(&kv_full[st], (cs / NS) & 1u, abort_flag, a.status)) { ok = false; break; }
-                    if (!mbar_wait(&s_free[sb], ((cs >> 1) & 1u) ^ 1u, abort_flag, a.status)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t kbase = sbase + st * PAGE_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t ad = umma_desc_sw128(kbase + (kk >> 2) * REGION + (kk & 3) * 32);
-                        const uint64_t bd = umma_desc_sw128(qbase + (kk >> 2) * (NQ * 128) + (kk & 3) * 32);
-                        umma_bf16(tmem + sb * NQ, ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&s_full[sb]);
-                    if (c == it.npages - 1) umma_commit(q_empty);
-                    if (c > 0 && !issue_pv(cs - 1, c == 1)) { ok = false; break; }
-                }
-                if (!ok) break;
-                if (!issue_pv(cs - 1, it.npages == 1)) { ok = false; break; }
+                for (int kk = 1; kk < 8; ++kk)
+                    umma_bf16_c<true>(d, ad + (uint64_t)(((kk >> 2) * REGION + (kk & 3) * 32) >> 4),
+                                      bd + (uint64_t)(((kk >> 2) * (NQ * 128) + (kk & 3) * 32) >> 4), C::IDESC_S);
+                umma_commit(&s_full[sb]);
+                if (x.j == x.it.npages - 1) umma_commit(q_empty);
             }
-            umma_commit(drain);
+            return true;
+        };
+        auto issue_pv = [&](const PageCursor& x) -> bool {
+            const uint32_t pb = x.cs % NPB, sv = x.cs % NSV;
+            const bool first = x.j == 0;
+            if (!wait_bcast(&p_full[pb], (x.cs / NPB) & 1u, abort_flag, a.status, lane)) return false;
+            if (!wait_bcast(&v_full[sv], (x.cs / NSV) & 1u, abort_flag, a.status, lane)) return false;
+            if (first && !wait_bcast(o_free, (x.ni & 1u) ^ 1u, abort_flag, a.status, lane)) return false;
+            tc_fence_after();
+            const uint64_t ad = vd0 + ((sv * HALF_PAGE) >> 4);
+            const uint64_t bd = pd0 + ((pb * C::PB) >> 4);
+            const uint32_t d = tmem + C::O_COL;
+            if (elect_one()) {
+                if (first) umma_bf16_c<false>(d, ad, bd, C::IDESC_PV);
+                else umma_bf16_c<true>(d, ad, bd, C::IDESC_PV);
+#pragma unroll
+                for (int kk = 1; kk < ROWS / 16; ++kk)
+                    umma_bf16_c<true>(d, ad + (uint64_t)((kk * 2048) >> 4),
+                                      bd + (uint64_t)(((kk >> 2) * (NQ * 128) + (kk & 3) * 32) >> 4), C::IDESC_PV);
+                umma_commit(&pv_done[pb]);
+            }
+            return true;
+        };
+        while (ok && pc.valid) {
+            while (ok && sc.valid && sc.cs <= pc.cs + (uint32_t)C::LOOK) {
+                // the first page of a later request waits for its Q only when P V has nothing to do
+                if (sc.j == 0 && sc.cs > pc.cs && !test_bcast(q_full, sc.ni & 1u, lane)) break;
+                ok = issue_s(sc);
+                cursor_next(sc, a, hi);
+            }
+            if (!ok) break;
+            ok = issue_pv(pc);
+            cursor_next(pc, a, hi);
+        }
+        if (elect_one()) umma_commit(drain);
+        __syncwarp();
+        if (lane == 0) {
             volatile int quiet = 0;
             mbar_wait(drain, 0, &quiet, nullptr);
         }
@@ -262,18 +348,24 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int i = 0; i < G; ++i) { m[i] = -INFINITY; lp[i] = 0.f; }
             for (int c = 0; c < it.npages; ++c, ++cs) {
-                const uint32_t sb = cs & 1u;
-                bool okc = wait_bcast(&s_full[sb], (cs >> 1) & 1u, abort_flag, a.status, lane);
+                const uint32_t sb = cs % NSB;
+                bool okc = wait_bcast(&s_full[sb], (cs / NSB) & 1u, abort_flag, a.status, lane);
                 float sw[2 * G];  // scores of the warp's two heads' query columns
 #pragma unroll
                 for (int i = 0; i < 2 * G; ++i) sw[i] = -INFINITY;
                 if (okc) {
                     tc_fence_after();
+                    // the 2G score columns of this warp's two heads (constant indices in both
+                    // branches keep tmp in registers)
                     float tmp[16];
                     tmem_ld16(tmem + lane_addr + sb * NQ + ((2 * q * G) & ~15), tmp);
-                    const int off = (2 * q * G) & 15;
+                    if (((2 * q * G) & 15) != 0) {
 #pragma unroll
-                    for (int i = 0; i < 2 * G; ++i) sw[i] = tmp[(off + i) & 15];
+                        for (int i = 0; i < 2 * G && i + 8 < 16; ++i) sw[i] = tmp[i + 8];
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 2 * G; ++i) sw[i] = tmp[i];
+                    }
                     tc_fence_before();
                 }
                 __syncwarp();
@@ -307,17 +399,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                         }
                         bar_sync_n(2, 128);
                         // the previous page's P V must have landed in O^T before it is rescaled
-                        okc = okc && wait_bcast(&pv_done[(cs - 1) & 1u], ((cs - 1) >> 1) & 1u, abort_flag,
+                        okc = okc && wait_bcast(&pv_done[(cs - 1) % NPB], ((cs - 1) / NPB) & 1u, abort_flag,
                                                 a.status, lane);
                         if (okc) {
                             tc_fence_after();
 #pragma unroll
                             for (int c16 = 0; c16 < NQ / 16; ++c16) {
                                 float o[16];
-                                tmem_ld16(tmem + lane_addr + 2 * NQ + c16 * 16, o);
+                                tmem_ld16(tmem + lane_addr + C::O_COL + c16 * 16, o);
 #pragma unroll
                                 for (int i = 0; i < 16; ++i) o[i] *= cfs[c16 * 16 + i];
-                                tmem_st16(tmem + lane_addr + 2 * NQ + c16 * 16, o);
+                                tmem_st16(tmem + lane_addr + C::O_COL + c16 * 16, o);
                             }
                             tc_fence_before();
                         }
@@ -325,8 +417,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
                 // P entries of this row (its G query heads) into this page's P buffer
-                const uint32_t pb = cs & 1u;
-                if (cs >= 2) okc = okc && wait_bcast(&pv_done[pb], ((cs - 2) >> 1) & 1u, abort_flag, a.status, lane);
+                const uint32_t pb = cs % NPB;
+                if (cs >= (uint32_t)NPB)
+                    okc = okc && wait_bcast(&pv_done[pb], ((cs - NPB) / NPB) & 1u, abort_flag, a.status, lane);
                 if (okc) {
                     uint8_t* pbuf = smem + C::OFF_P + pb * C::PB + (t >> 6) * (NQ * 128);
 #pragma unroll
@@ -336,14 +429,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                         *reinterpret_cast<__nv_bfloat16*>(pbuf + sw128_offset(h * G + i, t & 63)) =
                             __float2bfloat16_rn(p);
                     }
-                    if (c * 16 + k >= it.nkeys) {
-                        // V row of a key past the request: zero it so that 0 * garbage cannot occur
-                        uint8_t* vrow = smem + (cs % NS) * PAGE_BYTES + 2 * REGION + t * 128;
+                    if ((it.nkeys & 15) != 0 && c == it.npages - 1) {  // CTA-uniform
+                        // V rows of keys past the request in the last page: zero them (once the
+                        // V half has landed) so that 0 * garbage cannot occur in P V
+                        okc = okc && wait_bcast(&v_full[cs % NSV], (cs / NSV) & 1u, abort_flag, a.status, lane);
+                        if (okc && c * 16 + k >= it.nkeys) {
+                            uint8_t* vrow = smem + C::OFF_V + (cs % NSV) * HALF_PAGE + t * 128;
 #pragma unroll
-                        for (int b = 0; b < 2; ++b)
+                            for (int b = 0; b < 2; ++b)
 #pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                reinterpret_cast<uint4*>(vrow + b * REGION)[i] = make_uint4(0u, 0u, 0u, 0u);
+                                for (int i = 0; i < 8; ++i)
+                                    reinterpret_cast<uint4*>(vrow + b * REGION)[i] = make_uint4(0u, 0u, 0u, 0u);
+                        }
                     }
                 }
                 fence_proxy_async_smem();
@@ -360,7 +457,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
                 if (k == 0) cfs[h * G + i] = x;
             }
-            bool okc = wait_bcast(&pv_done[(cs - 1) & 1u], ((cs - 1) >> 1) & 1u, abort_flag, a.status, lane);
+            bool okc = wait_bcast(&pv_done[(cs - 1) % NPB], ((cs - 1) / NPB) & 1u, abort_flag, a.status, lane);
             bar_sync_n(2, 128);
             uint16_t* ob = a.out + (size_t)it.r * NQ * 128 + t;  // thread t writes d = t of every head
             if (okc) tc_fence_after();
@@ -370,7 +467,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                 for (int i = 0; i < 16; ++i) o[i] = 0.f;
                 if (okc) {
-                    tmem_ld16(tmem + lane_addr + 2 * NQ + c16 * 16, o);
+                    tmem_ld16(tmem + lane_addr + C::O_COL + c16 * 16, o);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) ob[(size_t)(c16 * 16 + i) * 128] = f2bf(o[i] / cfs[c16 * 16 + i]);
                 }
