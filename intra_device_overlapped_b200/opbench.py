@@ -1,0 +1,94 @@
+"""Time one operation of the serving iteration alone, through the C ABI.
+
+    python -m intra_device_overlapped_b200.opbench --op decode_attention --workload llama3_8b_layer \
+        --requests 64 --sm 16 --reps 5
+
+Ops: ``decode_attention`` (requests [0, --requests) of the workload's decode batch, KV read from the
+paged pool), ``prefill_attention`` (the workload's prefill chunk), ``gemm`` (--m x --n x --k bf16,
+random operands). ``--sm`` is the persistent grid (0 = every SM). The printed line holds the mean
+launch time over --reps launches (CUDA events on the launching stream, after --warmup launches) and
+the algorithmic bytes or FLOPs of one launch, so that a profiler can target a small, known case.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import numpy as np
+import torch
+
+from . import check, nf_op_decode_attention, nf_op_gemm_bf16, nf_op_prefill_attention
+
+
+def _time(launch, reps: int, warmup: int, stream) -> float:
+    for _ in range(warmup):
+        launch()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        launch()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1000.0 / reps
+
+
+def main(argv=None) -> dict:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--op", choices=["decode_attention", "prefill_attention", "gemm"], required=True)
+    ap.add_argument("--workload", default="llama3_8b_layer")
+    ap.add_argument("--requests", type=int, default=0, help="decode requests (0 = all)")
+    ap.add_argument("--sm", type=int, default=0)
+    ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=2)
+    ap.add_argument("--m", type=int, default=1536)
+    ap.add_argument("--n", type=int, default=4096)
+    ap.add_argument("--k", type=int, default=4096)
+    args = ap.parse_args(argv)
+    dev = "cuda:0"
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    out = {"op": args.op, "sm": args.sm}
+
+    if args.op == "gemm":
+        M, N, K = args.m, args.n, args.k
+        g = torch.Generator(device=dev).manual_seed(0)
+        a = torch.randn((M, K), device=dev, generator=g).to(torch.bfloat16)
+        b = (torch.randn((N, K), device=dev, generator=g) * 0.02).to(torch.bfloat16)
+        c = torch.empty((M, N), dtype=torch.float32, device=dev)
+        us = _time(lambda: check(nf_op_gemm_bf16(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, args.sm,
+                                                 stream.cuda_stream), "gemm"), args.reps, args.warmup, stream)
+        out.update({"shape": [M, N, K], "us": round(us, 2), "tflops": round(2.0 * M * N * K / us / 1e6, 1)})
+    else:
+        from synth.workloads import WORKLOADS
+        from .harness import DeviceWorkload
+        w = WORKLOADS[args.workload]
+        dw = DeviceWorkload(w, dev, keep_logits=False)
+        s, bt = w.shape, dw.batch
+        q = torch.zeros((dw.T, s.n_q_heads, s.head_dim), dtype=torch.bfloat16, device=dev)
+        o = torch.zeros_like(q)
+        if args.op == "decode_attention":
+            R = args.requests or bt.num_decode
+            pages = sum(-(-(int(c) + 1) // s.page_size) for c in bt.ctx_lens[:R])
+            nbytes = pages * 2 * s.n_kv_heads * s.page_size * s.head_dim * 2
+            us = _time(lambda: check(nf_op_decode_attention(dw.model, q.data_ptr(), o.data_ptr(), dw.io, 0, 0, R,
+                                                            args.sm, stream.cuda_stream), "decode"),
+                       args.reps, args.warmup, stream)
+            out.update({"workload": args.workload, "requests": R, "kv_bytes": nbytes, "us": round(us, 2),
+                        "gbs": round(nbytes / us / 1e3, 1)})
+        else:
+            R, C = bt.num_decode, bt.prefill_len
+            flops = 4.0 * s.n_q_heads * s.head_dim * C * (C + 1) / 2
+            us = _time(lambda: check(nf_op_prefill_attention(dw.model, q.data_ptr(), o.data_ptr(), dw.io, 0, R, C,
+                                                             args.sm, stream.cuda_stream), "prefill"),
+                       args.reps, args.warmup, stream)
+            out.update({"workload": args.workload, "chunk": C, "flops": flops, "us": round(us, 2),
+                        "tflops": round(flops / us / 1e6, 2)})
+        check(dw.sync(), "status")
+        dw.close()
+    print(json.dumps(out), flush=True)
+    return out
+
+
+if __name__ == "__main__":
+    main()
