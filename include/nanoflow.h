@@ -299,6 +299,41 @@ nf_status nf_op_prefill_attention(nf_model* m, const void* q, void* out, const n
  * outcome) after the kernel has given up and exited, or NF_OK if the flag was set. */
 nf_status nf_op_wait_flag_test(int32_t* flag_device, uint64_t limit_ns, void* stream);
 
+/* Largest num_requests nf_decode_attention_noalloc accepts (size of its static scratch). */
+#define NF_NOALLOC_MAX_REQUESTS 16384
+
+/* Decode attention that allocates nothing. The paper has no counterpart: this entry point
+ * exists for callers that cannot allocate device memory where they call it (code between
+ * the capture calls of a CUDA graph, allocator-free runtimes, processes whose device memory
+ * all belongs to their own pool), and therefore cannot create an nf_model.
+ *
+ * Computes, for each decode request r < num_requests and query head h, the softmax
+ * attention of q[r][h] over the ctx_len[r] + 1 cached keys of KV head h / (nq / nkv),
+ * gathered through the page table (the operation nf_forward_iteration runs as its decode
+ * attention step), with the same tensor-core kernel as nf_op_decode_attention.
+ *   q, out        device bf16 [num_requests x n_q_heads x head_dim], row r = request r.
+ *   kv_pool       device bf16 pool of one layer, num_pages pages in the physical page layout
+ *                 described for nf_iter_io.kv_pools.
+ *   ctx_len       device int32 [num_requests]; page_indptr device int32 [num_requests + 1];
+ *   page_indices  device int32 (CSR page table; request r owns page_indices[page_indptr[r] ..]).
+ *   sm_count      persistent grid (0 = every SM).
+ *   status_device optional device int32 the caller zeroes; receives the first device-detected
+ *                 error (NF_ERR_DEVICE_BOUNDS for a page index outside the pool,
+ *                 NF_ERR_DEVICE_TIMEOUT for a pipeline wait that passed its limit). NULL: the
+ *                 errors go to the library's scratch only.
+ * Supported shapes: head_dim 128, n_kv_heads 8, n_q_heads 32 or 64 (else NF_ERR_UNSUPPORTED).
+ * num_requests > NF_NOALLOC_MAX_REQUESTS returns NF_ERR_INVALID_ARGUMENT.
+ * Scratch: a static device array of 66 KB per device (status word and the per-request page
+ * prefix), shared by every call: calls that overlap on the GPU race on it and must be
+ * serialised. The first call on each device looks up the array's address
+ * (cudaGetSymbolAddress); make that first call before any stream capture. Asynchronous on
+ * `stream`; no call allocates device or pinned memory. */
+nf_status nf_decode_attention_noalloc(const void* q, void* out, const void* kv_pool, int32_t num_pages,
+                                      const int32_t* ctx_len, const int32_t* page_indptr,
+                                      const int32_t* page_indices, int32_t num_requests, int32_t n_q_heads,
+                                      int32_t n_kv_heads, int32_t head_dim, int32_t sm_count,
+                                      int32_t* status_device, void* stream);
+
 /* Library version string. */
 const char* nf_version(void);
 

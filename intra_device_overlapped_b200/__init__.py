@@ -133,6 +133,8 @@ def _load():
         "nf_op_decode_attention": ([_vp, _vp, _vp, P(nf_iter_io), _i32, _i32, _i32, _i32, _vp], ctypes.c_int),
         "nf_op_prefill_attention": ([_vp, _vp, _vp, P(nf_iter_io), _i32, _i32, _i32, _i32, _vp], ctypes.c_int),
         "nf_op_wait_flag_test": ([_vp, _u64, _vp], ctypes.c_int),
+        "nf_decode_attention_noalloc": ([_vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp],
+                                        ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -146,7 +148,20 @@ EXPORTED = ("nf_status_string", "nf_version", "nf_init_model", "nf_set_layer_wei
             "nf_destroy_model", "nf_plan_iteration", "nf_plan_for_config", "nf_forward_iteration", "nf_sync_status", "nf_calibrate",
             "nf_get_cost_model", "nf_set_cost_model",
             "nf_set_trace", "nf_get_trace", "nf_set_timing", "nf_get_op_times", "nf_op_gemm_bf16", "nf_op_decode_attention",
-            "nf_op_prefill_attention", "nf_op_wait_flag_test")
+            "nf_op_prefill_attention", "nf_op_wait_flag_test", "nf_decode_attention_noalloc")
+
+
+NF_NOALLOC_MAX_REQUESTS = 16384
+
+
+def nf_decode_attention_noalloc(q_ptr: int, out_ptr: int, kv_pool_ptr: int, num_pages: int, ctx_len_ptr: int,
+                                page_indptr_ptr: int, page_indices_ptr: int, num_requests: int, n_q_heads: int,
+                                n_kv_heads: int, head_dim: int, sm_count: int = 0, status_ptr: int = 0,
+                                stream: int = 0) -> int:
+    """Decode attention from plain device pointers; allocates nothing (static scratch, see nanoflow.h)."""
+    return _lib.nf_decode_attention_noalloc(q_ptr, out_ptr, kv_pool_ptr, num_pages, ctx_len_ptr, page_indptr_ptr,
+                                            page_indices_ptr, num_requests, n_q_heads, n_kv_heads, head_dim,
+                                            sm_count, status_ptr or None, stream or None)
 
 
 class NanoflowError(RuntimeError):
