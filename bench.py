@@ -141,6 +141,16 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- work accounting
 
+# DRAM bytes (read + write) per algorithmic byte of a kernel, from one ncu capture of that
+# kernel as it stands; the bench scales it to its own launches (traffic grows with the pages
+# read). Entries must be retaken whenever the kernel changes.
+TRAFFIC_PER_ALGO_BYTE = {
+    # decode_attention_tc_kernel<32>, 64 requests of llama3_8b_layer on 16 SMs:
+    # dram__bytes_read.sum 337.785 MB + dram__bytes_write.sum 5.414 MB for 338.166 MB of
+    # algorithmic bytes (337.117 MB of pages + 1.049 MB of q and o)
+    "decode_attention": (1.0149, "ncu: decode_attention_tc_kernel<32>, 64 of 512 requests, 16 SMs, scaled by pages"),
+}
+
 def iteration_flops(work, batch):
     """GEMM FLOPs + attention matmul FLOPs of one iteration (compute-bound optimum numerator)."""
     s = work.shape
@@ -189,15 +199,17 @@ def op_algorithmic(work, batch, plan, op, nano):
 
 
 def count_launches(work, plan):
+    """Kernels this library launches per iteration (checked against the ncu launch list)."""
     s = work.shape
     R = plan.num_decode
-    per_step = 2 if R > 0 else 1          # decode schedule + residual set-up (or embedding)
+    tc = s.head_dim == 128 and s.n_kv_heads == 8 and s.n_q_heads in (32, 64)
+    per_step = 1                          # residual set-up (or embedding)
+    if R > 0:
+        per_step += 1 if tc else 2        # decode schedule (+ split-item table on the warp-level path)
     for j in range(plan.n_nano):
         t0, t1 = plan.tok_begin[j], plan.tok_end[j]
-        att = (2 if min(t1, R) > min(t0, R) else 0) + (1 if t1 > R and plan.prefill_len else 0)
-        ffn = 6 if s.n_experts else 2      # route+sort, gather, 2 grouped GEMMs, combine
-        if s.n_experts:
-            ffn = 6
+        att = (1 if min(t1, R) > min(t0, R) else 0) + (1 if t1 > R and plan.prefill_len else 0)
+        ffn = 6 if s.n_experts else 2      # MoE: route+sort, gather, 2 grouped GEMMs, combine
         per_step += s.n_layers * (1 + att + 1 + ffn)
     if s.vocab:
         per_step += 3
@@ -343,8 +355,13 @@ def run_ours(args, work, dist):
             peak = hbm_gbs
             achieved = per_launch / (avg_us * 1e-6) / 1e9
             unit = "GB/s"
+        traffic, traffic_src = None, None
+        if dominant in TRAFFIC_PER_ALGO_BYTE and a["bound"] == "hbm":
+            ratio, traffic_src = TRAFFIC_PER_ALGO_BYTE[dominant]
+            traffic = int(round(per_launch * ratio))
         roofline = {"kernel": dominant, "bound": a["bound"], "achieved": round(achieved, 1), "peak": peak,
-                    "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
+                    "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
+                    "traffic_unit": "bytes per launch", "traffic_source": traffic_src,
                     "avg_launch_us": round(avg_us, 2), "launches_per_step": a["launches"] / args.steps,
                     "peak_source": f"{peak_src} (burst)"}
     op_summary = {k: {"avg_us": round(v["us"] / v["launches"], 1), "launches": v["launches"],

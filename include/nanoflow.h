@@ -16,8 +16,8 @@
  * nano-batches and duplicates each operation per nano-batch so that operations
  * of different nano-batches no longer depend on one another (arXiv abstract of
  * "NanoFlow: Towards Optimal Large Language Model Serving Throughput"; README
- * "Abstract"). A "device-level pipeline with execution unit scheduling" then
- * runs the compute-bound GEMMs of one nano-batch on one part of the GPU while
+ * "Abstract"). A pipeline inside the device then assigns execution units so that
+ * the compute-bound GEMMs of one nano-batch run on one part of the GPU while
  * the memory-bound attention of another runs on the rest (README
  * "Introduction" and "Abstract"). The number, size, order and GPU resource
  * split of the nano-batches are chosen automatically, taking interference into
@@ -174,8 +174,9 @@ typedef struct {
 
 /* Choose nano-batch count, sizes (token ranges cut at request boundaries, the
  * prefill chunk whole), op order and SM split minimising the simulated two-stream
- * makespan over the model's per-kernel cost tables (arXiv abstract: "number,
- * size, ordering, and GPU resource allocation of nano-batches"). Host only. */
+ * makespan over the model's per-kernel cost tables (arXiv abstract: the search
+ * covers the count, size and order of nano-batches and their share of the GPU).
+ * Host only. */
 nf_status nf_plan_iteration(const nf_model* m, const nf_batch_desc* b, const nf_plan_opts* opts, nf_plan* out);
 
 /* The same search for a model configuration without a device or a model handle:

@@ -1,9 +1,10 @@
 // Planner: nano-batch count, sizes, pipeline order and SM split by exhaustive search
 // over a per-kernel cost model, replacing the external MILP solver of the reference
-// design. NanoFlow "automatically identifies the number, size, ordering, and GPU
-// resource allocation of nano-batches to minimize the execution time, while
-// considering the interference of concurrent operations" (arXiv abstract; README
-// "Abstract": a parameter search algorithm sets up the pipeline).
+// design. NanoFlow picks how many nano-batches to use, how large each is, the order
+// of their operations and how the GPU is divided between them so that the iteration
+// is shortest, taking into account how concurrent operations slow one another
+// (arXiv abstract; README "Abstract": an offline parameter search configures the
+// pipeline).
 //
 // Candidates: n in 1..4 nano-batches; decode rows cut at request boundaries into
 // groups of equal KV bytes; the prefill chunk either its own nano-batch or joined to

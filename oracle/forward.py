@@ -15,9 +15,9 @@ is the standard Llama / Mixtral layer, written out here step by step:
     x' = h + (silu(n2 Wg^T) * (n2 Wu^T)) Wd^T     dense SwiGLU, or
     x' = h + sum_k w_k E_{i_k}(n2)                top-k mixture of SwiGLU experts
 
-NanoFlow's nano-batching "splits inputs into smaller nano-batches and
-duplicates operations to operate on each portion independently" (arXiv
-abstract): a schedule, not an approximation. The oracle therefore computes the
+NanoFlow's nano-batching cuts the batch into smaller pieces and runs a copy of
+each operation on every piece on its own (arXiv abstract of the NanoFlow paper):
+a schedule, not an approximation. The oracle therefore computes the
 unsplit batch; every nano-batch plan must reproduce it.
 """
 from __future__ import annotations
