@@ -261,7 +261,11 @@ def run_reference(args, work, dist):
         return
     from synth.workloads import make_batch
     batch = make_batch(work)
-    n = args.cpu_sample or min(128, batch.num_decode)
+    # each step is a bounded sample of decode requests, sized from a timed probe of 4 requests
+    # so that the warm-up and timed steps together take about 90 s of host time
+    probe, _ = cpu_oracle_sample(work, batch, min(4, batch.num_decode), repeats=1)
+    per_req = probe[0] / min(4, batch.num_decode)
+    n = args.cpu_sample or int(max(1, min(128, batch.num_decode, 90.0 / ((args.steps + args.warmup) * per_req))))
     cpu_oracle_sample(work, batch, n, repeats=max(1, args.warmup))  # warm-up
     times, threads = cpu_oracle_sample(work, batch, n, repeats=args.steps)
     tot = sum(times)
