@@ -160,6 +160,7 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) {
     m->cost = nf::default_cost_model(m->sm_count);
     m->layers.resize(d.L);
     m->decode_tc = nf::decode_tc_supported(d.nq, d.nkv, d.d);
+    m->prefill_tc = nf::prefill_tc_supported(d.d);
 
     const size_t T = (size_t)cfg->max_tokens;
     const size_t TK = T * (size_t)d.K;
@@ -227,6 +228,7 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) {
          nf::make_tmap_bf16_2d(&m->tm_act, m->act, act_rows, d.F, nf::kGemmBM);
     if (ok && cfg->vocab > 0) ok = nf::make_tmap_bf16_2d(&m->tm_lm_in, m->lm_in, lm_rows, d.H, nf::kGemmBM);
     if (ok && m->decode_tc) ok = nf::make_tmap_bf16_2d(&m->tm_q, m->q, T * d.nq, d.d, (uint32_t)d.nq);
+    if (ok && m->prefill_tc) ok = nf::make_tmap_bf16_3d_heads(&m->tm_q3, m->q, T, d.nq, d.d, 128);
     if (ok && d.E > 0) ok = nf::make_tmap_bf16_2d(&m->tm_moe_a, m->moe_a, TK, d.H, nf::kGemmBM);
     if (!ok) { nf_destroy_model(m); return NF_ERR_CUDA; }
     *out = m;
@@ -418,6 +420,16 @@ cudaError_t launch_decode(nf_model* m, const nf_iter_io* io, const CUtensorMap& 
     return nf::launch_decode_attention(da, m->dims.d, grid, s);
 }
 
+// Prefill attention of layer `layer` reading q (rows [0, tokens), tensor map tmq3 when the
+// tensor-core kernel applies) and writing out.
+cudaError_t launch_prefill(nf_model* m, const nf_iter_io* io, const CUtensorMap& tmq3, const void* q, void* out,
+                           int layer, int R, int C, int grid, cudaStream_t s) {
+    nf::PrefillArgs pa = prefill_args(m, io, q, out, R, C);
+    pa.kv_pool = (const uint16_t*)io->kv_pools[layer];
+    if (m->prefill_tc) return nf::launch_prefill_attention_tc(tmq3, pa, grid, s);
+    return nf::launch_prefill_attention(pa, m->dims.d, grid, s);
+}
+
 nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::Op& op, int grid,
                  cudaStream_t s) {
     const nf::ModelDims& d = m->dims;
@@ -455,11 +467,7 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
             return NF_OK;
         }
         case nf::OP_PATT: {
-            if (t1 > R && C > 0) {
-                nf::PrefillArgs pa = prefill_args(m, io, m->q, m->attn_o, R, C);
-                pa.kv_pool = (const uint16_t*)io->kv_pools[l];
-                NF_CUDA_TRY(nf::launch_prefill_attention(pa, d.d, grid, s));
-            }
+            if (t1 > R && C > 0) NF_CUDA_TRY(launch_prefill(m, io, m->tm_q3, m->q, m->attn_o, l, R, C, grid, s));
             return NF_OK;
         }
         case nf::OP_O: {
@@ -792,9 +800,12 @@ extern "C" nf_status nf_op_prefill_attention(nf_model* m, const void* q, void* o
     nf_status st = check_pool(m, layer, io);
     if (st != NF_OK) return st;
     const int grid = sm_count > 0 ? std::min(sm_count, m->sm_count) : m->sm_count;
-    nf::PrefillArgs pa = prefill_args(m, io, q, out, num_decode, prefill_len);
-    pa.kv_pool = (const uint16_t*)io->kv_pools[layer];
-    NF_CUDA_TRY(nf::launch_prefill_attention(pa, m->dims.d, grid, (cudaStream_t)stream));
+    CUtensorMap tmq3;
+    std::memset(&tmq3, 0, sizeof(tmq3));
+    if (m->prefill_tc && !nf::make_tmap_bf16_3d_heads(&tmq3, q, (uint64_t)num_decode + prefill_len, m->dims.nq,
+                                                      m->dims.d, 128))
+        return NF_ERR_INVALID_ARGUMENT;
+    NF_CUDA_TRY(launch_prefill(m, io, tmq3, q, out, layer, num_decode, prefill_len, grid, (cudaStream_t)stream));
     return NF_OK;
 }
 
@@ -935,9 +946,7 @@ extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_
         const int q = std::max(8, S / 4);
         double t_p = 0;
         auto pre = [&]() -> nf_status {
-            nf::PrefillArgs pa = prefill_args(m, io, m->q, m->attn_o, R, C);
-            pa.kv_pool = (const uint16_t*)io->kv_pools[0];
-            return nf::launch_prefill_attention(pa, d.d, q, sg) == cudaSuccess ? NF_OK : NF_ERR_CUDA;
+            return launch_prefill(m, io, m->tm_q3, m->q, m->attn_o, 0, R, C, q, sg) == cudaSuccess ? NF_OK : NF_ERR_CUDA;
         };
         if ((st = time_us(sg, 3, pre, &t_p)) != NF_OK) return st;
         const double flops = 4.0 * d.nq * d.d * (double)C * (C + 1) / 2.0;

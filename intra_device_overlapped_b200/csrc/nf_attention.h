@@ -69,4 +69,10 @@ cudaError_t launch_prefill_attention(const PrefillArgs& a, int head_dim, int gri
 bool decode_tc_supported(int nq, int nkv, int head_dim);
 cudaError_t launch_decode_attention_tc(const CUtensorMap& tmQ, const DecodeArgs& a, int grid, cudaStream_t stream);
 
+// Tensor-core (tcgen05) causal attention of the prefill chunk for head dim 128 (any G):
+// 128 query positions of one head per unit; tmQ maps q as [tokens][nq][128] (3-D, boxes of
+// 64 x 1 x 128).
+bool prefill_tc_supported(int head_dim);
+cudaError_t launch_prefill_attention_tc(const CUtensorMap& tmQ, const PrefillArgs& a, int grid, cudaStream_t stream);
+
 }  // namespace nf

@@ -70,6 +70,10 @@ struct GemmArgs {
 // Encode a 2-D bf16 tensor map over a row-major [rows x cols] matrix with a box of
 // box_rows x 64 columns and 128-byte swizzle. Returns false on failure.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// [tokens][heads][head_dim] bf16 viewed as a 3-D map with boxes of 64 elements x 1 head x
+// box_tokens tokens (128-byte swizzle): one head's rows of consecutive tokens.
+bool make_tmap_bf16_3d_heads(CUtensorMap* map, const void* base, uint64_t tokens, uint64_t heads, uint64_t head_dim,
+                             uint32_t box_tokens);
 
 cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args, int grid,
                         cudaStream_t stream);

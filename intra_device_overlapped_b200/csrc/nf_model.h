@@ -69,6 +69,8 @@ struct nf_model {
     CUtensorMap tm_xb, tm_attn_o, tm_act, tm_lm_in, tm_moe_a;
     CUtensorMap tm_q;             // q as [T * nq rows x d], nq-row boxes (tensor-core decode attention Q loads)
     bool decode_tc = false;       // the tensor-core decode kernel handles this model's head shape
+    CUtensorMap tm_q3;            // q as [T][nq][d], 128-token boxes of one head (tensor-core prefill Q loads)
+    bool prefill_tc = false;      // the tensor-core prefill kernel handles this model's head dim
 
     int* status = nullptr;        // device status word
     int* trace_ctr = nullptr;

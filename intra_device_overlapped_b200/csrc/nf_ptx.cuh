@@ -111,6 +111,15 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 
 // 2-D tiled bulk tensor load global -> shared, completion counted on `bar` (bytes).
 // x is the innermost coordinate (element index); callers keep x * 2 bytes 16-byte aligned.
+// 3-D tiled bulk tensor load; x (innermost) * 2 bytes must be 16-byte aligned.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
@@ -172,6 +181,11 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
 // Instruction descriptor of kind::f16: bf16 A and B (K-major), fp32 accumulator.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Same with B MN-major (bit 16): B is stored with its N dimension contiguous.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32_bmn(int M, int N) {
+    return umma_idesc_bf16_f32(M, N) | (1u << 16);
 }
 
 // Same with A MN-major (bit 15): A is stored with its M dimension contiguous.
@@ -322,6 +336,14 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
     uint32_t d;
     asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
     return d;
+}
+
+// 2^x by the hardware approximation (relative error about 2^-22; 2^-inf = 0, flushes
+// subnormal results to zero). Used for softmax weights that are rounded to bf16 afterwards.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
