@@ -303,7 +303,11 @@ def run_ours(args, work, dist):
     dw = DeviceWorkload(work, dev, keep_logits=False)
     b = dw.batch
     cost = dw.calibrate()
-    plan = dw.plan(nano=args.nano, sm_attn=args.sm_attn, template=args.template)
+    forced = args.nano > 0 or args.sm_attn > 0 or args.template >= 0
+    if forced:
+        plan = dw.plan(nano=args.nano, sm_attn=args.sm_attn, template=args.template)
+    else:  # the planner's candidates measured on this batch, fastest kept (nf_tune_plan)
+        plan, _ = dw.tune(reps=5)
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(max(args.warmup, 3)):
@@ -458,6 +462,8 @@ def run_ours(args, work, dist):
             "config": {"workload": args.workload, "decode_requests": R, "prefill_len": b.prefill_len,
                        "tokens": b.num_tokens, "ctx": "uniform [1024,1536]" if args.workload.startswith("llama") else "",
                        "parallelism": f"replicas x{dist.world}", "plan": plan.describe(),
+                       "plan_choice": "forced on the command line" if forced else
+                       "planner candidates timed on this batch (nf_tune_plan), fastest kept",
                        "l2": "working set (KV cache + weights) > 126 MB L2 on every step; no flush"},
             "frac_of_compute_optimum": round(t_opt_ms / ms_step, 4),
             "t_opt_ms": round(t_opt_ms, 4), "iteration_tflop": round(flops / 1e12, 4),

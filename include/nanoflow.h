@@ -194,7 +194,10 @@ typedef struct {
     const int32_t* ctx_len;      /* [R] */
     const int32_t* page_indptr;  /* [R + 2] */
     const int32_t* page_indices; /* [page_indptr[R+1]] page ids < num_pages */
-    void* const* kv_pools;       /* host array [n_layers]: device [num_pages][2][nkv][16][d] bf16, updated in place */
+    void* const* kv_pools;       /* host array [n_layers]: device pool of num_pages pages, updated in place.
+                                  * Page layout (bf16): [K|V][half of d (64 columns)][KV head][16 slots]
+                                  * [8 chunks of 8 columns], logical chunk c of slot r stored at c ^ (r % 8);
+                                  * one page holds 2 * nkv * 16 * d elements. */
     int32_t num_pages;
     void* hidden_out;            /* [T x H] bf16, nullable */
     float* hidden_out_f32;       /* [T x H] fp32 residual stream after the last layer, nullable */
@@ -203,12 +206,26 @@ typedef struct {
     int32_t* topk_idx;           /* MoE: [n_layers x T x top_k] expert ids, nullable */
     float* topk_w;               /* MoE: [n_layers x T x top_k] routing weights, nullable */
     float* router_logits;        /* MoE: [n_layers x T x E] fp32, nullable */
+    float* layer_hidden_out;     /* [n_layers x T x H] fp32 residual stream after each layer, nullable
+                                  * (verification: copied row range by row range as each nano-batch
+                                  * finishes a layer) */
 } nf_iter_io;
 
 /* Run the iteration described by `plan` (made by nf_plan_iteration for the same
  * batch). GEMMs run on `stream`, attention on a model-owned second stream that
  * forks from and joins back into `stream`. Asynchronous. */
 nf_status nf_forward_iteration(nf_model* m, const nf_plan* plan, const nf_iter_io* io, void* stream);
+
+/* Plan choice by measurement. For each template and nano-batch count the planner's best
+ * plan (the SM split chosen by the cost model) is run on this batch: one warm-up and `reps`
+ * timed iterations (CUDA events on `stream`). The fastest plan is written to `out` and its
+ * mean iteration time in microseconds to `best_us` (nullable). This is the search over
+ * measured costs that the arXiv abstract describes, with the final choice between templates
+ * and counts made on the device, where the interference of co-running kernels is real.
+ * Runs nf_forward_iteration with `io` repeatedly: the new tokens' K/V slots are rewritten
+ * with the same values and the outputs are overwritten. Synchronizes `stream`. */
+nf_status nf_tune_plan(nf_model* m, const nf_batch_desc* b, const nf_iter_io* io, int32_t reps, void* stream,
+                       nf_plan* out, float* best_us);
 
 /* Wait for the model's streams and return (and clear) the latched device status. */
 nf_status nf_sync_status(nf_model* m);

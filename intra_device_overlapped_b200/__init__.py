@@ -78,7 +78,8 @@ class nf_iter_io(ctypes.Structure):
     _fields_ = [("token_ids", _vp), ("hidden_in", _vp), ("positions", _vp), ("ctx_len", _vp),
                 ("page_indptr", _vp), ("page_indices", _vp), ("kv_pools", ctypes.POINTER(_vp)),
                 ("num_pages", _i32), ("hidden_out", _vp), ("hidden_out_f32", _vp), ("logits", _vp),
-                ("next_token", _vp), ("topk_idx", _vp), ("topk_w", _vp), ("router_logits", _vp)]
+                ("next_token", _vp), ("topk_idx", _vp), ("topk_w", _vp), ("router_logits", _vp),
+                ("layer_hidden_out", _vp)]
 
 
 class nf_op_time(ctypes.Structure):
@@ -121,6 +122,7 @@ def _load():
         "nf_plan_for_config": ([P(nf_model_config), _i32, P(nf_batch_desc), P(nf_plan_opts), P(nf_plan)],
                                ctypes.c_int),
         "nf_forward_iteration": ([_vp, P(nf_plan), P(nf_iter_io), _vp], ctypes.c_int),
+        "nf_tune_plan": ([_vp, P(nf_batch_desc), P(nf_iter_io), _i32, _vp, P(nf_plan), P(_f32)], ctypes.c_int),
         "nf_sync_status": ([_vp], ctypes.c_int),
         "nf_calibrate": ([_vp, P(nf_batch_desc), P(nf_iter_io), _vp], ctypes.c_int),
         "nf_get_cost_model": ([_vp, P(nf_cost_model)], ctypes.c_int),
@@ -145,7 +147,7 @@ def _load():
 
 _lib = _load()
 EXPORTED = ("nf_status_string", "nf_version", "nf_init_model", "nf_set_layer_weights", "nf_set_global_weights",
-            "nf_destroy_model", "nf_plan_iteration", "nf_plan_for_config", "nf_forward_iteration", "nf_sync_status", "nf_calibrate",
+            "nf_destroy_model", "nf_plan_iteration", "nf_plan_for_config", "nf_forward_iteration", "nf_tune_plan", "nf_sync_status", "nf_calibrate",
             "nf_get_cost_model", "nf_set_cost_model",
             "nf_set_trace", "nf_get_trace", "nf_set_timing", "nf_get_op_times", "nf_op_gemm_bf16", "nf_op_decode_attention",
             "nf_op_prefill_attention", "nf_op_wait_flag_test", "nf_decode_attention_noalloc")
@@ -221,6 +223,15 @@ def nf_plan_for_config(cfg: nf_model_config, sm_count: int, batch: nf_batch_desc
 
 def nf_forward_iteration(model: int, plan: nf_plan, io: nf_iter_io, stream: int = 0) -> int:
     return _lib.nf_forward_iteration(model, ctypes.byref(plan), ctypes.byref(io), stream)
+
+
+def nf_tune_plan(model: int, desc: nf_batch_desc, io: nf_iter_io, reps: int = 5, stream: int = 0):
+    """(status, fastest measured plan, its mean iteration time in us)."""
+    plan = nf_plan()
+    us = ctypes.c_float(0.0)
+    st = _lib.nf_tune_plan(model, ctypes.byref(desc), ctypes.byref(io), reps, stream, ctypes.byref(plan),
+                           ctypes.byref(us))
+    return st, plan, us.value
 
 
 def nf_sync_status(model: int) -> int:

@@ -642,6 +642,15 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
         NF_CUDA_TRY(tm.begin(s));
         if ((st = run_op(m, p, io, op, grid, s)) != NF_OK) return st;
         NF_CUDA_TRY(tm.end(s, kTimingKind[op.kind], op.nano, op.layer, op.stream, grid));
+        if (io->layer_hidden_out && (op.kind == nf::OP_D || op.kind == nf::OP_MOE)) {
+            // the nano-batch's rows have finished this layer: copy them out before any later op
+            // (ordered after this one on this stream or through the event below) changes them
+            const int t0 = p->tok_begin[op.nano], t1 = p->tok_end[op.nano];
+            if (t1 > t0)
+                NF_CUDA_TRY(cudaMemcpyAsync(io->layer_hidden_out + ((size_t)op.layer * T + t0) * d.H,
+                                            m->resid + (size_t)t0 * d.H, (size_t)(t1 - t0) * d.H * 4,
+                                            cudaMemcpyDeviceToDevice, s));
+        }
         if (op.signal) NF_CUDA_TRY(cudaEventRecord(m->events[i], s));
     }
     NF_CUDA_TRY(cudaEventRecord(m->ev_join, sa));
@@ -671,6 +680,59 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     if (io->hidden_out_f32)
         NF_CUDA_TRY(cudaMemcpyAsync(io->hidden_out_f32, m->resid, (size_t)T * d.H * 4, cudaMemcpyDeviceToDevice, sg));
     return NF_OK;
+}
+
+// Search over measured costs: the planner's best plan for every (template, nano-batch count) is
+// run on this batch and timed; the fastest is returned. The simulated cost model ranks plans
+// within a template well but misjudges how much co-running kernels slow one another, so the
+// final choice between templates and counts is made on the device.
+extern "C" nf_status nf_tune_plan(nf_model* m, const nf_batch_desc* b, const nf_iter_io* io, int32_t reps,
+                                  void* stream, nf_plan* out, float* best_us) {
+    if (!m || !b || !io || !out || reps < 1) return NF_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaEvent_t e0 = nullptr, e1 = nullptr;
+    NF_CUDA_TRY(cudaEventCreate(&e0));
+    if (cudaEventCreate(&e1) != cudaSuccess) {
+        cudaEventDestroy(e0);
+        return NF_ERR_CUDA;
+    }
+    nf_status result = NF_ERR_INVALID_ARGUMENT;
+    float best = 0.f;
+    auto try_plan = [&](const nf_plan& p) -> nf_status {
+        nf_status st = nf_forward_iteration(m, &p, io, stream);  // warm-up of this plan's launch shapes
+        if (st != NF_OK) return st;
+        if (cudaEventRecord(e0, s) != cudaSuccess) return NF_ERR_CUDA;
+        for (int r = 0; r < reps; ++r)
+            if ((st = nf_forward_iteration(m, &p, io, stream)) != NF_OK) return st;
+        if (cudaEventRecord(e1, s) != cudaSuccess || cudaEventSynchronize(e1) != cudaSuccess) return NF_ERR_CUDA;
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, e0, e1) != cudaSuccess) return NF_ERR_CUDA;
+        const float us = 1000.f * ms / (float)reps;
+        if (result != NF_OK || us < best) {
+            best = us;
+            *out = p;
+            result = NF_OK;
+        }
+        return NF_OK;
+    };
+    nf_status st = NF_OK;
+    for (int t = NF_TEMPLATE_SEQUENTIAL; t <= NF_TEMPLATE_PREFILL_ON_GEMM && st == NF_OK; ++t) {
+        for (int n = 1; n <= NF_MAX_NANO && st == NF_OK; ++n) {
+            if (t == NF_TEMPLATE_SEQUENTIAL && n > 1) break;  // without overlap, splitting only adds launches
+            nf_plan_opts o;
+            std::memset(&o, 0, sizeof(o));
+            o.force_nano = n;
+            o.force_template = t;
+            nf_plan p;
+            if (nf_plan_iteration(m, b, &o, &p) != NF_OK) continue;  // e.g. more nano-batches than rows allow
+            st = try_plan(p);
+        }
+    }
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    if (st != NF_OK) return st;
+    if (result == NF_OK && best_us) *best_us = best;
+    return result;
 }
 
 extern "C" nf_status nf_sync_status(nf_model* m) {

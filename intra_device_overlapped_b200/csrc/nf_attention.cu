@@ -241,8 +241,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
             const float tA = fmaxf(s[0], s[2]), tB = fmaxf(s[1], s[3]);
             if (__any_sync(0xffffffffu, tA > mA + LAZY || tB > mB + LAZY)) {
                 const float xA = col_max(tA), xB = col_max(tB);
-                const float nA = fmaxf(mA, xA), nB = fmaxf(mB, xB);
-                const float cA = exp2f(mA - nA), cB = exp2f(mB - nB);
+                const float nA = softmax_max_update(mA, xA), nB = softmax_max_update(mB, xB);
+                const float cA = softmax_rescale(mA, nA), cB = softmax_rescale(mB, nB);
                 mA = nA;
                 mB = nB;
                 lA *= cA;
@@ -522,10 +522,10 @@ __global__ void __launch_bounds__(PRE_THREADS, 1)
                 }
                 mx0 = quad_max(mx0);
                 mx1 = quad_max(mx1);
-                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                const float mn0 = softmax_max_update(m0, mx0), mn1 = softmax_max_update(m1, mx1);
                 // rows whose keys in this tile are all masked keep m = -inf: guard the rescale
-                const float c0 = (mn0 == -INFINITY) ? 1.f : exp2f(m0 - mn0);
-                const float c1 = (mn1 == -INFINITY) ? 1.f : exp2f(m1 - mn1);
+                const float c0 = softmax_rescale(m0, mn0);
+                const float c1 = softmax_rescale(m1, mn1);
                 m0 = mn0;
                 m1 = mn1;
                 float ps0 = 0.f, ps1 = 0.f;

@@ -387,8 +387,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                         float x = s[i];
 #pragma unroll
                         for (int o = 8; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-                        const float nm = fmaxf(m[i], x);
-                        cf[i] = (nm == -INFINITY) ? 1.f : exp2f(m[i] - nm);
+                        const float nm = softmax_max_update(m[i], x);
+                        cf[i] = softmax_rescale(m[i], nm);
                         m[i] = nm;
                         lp[i] *= cf[i];
                     }
@@ -431,7 +431,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                     if ((it.nkeys & 15) != 0 && c == it.npages - 1) {  // CTA-uniform
                         // V rows of keys past the request in the last page: zero them (once the
-                        // V half has landed) so that 0 * garbage cannot occur in P V
+                        // V half has landed) so that 0 * garbage cannot occur in P V. The stage's
+                        // previous page (cs - NSV) must have been consumed first: with fewer V stages
+                        // than P buffers nothing else orders it, and until then the parity test
+                        // below could see that page's load as this one's.
+                        if (cs >= (uint32_t)NSV)
+                            okc = okc && wait_bcast(&pv_done[(cs - NSV) % NPB], ((cs - NSV) / NPB) & 1u, abort_flag,
+                                                    a.status, lane);
                         okc = okc && wait_bcast(&v_full[cs % NSV], (cs / NSV) & 1u, abort_flag, a.status, lane);
                         if (okc && c * 16 + k >= it.nkeys) {
                             uint8_t* vrow = smem + C::OFF_V + (cs % NSV) * HALF_PAGE + t * 128;

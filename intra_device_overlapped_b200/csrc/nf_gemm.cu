@@ -134,6 +134,16 @@ __device__ __forceinline__ void store_kv_row32(uint16_t* page, int kv, int g, in
     }
 }
 
+// Warp-uniform wait: every lane tests the phase; if it has not completed, lane 0 waits with
+// the time limit and the outcome is shared.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                          int lane) {
+    if (__all_sync(0xffffffffu, mbar_test_wait(smem_u32(bar), parity))) return true;
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 // ------------------------------------------------------------------ epilogues
 // Each is called by all 32 lanes of an epilogue warp (tcgen05.ld is warp-collective);
 // `valid` says whether this lane's row is inside the tile's row range.
@@ -345,36 +355,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------- MMA issuer
-            uint32_t stage = 0, phase = 0;
-            int local = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++local) {
-                const int acc = local & 1;
-                const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        // ---------------- MMA issuer: the whole warp follows the loop and one elected lane issues,
+        // with the stage's descriptors offset by constants and the accumulate flags fixed per MMA,
+        // so that issue keeps ahead of the tensor core
+        uint32_t stage = 0, phase = 0;
+        int local = 0;
+        bool ok = true;
+        const uint64_t desc0 = umma_desc_sw128(smem_u32(smem));
+        for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++local) {
+            const int acc = local & 1;
+            const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
+            if (!wait_warp(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, lane)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+            for (int kb = 0; kb < p.k_blocks; ++kb) {
+                if (!wait_warp(&full[stage], phase, abort_flag, p.status, lane)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-                    const uint64_t adesc = umma_desc_sw128(sa);
-                    const uint64_t bdesc = umma_desc_sw128(sa + A_BYTES);
+                const uint64_t adesc = desc0 + (uint64_t)((stage * STAGE_BYTES) >> 4);
+                const uint64_t bdesc = adesc + (uint64_t)(A_BYTES >> 4);
+                if (elect_one()) {
+                    // advance 16 bf16 = 32 bytes along K inside the 128-byte swizzle atom
+                    if (kb == 0) umma_bf16_c<false>(d_tmem, adesc, bdesc, IDESC);
+                    else umma_bf16_c<true>(d_tmem, adesc, bdesc, IDESC);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k) {
-                        // advance 16 bf16 = 32 bytes along K inside the 128-byte swizzle atom
-                        umma_bf16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), IDESC,
-                                  (kb | k) != 0 ? 1u : 0u);
-                    }
+                    for (int k = 1; k < BK / 16; ++k)
+                        umma_bf16_c<true>(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), IDESC);
                     umma_commit(&empty[stage]);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                if (ok) umma_commit(&tfull[acc]);
+                __syncwarp();
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
-            // All MMAs issued by this thread have completed once `drain` flips.
-            umma_commit(drain);
+            if (ok) {
+                if (elect_one()) umma_commit(&tfull[acc]);
+                __syncwarp();
+            }
+        }
+        // All MMAs issued by this warp have completed once `drain` flips.
+        if (elect_one()) umma_commit(drain);
+        __syncwarp();
+        if (lane == 0) {
             volatile int quiet = 0;
             mbar_wait(drain, 0, &quiet, nullptr);
         }

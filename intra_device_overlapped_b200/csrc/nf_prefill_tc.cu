@@ -275,8 +275,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * a.scale_log2;
                 const bool need = mx > m + LAZY;
                 if (__any_sync(0xffffffffu, need)) {
-                    const float nm = need ? fmaxf(m, mx) : m;
-                    const float cf = (nm == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - nm);
+                    const float nm = need ? softmax_max_update(m, mx) : m;
+                    const float cf = softmax_rescale(m, nm);
                     if (j > 0) {
                         // the previous key tile's P V must have landed in O before it is rescaled
                         if (!wait_warp(&pv_done[(x - 1) & 1u], ((x - 1) >> 1) & 1u, abort_flag, a.status, lane)) {

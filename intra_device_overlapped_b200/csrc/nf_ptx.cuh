@@ -338,6 +338,16 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
     return d;
 }
 
+// Online softmax in the log2 domain keeps its running maximum m integral: every rescale
+// 2^(m_old - m_new) is then an exact power of two, and the bf16 rounding of P = 2^(s - m)
+// does not depend on which integer m is current (bf16(2^k y) = 2^k bf16(y)).
+__device__ __forceinline__ float softmax_max_update(float m, float x) { return ceilf(fmaxf(m, x)); }
+__device__ __forceinline__ float softmax_rescale(float m_old, float m_new) {
+    if (m_new == -INFINITY) return 1.f;
+    if (m_old == -INFINITY) return 0.f;
+    return ldexpf(1.f, (int)(m_old - m_new));
+}
+
 // 2^x by the hardware approximation (relative error about 2^-22; 2^-inf = 0, flushes
 // subnormal results to zero). Used for softmax weights that are rounded to bf16 afterwards.
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -19,6 +19,7 @@ from synth.workloads import Workload, make_batch
 
 from . import (NF_OK, check, nf_calibrate, nf_get_cost_model, nf_batch_desc, nf_destroy_model, nf_forward_iteration, nf_global_weights,
                nf_init_model, nf_iter_io, nf_layer_weights, nf_model_config, nf_plan_iteration, nf_plan_opts,
+               nf_tune_plan,
                nf_set_global_weights, nf_set_layer_weights, nf_sync_status, nf_set_trace, nf_get_trace)
 
 _vp = ctypes.c_void_p
@@ -46,7 +47,7 @@ class DeviceWorkload:
     """One workload resident on a GPU: model (packed weights), KV pools, inputs and outputs."""
 
     def __init__(self, work: Workload, device: str = "cuda:0", batch=None, keep_logits: bool = True,
-                 moe_debug: bool = False):
+                 moe_debug: bool = False, layer_outputs: bool = False):
         self.work = work
         self.shape = s = work.shape
         self.device = torch.device(device)
@@ -86,6 +87,9 @@ class DeviceWorkload:
             if keep_logits:
                 self.logits = _empty_bf16((self.rows, s.vocab), self.device)
         self.topk_idx = self.topk_w = self.router_logits = None
+        # fp32 residual after every layer (verification of deep stacks layer by layer)
+        self.layer_hidden = (torch.empty((s.n_layers, T, s.hidden), dtype=torch.float32, device=self.device)
+                             if layer_outputs else None)
         if s.n_experts > 0 and moe_debug:
             self.topk_idx = torch.empty((s.n_layers, T, s.top_k), dtype=torch.int32, device=self.device)
             self.topk_w = torch.empty((s.n_layers, T, s.top_k), dtype=torch.float32, device=self.device)
@@ -158,6 +162,7 @@ class DeviceWorkload:
         io.topk_idx = p(self.topk_idx)
         io.topk_w = p(self.topk_w)
         io.router_logits = p(self.router_logits)
+        io.layer_hidden_out = p(self.layer_hidden)
         return io
 
     # -- running ----------------------------------------------------------------------------------
@@ -166,6 +171,13 @@ class DeviceWorkload:
         st, plan = nf_plan_iteration(self.model, self.desc, opts)
         check(st, "nf_plan_iteration")
         return plan
+
+    def tune(self, reps: int = 5, stream: Optional[torch.cuda.Stream] = None):
+        """Fastest plan measured on this batch (nf_tune_plan) and its iteration time in us."""
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        st, plan, us = nf_tune_plan(self.model, self.desc, self.io, reps, s.cuda_stream)
+        check(st, "nf_tune_plan")
+        return plan, us
 
     def forward(self, plan, stream: Optional[torch.cuda.Stream] = None, io: Optional[nf_iter_io] = None) -> None:
         s = stream.cuda_stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
