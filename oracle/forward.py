@@ -19,6 +19,17 @@ NanoFlow's nano-batching cuts the batch into smaller pieces and runs a copy of
 each operation on every piece on its own (arXiv abstract of the NanoFlow paper):
 a schedule, not an approximation. The oracle therefore computes the
 unsplit batch; every nano-batch plan must reproduce it.
+
+Precision. The model runs in bf16 with fp32 accumulation, so every tensor one
+operation hands to the next is a bf16 tensor. With ``bf16_act`` (the default) the
+oracle rounds exactly those tensors to bf16 and computes everything else in
+float64: the operand of each projection is the bf16 copy of the residual stream x
+(RMSNorm's 1/rms and gamma scale the product, so n = bf16(x) / rms(x) * gamma with
+rms taken over the unrounded x); q after RoPE; K and V in the cache; the attention
+output; the SwiGLU activation; and the attention weights that multiply V (see
+``attention``). The residual stream itself, the router logits, the softmax sums and
+all accumulations stay unrounded. With ``bf16_act=False`` nothing but the inputs,
+weights and cache is bf16.
 """
 from __future__ import annotations
 
@@ -69,11 +80,18 @@ def silu(z: np.ndarray) -> np.ndarray:
 
 # --- attention ------------------------------------------------------------------------------------
 
-def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_pos: np.ndarray, k_pos: np.ndarray) -> np.ndarray:
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_pos: np.ndarray, k_pos: np.ndarray,
+              bf16_p: bool = False) -> np.ndarray:
     """Scaled dot-product attention with a position mask (key j visible to query i iff k_pos[j] <= q_pos[i]).
 
     q is [Tq, nq, d]; k, v are [Tk, nkv, d]; query head h reads KV head h // (nq // nkv) (GQA).
     Softmax with max subtraction, all in float64. Returns [Tq, nq, d].
+
+    With bf16_p, the weights that multiply V form a bf16 matrix, as in a bf16 model: in the log2
+    domain x = s * log2(e), P = bf16(2^(x - M)) with M the integer ceiling of the row maximum, and
+    the output is (P V) / sum 2^(x - M) (the sum unrounded). For any integer M the bf16 rounding of
+    2^(x - M) differs only by the exact power of two 2^(M' - M), so this P is defined independently
+    of how an implementation blocks the keys, as long as its running maximum stays integral.
     """
     Tq, nq, d = q.shape
     nkv = k.shape[1]
@@ -84,6 +102,11 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_pos: np.ndarray, k_
         g = h // G
         s = (q[:, h, :] @ k[:, g, :].T) / math.sqrt(d)
         s = np.where(visible, s, -np.inf)
+        if bf16_p:
+            x = s * math.log2(math.e)
+            p = np.exp2(x - np.ceil(x.max(axis=1, keepdims=True)))
+            out[:, h, :] = (bf16_round(p) @ v[:, g, :]) / p.sum(axis=1, keepdims=True)
+            continue
         s = s - s.max(axis=1, keepdims=True)
         p = np.exp(s)
         p = p / p.sum(axis=1, keepdims=True)
@@ -91,23 +114,29 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_pos: np.ndarray, k_
     return out
 
 
-def decode_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
+def decode_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, bf16_p: bool = False) -> np.ndarray:
     """One decode query [nq, d] over all of its request's keys [n, nkv, d] (its own new key included)."""
     n = k.shape[0]
-    return attention(q[None], k, v, np.array([n - 1]), np.arange(n))[0]
+    return attention(q[None], k, v, np.array([n - 1]), np.arange(n), bf16_p)[0]
 
 
-def prefill_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, prefix_len: int = 0) -> np.ndarray:
+def prefill_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, prefix_len: int = 0,
+                      bf16_p: bool = False) -> np.ndarray:
     """Causal attention of a prefill chunk: query at position prefix+i sees keys 0..prefix+i."""
     C = q.shape[0]
-    return attention(q, k, v, prefix_len + np.arange(C), np.arange(k.shape[0]))
+    return attention(q, k, v, prefix_len + np.arange(C), np.arange(k.shape[0]), bf16_p)
 
 
 # --- feed-forward ---------------------------------------------------------------------------------
 
-def swiglu_ffn(n: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
-    """SwiGLU FFN (Shazeer 2020): (silu(n Wg^T) * (n Wu^T)) Wd^T."""
-    return (silu(n @ w_gate.T) * (n @ w_up.T)) @ w_down.T
+def swiglu_ffn(n: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray, w_down: np.ndarray,
+               bf16_act: bool = False) -> np.ndarray:
+    """SwiGLU FFN (Shazeer 2020): (silu(n Wg^T) * (n Wu^T)) Wd^T; with bf16_act the activation
+    silu(n Wg^T) * (n Wu^T), the tensor handed to the down projection, is a bf16 tensor."""
+    act = silu(n @ w_gate.T) * (n @ w_up.T)
+    if bf16_act:
+        act = bf16_round(act)
+    return act @ w_down.T
 
 
 def moe_route(z: np.ndarray, top_k: int):
@@ -122,21 +151,32 @@ def moe_route(z: np.ndarray, top_k: int):
     return idx, w
 
 
-def moe_ffn(n: np.ndarray, experts: Sequence, idx: np.ndarray, w: np.ndarray) -> np.ndarray:
-    """sum_k w[t,k] * SwiGLU_{idx[t,k]}(n[t]); experts[e] = (w_gate, w_up, w_down)."""
+def moe_ffn(n: np.ndarray, experts: Sequence, idx: np.ndarray, w: np.ndarray, bf16_act: bool = False) -> np.ndarray:
+    """sum_k w[t,k] * SwiGLU_{idx[t,k]}(n[t]) with k ascending; experts[e] = (w_gate, w_up, w_down)."""
     T, K = idx.shape
     y = np.zeros((T, experts[0][2].shape[0]), dtype=np.float64)
     for e, (wg, wu, wd) in enumerate(experts):
         for kk in range(K):
             rows = np.nonzero(idx[:, kk] == e)[0]
             if rows.size:
-                y[rows] += w[rows, kk:kk + 1] * swiglu_ffn(n[rows], wg, wu, wd)
+                y[rows] += w[rows, kk:kk + 1] * swiglu_ffn(n[rows], wg, wu, wd, bf16_act)
     return y
 
 
-def lm_head_argmax(x: np.ndarray, final_norm: np.ndarray, lm_head: np.ndarray, eps: float):
+def norm_operand(x: np.ndarray, gamma: np.ndarray, eps: float, bf16_act: bool) -> np.ndarray:
+    """RMSNorm(x) * gamma as a projection consumes it: with bf16_act the product's operand is the
+    bf16 copy of x, scaled by 1/rms of the unrounded x and by gamma."""
+    if not bf16_act:
+        return rmsnorm(x, gamma, eps)
+    x = np.asarray(x, dtype=np.float64)
+    rs = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return bf16_round(x) * rs * gamma
+
+
+def lm_head_argmax(x: np.ndarray, final_norm: np.ndarray, lm_head: np.ndarray, eps: float,
+                   bf16_act: bool = False):
     """logits = RMSNorm(x) * gamma_final  E_out^T; greedy next token = first index of the maximum."""
-    logits = rmsnorm(x, final_norm, eps) @ lm_head.T
+    logits = norm_operand(x, final_norm, eps, bf16_act) @ lm_head.T
     return logits, np.argmax(logits, axis=1).astype(np.int64)
 
 
@@ -184,19 +224,21 @@ def _request_of_token(t: int, R: int) -> int:
     return t if t < R else R
 
 
-def layer_forward(s, lw: dict, x: np.ndarray, batch, kv: PagedKV, layer: int):
+def layer_forward(s, lw: dict, x: np.ndarray, batch, kv: PagedKV, layer: int, bf16_act: bool = True):
     """One transformer layer over the whole batch (decode rows first, then the prefill chunk)."""
     T, R, C = batch.num_tokens, batch.num_decode, batch.prefill_len
     nq, nkv, d, P = s.n_q_heads, s.n_kv_heads, s.head_dim, s.page_size
     pos = np.asarray(batch.positions, dtype=np.int64)
 
-    n = rmsnorm(x, lw["attn_norm"], s.rms_eps)
+    n = norm_operand(x, lw["attn_norm"], s.rms_eps, bf16_act)
     q = (n @ lw["wq"].T).reshape(T, nq, d)
     k = (n @ lw["wk"].T).reshape(T, nkv, d)
     v = (n @ lw["wv"].T).reshape(T, nkv, d)
     cos, sin = rope_cos_sin(pos, d, s.rope_theta)
     q = apply_rope(q, cos, sin)
     k = apply_rope(k, cos, sin)
+    if bf16_act:
+        q = bf16_round(q)
 
     # New K/V of every token go to slot pos % P of page page_table[req][pos // P].
     written = {}
@@ -210,22 +252,25 @@ def layer_forward(s, lw: dict, x: np.ndarray, batch, kv: PagedKV, layer: int):
     for r in range(R):
         pages = batch.page_indices[batch.page_indptr[r]:batch.page_indptr[r + 1]]
         K, V = kv.read(layer, pages, int(pos[r]) + 1)
-        o[r] = decode_attention(q[r], K, V)
+        o[r] = decode_attention(q[r], K, V, bf16_act)
     if C > 0:
         pages = batch.page_indices[batch.page_indptr[R]:batch.page_indptr[R + 1]]
         K, V = kv.read(layer, pages, C)
-        o[R:] = prefill_attention(q[R:], K, V)
+        o[R:] = prefill_attention(q[R:], K, V, bf16_p=bf16_act)
 
+    if bf16_act:
+        o = bf16_round(o)
     h = x + o.reshape(T, nq * d) @ lw["wo"].T
-    n2 = rmsnorm(h, lw["ffn_norm"], s.rms_eps)
+    n2 = norm_operand(h, lw["ffn_norm"], s.rms_eps, bf16_act)
     extras = {"written": written}
     if s.n_experts == 0:
-        y = swiglu_ffn(n2, lw["w_gate"], lw["w_up"], lw["w_down"])
+        y = swiglu_ffn(n2, lw["w_gate"], lw["w_up"], lw["w_down"], bf16_act)
     else:
-        z = n2 @ lw["router"].T + lw["router_bias"]
+        # router logits from the unrounded residual
+        z = rmsnorm(h, lw["ffn_norm"], s.rms_eps) @ lw["router"].T + lw["router_bias"]
         idx, w = moe_route(z, s.top_k)
         experts = [(lw[f"e{e}_gate"], lw[f"e{e}_up"], lw[f"e{e}_down"]) for e in range(s.n_experts)]
-        y = moe_ffn(n2, experts, idx, w)
+        y = moe_ffn(n2, experts, idx, w, bf16_act)
         extras.update(router_logits=z, topk_idx=idx, topk_w=w)
     return h + y, extras
 
@@ -234,7 +279,7 @@ def iteration_forward(s, batch, layer_weights: Callable[[int], dict], kv: PagedK
                       x_in: Optional[np.ndarray] = None,
                       embed_rows: Optional[Callable[[np.ndarray], np.ndarray]] = None,
                       final_norm: Optional[np.ndarray] = None, lm_head: Optional[np.ndarray] = None,
-                      keep_layer_inputs: bool = False):
+                      keep_layer_inputs: bool = False, bf16_act: bool = True):
     """The whole iteration. Layer slices take ``x_in`` [T, H]; full models embed ``batch.tokens``
     and finish with the final norm, the LM head over the decode rows plus the chunk's last row,
     and greedy argmax."""
@@ -246,13 +291,13 @@ def iteration_forward(s, batch, layer_weights: Callable[[int], dict], kv: PagedK
     for layer in range(s.n_layers):
         if keep_layer_inputs:
             out.setdefault("layer_inputs", []).append(x.copy())
-        x, extras = layer_forward(s, layer_weights(layer), x, batch, kv, layer)
+        x, extras = layer_forward(s, layer_weights(layer), x, batch, kv, layer, bf16_act)
         out["layers"].append(extras)
     out["hidden"] = x
     if s.vocab > 0:
         rows = lm_rows(batch)
         out["lm_rows"] = rows
-        out["logits"], out["next_token"] = lm_head_argmax(x[rows], final_norm, lm_head, s.rms_eps)
+        out["logits"], out["next_token"] = lm_head_argmax(x[rows], final_norm, lm_head, s.rms_eps, bf16_act)
     return out
 
 

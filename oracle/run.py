@@ -24,7 +24,7 @@ def make_kv(shape) -> PagedKV:
 
 
 def run_oracle(work: Workload, batch=None, requests=None, keep_prefill: bool = True,
-               keep_layer_inputs: bool = False, weights_cache: dict | None = None):
+               keep_layer_inputs: bool = False, weights_cache: dict | None = None, bf16_act: bool = True):
     """Oracle outputs for ``work``; with ``requests`` only those decode rows (and the chunk if kept).
 
     Returns (sub-batch actually computed, result dict, kv cache object).
@@ -56,5 +56,6 @@ def run_oracle(work: Workload, batch=None, requests=None, keep_prefill: bool = T
             if keep_prefill:
                 rows += list(range(full.num_decode, full.num_tokens))
             x_in = bf16_to_f64(W.host_input_rows(s, np.array(rows, dtype=np.int64)))
-    res = iteration_forward(s, b, lw, kv, x_in=x_in, keep_layer_inputs=keep_layer_inputs, **kwargs)
+    res = iteration_forward(s, b, lw, kv, x_in=x_in, keep_layer_inputs=keep_layer_inputs, bf16_act=bf16_act,
+                            **kwargs)
     return b, res, kv

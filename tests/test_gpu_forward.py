@@ -189,3 +189,21 @@ def test_gqa8_iteration_matches_oracle_and_is_invariant():
             assert np.array_equal(o, outs[0])
     finally:
         dw.close()
+
+
+def test_tuned_plan_is_bitwise_equal_to_sequential():
+    """nf_tune_plan returns one of the planner's plans, timed on the device; any plan gives the same bits."""
+    from intra_device_overlapped_b200.harness import DeviceWorkload
+    w = TEST_WORKLOADS["small_gqa8"]
+    dw = DeviceWorkload(w, DEV)
+    try:
+        _reset_kv(dw)
+        _run(dw, dw.plan(nano=1, template=0))
+        ref = _bits(dw.hidden_out_f32)
+        plan, us = dw.tune(reps=2)
+        assert us > 0 and 1 <= plan.n_nano <= 4
+        _reset_kv(dw)
+        _run(dw, plan)
+        assert np.array_equal(_bits(dw.hidden_out_f32), ref)
+    finally:
+        dw.close()

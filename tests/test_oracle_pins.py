@@ -315,19 +315,19 @@ def test_planted_mistakes_are_caught(monkeypatch):
     # a wrong GQA head map (h % nkv) breaks the brute-force GQA pin
     orig = F.attention
 
-    def attention_wrong_map(q, k, v, q_pos, k_pos):
+    def attention_wrong_map(q, k, v, q_pos, k_pos, bf16_p=False):
         nq, nkv = q.shape[1], k.shape[1]
         kk = k[:, [h % nkv for h in range(nq)], :]
         vv = v[:, [h % nkv for h in range(nq)], :]
-        return orig(q, kk, vv, q_pos, k_pos)
+        return orig(q, kk, vv, q_pos, k_pos, bf16_p)
     monkeypatch.setattr(F, "attention", attention_wrong_map)
     with pytest.raises(AssertionError):
         test_attention_matches_brute_force_gqa_causal()
     monkeypatch.undo()
 
     # a dropped causal mask breaks the causal brute-force pin
-    def attention_no_mask(q, k, v, q_pos, k_pos):
-        return orig(q, k, v, np.full_like(np.asarray(q_pos), 10 ** 9), k_pos)
+    def attention_no_mask(q, k, v, q_pos, k_pos, bf16_p=False):
+        return orig(q, k, v, np.full_like(np.asarray(q_pos), 10 ** 9), k_pos, bf16_p)
     monkeypatch.setattr(F, "attention", attention_no_mask)
     with pytest.raises(AssertionError):
         test_attention_matches_brute_force_gqa_causal()
@@ -337,3 +337,37 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(F, "rmsnorm", lambda x, g, eps: x / np.sqrt(np.mean(x * x, axis=0, keepdims=True) + eps) * g)
     with pytest.raises(AssertionError):
         test_rmsnorm_constant_rows_closed_form()
+
+
+def test_bf16_p_attention_definition():
+    """Attention of the bf16 model: P = bf16(2^(x - M)), M the integer ceiling of the row maximum, output
+    (P V) / sum 2^(x - M). Any other integer M gives the same result (exact power-of-two scaling of
+    bf16 values); it stays within bf16 resolution of exact attention; scores that make every weight a
+    power of two (no rounding) reproduce exact attention to double precision."""
+    import math
+    from oracle import forward as F
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((3, 4, 16))
+    k = rng.standard_normal((40, 2, 16))
+    v = rng.standard_normal((40, 2, 16))
+    qp, kp = np.array([39, 20, 5]), np.arange(40)
+    got = F.attention(q, k, v, qp, kp, bf16_p=True)
+    exact = F.attention(q, k, v, qp, kp)
+    assert np.abs(got - exact).max() < 4e-3 * np.abs(v).max()
+    # the same definition written with M + 7 instead of M
+    man = np.zeros_like(got)
+    for h in range(4):
+        g = h // 2
+        s = (q[:, h, :] @ k[:, g, :].T) / math.sqrt(16)
+        x = np.where(kp[None, :] <= qp[:, None], s, -np.inf) * math.log2(math.e)
+        p = np.exp2(x - (np.ceil(x.max(axis=1, keepdims=True)) + 7))
+        man[:, h, :] = (F.bf16_round(p) @ v[:, g, :]) / p.sum(axis=1, keepdims=True)
+    assert np.abs(got - man).max() < 1e-12   # (x - M - 7) and (x - M) round differently only in the last bit
+    # integer log2 scores: every weight is an exact power of two, so bf16 P is exact
+    d = 16
+    qi = np.zeros((1, 1, d)); qi[0, 0, 0] = math.sqrt(d) / math.log2(math.e)
+    ki = np.zeros((8, 1, d)); ki[:, 0, 0] = rng.integers(-6, 3, size=8)
+    vi = rng.standard_normal((8, 1, d))
+    a = F.attention(qi, ki, vi, np.array([7]), np.arange(8), bf16_p=True)
+    b = F.attention(qi, ki, vi, np.array([7]), np.arange(8))
+    assert np.abs(a - b).max() < 1e-12
