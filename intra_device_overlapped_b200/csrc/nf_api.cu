@@ -71,8 +71,21 @@ void set_tiles(GemmArgs& a, int M, int N, int K) {
 }
 
 int gemm_grid(const GemmArgs& a, int grid) {
-    const int tiles = a.m_tiles * a.n_tiles;
-    return std::max(1, std::min(grid, tiles));
+    const int units = a.m_tiles * a.n_tiles * (a.k_split == 2 ? 2 : 1);
+    return std::max(1, std::min(grid, units));
+}
+
+// Residual GEMMs (O and down projections, N = hidden) have few tiles per SM; a long one (at least
+// 160 k blocks of 64, e.g. the down projection of a 14336-wide FFN) splits K in two so that the
+// last wave is not mostly idle. Shorter ones lose more to the extra fill and partial traffic than
+// they gain. The rule depends only on K, so every plan gives the same bits.
+void set_splitk(nf_model* m, GemmArgs& a) {
+    if (a.k_blocks >= 160 && a.k_blocks % 2 == 0) {
+        a.k_split = 2;
+        a.splitk_ws = m->splitk_ws;
+        a.splitk_flags = m->splitk_flags;
+        a.splitk_epoch = ++m->splitk_epoch;
+    }
 }
 
 bool valid_config(const nf_model_config& c) {
@@ -176,6 +189,12 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) {
     ok &= (m->rope_cos = dalloc<float>(m, (size_t)cfg->max_position * d.d / 2)) != nullptr;
     ok &= (m->rope_sin = dalloc<float>(m, (size_t)cfg->max_position * d.d / 2)) != nullptr;
     ok &= (m->item_off = dalloc<int>(m, (size_t)cfg->max_requests + 1)) != nullptr;
+    {  // split-K workspace of the residual GEMMs (O and down: N = hidden)
+        const size_t tiles = (size_t)((T + nf::kGemmBM - 1) / nf::kGemmBM) * (d.H / nf::kGemmBN);
+        ok &= (m->splitk_ws = dalloc<float>(m, tiles * nf::kGemmBM * nf::kGemmBN)) != nullptr;
+        ok &= (m->splitk_flags = dalloc<int>(m, tiles)) != nullptr;
+        if (ok) ok = cudaMemset(m->splitk_flags, 0, tiles * sizeof(int)) == cudaSuccess;
+    }
     ok &= (m->merge_cnt = dalloc<int>(m, ((size_t)cfg->max_requests + 1) * d.nkv)) != nullptr;
     ok &= (m->status = dalloc<int>(m, 1)) != nullptr;
     m->trace_cap = 65536;
@@ -476,6 +495,7 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
             a.out_bf16 = m->xb;
             a.ld_bf16 = d.H;
             a.out_partials = m->partials;
+            set_splitk(m, a);
             NF_CUDA_TRY(nf::launch_gemm(nf::EPI_RESID, m->tm_attn_o, W.tm_o, a, gemm_grid(a, grid), s));
             return NF_OK;
         }
@@ -493,6 +513,7 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
             a.out_bf16 = m->xb;
             a.ld_bf16 = d.H;
             a.out_partials = m->partials;
+            set_splitk(m, a);
             NF_CUDA_TRY(nf::launch_gemm(nf::EPI_RESID, m->tm_act, W.tm_d, a, gemm_grid(a, grid), s));
             return NF_OK;
         }

@@ -134,6 +134,15 @@ __device__ __forceinline__ void store_kv_row32(uint16_t* page, int kv, int g, in
     }
 }
 
+__device__ __forceinline__ int ld_acquire_gpu(const int* ptr) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* ptr, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+
 // Warp-uniform wait: every lane tests the phase; if it has not completed, lane 0 waits with
 // the time limit and the outcome is shared.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
@@ -150,7 +159,7 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volati
 
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, uint32_t tacc, int row,
-                                              bool valid) {
+                                              bool valid, const float* partial_row) {
     float v[32];
     const int n0 = t.n_blk * BN;
     if constexpr (EPI == EPI_F32) {
@@ -171,6 +180,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, 
 #pragma unroll 1
         for (int j = 0; j < BN / 32; ++j) {
             tmem_ld32(tacc + 32 * j, v);
+            if (partial_row) {  // split-K: first half's partial + this half, in that order
+                const float4* w4 = reinterpret_cast<const float4*>(partial_row + 32 * j);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 w = __ldcg(w4 + q);
+                    v[4 * q + 0] = w.x + v[4 * q + 0]; v[4 * q + 1] = w.y + v[4 * q + 1];
+                    v[4 * q + 2] = w.z + v[4 * q + 2]; v[4 * q + 3] = w.w + v[4 * q + 3];
+                }
+            }
             if (valid) {
                 float* rp = p.resid + base + 32 * j;
                 const float4* r4 = reinterpret_cast<const float4*>(rp);
@@ -324,6 +342,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int ntiles = total_tiles(p);
+    const int ks = (EPI == EPI_RESID && p.k_split == 2) ? 2 : 1;  // k halves per tile
+    const int nunits = ntiles * ks;
+    const int kb_per = p.k_blocks / ks;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -332,9 +353,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int pending[STAGES];
             for (int s = 0; s < STAGES; ++s) pending[s] = -1;  // parity of an unconsumed load, -1 = none
             bool ok = true;
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-                const Tile t = tile_at(p, tile);
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
+            for (int unit = blockIdx.x; unit < nunits && ok; unit += gridDim.x) {
+                const Tile t = tile_at(p, unit % ntiles);
+                const int kb0 = (unit / ntiles) * kb_per;
+                for (int kb = kb0; kb < kb0 + kb_per; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
                     pending[stage] = -1;
                     uint8_t* sa = smem + stage * STAGE_BYTES;
@@ -362,20 +384,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int local = 0;
         bool ok = true;
         const uint64_t desc0 = umma_desc_sw128(smem_u32(smem));
-        for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++local) {
+        for (int unit = blockIdx.x; unit < nunits && ok; unit += gridDim.x, ++local) {
             const int acc = local & 1;
             const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
             if (!wait_warp(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, lane)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-            for (int kb = 0; kb < p.k_blocks; ++kb) {
+            const int kb0 = (unit / ntiles) * kb_per;
+            for (int kb = kb0; kb < kb0 + kb_per; ++kb) {
                 if (!wait_warp(&full[stage], phase, abort_flag, p.status, lane)) { ok = false; break; }
                 tc_fence_after();
                 const uint64_t adesc = desc0 + (uint64_t)((stage * STAGE_BYTES) >> 4);
                 const uint64_t bdesc = adesc + (uint64_t)(A_BYTES >> 4);
                 if (elect_one()) {
                     // advance 16 bf16 = 32 bytes along K inside the 128-byte swizzle atom
-                    if (kb == 0) umma_bf16_c<false>(d_tmem, adesc, bdesc, IDESC);
+                    if (kb == kb0) umma_bf16_c<false>(d_tmem, adesc, bdesc, IDESC);
                     else umma_bf16_c<true>(d_tmem, adesc, bdesc, IDESC);
 #pragma unroll
                     for (int k = 1; k < BK / 16; ++k)
@@ -403,19 +426,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int quarter = warp & 3;
         const int row_in_tile = quarter * 32 + lane;
         int local = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
+        for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x, ++local) {
             const int acc = local & 1;
             const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
             int ok = 1;
             if (lane == 0) ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
+            // all four epilogue warps leave together, so that none waits alone at barrier 1 below
+            if (bar_red_or(1, 128, !ok)) break;
             tc_fence_after();
+            const int tile = unit % ntiles;
             const Tile t = tile_at(p, tile);
             const int row = t.row_begin + row_in_tile;
             const bool valid = row < t.row_end;
             const uint32_t tacc = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-            epilogue_tile<EPI>(p, t, tacc, row, valid);
+            if (ks == 2 && unit < ntiles) {
+                // first half of the k blocks: publish the fp32 partial for the second half
+                float* wrow = p.splitk_ws + ((size_t)tile * BM + row_in_tile) * BN;
+#pragma unroll 1
+                for (int j = 0; j < BN / 32; ++j) {
+                    float v[32];
+                    tmem_ld32(tacc + 32 * j, v);
+                    store_f32x32(wrow + 32 * j, v);
+                }
+                __threadfence();
+                bar_sync_n(1, 128);
+                if (warp == 2 && lane == 0) st_release_gpu(p.splitk_flags + tile, p.splitk_epoch);
+            } else {
+                const float* prow = nullptr;
+                if (ks == 2) {
+                    // second half: wait (bounded) until the first half of this tile is published
+                    if (warp == 2 && lane == 0) {
+                        const uint64_t t0 = globaltimer_ns();
+                        while (ld_acquire_gpu(p.splitk_flags + tile) != p.splitk_epoch) {
+                            if (*abort_flag) break;
+                            if (globaltimer_ns() - t0 > NF_WAIT_LIMIT_NS) {
+                                *abort_flag = 1;
+                                set_status(p.status, NF_ERR_DEVICE_TIMEOUT);
+                                break;
+                            }
+                            __nanosleep(128);
+                        }
+                    }
+                    bar_sync_n(1, 128);
+                    prow = p.splitk_ws + ((size_t)tile * BM + row_in_tile) * BN;
+                }
+                epilogue_tile<EPI>(p, t, tacc, row, valid, prow);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);

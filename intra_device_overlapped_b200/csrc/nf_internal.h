@@ -57,6 +57,14 @@ struct GemmArgs {
     const int* page_indptr;
     const int* page_indices;
     int num_decode;
+    // split-K (EPI_RESID only): with k_split = 2 work unit u < tiles is the first half of the k
+    // blocks of tile u and writes its fp32 partial to splitk_ws, publishing splitk_flags[u] =
+    // splitk_epoch; unit tiles + u is the second half and adds that partial (in this fixed order)
+    // before the residual epilogue. Units of first halves come first in every CTA's order.
+    int k_split;
+    float* splitk_ws;     // [tiles x BM x BN] fp32
+    int* splitk_flags;    // [tiles]
+    int splitk_epoch;
     // EPI_LMHEAD
     float* tile_max;  // [rows x n_tiles]
     int* tile_arg;

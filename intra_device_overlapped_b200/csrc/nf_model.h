@@ -46,6 +46,9 @@ struct nf_model {
     float* rope_cos = nullptr;    // [max_position x d/2]
     float* rope_sin = nullptr;
     int* item_off = nullptr;      // [max_requests + 1]
+    float* splitk_ws = nullptr;   // split-K partials of the residual GEMMs: [tiles x 128 x 256] fp32
+    int* splitk_flags = nullptr;  // [tiles]: epoch of the last published first half
+    int splitk_epoch = 0;         // incremented per split-K launch
     int* merge_cnt = nullptr;     // [max_requests x nkv] split-KV arrival counters
     float* part_o = nullptr;      // split-KV partials
     float* part_lse = nullptr;
