@@ -217,6 +217,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t cs = 0, ni = 0;
         bool ok = true;
         const char* pool = reinterpret_cast<const char*>(a.kv_pool) + (is_k ? 0 : HALF_PAGE);
+        // each page is read once per launch: stream it through L2 without displacing reused data
+        const uint64_t stream_policy = l2_policy_evict_first();
         for (; it.valid && ok; req_next(it, a, hi), ++ni) {
             const int base = a.page_indptr[it.r];
             if (is_k) {
@@ -246,7 +248,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[st], HALF_PAGE);
-                    bulk_load(ring + st * HALF_PAGE, pool + (size_t)pg * PAGE_BYTES, HALF_PAGE, &full[st]);
+                    bulk_load_hint(ring + st * HALF_PAGE, pool + (size_t)pg * PAGE_BYTES, HALF_PAGE, &full[st],
+                                   stream_policy);
                 }
             }
         }

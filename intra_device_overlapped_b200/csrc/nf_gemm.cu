@@ -348,7 +348,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------- TMA producer
+            // ---------------- TMA producer. A (activations) is re-read by every column block: keep
+            // it in L2 over the KV pages that attention streams beside this GEMM.
+            const uint64_t a_policy = l2_policy_evict_last();
             uint32_t stage = 0, phase = 0;
             int pending[STAGES];
             for (int s = 0; s < STAGES; ++s) pending[s] = -1;  // parity of an unconsumed load, -1 = none
@@ -362,7 +364,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     uint8_t* sa = smem + stage * STAGE_BYTES;
                     uint8_t* sb = sa + A_BYTES;
                     mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-                    tma_load_2d(sa, &tmA, &full[stage], kb * BK, t.a_row);
+                    tma_load_2d_hint(sa, &tmA, &full[stage], kb * BK, t.a_row, a_policy);
                     tma_load_2d(sb, &tmB, &full[stage], kb * BK, t.b_row);
                     pending[stage] = (int)phase;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
