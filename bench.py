@@ -146,9 +146,9 @@ class ClockSampler:
 # read). Entries must be retaken whenever the kernel changes.
 TRAFFIC_PER_ALGO_BYTE = {
     # decode_attention_tc_kernel<32>, 64 requests of llama3_8b_layer on 16 SMs:
-    # dram__bytes_read.sum 337.738 MB + dram__bytes_write.sum 4.647 MB for 338.166 MB of
+    # dram__bytes_read.sum 337.759 MB + dram__bytes_write.sum 5.042 MB for 338.166 MB of
     # algorithmic bytes (337.117 MB of pages + 1.049 MB of q and o)
-    "decode_attention": (1.0125, "ncu: decode_attention_tc_kernel<32>, 64 of 512 requests, 16 SMs, scaled by pages"),
+    "decode_attention": (1.0137, "ncu: decode_attention_tc_kernel<32>, 64 of 512 requests, 16 SMs, scaled by pages"),
 }
 
 def iteration_flops(work, batch):
