@@ -75,12 +75,15 @@ int gemm_grid(const GemmArgs& a, int grid) {
     return std::max(1, std::min(grid, units));
 }
 
-// Residual GEMMs (O and down projections, N = hidden) have few tiles per SM; a long one (at least
-// 160 k blocks of 64, e.g. the down projection of a 14336-wide FFN) splits K in two so that the
-// last wave is not mostly idle. Shorter ones lose more to the extra fill and partial traffic than
-// they gain. The rule depends only on K, so every plan gives the same bits.
+// Residual GEMMs (O and down projections, N = hidden) have few tiles per SM (192 tiles of 128 x 256
+// for 1536 rows of a 4096-wide model: 1.3 waves on 148 SMs); one with at least
+// NF_SPLITK_MIN_KBLOCKS k blocks of 64 splits K in two so that the last wave is not mostly idle.
+// The rule depends only on K, so every plan gives the same bits.
+#ifndef NF_SPLITK_MIN_KBLOCKS
+#define NF_SPLITK_MIN_KBLOCKS 64
+#endif
 void set_splitk(nf_model* m, GemmArgs& a) {
-    if (a.k_blocks >= 160 && a.k_blocks % 2 == 0) {
+    if (a.k_blocks >= NF_SPLITK_MIN_KBLOCKS && a.k_blocks % 2 == 0) {
         a.k_split = 2;
         a.splitk_ws = m->splitk_ws;
         a.splitk_flags = m->splitk_flags;

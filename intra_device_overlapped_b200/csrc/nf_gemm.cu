@@ -134,6 +134,22 @@ __device__ __forceinline__ void store_kv_row32(uint16_t* page, int kv, int g, in
     }
 }
 
+// Per-warp staging of a 32 x 32 fp32 block of the accumulator. After tcgen05.ld lane l holds
+// row l; global rows are contiguous along columns, so the block is turned around in shared
+// memory: afterwards lane l serves column quad (l & 7) of rows 4 i + (l >> 3), i = 0..7, and
+// eight lanes cover one 128-byte row segment (four rows per warp access instead of 32). The
+// 16-byte chunks of a row are XOR-swizzled by the row so that the row-wise writes and the
+// column-quad reads are both free of bank conflicts.
+__device__ __forceinline__ void stage_rows32(float* stg, int lane, const float* v) {
+    float4* s4 = reinterpret_cast<float4*>(stg) + lane * 8;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) s4[q ^ (lane & 7)] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+__device__ __forceinline__ float4 staged_quad(const float* stg, int r, int c4) {
+    return reinterpret_cast<const float4*>(stg)[r * 8 + (c4 ^ (r & 7))];
+}
+
 __device__ __forceinline__ int ld_acquire_gpu(const int* ptr) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
@@ -154,12 +170,123 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volati
 }
 
 // ------------------------------------------------------------------ epilogues
+// Residual epilogue of one warp's 32 rows (rows rbase .. rbase + 31 of the tile), through the
+// warp's staging block so that every global access is row-contiguous:
+//   publish != null (first k half of a split tile): the fp32 partial goes to the workspace;
+//   otherwise h = (part + acc) + resid, written back to resid (fp32), to out_bf16 and, if set,
+//   out_f32; the row's sum of squares over this column block goes to out_partials.
+// The global reads of a 32-column block (residual, first-half partial) are issued together one
+// block ahead of their use, so that their latency overlaps the previous block's work instead of
+// being paid once per row behind that row's stores.
+struct ResidCtx {
+    const GemmArgs* p;
+    const Tile* t;
+    uint32_t tacc;
+    int rbase, lane;
+    float* stg;
+    const float* part;
+};
+
+__device__ __forceinline__ void resid_load(const ResidCtx& c, int j, float4 (&r)[8], float4 (&w)[8]) {
+    const GemmArgs& p = *c.p;
+    const int n0 = c.t->n_blk * BN;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int rt = c.rbase + 4 * i + (c.lane >> 3);
+        const int col = 32 * j + 4 * (c.lane & 7);
+        if (c.part != nullptr) w[i] = __ldcg(reinterpret_cast<const float4*>(c.part + (size_t)rt * BN + col));
+        const int row = c.t->row_begin + rt;
+        if (row < c.t->row_end)
+            r[i] = __ldcg(reinterpret_cast<const float4*>(p.resid + (size_t)(p.tok0 + row) * p.N + n0 + col));
+    }
+}
+
+__device__ __forceinline__ void resid_block(const ResidCtx& c, int j, const float4 (&r)[8], const float4 (&w)[8],
+                                            float (&ss)[8]) {
+    const GemmArgs& p = *c.p;
+    const int n0 = c.t->n_blk * BN;
+    float v[32];
+    tmem_ld32(c.tacc + 32 * j, v);
+    stage_rows32(c.stg, c.lane, v);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int rt = c.rbase + 4 * i + (c.lane >> 3);
+        const int col = 32 * j + 4 * (c.lane & 7);
+        float4 x = staged_quad(c.stg, 4 * i + (c.lane >> 3), c.lane & 7);
+        if (c.part != nullptr)  // split-K: first half's partial + this half, in that order
+            x = make_float4(w[i].x + x.x, w[i].y + x.y, w[i].z + x.z, w[i].w + x.w);
+        const int row = c.t->row_begin + rt;
+        if (row < c.t->row_end) {
+            const size_t g = (size_t)(p.tok0 + row);
+            x = make_float4(x.x + r[i].x, x.y + r[i].y, x.z + r[i].z, x.w + r[i].w);
+            ss[i] += x.x * x.x;
+            ss[i] += x.y * x.y;
+            ss[i] += x.z * x.z;
+            ss[i] += x.w * x.w;
+            *reinterpret_cast<float4*>(p.resid + g * p.N + n0 + col) = x;
+            *reinterpret_cast<uint2*>(p.out_bf16 + g * p.ld_bf16 + n0 + col) =
+                make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+            if (p.out_f32) *reinterpret_cast<float4*>(p.out_f32 + g * p.ld_f32 + n0 + col) = x;
+        }
+    }
+    __syncwarp();  // the next block overwrites the staging buffer
+}
+
+static_assert((BN / 32) % 2 == 0, "the residual epilogue walks column blocks in pairs");
+
+__device__ __forceinline__ void epilogue_resid(const GemmArgs& p, const Tile& t, uint32_t tacc, int rbase, int lane,
+                                               float* stg, const float* part, float* publish) {
+    if (publish != nullptr) {
+#pragma unroll 1
+        for (int j = 0; j < BN / 32; ++j) {
+            float v[32];
+            tmem_ld32(tacc + 32 * j, v);
+            stage_rows32(stg, lane, v);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int rt = rbase + 4 * i + (lane >> 3);
+                __stcg(reinterpret_cast<float4*>(publish + (size_t)rt * BN + 32 * j + 4 * (lane & 7)),
+                       staged_quad(stg, 4 * i + (lane >> 3), lane & 7));
+            }
+            __syncwarp();
+        }
+        return;
+    }
+    const ResidCtx c{&p, &t, tacc, rbase, lane, stg, part};
+    float ss[8];
+    float4 ra[8], wa[8], rb[8], wb[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        ss[i] = 0.f;
+        ra[i] = rb[i] = wa[i] = wb[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    resid_load(c, 0, ra, wa);
+#pragma unroll 1
+    for (int j = 0; j < BN / 32; j += 2) {
+        resid_load(c, j + 1, rb, wb);
+        resid_block(c, j, ra, wa, ss);
+        if (j + 2 < BN / 32) resid_load(c, j + 2, ra, wa);
+        resid_block(c, j + 1, rb, wb, ss);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float x = ss[i];
+        x += __shfl_xor_sync(0xffffffffu, x, 1);
+        x += __shfl_xor_sync(0xffffffffu, x, 2);
+        x += __shfl_xor_sync(0xffffffffu, x, 4);
+        const int row = t.row_begin + rbase + 4 * i + (lane >> 3);
+        if ((lane & 7) == 0 && row < t.row_end) p.out_partials[(size_t)(p.tok0 + row) * p.n_tiles + t.n_blk] = x;
+    }
+}
+
 // Each is called by all 32 lanes of an epilogue warp (tcgen05.ld is warp-collective);
 // `valid` says whether this lane's row is inside the tile's row range.
 
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, uint32_t tacc, int row,
-                                              bool valid, const float* partial_row) {
+                                              bool valid) {
     float v[32];
     const int n0 = t.n_blk * BN;
     if constexpr (EPI == EPI_F32) {
@@ -174,37 +301,6 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, 
                 store_f32x32(dst + 32 * j, v);
             }
         }
-    } else if constexpr (EPI == EPI_RESID) {
-        const size_t base = (size_t)(p.tok0 + row) * p.N + n0;
-        float ss = 0.f;
-#pragma unroll 1
-        for (int j = 0; j < BN / 32; ++j) {
-            tmem_ld32(tacc + 32 * j, v);
-            if (partial_row) {  // split-K: first half's partial + this half, in that order
-                const float4* w4 = reinterpret_cast<const float4*>(partial_row + 32 * j);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 w = __ldcg(w4 + q);
-                    v[4 * q + 0] = w.x + v[4 * q + 0]; v[4 * q + 1] = w.y + v[4 * q + 1];
-                    v[4 * q + 2] = w.z + v[4 * q + 2]; v[4 * q + 3] = w.w + v[4 * q + 3];
-                }
-            }
-            if (valid) {
-                float* rp = p.resid + base + 32 * j;
-                const float4* r4 = reinterpret_cast<const float4*>(rp);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 x = r4[q];
-                    v[4 * q + 0] += x.x; v[4 * q + 1] += x.y; v[4 * q + 2] += x.z; v[4 * q + 3] += x.w;
-                }
-#pragma unroll
-                for (int e = 0; e < 32; ++e) ss += v[e] * v[e];
-                store_f32x32(rp, v);
-                store_bf16x32(p.out_bf16 + (size_t)(p.tok0 + row) * p.ld_bf16 + n0 + 32 * j, v);
-                if (p.out_f32) store_f32x32(p.out_f32 + (size_t)(p.tok0 + row) * p.ld_f32 + n0 + 32 * j, v);
-            }
-        }
-        if (valid) p.out_partials[(size_t)(p.tok0 + row) * p.n_tiles + t.n_blk] = ss;
     } else if constexpr (EPI == EPI_SWIGLU) {
         const float rs = valid ? row_scale(p, row) : 1.f;
         float u[32];
@@ -267,26 +363,36 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, 
             }
         }
         const int slot = pos & 15;
-        float x2[32];
+        // the rotation angles depend on the position and the column pair only: each column
+        // block's cos / sin row segment is loaded once (16-byte loads) for both heads of the tile
+        const bool any_rope = n0 / d < p.nq + p.nkv;
+        float x2[32], cs[32], sn[32];
 #pragma unroll 1
-        for (int hc = 0; hc < BN / d; ++hc) {
-            const int head = (n0 + hc * d) / d;
-            const int kind = head < p.nq ? 0 : (head < p.nq + p.nkv ? 1 : 2);
-            const int g = kind == 1 ? head - p.nq : head - p.nq - p.nkv;
+        for (int j = 0; j < half / 32; ++j) {
+            if (ok && any_rope) {
+                const float4* c4 = reinterpret_cast<const float4*>(p.rope_cos + (size_t)pos * half + 32 * j);
+                const float4* s4 = reinterpret_cast<const float4*>(p.rope_sin + (size_t)pos * half + 32 * j);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 c = __ldg(c4 + q), sv = __ldg(s4 + q);
+                    cs[4 * q] = c.x; cs[4 * q + 1] = c.y; cs[4 * q + 2] = c.z; cs[4 * q + 3] = c.w;
+                    sn[4 * q] = sv.x; sn[4 * q + 1] = sv.y; sn[4 * q + 2] = sv.z; sn[4 * q + 3] = sv.w;
+                }
+            }
 #pragma unroll 1
-            for (int j = 0; j < half / 32; ++j) {
+            for (int hc = 0; hc < BN / d; ++hc) {
+                const int head = (n0 + hc * d) / d;
+                const int kind = head < p.nq ? 0 : (head < p.nq + p.nkv ? 1 : 2);
+                const int g = kind == 1 ? head - p.nq : head - p.nq - p.nkv;
                 tmem_ld32(tacc + hc * d + 32 * j, v);
                 tmem_ld32(tacc + hc * d + half + 32 * j, x2);
                 if (!ok || (kind != 0 && page_base < 0)) continue;
                 if (kind < 2) {
-                    const float* cs = p.rope_cos + (size_t)pos * half + 32 * j;
-                    const float* sn = p.rope_sin + (size_t)pos * half + 32 * j;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const float a = v[e] * rs, b = x2[e] * rs;
-                        const float c = cs[e], s = sn[e];
-                        v[e] = a * c - b * s;
-                        x2[e] = b * c + a * s;
+                        v[e] = a * cs[e] - b * sn[e];
+                        x2[e] = b * cs[e] + a * sn[e];
                     }
                 } else {
 #pragma unroll
@@ -311,6 +417,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const __grid_constant__ GemmArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // barriers in the kGemmBarrierBytes after the ring, then the epilogue warps' staging blocks
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;   // [2]
@@ -442,38 +549,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int row = t.row_begin + row_in_tile;
             const bool valid = row < t.row_end;
             const uint32_t tacc = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-            if (ks == 2 && unit < ntiles) {
-                // first half of the k blocks: publish the fp32 partial for the second half
-                float* wrow = p.splitk_ws + ((size_t)tile * BM + row_in_tile) * BN;
-#pragma unroll 1
-                for (int j = 0; j < BN / 32; ++j) {
-                    float v[32];
-                    tmem_ld32(tacc + 32 * j, v);
-                    store_f32x32(wrow + 32 * j, v);
-                }
-                __threadfence();
-                bar_sync_n(1, 128);
-                if (warp == 2 && lane == 0) st_release_gpu(p.splitk_flags + tile, p.splitk_epoch);
-            } else {
-                const float* prow = nullptr;
-                if (ks == 2) {
-                    // second half: wait (bounded) until the first half of this tile is published
-                    if (warp == 2 && lane == 0) {
-                        const uint64_t t0 = globaltimer_ns();
-                        while (ld_acquire_gpu(p.splitk_flags + tile) != p.splitk_epoch) {
-                            if (*abort_flag) break;
-                            if (globaltimer_ns() - t0 > NF_WAIT_LIMIT_NS) {
-                                *abort_flag = 1;
-                                set_status(p.status, NF_ERR_DEVICE_TIMEOUT);
-                                break;
-                            }
-                            __nanosleep(128);
-                        }
-                    }
+            if constexpr (EPI == EPI_RESID) {
+                float* stg = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + kGemmBarrierBytes) + quarter * 1024;
+                float* ws = p.splitk_ws + (size_t)tile * BM * BN;
+                if (ks == 2 && unit < ntiles) {
+                    // first half of the k blocks: publish the fp32 partial for the second half
+                    epilogue_resid(p, t, tacc, quarter * 32, lane, stg, nullptr, ws);
+                    __threadfence();
                     bar_sync_n(1, 128);
-                    prow = p.splitk_ws + ((size_t)tile * BM + row_in_tile) * BN;
+                    if (warp == 2 && lane == 0) st_release_gpu(p.splitk_flags + tile, p.splitk_epoch);
+                } else {
+                    if (ks == 2) {
+                        // second half: wait (bounded) until the first half of this tile is published
+                        if (warp == 2 && lane == 0) {
+                            const uint64_t t0 = globaltimer_ns();
+                            while (ld_acquire_gpu(p.splitk_flags + tile) != p.splitk_epoch) {
+                                if (*abort_flag) break;
+                                if (globaltimer_ns() - t0 > NF_WAIT_LIMIT_NS) {
+                                    *abort_flag = 1;
+                                    set_status(p.status, NF_ERR_DEVICE_TIMEOUT);
+                                    break;
+                                }
+                                __nanosleep(128);
+                            }
+                        }
+                        bar_sync_n(1, 128);
+                    }
+                    epilogue_resid(p, t, tacc, quarter * 32, lane, stg, ks == 2 ? ws : nullptr, nullptr);
                 }
-                epilogue_tile<EPI>(p, t, tacc, row, valid, prow);
+            } else {
+                epilogue_tile<EPI>(p, t, tacc, row, valid);
             }
             tc_fence_before();
             __syncwarp();

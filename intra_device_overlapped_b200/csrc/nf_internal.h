@@ -13,7 +13,10 @@ constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 64;
 constexpr int kGemmStages = 4;
 constexpr int kGemmThreads = 192;
-constexpr int kGemmSmemBytes = kGemmStages * (kGemmBM + kGemmBN) * kGemmBK * 2 + 1024 + 256;
+constexpr int kGemmBarrierBytes = 256;
+constexpr int kGemmStagingBytes = 4 * 32 * 32 * 4;  // residual epilogue: 32 x 32 fp32 per epilogue warp
+constexpr int kGemmSmemBytes =
+    kGemmStages * (kGemmBM + kGemmBN) * kGemmBK * 2 + 1024 + kGemmBarrierBytes + kGemmStagingBytes;
 
 enum EpiKind : int {
     EPI_F32 = 0,     // out_f32 = acc (* rs if partials)
