@@ -750,6 +750,16 @@ extern "C" nf_status nf_tune_plan(nf_model* m, const nf_batch_desc* b, const nf_
             nf_plan p;
             if (nf_plan_iteration(m, b, &o, &p) != NF_OK) continue;  // e.g. more nano-batches than rows allow
             st = try_plan(p);
+            if (t == NF_TEMPLATE_PREFILL_ON_GEMM && n == 1) {
+                // decode attention beside prefill attention: the split is decided by how many SMs
+                // keep decode attention at full HBM bandwidth, which the cost model only estimates
+                static const int kPrefillSms[] = {8, 16, 24, 32, 48};
+                for (int k : kPrefillSms) {
+                    if (st != NF_OK || k > m->sm_count - 8) break;
+                    o.force_sm_attn = m->sm_count - k;
+                    if (nf_plan_iteration(m, b, &o, &p) == NF_OK) st = try_plan(p);
+                }
+            }
         }
     }
     cudaEventDestroy(e0);

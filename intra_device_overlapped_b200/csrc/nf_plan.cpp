@@ -9,8 +9,10 @@
 // Candidates: n in 1..4 nano-batches; decode rows cut at request boundaries into
 // groups of equal KV bytes; the prefill chunk either its own nano-batch or joined to
 // the last decode group; pipeline order natural or prefill first; SM split for
-// attention in steps of 4; template sequential or pipelined. Each candidate's op list
-// (build_ops) is simulated on two streams; the minimum makespan wins.
+// attention in steps of 4; template sequential or pipelined. With one nano-batch the
+// prefill-on-GEMM template still overlaps something: the decode attention (HBM-bound) on
+// sm_attn SMs beside the prefill attention (tensor-bound) on the others. Each candidate's
+// op list (build_ops) is simulated on two streams; the minimum makespan wins.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -371,7 +373,10 @@ nf_status plan_impl(const nf_model* m, const nf_batch_desc* b, const nf_plan_opt
                 for (int i = 0; i < n; ++i) p.nano_order[i] = perm[i];
                 for (int tmpl = 0; tmpl <= 2; ++tmpl) {
                     if (o.force_template >= 0 && tmpl != o.force_template) continue;
-                    if (tmpl != NF_TEMPLATE_SEQUENTIAL && n < 2) continue;
+                    // one nano-batch overlaps only with the prefill attention on the GEMM stream beside
+                    // the decode attention (two attention kernels bound by different units)
+                    if (tmpl != NF_TEMPLATE_SEQUENTIAL && n < 2 && !(tmpl == NF_TEMPLATE_PREFILL_ON_GEMM && R > 0))
+                        continue;
                     if (tmpl == NF_TEMPLATE_PREFILL_ON_GEMM && C == 0) continue;
                     if (tmpl == NF_TEMPLATE_SEQUENTIAL && perm[0] != 0) continue;  // order is irrelevant
                     p.order_template = tmpl;

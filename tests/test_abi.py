@@ -94,7 +94,8 @@ def test_planner_produces_valid_plans(nf, name):
     d, keep = _desc(nf, b)
     for opts in (nf.nf_plan_opts(force_template=-1), nf.nf_plan_opts(force_nano=2, force_template=1),
                  nf.nf_plan_opts(force_nano=4, force_template=1, force_sm_attn=40),
-                 nf.nf_plan_opts(force_nano=1, force_template=0)):
+                 nf.nf_plan_opts(force_nano=1, force_template=0),
+                 nf.nf_plan_opts(force_nano=1, force_template=2, force_sm_attn=124)):
         st, p = nf.nf_plan_for_config(model_config(w), 148, d, opts)
         assert st == 0
         T = b.num_tokens

@@ -45,7 +45,7 @@ def tiny():
 
 PLANS = [dict(nano=1, template=0), dict(nano=2, template=1, sm_attn=16), dict(nano=3, template=1, sm_attn=40),
          dict(nano=4, template=1, sm_attn=64), dict(nano=2, template=0), dict(nano=2, template=2, sm_attn=24),
-         dict(nano=3, template=2, sm_attn=52)]
+         dict(nano=3, template=2, sm_attn=52), dict(nano=1, template=2, sm_attn=120)]
 
 
 @pytest.mark.parametrize("opts", PLANS)
