@@ -209,6 +209,14 @@ typedef struct {
     float* layer_hidden_out;     /* [n_layers x T x H] fp32 residual stream after each layer, nullable
                                   * (verification: copied row range by row range as each nano-batch
                                   * finishes a layer) */
+    /* Token feedback on the device (vocab > 0), for a CPU that forms iteration i+1 before it has
+     * read iteration i's tokens. token_src NULL: every token comes from token_ids. Otherwise
+     * row t's token is prev_token[token_src[t]] when token_src[t] >= 0 (prev_token: the previous
+     * iteration's next_token, prev_rows entries), else token_ids[t]. A token_src entry >=
+     * prev_rows latches NF_ERR_DEVICE_BOUNDS and reads token 0. */
+    const int32_t* token_src;    /* [T] device, nullable */
+    const int32_t* prev_token;   /* [prev_rows] device */
+    int32_t prev_rows;
 } nf_iter_io;
 
 /* Run the iteration described by `plan` (made by nf_plan_iteration for the same
@@ -351,6 +359,83 @@ nf_status nf_decode_attention_noalloc(const void* q, void* out, const void* kv_p
                                       const int32_t* page_indices, int32_t num_requests, int32_t n_q_heads,
                                       int32_t n_kv_heads, int32_t head_dim, int32_t sm_count,
                                       int32_t* status_device, void* stream);
+
+/* ------------------------------------------------------------------ serving scheduler (host)
+ *
+ * The CPU control flow around nf_forward_iteration for a stream of requests (prompt, then greedy
+ * decoding). The CPU forms iteration i+1 while the GPU runs iteration i (README "Abstract",
+ * arXiv abstract: NanoFlow's asynchronous CPU scheduling), so a request whose last token comes out
+ * of iteration i is decoded once more in iteration i+1; that token is dropped and the request
+ * leaves the batch from iteration i+2 on. Decode rows take their input token from the previous
+ * iteration's next_token on the device (nf_iter_io.token_src), so forming a batch never waits for
+ * the GPU. Host only: no call touches a device.
+ *
+ * Policy: first come first served; one prompt per iteration, whole, as the prefill chunk; a
+ * request is admitted when a running slot and ceil((prompt_len + max_new_tokens) / 16) free pages
+ * exist, and keeps those pages until the host learns that it finished. Admitted requests decode
+ * in every iteration (rows in admission order), so none waits for a page or is preempted. */
+typedef struct nf_sched nf_sched; /* opaque */
+
+typedef struct {
+    int32_t num_pages;    /* pages in each layer's KV pool, numbered 0 .. num_pages - 1 */
+    int32_t max_running;  /* decode rows per iteration at most (<= the model's max_requests) */
+    int32_t chunk_len;    /* prefill tokens per iteration at most; a prompt must fit one chunk.
+                           * The model's max_tokens must be >= max_running + chunk_len. */
+    int32_t max_position; /* prompt_len + max_new_tokens must not exceed it (the model's RoPE table) */
+    int32_t lag;          /* 1: iteration i+1 is formed before iteration i completes (asynchronous);
+                           * 0: after (synchronous) */
+} nf_sched_config;
+
+/* One formed iteration. The arrays belong to the scheduler and stay valid until the next
+ * nf_sched_next call; they map one to one onto nf_batch_desc and nf_iter_io. */
+typedef struct {
+    int64_t iteration;           /* sequence number (0, 1, ...), -1 when num_tokens == 0 */
+    int32_t num_decode;          /* R */
+    int32_t prefill_len;         /* C (0: no prompt this iteration) */
+    int32_t num_tokens;          /* T = R + C; 0: nothing to run now */
+    int32_t rows;                /* next_token rows: R + (C > 0) */
+    int32_t num_page_entries;    /* page_indptr[R + 1] */
+    const int32_t* ctx_len;      /* [R] cached tokens per decode row */
+    const int32_t* positions;    /* [T] */
+    const int32_t* token_ids;    /* [T] prompt tokens on the chunk rows, -1 on decode rows */
+    const int32_t* token_src;    /* [T] decode rows: their row in the previous iteration's next_token;
+                                  * chunk rows: -1 */
+    const int32_t* page_indptr;  /* [R + 2], prefill request last */
+    const int32_t* page_indices; /* [num_page_entries] */
+    const int64_t* row_request;  /* [rows] request id of each next_token row */
+} nf_sched_iter;
+
+typedef struct {
+    int32_t waiting, running, finished, free_pages, inflight;
+    int64_t iterations;       /* iterations formed */
+    int64_t discarded_tokens; /* tokens decoded after a request's last one (one per request at lag 1) */
+} nf_sched_stats;
+
+/* NF_ERR_INVALID_ARGUMENT for a bad configuration. */
+nf_status nf_sched_create(const nf_sched_config* cfg, nf_sched** out);
+void nf_sched_destroy(nf_sched* s);
+
+/* Queue a request; the prompt is copied. eos_token < 0: none. NF_ERR_INVALID_ARGUMENT when
+ * the request could never run (prompt longer than a chunk, prompt_len + max_new_tokens above
+ * max_position, more pages than the pool). */
+nf_status nf_sched_add_request(nf_sched* s, const int32_t* prompt, int32_t prompt_len, int32_t max_new_tokens,
+                               int32_t eos_token, int64_t* id_out);
+
+/* Form the next iteration. Iteration k may be formed only after iteration k - 1 - lag was
+ * completed (else NF_ERR_INVALID_ARGUMENT). num_tokens == 0: nothing can run before another
+ * completion (or every request has finished). */
+nf_status nf_sched_next(nf_sched* s, nf_sched_iter* out);
+
+/* Hand over the host copy of an iteration's next_token ([rows]); iterations complete in the
+ * order they were formed. Finished requests release their pages. */
+nf_status nf_sched_complete(nf_sched* s, int64_t iteration, const int32_t* next_token, int32_t rows);
+
+/* Tokens generated so far for request `id` (the first min(cap, *len) are copied to out), and
+ * whether it has finished (nullable). */
+nf_status nf_sched_request_tokens(const nf_sched* s, int64_t id, int32_t* out, int32_t cap, int32_t* len,
+                                  int32_t* finished);
+
+nf_status nf_sched_get_stats(const nf_sched* s, nf_sched_stats* out);
 
 /* Library version string. */
 const char* nf_version(void);

@@ -79,7 +79,28 @@ class nf_iter_io(ctypes.Structure):
                 ("page_indptr", _vp), ("page_indices", _vp), ("kv_pools", ctypes.POINTER(_vp)),
                 ("num_pages", _i32), ("hidden_out", _vp), ("hidden_out_f32", _vp), ("logits", _vp),
                 ("next_token", _vp), ("topk_idx", _vp), ("topk_w", _vp), ("router_logits", _vp),
-                ("layer_hidden_out", _vp)]
+                ("layer_hidden_out", _vp), ("token_src", _vp), ("prev_token", _vp), ("prev_rows", _i32)]
+
+
+class nf_sched_config(ctypes.Structure):
+    _fields_ = [("num_pages", _i32), ("max_running", _i32), ("chunk_len", _i32), ("max_position", _i32),
+                ("lag", _i32)]
+
+
+class nf_sched_iter(ctypes.Structure):
+    _fields_ = [("iteration", _i64), ("num_decode", _i32), ("prefill_len", _i32), ("num_tokens", _i32),
+                ("rows", _i32), ("num_page_entries", _i32), ("ctx_len", ctypes.POINTER(_i32)),
+                ("positions", ctypes.POINTER(_i32)), ("token_ids", ctypes.POINTER(_i32)),
+                ("token_src", ctypes.POINTER(_i32)), ("page_indptr", ctypes.POINTER(_i32)),
+                ("page_indices", ctypes.POINTER(_i32)), ("row_request", ctypes.POINTER(_i64))]
+
+
+class nf_sched_stats(ctypes.Structure):
+    _fields_ = [("waiting", _i32), ("running", _i32), ("finished", _i32), ("free_pages", _i32), ("inflight", _i32),
+                ("iterations", _i64), ("discarded_tokens", _i64)]
+
+    def as_dict(self) -> dict:
+        return {f: getattr(self, f) for f, _ in self._fields_}
 
 
 class nf_op_time(ctypes.Structure):
@@ -137,6 +158,13 @@ def _load():
         "nf_op_wait_flag_test": ([_vp, _u64, _vp], ctypes.c_int),
         "nf_decode_attention_noalloc": ([_vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp],
                                         ctypes.c_int),
+        "nf_sched_create": ([P(nf_sched_config), P(_vp)], ctypes.c_int),
+        "nf_sched_destroy": ([_vp], None),
+        "nf_sched_add_request": ([_vp, P(_i32), _i32, _i32, _i32, P(_i64)], ctypes.c_int),
+        "nf_sched_next": ([_vp, P(nf_sched_iter)], ctypes.c_int),
+        "nf_sched_complete": ([_vp, _i64, P(_i32), _i32], ctypes.c_int),
+        "nf_sched_request_tokens": ([_vp, _i64, P(_i32), _i32, P(_i32), P(_i32)], ctypes.c_int),
+        "nf_sched_get_stats": ([_vp, P(nf_sched_stats)], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -150,7 +178,9 @@ EXPORTED = ("nf_status_string", "nf_version", "nf_init_model", "nf_set_layer_wei
             "nf_destroy_model", "nf_plan_iteration", "nf_plan_for_config", "nf_forward_iteration", "nf_tune_plan", "nf_sync_status", "nf_calibrate",
             "nf_get_cost_model", "nf_set_cost_model",
             "nf_set_trace", "nf_get_trace", "nf_set_timing", "nf_get_op_times", "nf_op_gemm_bf16", "nf_op_decode_attention",
-            "nf_op_prefill_attention", "nf_op_wait_flag_test", "nf_decode_attention_noalloc")
+            "nf_op_prefill_attention", "nf_op_wait_flag_test", "nf_decode_attention_noalloc",
+            "nf_sched_create", "nf_sched_destroy", "nf_sched_add_request", "nf_sched_next", "nf_sched_complete",
+            "nf_sched_request_tokens", "nf_sched_get_stats")
 
 
 NF_NOALLOC_MAX_REQUESTS = 16384
@@ -296,3 +326,53 @@ def nf_op_prefill_attention(model: int, q_ptr: int, out_ptr: int, io: nf_iter_io
 
 def nf_op_wait_flag_test(flag_ptr: int, limit_ns: int, stream: int = 0) -> int:
     return _lib.nf_op_wait_flag_test(flag_ptr, limit_ns, stream)
+
+
+def _i32_array(values) -> "ctypes.Array":
+    vals = [int(v) for v in values]
+    return (_i32 * max(1, len(vals)))(*vals)
+
+
+def nf_sched_create(cfg: nf_sched_config):
+    """Returns (status, scheduler handle)."""
+    h = _vp()
+    st = _lib.nf_sched_create(ctypes.byref(cfg), ctypes.byref(h))
+    return st, h.value
+
+
+def nf_sched_destroy(sched: int) -> None:
+    _lib.nf_sched_destroy(sched)
+
+
+def nf_sched_add_request(sched: int, prompt, max_new_tokens: int, eos_token: int = -1):
+    """Returns (status, request id)."""
+    arr = _i32_array(prompt)
+    rid = _i64()
+    st = _lib.nf_sched_add_request(sched, arr, len(prompt), max_new_tokens, eos_token, ctypes.byref(rid))
+    return st, rid.value
+
+
+def nf_sched_next(sched: int):
+    """Returns (status, nf_sched_iter); the arrays it points to live until the next call."""
+    it = nf_sched_iter()
+    st = _lib.nf_sched_next(sched, ctypes.byref(it))
+    return st, it
+
+
+def nf_sched_complete(sched: int, iteration: int, next_token) -> int:
+    arr = _i32_array(next_token)
+    return _lib.nf_sched_complete(sched, iteration, arr, len(next_token))
+
+
+def nf_sched_request_tokens(sched: int, rid: int, cap: int = 1 << 16):
+    """Returns (status, generated tokens, finished)."""
+    buf = (_i32 * max(1, cap))()
+    n, fin = _i32(), _i32()
+    st = _lib.nf_sched_request_tokens(sched, rid, buf, cap, ctypes.byref(n), ctypes.byref(fin))
+    return st, list(buf[:min(n.value, cap)]), bool(fin.value)
+
+
+def nf_sched_get_stats(sched: int):
+    out = nf_sched_stats()
+    st = _lib.nf_sched_get_stats(sched, ctypes.byref(out))
+    return st, out

@@ -192,6 +192,7 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) {
     ok &= (m->rope_cos = dalloc<float>(m, (size_t)cfg->max_position * d.d / 2)) != nullptr;
     ok &= (m->rope_sin = dalloc<float>(m, (size_t)cfg->max_position * d.d / 2)) != nullptr;
     ok &= (m->item_off = dalloc<int>(m, (size_t)cfg->max_requests + 1)) != nullptr;
+    if (cfg->vocab > 0) ok &= (m->tok_feedback = dalloc<int>(m, T)) != nullptr;
     {  // split-K workspace of the residual GEMMs (O and down: N = hidden)
         const size_t tiles = (size_t)((T + nf::kGemmBM - 1) / nf::kGemmBM) * (d.H / nf::kGemmBN);
         ok &= (m->splitk_ws = dalloc<float>(m, tiles * nf::kGemmBM * nf::kGemmBN)) != nullptr;
@@ -607,6 +608,8 @@ nf_status validate_forward(const nf_model* m, const nf_plan* p, const nf_iter_io
         return NF_ERR_INVALID_ARGUMENT;
     if (R > 0 && !io->ctx_len) return NF_ERR_INVALID_ARGUMENT;
     if (m->cfg.vocab > 0 && (!io->token_ids || !m->globals_loaded)) return NF_ERR_INVALID_ARGUMENT;
+    if (m->cfg.vocab > 0 && io->token_src && (io->prev_rows < 0 || (io->prev_rows > 0 && !io->prev_token)))
+        return NF_ERR_INVALID_ARGUMENT;
     if (m->cfg.vocab == 0 && !io->hidden_in) return NF_ERR_INVALID_ARGUMENT;
     for (int l = 0; l < m->dims.L; ++l)
         if (!m->layers[l].loaded || io->kv_pools[l] == nullptr) return NF_ERR_INVALID_ARGUMENT;
@@ -636,7 +639,13 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     // prologue: decode work items, residual stream set-up
     NF_CUDA_TRY(decode_prologue(m, io, R, sg));
     if (m->cfg.vocab > 0) {
-        NF_CUDA_TRY(nf::launch_embed(io->token_ids, m->embed, T, d.H, m->cfg.vocab, m->resid, m->xb, m->partials,
+        const int* tokens = io->token_ids;
+        if (io->token_src) {
+            NF_CUDA_TRY(nf::launch_gather_tokens(io->token_ids, io->token_src, io->prev_token, io->prev_rows, T,
+                                                 m->tok_feedback, m->status, sg));
+            tokens = m->tok_feedback;
+        }
+        NF_CUDA_TRY(nf::launch_embed(tokens, m->embed, T, d.H, m->cfg.vocab, m->resid, m->xb, m->partials,
                                      m->status, S * 4, sg));
     } else {
         NF_CUDA_TRY(nf::launch_prep_hidden((const uint16_t*)io->hidden_in, T, d.H, m->resid, m->xb, m->partials, S * 4,

@@ -66,6 +66,26 @@ __global__ void embed_kernel(const int* __restrict__ tokens, const uint16_t* __r
     }
 }
 
+// Token feedback: out[t] = prev_token[src[t]] for src[t] >= 0 (the previous iteration's greedy
+// token of that request), else token_ids[t] (a prompt token).
+__global__ void gather_tokens_kernel(const int* __restrict__ token_ids, const int* __restrict__ src,
+                                     const int* __restrict__ prev_token, int prev_rows, int T, int* out,
+                                     int* status) {
+    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
+        const int s = src[t];
+        int tok;
+        if (s < 0) {
+            tok = token_ids[t];
+        } else if (s < prev_rows) {
+            tok = prev_token[s];
+        } else {
+            set_status(status, NF_ERR_DEVICE_BOUNDS);
+            tok = 0;
+        }
+        out[t] = tok;
+    }
+}
+
 // LM-head input rows: every decode row, then (if present) the chunk's last row.
 __global__ void lm_gather_kernel(const uint16_t* __restrict__ xb, const float* __restrict__ partials, int R,
                                  int T, int rows, int H, uint16_t* out, float* out_partials) {
@@ -159,6 +179,13 @@ cudaError_t launch_embed(const int* tokens, const uint16_t* table, int T, int H,
     if (T <= 0) return cudaSuccess;
     embed_kernel<<<grid_for((size_t)T * (H / 256), 8, max_blocks), 256, 0, s>>>(tokens, table, T, H, V, resid, xb,
                                                                                   partials, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_tokens(const int* token_ids, const int* src, const int* prev_token, int prev_rows, int T,
+                                 int* out, int* status, cudaStream_t s) {
+    if (T <= 0) return cudaSuccess;
+    gather_tokens_kernel<<<(T + 255) / 256, 256, 0, s>>>(token_ids, src, prev_token, prev_rows, T, out, status);
     return cudaGetLastError();
 }
 

@@ -9,6 +9,8 @@ cudaError_t launch_prep_hidden(const uint16_t* in, int T, int H, float* resid, u
                                int max_blocks, cudaStream_t s);
 cudaError_t launch_embed(const int* tokens, const uint16_t* table, int T, int H, int V, float* resid, uint16_t* xb,
                          float* partials, int* status, int max_blocks, cudaStream_t s);
+cudaError_t launch_gather_tokens(const int* token_ids, const int* src, const int* prev_token, int prev_rows, int T,
+                                 int* out, int* status, cudaStream_t s);
 cudaError_t launch_lm_gather(const uint16_t* xb, const float* partials, int R, int T, int rows, int H, uint16_t* out,
                              float* out_partials, int max_blocks, cudaStream_t s);
 cudaError_t launch_argmax_reduce(const float* tile_max, const int* tile_arg, int rows, int ntiles, int* next,

@@ -46,6 +46,7 @@ struct nf_model {
     float* rope_cos = nullptr;    // [max_position x d/2]
     float* rope_sin = nullptr;
     int* item_off = nullptr;      // [max_requests + 1]
+    int* tok_feedback = nullptr;  // [T] token ids gathered from the previous iteration's next_token
     float* splitk_ws = nullptr;   // split-K partials of the residual GEMMs: [tiles x 128 x 256] fp32
     int* splitk_flags = nullptr;  // [tiles]: epoch of the last published first half
     int splitk_epoch = 0;         // incremented per split-K launch
