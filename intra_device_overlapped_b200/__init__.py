@@ -104,7 +104,7 @@ class nf_sched_stats(ctypes.Structure):
 
 
 class nf_op_time(ctypes.Structure):
-    _fields_ = [("kernel_kind", _i32), ("nano", _i32), ("layer", _i32), ("stream", _i32), ("grid", _i32),
+    _fields_ = [("kind", _i32), ("nano", _i32), ("layer", _i32), ("stream", _i32), ("grid", _i32),
                 ("us", _f32)]
 
 
@@ -304,7 +304,7 @@ def nf_get_op_times(model: int, capacity: int = 8192):
     n = _lib.nf_get_op_times(model, buf, capacity)
     if n < 0:
         return int(-n), []
-    return NF_OK, [(NF_OP_NAMES[e.kernel_kind], e.nano, e.layer, e.stream, e.grid, e.us) for e in buf[:n]]
+    return NF_OK, [(NF_OP_NAMES[e.kind], e.nano, e.layer, e.stream, e.grid, e.us) for e in buf[:n]]
 
 
 def nf_op_gemm_bf16(a_ptr: int, b_ptr: int, c_ptr: int, M: int, N: int, K: int, sm_count: int = 0,
