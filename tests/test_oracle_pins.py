@@ -297,6 +297,51 @@ def test_written_kv_slots_follow_page_table(tiny_full):
         assert w[t] == (int(b.page_indices[b.page_indptr[r] + pos // 16]), pos % 16)
 
 
+def _lm_forward(s, batch, kv, bf16_act):
+    from oracle.run import layer_weights_f64
+    from synth import bf16_to_f64
+    from synth import weights as SW
+    g = SW.global_specs(s)
+    return F.iteration_forward(s, batch, lambda l: layer_weights_f64(s, l), kv,
+                               embed_rows=lambda t: bf16_to_f64(SW.host_rows(g["embed"], t)),
+                               final_norm=bf16_to_f64(SW.host_tensor(g["final_norm"])),
+                               lm_head=bf16_to_f64(SW.host_tensor(g["lm_head"])), bf16_act=bf16_act)
+
+
+def test_cached_decode_step_equals_full_sequence_recompute():
+    """Greedy decoding with a KV cache (prefill, then one decode row reading the cached pages)
+    gives the same logits as running prompt + token as one fresh prompt with no cache: the
+    identity that lets plain recomputation serve as the greedy-decoding reference."""
+    from oracle.run import make_kv
+    from synth.workloads import Batch
+    s = TEST_WORKLOADS["tiny_lm"].shape
+    prompt = RNG.integers(0, s.vocab, 21).tolist()
+    L = len(prompt)
+    npg = (L + 1 + 15) // 16
+    pages = np.array([3, 0, 5][:npg], dtype=np.int32)  # scattered pages of a larger pool
+    kv = make_kv(s)
+    pre = Batch(num_decode=0, prefill_len=L, ctx_lens=np.zeros(0, np.int32), page_size=16, num_pages=6,
+                page_indptr=np.array([0, npg], np.int32), page_indices=pages,
+                positions=np.arange(L, dtype=np.int32), tokens=np.array(prompt, np.int32))
+    r1 = _lm_forward(s, pre, kv, bf16_act=False)
+    tok = int(r1["next_token"][0])
+    dec = Batch(num_decode=1, prefill_len=0, ctx_lens=np.array([L], np.int32), page_size=16, num_pages=6,
+                page_indptr=np.array([0, npg, npg], np.int32), page_indices=pages,
+                positions=np.array([L], np.int32), tokens=np.array([tok], np.int32))
+    r2 = _lm_forward(s, dec, kv, bf16_act=False)
+    full = Batch(num_decode=0, prefill_len=L + 1, ctx_lens=np.zeros(0, np.int32), page_size=16, num_pages=npg,
+                 page_indptr=np.array([0, npg], np.int32), page_indices=np.arange(npg, dtype=np.int32),
+                 positions=np.arange(L + 1, dtype=np.int32), tokens=np.array(prompt + [tok], np.int32))
+    r3 = _lm_forward(s, full, make_kv(s), bf16_act=False)
+    assert np.allclose(r2["logits"][0], r3["logits"][0], rtol=0, atol=1e-9)
+    assert int(r2["next_token"][0]) == int(r3["next_token"][0])
+    # the first token agrees with the full recompute of the prompt alone, too
+    full_p = dataclasses.replace(full, prefill_len=L, positions=np.arange(L, dtype=np.int32),
+                                 tokens=np.array(prompt, np.int32))
+    assert np.allclose(_lm_forward(s, full_p, make_kv(s), bf16_act=False)["logits"][0], r1["logits"][0],
+                       rtol=0, atol=1e-9)
+
+
 # --- planted mistakes must be caught by the pins above --------------------------------------------
 
 def test_planted_mistakes_are_caught(monkeypatch):
