@@ -27,7 +27,8 @@
  * search over per-kernel costs.
  *
  * Conventions.
- *  - Every call returns an nf_status; nothing aborts or prints.
+ *  - Every call returns an nf_status; nothing aborts or prints. No C++ exception leaves the
+ *    library: a failed host allocation returns NF_ERR_OUT_OF_MEMORY.
  *  - bf16 tensors are passed as raw 16-bit patterns (void*), row-major.
  *  - Device pointers are owned by the caller unless stated otherwise; the model
  *    owns its packed weights and workspace (freed by nf_destroy_model).
@@ -411,7 +412,8 @@ typedef struct {
     int64_t discarded_tokens; /* tokens decoded after a request's last one (one per request at lag 1) */
 } nf_sched_stats;
 
-/* NF_ERR_INVALID_ARGUMENT for a bad configuration. */
+/* NF_ERR_INVALID_ARGUMENT for a bad configuration. After NF_ERR_OUT_OF_MEMORY from any
+ * nf_sched_* call the scheduler's state is unspecified: destroy it. */
 nf_status nf_sched_create(const nf_sched_config* cfg, nf_sched** out);
 void nf_sched_destroy(nf_sched* s);
 

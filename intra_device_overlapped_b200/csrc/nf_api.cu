@@ -143,7 +143,7 @@ extern "C" void nf_destroy_model(nf_model* m) {
     delete m;
 }
 
-extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) {
+extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) try {
     if (cfg == nullptr || out == nullptr) return NF_ERR_INVALID_ARGUMENT;
     *out = nullptr;
     if (!valid_config(*cfg)) {
@@ -256,9 +256,13 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) {
     if (!ok) { nf_destroy_model(m); return NF_ERR_CUDA; }
     *out = m;
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" nf_status nf_set_layer_weights(nf_model* m, int32_t layer, const nf_layer_weights* w, void* stream) {
+extern "C" nf_status nf_set_layer_weights(nf_model* m, int32_t layer, const nf_layer_weights* w, void* stream) try {
     if (m == nullptr || w == nullptr || layer < 0 || layer >= m->dims.L) return NF_ERR_INVALID_ARGUMENT;
     const nf::ModelDims& d = m->dims;
     cudaStream_t s = (cudaStream_t)stream;
@@ -311,9 +315,13 @@ extern "C" nf_status nf_set_layer_weights(nf_model* m, int32_t layer, const nf_l
     if (!ok) return NF_ERR_CUDA;
     L.loaded = true;
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" nf_status nf_set_global_weights(nf_model* m, const nf_global_weights* w, void* stream) {
+extern "C" nf_status nf_set_global_weights(nf_model* m, const nf_global_weights* w, void* stream) try {
     if (m == nullptr || w == nullptr) return NF_ERR_INVALID_ARGUMENT;
     if (m->cfg.vocab <= 0) return NF_ERR_INVALID_ARGUMENT;
     if (!w->embed || !w->final_norm || !w->lm_head) return NF_ERR_INVALID_ARGUMENT;
@@ -329,6 +337,10 @@ extern "C" nf_status nf_set_global_weights(nf_model* m, const nf_global_weights*
     if (!nf::make_tmap_bf16_2d(&m->tm_lm, m->lm_head, V, H, nf::kGemmBN)) return NF_ERR_CUDA;
     m->globals_loaded = true;
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
 // ------------------------------------------------------------------ executor
@@ -620,7 +632,7 @@ nf_status validate_forward(const nf_model* m, const nf_plan* p, const nf_iter_io
 
 }  // namespace
 
-extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const nf_iter_io* io, void* stream) {
+extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const nf_iter_io* io, void* stream) try {
     nf_status st = validate_forward(m, p, io);
     if (st != NF_OK) return st;
     const nf::ModelDims& d = m->dims;
@@ -713,6 +725,10 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     if (io->hidden_out_f32)
         NF_CUDA_TRY(cudaMemcpyAsync(io->hidden_out_f32, m->resid, (size_t)T * d.H * 4, cudaMemcpyDeviceToDevice, sg));
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
 // Search over measured costs: the planner's best plan for every (template, nano-batch count) is
@@ -720,7 +736,7 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
 // within a template well but misjudges how much co-running kernels slow one another, so the
 // final choice between templates and counts is made on the device.
 extern "C" nf_status nf_tune_plan(nf_model* m, const nf_batch_desc* b, const nf_iter_io* io, int32_t reps,
-                                  void* stream, nf_plan* out, float* best_us) {
+                                  void* stream, nf_plan* out, float* best_us) try {
     if (!m || !b || !io || !out || reps < 1) return NF_ERR_INVALID_ARGUMENT;
     cudaStream_t s = (cudaStream_t)stream;
     cudaEvent_t e0 = nullptr, e1 = nullptr;
@@ -776,9 +792,13 @@ extern "C" nf_status nf_tune_plan(nf_model* m, const nf_batch_desc* b, const nf_
     if (st != NF_OK) return st;
     if (result == NF_OK && best_us) *best_us = best;
     return result;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" nf_status nf_sync_status(nf_model* m) {
+extern "C" nf_status nf_sync_status(nf_model* m) try {
     if (m == nullptr) return NF_ERR_INVALID_ARGUMENT;
     if (cudaStreamSynchronize(m->s_attn) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
         cudaGetLastError();
@@ -788,15 +808,23 @@ extern "C" nf_status nf_sync_status(nf_model* m) {
     if (cudaMemcpy(&h, m->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return NF_ERR_CUDA;
     if (h != 0) cudaMemset(m->status, 0, sizeof(int));
     return (nf_status)h;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" nf_status nf_set_trace(nf_model* m, int32_t enable) {
+extern "C" nf_status nf_set_trace(nf_model* m, int32_t enable) try {
     if (m == nullptr) return NF_ERR_INVALID_ARGUMENT;
     m->trace_on = enable != 0;
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" int64_t nf_get_trace(nf_model* m, nf_trace_entry* out, int64_t capacity) {
+extern "C" int64_t nf_get_trace(nf_model* m, nf_trace_entry* out, int64_t capacity) try {
     if (m == nullptr || out == nullptr || capacity < 0) return -(int64_t)NF_ERR_INVALID_ARGUMENT;
     if (cudaDeviceSynchronize() != cudaSuccess) return -(int64_t)NF_ERR_CUDA;
     int n = 0;
@@ -805,16 +833,24 @@ extern "C" int64_t nf_get_trace(nf_model* m, nf_trace_entry* out, int64_t capaci
     if (n > 0 && cudaMemcpy(out, m->trace, (size_t)n * sizeof(nf_trace_entry), cudaMemcpyDeviceToHost) != cudaSuccess)
         return -(int64_t)NF_ERR_CUDA;
     return n;
+} catch (const std::bad_alloc&) {
+    return -(int64_t)NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return -(int64_t)NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" nf_status nf_set_timing(nf_model* m, int32_t enable) {
+extern "C" nf_status nf_set_timing(nf_model* m, int32_t enable) try {
     if (m == nullptr) return NF_ERR_INVALID_ARGUMENT;
     m->timing_on = enable != 0;
     m->t_ops.clear();
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" int64_t nf_get_op_times(nf_model* m, nf_op_time* out, int64_t capacity) {
+extern "C" int64_t nf_get_op_times(nf_model* m, nf_op_time* out, int64_t capacity) try {
     if (m == nullptr || out == nullptr || capacity < 0) return -(int64_t)NF_ERR_INVALID_ARGUMENT;
     if (cudaStreamSynchronize(m->s_attn) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
         return -(int64_t)NF_ERR_CUDA;
@@ -826,6 +862,10 @@ extern "C" int64_t nf_get_op_times(nf_model* m, nf_op_time* out, int64_t capacit
         out[i].us = ms * 1000.f;
     }
     return n;
+} catch (const std::bad_alloc&) {
+    return -(int64_t)NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return -(int64_t)NF_ERR_INVALID_ARGUMENT;
 }
 
 // ------------------------------------------------------------------ single ops
@@ -844,7 +884,7 @@ nf_status op_status_word(int** out) {
 }  // namespace
 
 extern "C" nf_status nf_op_gemm_bf16(const void* A, const void* B, float* C, int32_t M, int32_t N, int32_t K,
-                                     int32_t sm_count, void* stream) {
+                                     int32_t sm_count, void* stream) try {
     if (!A || !B || !C || M < 1 || N < 256 || N % 256 != 0 || K < 64 || K % 64 != 0) return NF_ERR_INVALID_ARGUMENT;
     int* status = nullptr;
     nf_status st = op_status_word(&status);
@@ -864,10 +904,14 @@ extern "C" nf_status nf_op_gemm_bf16(const void* A, const void* B, float* C, int
     const int grid = sm_count > 0 ? std::min(sm_count, sms) : sms;
     NF_CUDA_TRY(nf::launch_gemm(nf::EPI_F32, ta, tb, a, gemm_grid(a, grid), (cudaStream_t)stream));
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
 extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* out, const nf_iter_io* io, int32_t layer,
-                                            int32_t req_begin, int32_t req_end, int32_t sm_count, void* stream) {
+                                            int32_t req_begin, int32_t req_end, int32_t sm_count, void* stream) try {
     if (!m || !q || !out || !io || !io->ctx_len || !io->page_indptr || !io->page_indices || !io->kv_pools)
         return NF_ERR_INVALID_ARGUMENT;
     if (layer < 0 || layer >= m->dims.L || req_begin < 0 || req_end < req_begin || req_end > m->cfg.max_requests)
@@ -893,11 +937,15 @@ extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* ou
     const int grid = sm_count > 0 ? std::min(sm_count, m->sm_count) : m->sm_count;
     NF_CUDA_TRY(launch_decode(m, io, tmq, q, out, layer, req_begin, req_end, grid, s));
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
 extern "C" nf_status nf_op_prefill_attention(nf_model* m, const void* q, void* out, const nf_iter_io* io,
                                              int32_t layer, int32_t num_decode, int32_t prefill_len, int32_t sm_count,
-                                             void* stream) {
+                                             void* stream) try {
     if (!m || !q || !out || !io || !io->page_indptr || !io->page_indices || !io->kv_pools)
         return NF_ERR_INVALID_ARGUMENT;
     if (layer < 0 || layer >= m->dims.L || num_decode < 0 || prefill_len < 0) return NF_ERR_INVALID_ARGUMENT;
@@ -912,9 +960,13 @@ extern "C" nf_status nf_op_prefill_attention(nf_model* m, const void* q, void* o
         return NF_ERR_INVALID_ARGUMENT;
     NF_CUDA_TRY(launch_prefill(m, io, tmq3, q, out, layer, num_decode, prefill_len, grid, (cudaStream_t)stream));
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" nf_status nf_op_wait_flag_test(int32_t* flag_device, uint64_t limit_ns, void* stream) {
+extern "C" nf_status nf_op_wait_flag_test(int32_t* flag_device, uint64_t limit_ns, void* stream) try {
     if (flag_device == nullptr || limit_ns == 0 || limit_ns > 10000000000ull) return NF_ERR_INVALID_ARGUMENT;
     int* status = nullptr;
     nf_status st = op_status_word(&status);
@@ -926,6 +978,10 @@ extern "C" nf_status nf_op_wait_flag_test(int32_t* flag_device, uint64_t limit_n
     NF_CUDA_TRY(cudaMemcpyAsync(&h, status, sizeof(int), cudaMemcpyDeviceToHost, s));
     NF_CUDA_TRY(cudaStreamSynchronize(s));
     return (nf_status)h;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
 namespace {
@@ -950,7 +1006,7 @@ nf_status time_us(cudaStream_t s, int reps, F fn, double* out) {
 
 }  // namespace
 
-extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_iter_io* io, void* stream) {
+extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_iter_io* io, void* stream) try {
     if (m == nullptr || b == nullptr || io == nullptr) return NF_ERR_INVALID_ARGUMENT;
     const nf::ModelDims& d = m->dims;
     const int R = b->num_decode, C = b->prefill_len, T = R + C;
@@ -1061,17 +1117,25 @@ extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_
     c.calibrated = 1;
     m->cost = c;
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" nf_status nf_get_cost_model(const nf_model* m, nf_cost_model* out) {
+extern "C" nf_status nf_get_cost_model(const nf_model* m, nf_cost_model* out) try {
     if (m == nullptr || out == nullptr) return NF_ERR_INVALID_ARGUMENT;
     const nf::CostModel& c = m->cost;
     *out = nf_cost_model{c.gemm_flops_per_sm, c.gemm_tile_us, c.gemm_launch_us, c.hbm_bw, c.attn_bw_per_sm,
                          c.attn_launch_us, c.attn_flops_per_sm, c.interference, c.calibrated};
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" nf_status nf_set_cost_model(nf_model* m, const nf_cost_model* in) {
+extern "C" nf_status nf_set_cost_model(nf_model* m, const nf_cost_model* in) try {
     if (m == nullptr || in == nullptr) return NF_ERR_INVALID_ARGUMENT;
     if (!(in->gemm_flops_per_sm > 0) || !(in->hbm_bw > 0) || !(in->attn_bw_per_sm > 0) ||
         !(in->attn_flops_per_sm > 0) || in->interference < 0)
@@ -1080,4 +1144,8 @@ extern "C" nf_status nf_set_cost_model(nf_model* m, const nf_cost_model* in) {
                             in->attn_bw_per_sm, in->attn_launch_us, in->attn_flops_per_sm, in->interference,
                             in->calibrated};
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }

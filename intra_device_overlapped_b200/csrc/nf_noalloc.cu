@@ -12,6 +12,7 @@
 // Every call on a device shares that one array: two calls that overlap on the GPU (on
 // different streams, or from different host threads) race on it and may produce wrong
 // output. Serialise them.
+#include <new>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -59,7 +60,7 @@ extern "C" nf_status nf_decode_attention_noalloc(const void* q, void* out, const
                                                  const int32_t* ctx_len, const int32_t* page_indptr,
                                                  const int32_t* page_indices, int32_t num_requests,
                                                  int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
-                                                 int32_t sm_count, int32_t* status_device, void* stream) {
+                                                 int32_t sm_count, int32_t* status_device, void* stream) try {
     if (!q || !out || !kv_pool || !ctx_len || !page_indptr || !page_indices) return NF_ERR_INVALID_ARGUMENT;
     if (num_pages <= 0 || num_requests < 0 || sm_count < 0) return NF_ERR_INVALID_ARGUMENT;
     if (num_requests > NF_NOALLOC_MAX_REQUESTS) return NF_ERR_INVALID_ARGUMENT;  // scratch holds at most this many
@@ -107,4 +108,8 @@ extern "C" nf_status nf_decode_attention_noalloc(const void* q, void* out, const
     a.status = status;
     if (nf::launch_decode_attention_tc(tmq, a, grid, s) != cudaSuccess) return NF_ERR_CUDA;
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }

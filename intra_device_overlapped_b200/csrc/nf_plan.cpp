@@ -13,6 +13,7 @@
 // prefill-on-GEMM template still overlaps something: the decode attention (HBM-bound) on
 // sm_attn SMs beside the prefill attention (tensor-bound) on the others. Each candidate's
 // op list (build_ops) is simulated on two streams; the minimum makespan wins.
+#include <new>
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -286,12 +287,16 @@ nf_status plan_impl(const nf_model* m, const nf_batch_desc* b, const nf_plan_opt
 }
 
 extern "C" nf_status nf_plan_iteration(const nf_model* m, const nf_batch_desc* b, const nf_plan_opts* opts,
-                                       nf_plan* out) {
+                                       nf_plan* out) try {
     return plan_impl(m, b, opts, out);
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
 extern "C" nf_status nf_plan_for_config(const nf_model_config* cfg, int32_t sm_count, const nf_batch_desc* b,
-                                        const nf_plan_opts* opts, nf_plan* out) {
+                                        const nf_plan_opts* opts, nf_plan* out) try {
     if (cfg == nullptr || sm_count <= 0) return NF_ERR_INVALID_ARGUMENT;
     nf_model m;
     m.cfg = *cfg;
@@ -308,6 +313,10 @@ extern "C" nf_status nf_plan_for_config(const nf_model_config* cfg, int32_t sm_c
     m.cost = nf::default_cost_model(sm_count);
     if (m.dims.nkv <= 0 || m.dims.L <= 0) return NF_ERR_INVALID_ARGUMENT;
     return plan_impl(&m, b, opts, out);
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
 namespace {

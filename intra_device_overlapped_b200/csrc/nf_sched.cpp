@@ -71,7 +71,7 @@ bool valid_config(const nf_sched_config& c) {
 
 }  // namespace
 
-extern "C" nf_status nf_sched_create(const nf_sched_config* cfg, nf_sched** out) {
+extern "C" nf_status nf_sched_create(const nf_sched_config* cfg, nf_sched** out) try {
     if (!cfg || !out || !valid_config(*cfg)) return NF_ERR_INVALID_ARGUMENT;
     nf_sched* s = new (std::nothrow) nf_sched();
     if (!s) return NF_ERR_OUT_OF_MEMORY;
@@ -80,12 +80,16 @@ extern "C" nf_status nf_sched_create(const nf_sched_config* cfg, nf_sched** out)
     for (int32_t p = cfg->num_pages - 1; p >= 0; --p) s->free_pages.push_back(p);  // page 0 handed out first
     *out = s;
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
 extern "C" void nf_sched_destroy(nf_sched* s) { delete s; }
 
 extern "C" nf_status nf_sched_add_request(nf_sched* s, const int32_t* prompt, int32_t prompt_len,
-                                          int32_t max_new_tokens, int32_t eos_token, int64_t* id_out) {
+                                          int32_t max_new_tokens, int32_t eos_token, int64_t* id_out) try {
     if (!s || !prompt || !id_out || prompt_len < 1 || max_new_tokens < 1) return NF_ERR_INVALID_ARGUMENT;
     if (prompt_len > s->cfg.chunk_len) return NF_ERR_INVALID_ARGUMENT;          // one prompt = one chunk
     if ((int64_t)prompt_len + max_new_tokens > s->cfg.max_position) return NF_ERR_INVALID_ARGUMENT;
@@ -100,9 +104,13 @@ extern "C" nf_status nf_sched_add_request(nf_sched* s, const int32_t* prompt, in
     s->waiting.push_back(id);
     *id_out = id;
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" nf_status nf_sched_next(nf_sched* s, nf_sched_iter* out) {
+extern "C" nf_status nf_sched_next(nf_sched* s, nf_sched_iter* out) try {
     if (!s || !out) return NF_ERR_INVALID_ARGUMENT;
     // the batch of iteration k may only be formed once iteration k - 1 - lag has completed
     if (s->next_complete < s->next_iter - s->cfg.lag) return NF_ERR_INVALID_ARGUMENT;
@@ -184,9 +192,13 @@ extern "C" nf_status nf_sched_next(nf_sched* s, nf_sched_iter* out) {
         out->iteration = -1;  // nothing to run: no sequence number is used
     }
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" nf_status nf_sched_complete(nf_sched* s, int64_t iteration, const int32_t* next_token, int32_t rows) {
+extern "C" nf_status nf_sched_complete(nf_sched* s, int64_t iteration, const int32_t* next_token, int32_t rows) try {
     if (!s || !next_token || s->inflight.empty()) return NF_ERR_INVALID_ARGUMENT;
     const nf_sched::Inflight& it = s->inflight.front();
     if (iteration != it.iteration || rows != (int32_t)it.row_request.size()) return NF_ERR_INVALID_ARGUMENT;
@@ -211,10 +223,14 @@ extern "C" nf_status nf_sched_complete(nf_sched* s, int64_t iteration, const int
     s->inflight.pop_front();
     s->next_complete = iteration + 1;
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
 extern "C" nf_status nf_sched_request_tokens(const nf_sched* s, int64_t id, int32_t* out, int32_t cap, int32_t* len,
-                                             int32_t* finished) {
+                                             int32_t* finished) try {
     if (!s || !len || cap < 0 || (cap > 0 && !out)) return NF_ERR_INVALID_ARGUMENT;
     auto f = s->reqs.find(id);
     if (f == s->reqs.end()) return NF_ERR_INVALID_ARGUMENT;
@@ -224,9 +240,13 @@ extern "C" nf_status nf_sched_request_tokens(const nf_sched* s, int64_t id, int3
     *len = (int32_t)o.size();
     if (finished) *finished = f->second.finished ? 1 : 0;
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
 
-extern "C" nf_status nf_sched_get_stats(const nf_sched* s, nf_sched_stats* out) {
+extern "C" nf_status nf_sched_get_stats(const nf_sched* s, nf_sched_stats* out) try {
     if (!s || !out) return NF_ERR_INVALID_ARGUMENT;
     out->waiting = (int32_t)s->waiting.size();
     out->running = (int32_t)s->running.size();
@@ -236,4 +256,8 @@ extern "C" nf_status nf_sched_get_stats(const nf_sched* s, nf_sched_stats* out) 
     out->iterations = s->next_iter;
     out->discarded_tokens = s->discarded;
     return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
 }
