@@ -203,3 +203,14 @@ def test_batch_layout_matches_the_forward_contract():
         assert np.ctypeslib.as_array(it.row_request, shape=(2,)).tolist() == [0, 1]
     finally:
         nf.nf_sched_destroy(s)
+
+
+def test_serving_plan_shape_policy():
+    """Decode attention beside prefill attention only when both are present; one nano-batch."""
+    from intra_device_overlapped_b200.serving import default_plan_opts
+    pick = default_plan_opts(148, prefill_sms=8)
+    both, dec, pre = pick(7, 20), pick(8, 0), pick(0, 32)
+    assert (both.force_nano, both.force_template, both.force_sm_attn) == (1, nf.NF_TEMPLATE_PREFILL_ON_GEMM, 140)
+    for o in (dec, pre):
+        assert (o.force_nano, o.force_template) == (1, nf.NF_TEMPLATE_SEQUENTIAL)
+    assert default_plan_opts(12)(4, 4).force_template == nf.NF_TEMPLATE_SEQUENTIAL  # too few SMs to split
