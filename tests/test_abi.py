@@ -138,3 +138,49 @@ def test_planner_prefers_overlap_on_the_8b_layer(nf):
     assert st == 0 and p.order_template != nf.NF_TEMPLATE_SEQUENTIAL and p.n_nano >= 2
     st, seq = nf.nf_plan_for_config(model_config(w), 148, d, nf.nf_plan_opts(force_nano=1, force_template=0))
     assert p.predicted_us < seq.predicted_us
+
+
+def test_planner_fuzz_returns_valid_plans_or_invalid_argument(nf):
+    """Random batches (including empty decode sets, no prefill, tiny and long contexts, short page
+    tables) and random forced options: every call returns a plan that covers the batch with the
+    chunk whole, or NF_ERR_INVALID_ARGUMENT; none crashes."""
+    from intra_device_overlapped_b200.harness import model_config
+    from synth.workloads import WORKLOADS
+    rng = np.random.default_rng(99)
+    cfg = model_config(WORKLOADS["llama3_8b_layer"])
+    ok = 0
+    for case in range(300):
+        R = int(rng.choice([0, 1, 2, 7, 64, 300]))
+        C = int(rng.choice([0, 1, 17, 128, 1000]))
+        if R + C == 0:
+            continue
+        ctx = rng.integers(0, 3000, R).astype(np.int32)
+        counts = [(int(c) + 1 + 15) // 16 for c in ctx] + [(C + 15) // 16]
+        if rng.random() < 0.1 and R:
+            counts[int(rng.integers(0, R))] -= 1  # one request short of a page: must be rejected
+        indptr = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+        d = nf.nf_batch_desc(num_decode=R, prefill_len=C, prefix_len=0,
+                             ctx_len=ctx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                             page_indptr=indptr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                             num_pages=max(int(indptr[-1]), 1))
+        opts = nf.nf_plan_opts(force_nano=int(rng.integers(0, 5)), force_sm_attn=int(rng.choice([0, 8, 64, 140])),
+                               force_template=int(rng.integers(-1, 3)))
+        if opts.force_nano == 0 and opts.force_template == -1:
+            opts.force_nano = 1  # keep the full search (milliseconds per call) out of the loop
+        st, p = nf.nf_plan_for_config(cfg, 148, d, opts)
+        assert st in (0, nf.NF_ERR_INVALID_ARGUMENT), (case, st)
+        short = any(c < ((int(x) + 1 + 15) // 16) for c, x in zip(counts[:R], ctx))
+        if short:
+            assert st == nf.NF_ERR_INVALID_ARGUMENT, case
+        if st != 0:
+            continue
+        ok += 1
+        T = R + C
+        assert p.num_tokens == T and p.tok_begin[0] == 0 and p.tok_end[p.n_nano - 1] == T
+        for j in range(p.n_nano):
+            assert p.tok_end[j] > p.tok_begin[j]
+            assert not (R < p.tok_begin[j] < T)
+        assert sorted(p.nano_order[i] for i in range(p.n_nano)) == list(range(p.n_nano))
+        if p.order_template != nf.NF_TEMPLATE_SEQUENTIAL:
+            assert 1 <= p.sm_attn and p.sm_attn + p.sm_gemm <= 148
+    assert ok > 100
