@@ -131,7 +131,12 @@ void nf_destroy_model(nf_model* m);
 
 /* ------------------------------------------------------------------ plan */
 
-/* Host-side description of the iteration's batch. */
+/* Host-side description of the iteration's batch (host copies of the page table that the
+ * device copies in nf_iter_io hold). nf_plan_iteration, nf_tune_plan and nf_calibrate validate
+ * it before anything is launched: every request holds at least ceil(keys / 16) pages
+ * (keys = ctx_len[r] + 1 for a decode request, C for the chunk), the offsets start at 0 and
+ * grow, and every page id of every request lies in [0, num_pages); else
+ * NF_ERR_INVALID_ARGUMENT. */
 typedef struct {
     int32_t num_decode;        /* R >= 0 */
     int32_t prefill_len;       /* C >= 0 */
@@ -139,6 +144,7 @@ typedef struct {
     const int32_t* ctx_len;    /* host [R]: cached tokens per decode request (>= 0) */
     const int32_t* page_indptr; /* host [R + 2]: CSR offsets of each request's pages (prefill last) */
     int32_t num_pages;         /* pages in each layer's pool */
+    const int32_t* page_indices; /* host [page_indptr[R + 1]]: the page ids (required) */
 } nf_batch_desc;
 
 #define NF_MAX_NANO 4

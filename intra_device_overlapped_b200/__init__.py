@@ -51,7 +51,8 @@ class nf_global_weights(ctypes.Structure):
 
 class nf_batch_desc(ctypes.Structure):
     _fields_ = [("num_decode", _i32), ("prefill_len", _i32), ("prefix_len", _i32),
-                ("ctx_len", ctypes.POINTER(_i32)), ("page_indptr", ctypes.POINTER(_i32)), ("num_pages", _i32)]
+                ("ctx_len", ctypes.POINTER(_i32)), ("page_indptr", ctypes.POINTER(_i32)), ("num_pages", _i32),
+                ("page_indices", ctypes.POINTER(_i32))]
 
 
 class nf_plan_opts(ctypes.Structure):

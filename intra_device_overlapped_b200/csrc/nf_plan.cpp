@@ -335,6 +335,10 @@ nf_status plan_impl(const nf_model* m, const nf_batch_desc* b, const nf_plan_opt
         if (have < 0 || have < (keys + 15) / 16) return NF_ERR_INVALID_ARGUMENT;
     }
     if (b->page_indptr[0] != 0 || b->num_pages <= 0) return NF_ERR_INVALID_ARGUMENT;
+    // every page id a request owns must address the pool (checked here, before any launch)
+    if (b->page_indices == nullptr && b->page_indptr[R + 1] > 0) return NF_ERR_INVALID_ARGUMENT;
+    for (int i = 0; i < b->page_indptr[R + 1]; ++i)
+        if (b->page_indices[i] < 0 || b->page_indices[i] >= b->num_pages) return NF_ERR_INVALID_ARGUMENT;
 
     nf_plan_opts o;
     if (opts) o = *opts; else { std::memset(&o, 0, sizeof(o)); o.force_template = -1; }

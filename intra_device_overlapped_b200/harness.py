@@ -97,10 +97,12 @@ class DeviceWorkload:
         self.io = self.make_io()
         self._ctx_host = np.ascontiguousarray(b.ctx_lens, dtype=np.int32)
         self._indptr_host = np.ascontiguousarray(b.page_indptr, dtype=np.int32)
+        self._pages_host = np.ascontiguousarray(b.page_indices, dtype=np.int32)
         self.desc = nf_batch_desc(num_decode=R, prefill_len=C, prefix_len=0,
                                   ctx_len=self._ctx_host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                                   page_indptr=self._indptr_host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
-                                  num_pages=b.num_pages)
+                                  num_pages=b.num_pages,
+                                  page_indices=self._pages_host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
         torch.cuda.synchronize(self.device)
 
     # -- set-up -----------------------------------------------------------------------------------

@@ -103,7 +103,8 @@ class ServingSession:
                 if n:
                     d[key][:n].copy_(h[key][:n], non_blocking=True)
         desc = nf_batch_desc(num_decode=R, prefill_len=C, prefix_len=0, ctx_len=it.ctx_len,
-                             page_indptr=it.page_indptr, num_pages=self.num_pages)
+                             page_indptr=it.page_indptr, num_pages=self.num_pages,
+                             page_indices=it.page_indices)
         st, plan = nf_plan_iteration(self.model, desc, self.plan_opts(R, C))
         check(st, "nf_plan_iteration")
         io = nf_iter_io()

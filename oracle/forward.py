@@ -44,7 +44,8 @@ import numpy as np
 def bf16_round(x) -> np.ndarray:
     """Round float64 values to the nearest bf16 value (8 significant bits, ties to even).
 
-    Used only where the data format is bf16 (the paged KV cache).
+    Applied where the data format is bf16: the paged KV cache, and (bf16 model) the tensors one
+    operation hands to the next.
     """
     x = np.asarray(x, dtype=np.float64)
     m, e = np.frexp(x)                      # x = m * 2**e with 0.5 <= |m| < 1
@@ -224,9 +225,17 @@ def _request_of_token(t: int, R: int) -> int:
     return t if t < R else R
 
 
-def layer_forward(s, lw: dict, x: np.ndarray, batch, kv: PagedKV, layer: int, bf16_act: bool = True):
-    """One transformer layer over the whole batch (decode rows first, then the prefill chunk)."""
+def layer_forward(s, lw: dict, x: np.ndarray, batch, kv: PagedKV, layer: int, bf16_act: bool = True,
+                  rows: Optional[Sequence[int]] = None):
+    """One transformer layer over the whole batch (decode rows first, then the prefill chunk).
+
+    With ``rows`` only those token rows of the output are computed (and returned, in that order):
+    K/V of every token are still projected and written, since attention reads them, but attention,
+    the output projection and the FFN run on the listed rows only. Rows are independent after
+    attention, so these rows equal the same rows of the full computation.
+    """
     T, R, C = batch.num_tokens, batch.num_decode, batch.prefill_len
+    sel = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
     nq, nkv, d, P = s.n_q_heads, s.n_kv_heads, s.head_dim, s.page_size
     pos = np.asarray(batch.positions, dtype=np.int64)
 
@@ -248,18 +257,25 @@ def layer_forward(s, lw: dict, x: np.ndarray, batch, kv: PagedKV, layer: int, bf
         kv.write(layer, page, int(pos[t] % P), k[t], v[t])
         written[t] = (page, int(pos[t] % P))
 
-    o = np.zeros((T, nq, d), dtype=np.float64)
-    for r in range(R):
-        pages = batch.page_indices[batch.page_indptr[r]:batch.page_indptr[r + 1]]
-        K, V = kv.read(layer, pages, int(pos[r]) + 1)
-        o[r] = decode_attention(q[r], K, V, bf16_act)
-    if C > 0:
+    o = np.zeros((len(sel), nq, d), dtype=np.float64)
+    for i, t in enumerate(sel):
+        if t < R:
+            pages = batch.page_indices[batch.page_indptr[t]:batch.page_indptr[t + 1]]
+            K, V = kv.read(layer, pages, int(pos[t]) + 1)
+            o[i] = decode_attention(q[t], K, V, bf16_act)
+    pre = np.nonzero(sel >= R)[0]
+    if C > 0 and pre.size:
         pages = batch.page_indices[batch.page_indptr[R]:batch.page_indptr[R + 1]]
         K, V = kv.read(layer, pages, C)
-        o[R:] = prefill_attention(q[R:], K, V, bf16_p=bf16_act)
+        if rows is None:
+            o[pre] = prefill_attention(q[R:], K, V, bf16_p=bf16_act)
+        else:  # chunk rows at positions sel - R, causal over the chunk's keys
+            o[pre] = attention(q[sel[pre]], K, V, sel[pre] - R, np.arange(C), bf16_act)
 
     if bf16_act:
         o = bf16_round(o)
+    x = x[sel]
+    T = len(sel)
     h = x + o.reshape(T, nq * d) @ lw["wo"].T
     n2 = norm_operand(h, lw["ffn_norm"], s.rms_eps, bf16_act)
     extras = {"written": written}

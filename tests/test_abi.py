@@ -78,10 +78,12 @@ def test_init_without_device_or_with_bad_config(nf):
 def _desc(nf, b):
     ctx = np.ascontiguousarray(b.ctx_lens, dtype=np.int32)
     ip = np.ascontiguousarray(b.page_indptr, dtype=np.int32)
+    pg = np.ascontiguousarray(b.page_indices, dtype=np.int32)
     d = nf.nf_batch_desc(num_decode=b.num_decode, prefill_len=b.prefill_len, prefix_len=0,
                          ctx_len=ctx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
-                         page_indptr=ip.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), num_pages=b.num_pages)
-    return d, (ctx, ip)
+                         page_indptr=ip.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), num_pages=b.num_pages,
+                         page_indices=pg.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+    return d, (ctx, ip, pg)
 
 
 @pytest.mark.parametrize("name", ["tiny_layer", "llama3_8b_layer", "llama3_8b_full", "llama2_70b_slice",
@@ -128,6 +130,26 @@ def test_planner_rejects_short_page_table(nf):
     assert st == nf.NF_ERR_INVALID_ARGUMENT
 
 
+@pytest.mark.parametrize("bad", [-1, "num_pages", "missing"])
+def test_planner_rejects_page_ids_outside_the_pool(nf, bad):
+    """A page id < 0 or >= num_pages anywhere in the host page table (or no host table at all) is
+    rejected on the host with NF_ERR_INVALID_ARGUMENT, before any launch."""
+    from intra_device_overlapped_b200.harness import model_config
+    from synth.workloads import WORKLOADS, make_batch
+    w = WORKLOADS["tiny_layer"]
+    b = make_batch(w)
+    d, keep = _desc(nf, b)
+    st, _ = nf.nf_plan_for_config(model_config(w), 148, d, None)
+    assert st == 0
+    pg = keep[2]
+    if bad == "missing":
+        d.page_indices = ctypes.POINTER(ctypes.c_int32)()
+    else:
+        pg[int(b.page_indptr[3]) + 1] = -1 if bad == -1 else b.num_pages   # one id of request 3
+    st, _ = nf.nf_plan_for_config(model_config(w), 148, d, None)
+    assert st == nf.NF_ERR_INVALID_ARGUMENT
+
+
 def test_planner_prefers_overlap_on_the_8b_layer(nf):
     from intra_device_overlapped_b200.harness import model_config
     from synth.workloads import WORKLOADS, make_batch
@@ -159,10 +181,12 @@ def test_planner_fuzz_returns_valid_plans_or_invalid_argument(nf):
         if rng.random() < 0.1 and R:
             counts[int(rng.integers(0, R))] -= 1  # one request short of a page: must be rejected
         indptr = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+        pages = rng.permutation(max(int(indptr[-1]), 1)).astype(np.int32)
         d = nf.nf_batch_desc(num_decode=R, prefill_len=C, prefix_len=0,
                              ctx_len=ctx.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                              page_indptr=indptr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
-                             num_pages=max(int(indptr[-1]), 1))
+                             num_pages=max(int(indptr[-1]), 1),
+                             page_indices=pages.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
         opts = nf.nf_plan_opts(force_nano=int(rng.integers(0, 5)), force_sm_attn=int(rng.choice([0, 8, 64, 140])),
                                force_template=int(rng.integers(-1, 3)))
         if opts.force_nano == 0 and opts.force_template == -1:
