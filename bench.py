@@ -145,10 +145,6 @@ class ClockSampler:
 # kernel as it stands; the bench scales it to its own launches (traffic grows with the pages
 # read). Entries must be retaken whenever the kernel changes.
 TRAFFIC_PER_ALGO_BYTE = {
-    # decode_attention_tc_kernel<32>, 64 requests of llama3_8b_layer on 16 SMs:
-    # dram__bytes_read.sum 337.759 MB + dram__bytes_write.sum 5.042 MB for 338.166 MB of
-    # algorithmic bytes (337.117 MB of pages + 1.049 MB of q and o)
-    "decode_attention": (1.0137, "ncu: decode_attention_tc_kernel<32>, 64 of 512 requests, 16 SMs, scaled by pages"),
 }
 
 def iteration_flops(work, batch):
@@ -185,13 +181,12 @@ def op_algorithmic(work, batch, plan, op, nano):
     if op == "lm_head":
         return "tensor", 2.0 * (batch.num_decode + (1 if batch.prefill_len else 0)) * H * s.vocab
     if op == "decode_attention":
-        # K and V pages of every KV head of the decode requests, plus q in and o out
+        # K and V of every KV head for the ctx + 1 keys of each decode request: (ctx + 1) * 4096 B at
+        # the Llama-3-8B shape (8 KV heads x 128 x bf16 x 2)
         R = batch.num_decode
         r0, r1 = min(t0, R), min(t1, R)
-        pages = sum((int(batch.ctx_lens[r]) + 1 + 15) // 16 for r in range(r0, r1))
-        kv = pages * 2 * nkv * 16 * d * 2
-        qo = (r1 - r0) * nq * d * 2 * 2
-        return "hbm", float(kv + qo)
+        keys = sum(int(batch.ctx_lens[r]) + 1 for r in range(r0, r1))
+        return "hbm", float(keys * 2 * nkv * d * 2)
     if op == "prefill_attention":
         C = batch.prefill_len
         return "tensor", 4.0 * nq * d * C * (C + 1) / 2.0
@@ -208,7 +203,9 @@ def count_launches(work, plan):
         per_step += 1 if tc else 2        # decode schedule (+ split-item table on the warp-level path)
     for j in range(plan.n_nano):
         t0, t1 = plan.tok_begin[j], plan.tok_end[j]
-        att = (1 if min(t1, R) > min(t0, R) else 0) + (1 if t1 > R and plan.prefill_len else 0)
+        dec = 1 if min(t1, R) > min(t0, R) else 0
+        # tensor-core decode: the attention kernel and its split-KV merge pass
+        att = dec * (2 if tc else 1) + (1 if t1 > R and plan.prefill_len else 0)
         ffn = 6 if s.n_experts else 2      # MoE: route+sort, gather, 2 grouped GEMMs, combine
         per_step += s.n_layers * (1 + att + 1 + ffn)
     if s.vocab:
@@ -310,13 +307,21 @@ def run_ours(args, work, dist):
         plan, _ = dw.tune(reps=5)
     stream = torch.cuda.current_stream(dev)
 
-    for _ in range(max(args.warmup, 3)):
-        dw.forward(plan, stream)
+    # clocks are sampled (every 50 ms) from the start of the warm-up to the end of the timed region;
+    # the warm-up runs at least W steps and at least one second, so that the record holds samples
+    # under load even when the K timed steps take only milliseconds
+    clocks = ClockSampler(dist.local)
+    clocks.start()
+    t_warm = time.perf_counter()
+    nwarm = 0
+    while nwarm < max(args.warmup, 3) or time.perf_counter() - t_warm < 1.0:
+        for _ in range(8):
+            dw.forward(plan, stream)
+        nwarm += 8
+        torch.cuda.synchronize(dev)
     nf.check(dw.sync(), "warm-up")
 
     # ---- timed region: K iterations back to back (no per-op instrumentation inside it)
-    clocks = ClockSampler(dist.local)
-    clocks.start()
     dist.barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -410,6 +415,30 @@ def run_ours(args, work, dist):
                                 "sum_isolated_gemm_ms": round(sum(v for k, v in iso.items() if k not in att) / 1000, 4),
                                 "sum_isolated_attention_ms": round(sum(iso.get(k, 0.0) for k in att) / 1000, 4)}
 
+        # ---- each op alone at the plan's SM shares: the same sequential iteration restricted to the
+        # attention share (decode attention's time) and to the GEMM share (every other op's time)
+        if plan.order_template != nf.NF_TEMPLATE_SEQUENTIAL:
+            share = {}
+            for sms, keep in ((plan.sm_attn, lambda k: k == "decode_attention"),
+                              (plan.sm_gemm, lambda k: k != "decode_attention")):
+                sp = dw.plan(nano=1, template=0, sm_total=sms)
+                for _ in range(2):
+                    dw.forward(sp, stream)
+                nf.check(nf.nf_set_timing(dw.model, True), "timing")
+                nrep = max(3, args.steps // 4)
+                for _ in range(nrep):
+                    dw.forward(sp, stream)
+                torch.cuda.synchronize(dev)
+                st, sh_ops = nf.nf_get_op_times(dw.model, 1 << 20)
+                nf.nf_set_timing(dw.model, False)
+                for (name, nano, layer, stream_id, grid, us) in sh_ops:
+                    if keep(name):
+                        share[name] = share.get(name, 0.0) + us / nrep
+            extras["sequential"]["isolated_op_ms_at_plan_share"] = {
+                "sm_attn": plan.sm_attn, "sm_gemm": plan.sm_gemm,
+                "ops": {k: round(v / 1000, 4) for k, v in share.items()},
+                "sum_ms": round(sum(share.values()) / 1000, 4)}
+
         # ---- end to end through the C ABI with host buffers: every step copies its inputs from pinned
         # host memory to the device and reads its result back. As a serving loop does, the copies
         # of neighbouring steps overlap the compute of this one: two device input/output sets, the
@@ -486,7 +515,8 @@ def run_ours(args, work, dist):
                          f"inputs pre-generated, {times[0]:.1f} s"}
 
     line = {"metric": METRIC, "value": value, "unit": "decode tokens/s", "n_gpus": dist.world,
-            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 4),
+            "steps": args.steps, "warmup": max(args.warmup, 3), "warmup_steps_run": nwarm,
+            "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded random-init weights, seeded paged KV cache)",
             "config": {"workload": args.workload, "decode_requests": R, "prefill_len": b.prefill_len,

@@ -260,8 +260,16 @@ typedef struct {
     double attn_bw_per_sm;     /* bytes/s one SM of decode attention pulls */
     double attn_launch_us;
     double attn_flops_per_sm;  /* prefill attention FLOP/s per SM */
-    double interference;       /* fractional slow-down of a GEMM and an attention kernel co-running */
+    double interference;       /* fractional slow-down of a GEMM and an attention kernel co-running (mean of
+                                * the tables below; used where a table entry is missing) */
     int32_t calibrated;
+    /* Measured by nf_calibrate (zero = not measured): decode attention bytes/s on grids of 1/8, 1/4,
+     * 1/2, 3/4 and all of the SMs, and the fractional slow-downs of decode attention and of a GEMM on
+     * the remaining SMs when the two co-run with attention on 1/4, 1/2 and 3/4 of the SMs. The
+     * planner interpolates them linearly in the attention share. */
+    double attn_bw_at[5];
+    double interf_attn[3];
+    double interf_gemm[3];
 } nf_cost_model;
 
 nf_status nf_get_cost_model(const nf_model* m, nf_cost_model* out);
@@ -332,6 +340,25 @@ nf_status nf_op_prefill_attention(nf_model* m, const void* q, void* out, const n
  * outcome) after the kernel has given up and exited, or NF_OK if the flag was set. */
 nf_status nf_op_wait_flag_test(int32_t* flag_device, uint64_t limit_ns, void* stream);
 
+/* ------------------------------------------------------------------ KV offload
+ *
+ * Offload of a finished request's KV cache to host memory (hysenlabs review, "KV-cache offload to
+ * SSD": NanoFlow moves the KV cache of finished requests off the GPU so that a later turn of the
+ * same conversation can resume from it; only the device-to-host half is built here, the storage
+ * tiers are not). For every layer l in [layer_begin, layer_end), the n_pages pages listed in
+ * pages_host (host int32, each in [0, num_pool_pages)) of kv_pools[l] are copied, in list order,
+ * to host_dst + ((l - layer_begin) * n_pages + i) * page_bytes, page_bytes = 2 * nkv * 16 * d * 2
+ * (the physical page image described for nf_iter_io.kv_pools). Layer by layer, a gather kernel
+ * packs the pages into a model-owned staging buffer and one cudaMemcpyAsync moves them to the host,
+ * all on `stream`: issued on a stream of its own, the offload runs on the copy engine beside the
+ * next iterations. host_dst must be pinned (page-locked) host memory for the copies to overlap.
+ * The caller must not let an iteration rewrite the pages before the offload has completed (e.g.
+ * keep them out of the free pool until an event recorded on `stream` has passed). Asynchronous;
+ * NF_ERR_INVALID_ARGUMENT for a page id outside the pool, an empty or out-of-range layer range or
+ * a null pointer; NF_ERR_OUT_OF_MEMORY if the staging buffer cannot grow. Not thread-safe per model. */
+nf_status nf_offload_kv(nf_model* m, void* const* kv_pools, int32_t num_pool_pages, const int32_t* pages_host,
+                        int32_t n_pages, int32_t layer_begin, int32_t layer_end, void* host_dst, void* stream);
+
 /* Largest num_requests nf_decode_attention_noalloc accepts (size of its static scratch). */
 #define NF_NOALLOC_MAX_REQUESTS 16384
 
@@ -343,24 +370,30 @@ nf_status nf_op_wait_flag_test(int32_t* flag_device, uint64_t limit_ns, void* st
  * Computes, for each decode request r < num_requests and query head h, the softmax
  * attention of q[r][h] over the ctx_len[r] + 1 cached keys of KV head h / (nq / nkv),
  * gathered through the page table (the operation nf_forward_iteration runs as its decode
- * attention step), with the same tensor-core kernel as nf_op_decode_attention.
+ * attention step), with the same tensor-core kernel as nf_op_decode_attention. Each request is
+ * one work item here (no split along the keys, whose partials would need scratch that grows
+ * with the batch), so the result equals nf_op_decode_attention's bit for bit for requests of at
+ * most 512 keys (which that entry point does not split either) and within rounding otherwise.
  *   q, out        device bf16 [num_requests x n_q_heads x head_dim], row r = request r.
  *   kv_pool       device bf16 pool of one layer, num_pages pages in the physical page layout
  *                 described for nf_iter_io.kv_pools.
  *   ctx_len       device int32 [num_requests]; page_indptr device int32 [num_requests + 1];
- *   page_indices  device int32 (CSR page table; request r owns page_indices[page_indptr[r] ..]).
+ *   page_indices  device int32 (CSR page table; request r owns page_indices[page_indptr[r] ..],
+ *                 at least ceil((ctx_len[r] + 1) / 16) entries).
  *   sm_count      persistent grid (0 = every SM).
- *   status_device optional device int32 the caller zeroes; receives the first device-detected
- *                 error (NF_ERR_DEVICE_BOUNDS for a page index outside the pool,
- *                 NF_ERR_DEVICE_TIMEOUT for a pipeline wait that passed its limit). NULL: the
- *                 errors go to the library's scratch only.
+ *   status_device device int32 the caller zeroes (required; NULL gives NF_ERR_INVALID_ARGUMENT);
+ *                 receives the first device-detected error: NF_ERR_DEVICE_BOUNDS for a page id
+ *                 outside the pool, a request row shorter than its keys need (page 0 is read in
+ *                 its place) or a negative ctx_len (read as 0); NF_ERR_DEVICE_TIMEOUT for a
+ *                 pipeline wait that passed its limit.
  * Supported shapes: head_dim 128, n_kv_heads 8, n_q_heads 32 or 64 (else NF_ERR_UNSUPPORTED).
  * num_requests > NF_NOALLOC_MAX_REQUESTS returns NF_ERR_INVALID_ARGUMENT.
- * Scratch: a static device array of 66 KB per device (status word and the per-request page
- * prefix), shared by every call: calls that overlap on the GPU race on it and must be
- * serialised. The first call on each device looks up the array's address
- * (cudaGetSymbolAddress); make that first call before any stream capture. Asynchronous on
- * `stream`; no call allocates device or pinned memory. */
+ * Scratch: a static device array of 64 KB per device (the per-request page prefix), shared by
+ * every call: calls that overlap on the GPU race on it and must be serialised. The first call
+ * on each device looks up the array's address (cudaGetSymbolAddress) and keeps it for the life
+ * of the process; make that first call before any stream capture, and do not call the entry
+ * point again on a device after cudaDeviceReset (the kept address would be stale). Asynchronous
+ * on `stream`; no call allocates device or pinned memory. */
 nf_status nf_decode_attention_noalloc(const void* q, void* out, const void* kv_pool, int32_t num_pages,
                                       const int32_t* ctx_len, const int32_t* page_indptr,
                                       const int32_t* page_indices, int32_t num_requests, int32_t n_q_heads,

@@ -116,10 +116,16 @@ class nf_cost_model(ctypes.Structure):
     _fields_ = [("gemm_flops_per_sm", ctypes.c_double), ("gemm_tile_us", ctypes.c_double),
                 ("gemm_launch_us", ctypes.c_double), ("hbm_bw", ctypes.c_double),
                 ("attn_bw_per_sm", ctypes.c_double), ("attn_launch_us", ctypes.c_double),
-                ("attn_flops_per_sm", ctypes.c_double), ("interference", ctypes.c_double), ("calibrated", _i32)]
+                ("attn_flops_per_sm", ctypes.c_double), ("interference", ctypes.c_double), ("calibrated", _i32),
+                ("attn_bw_at", ctypes.c_double * 5), ("interf_attn", ctypes.c_double * 3),
+                ("interf_gemm", ctypes.c_double * 3)]
 
     def as_dict(self) -> dict:
-        return {f: getattr(self, f) for f, _ in self._fields_}
+        out = {}
+        for f, _ in self._fields_:
+            v = getattr(self, f)
+            out[f] = list(v) if isinstance(v, ctypes.Array) else v
+        return out
 
 
 class nf_trace_entry(ctypes.Structure):
@@ -159,6 +165,7 @@ def _load():
         "nf_op_wait_flag_test": ([_vp, _u64, _vp], ctypes.c_int),
         "nf_decode_attention_noalloc": ([_vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp],
                                         ctypes.c_int),
+        "nf_offload_kv": ([_vp, P(_vp), _i32, P(_i32), _i32, _i32, _i32, _vp, _vp], ctypes.c_int),
         "nf_sched_create": ([P(nf_sched_config), P(_vp)], ctypes.c_int),
         "nf_sched_destroy": ([_vp], None),
         "nf_sched_add_request": ([_vp, P(_i32), _i32, _i32, _i32, P(_i64)], ctypes.c_int),
@@ -179,6 +186,7 @@ EXPORTED = ("nf_status_string", "nf_version", "nf_init_model", "nf_set_layer_wei
             "nf_destroy_model", "nf_plan_iteration", "nf_plan_for_config", "nf_forward_iteration", "nf_tune_plan", "nf_sync_status", "nf_calibrate",
             "nf_get_cost_model", "nf_set_cost_model",
             "nf_set_trace", "nf_get_trace", "nf_set_timing", "nf_get_op_times", "nf_op_gemm_bf16", "nf_op_decode_attention",
+            "nf_offload_kv",
             "nf_op_prefill_attention", "nf_op_wait_flag_test", "nf_decode_attention_noalloc",
             "nf_sched_create", "nf_sched_destroy", "nf_sched_add_request", "nf_sched_next", "nf_sched_complete",
             "nf_sched_request_tokens", "nf_sched_get_stats")
@@ -195,6 +203,14 @@ def nf_decode_attention_noalloc(q_ptr: int, out_ptr: int, kv_pool_ptr: int, num_
     return _lib.nf_decode_attention_noalloc(q_ptr, out_ptr, kv_pool_ptr, num_pages, ctx_len_ptr, page_indptr_ptr,
                                             page_indices_ptr, num_requests, n_q_heads, n_kv_heads, head_dim,
                                             sm_count, status_ptr or None, stream or None)
+
+
+def nf_offload_kv(model: int, kv_pools, num_pool_pages: int, pages, layer_begin: int, layer_end: int,
+                  host_dst_ptr: int, stream: int = 0) -> int:
+    """KV pages of layers [layer_begin, layer_end) to pinned host memory (see nanoflow.h)."""
+    ids = (_i32 * len(pages))(*[int(p) for p in pages])
+    return _lib.nf_offload_kv(model, kv_pools, num_pool_pages, ids, len(pages), layer_begin, layer_end,
+                              host_dst_ptr, stream)
 
 
 class NanoflowError(RuntimeError):

@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstring>
 #include <new>
+#include <memory>
 #include <vector>
 
 #include <cuda.h>
@@ -71,7 +72,8 @@ void set_tiles(GemmArgs& a, int M, int N, int K) {
 }
 
 int gemm_grid(const GemmArgs& a, int grid) {
-    const int units = a.m_tiles * a.n_tiles * (a.k_split == 2 ? 2 : 1);
+    const int units = nf::gemm_units(a);
+    if (nf::gemm_uses_pairs(a) && grid >= 2) return std::max(2, std::min(grid, 2 * units) & ~1);
     return std::max(1, std::min(grid, units));
 }
 
@@ -158,8 +160,21 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) t
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     if (major < 10) return NF_ERR_UNSUPPORTED;
 
+    // RoPE angles pos * theta^(-2i/d) in double, stored as fp32 cos / sin: the host tables are built
+    // before any device memory exists, so a failed host allocation cannot strand device buffers.
+    const int half = cfg->head_dim / 2;
+    std::vector<float> rope_c((size_t)cfg->max_position * half), rope_s(rope_c.size());
+    for (int p = 0; p < cfg->max_position; ++p)
+        for (int i = 0; i < half; ++i) {
+            const double ang = (double)p * std::pow((double)cfg->rope_theta, -2.0 * i / cfg->head_dim);
+            rope_c[(size_t)p * half + i] = (float)std::cos(ang);
+            rope_s[(size_t)p * half + i] = (float)std::sin(ang);
+        }
+
     nf_model* m = new (std::nothrow) nf_model();
     if (m == nullptr) return NF_ERR_OUT_OF_MEMORY;
+    // owns the model until it is handed out: every early return, and any exception, frees it
+    std::unique_ptr<nf_model, void (*)(nf_model*)> guard(m, nf_destroy_model);
     m->cfg = *cfg;
     nf::ModelDims& d = m->dims;
     d.L = cfg->n_layers;
@@ -192,9 +207,12 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) t
     ok &= (m->rope_cos = dalloc<float>(m, (size_t)cfg->max_position * d.d / 2)) != nullptr;
     ok &= (m->rope_sin = dalloc<float>(m, (size_t)cfg->max_position * d.d / 2)) != nullptr;
     ok &= (m->item_off = dalloc<int>(m, (size_t)cfg->max_requests + 1)) != nullptr;
+    ok &= (m->chunk_off = dalloc<int>(m, (size_t)cfg->max_requests + 1)) != nullptr;
+    ok &= (m->tile_ctr = dalloc<int>(m, nf::kMaxCountedOps)) != nullptr;
     if (cfg->vocab > 0) ok &= (m->tok_feedback = dalloc<int>(m, T)) != nullptr;
     {  // split-K workspace of the residual GEMMs (O and down: N = hidden)
-        const size_t tiles = (size_t)((T + nf::kGemmBM - 1) / nf::kGemmBM) * (d.H / nf::kGemmBN);
+        // 128-row tiles, or two 128-row halves of each 256-row pair tile (at most one tile row more)
+        const size_t tiles = (size_t)((T + nf::kGemmBM - 1) / nf::kGemmBM + 1) * (d.H / nf::kGemmBN);
         ok &= (m->splitk_ws = dalloc<float>(m, tiles * nf::kGemmBM * nf::kGemmBN)) != nullptr;
         ok &= (m->splitk_flags = dalloc<int>(m, tiles)) != nullptr;
         if (ok) ok = cudaMemset(m->splitk_flags, 0, tiles * sizeof(int)) == cudaSuccess;
@@ -221,31 +239,20 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) t
         ok &= (m->moe_part = dalloc<float>(m, TK * m->n_part)) != nullptr;
         ok &= (m->moe_y = dalloc<float>(m, TK * d.H)) != nullptr;
     }
-    if (!ok) { nf_destroy_model(m); return NF_ERR_OUT_OF_MEMORY; }
+    if (!ok) return NF_ERR_OUT_OF_MEMORY;
 
-    // RoPE angles pos * theta^(-2i/d) in double, stored as fp32 cos / sin.
-    {
-        const int half = d.d / 2;
-        std::vector<float> c((size_t)cfg->max_position * half), s(c.size());
-        for (int p = 0; p < cfg->max_position; ++p)
-            for (int i = 0; i < half; ++i) {
-                const double ang = (double)p * std::pow((double)cfg->rope_theta, -2.0 * i / d.d);
-                c[(size_t)p * half + i] = (float)std::cos(ang);
-                s[(size_t)p * half + i] = (float)std::sin(ang);
-            }
-        if (cudaMemcpy(m->rope_cos, c.data(), c.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
-            cudaMemcpy(m->rope_sin, s.data(), s.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
-            nf_destroy_model(m);
-            return NF_ERR_CUDA;
-        }
-    }
-    if (cudaMemset(m->status, 0, sizeof(int)) != cudaSuccess ||
-        cudaStreamCreateWithFlags(&m->s_attn, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&m->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&m->ev_join, cudaEventDisableTiming) != cudaSuccess) {
-        nf_destroy_model(m);
+    // The attention stream has the highest priority: when an attention kernel and a GEMM wait for SMs
+    // at the same time, the attention kernel's CTAs are placed first.
+    int prio_least = 0, prio_greatest = 0;
+    if (cudaMemcpy(m->rope_cos, rope_c.data(), rope_c.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(m->rope_sin, rope_s.data(), rope_s.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
         return NF_ERR_CUDA;
-    }
+    if (cudaMemset(m->status, 0, sizeof(int)) != cudaSuccess ||
+        cudaDeviceGetStreamPriorityRange(&prio_least, &prio_greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&m->s_attn, cudaStreamNonBlocking, prio_greatest) != cudaSuccess ||
+        cudaEventCreateWithFlags(&m->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&m->ev_join, cudaEventDisableTiming) != cudaSuccess)
+        return NF_ERR_CUDA;
     ok = nf::make_tmap_bf16_2d(&m->tm_xb, m->xb, T, d.H, nf::kGemmBM) &&
          nf::make_tmap_bf16_2d(&m->tm_attn_o, m->attn_o, T, (uint64_t)d.nq * d.d, nf::kGemmBM) &&
          nf::make_tmap_bf16_2d(&m->tm_act, m->act, act_rows, d.F, nf::kGemmBM);
@@ -253,8 +260,8 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) t
     if (ok && m->decode_tc) ok = nf::make_tmap_bf16_2d(&m->tm_q, m->q, T * d.nq, d.d, (uint32_t)d.nq);
     if (ok && m->prefill_tc) ok = nf::make_tmap_bf16_3d_heads(&m->tm_q3, m->q, T, d.nq, d.d, 128);
     if (ok && d.E > 0) ok = nf::make_tmap_bf16_2d(&m->tm_moe_a, m->moe_a, TK, d.H, nf::kGemmBM);
-    if (!ok) { nf_destroy_model(m); return NF_ERR_CUDA; }
-    *out = m;
+    if (!ok) return NF_ERR_CUDA;
+    *out = guard.release();
     return NF_OK;
 } catch (const std::bad_alloc&) {
     return NF_ERR_OUT_OF_MEMORY;
@@ -308,10 +315,10 @@ extern "C" nf_status nf_set_layer_weights(nf_model* m, int32_t layer, const nf_l
         NF_CUDA_TRY(nf::launch_widen_scaled((const uint16_t*)w->router, L.router, d.E, d.H, fn, s));
         NF_CUDA_TRY(nf::launch_widen_scaled((const uint16_t*)w->router_bias, L.router_bias, 1, d.E, nullptr, s));
     }
-    bool ok = nf::make_tmap_bf16_2d(&L.tm_qkv, L.wqkv, d.qkv, d.H, nf::kGemmBN) &&
-              nf::make_tmap_bf16_2d(&L.tm_o, L.wo, d.H, qd, nf::kGemmBN) &&
-              nf::make_tmap_bf16_2d(&L.tm_gu, L.wgu, (uint64_t)E * 2 * d.F, d.H, nf::kGemmBN) &&
-              nf::make_tmap_bf16_2d(&L.tm_d, L.wd, (uint64_t)E * d.H, d.F, nf::kGemmBN);
+    bool ok = nf::make_tmap_bf16_2d(&L.tm_qkv, L.wqkv, d.qkv, d.H, nf::kGemmBBoxRows) &&
+              nf::make_tmap_bf16_2d(&L.tm_o, L.wo, d.H, qd, nf::kGemmBBoxRows) &&
+              nf::make_tmap_bf16_2d(&L.tm_gu, L.wgu, (uint64_t)E * 2 * d.F, d.H, nf::kGemmBBoxRows) &&
+              nf::make_tmap_bf16_2d(&L.tm_d, L.wd, (uint64_t)E * d.H, d.F, nf::kGemmBBoxRows);
     if (!ok) return NF_ERR_CUDA;
     L.loaded = true;
     return NF_OK;
@@ -334,7 +341,7 @@ extern "C" nf_status nf_set_global_weights(nf_model* m, const nf_global_weights*
     NF_CUDA_TRY(cudaMemcpyAsync(m->embed, w->embed, (size_t)V * H * 2, cudaMemcpyDeviceToDevice, s));
     NF_CUDA_TRY(nf::launch_pack_rows((const uint16_t*)w->lm_head, m->lm_head, V, H,
                                      (const uint16_t*)w->final_norm, V, 0, 0, s));
-    if (!nf::make_tmap_bf16_2d(&m->tm_lm, m->lm_head, V, H, nf::kGemmBN)) return NF_ERR_CUDA;
+    if (!nf::make_tmap_bf16_2d(&m->tm_lm, m->lm_head, V, H, nf::kGemmBBoxRows)) return NF_ERR_CUDA;
     m->globals_loaded = true;
     return NF_OK;
 } catch (const std::bad_alloc&) {
@@ -360,8 +367,11 @@ nf_status ensure_part_capacity(nf_model* m, int64_t items) {
     dfree(m, m->part_o);
     dfree(m, m->part_lse);
     dfree(m, m->item_tab);
-    m->part_o = dalloc<float>(m, (size_t)cap * m->dims.nq / m->dims.nkv * m->dims.d);
-    m->part_lse = dalloc<float>(m, (size_t)cap * m->dims.nq / m->dims.nkv);
+    // per item: the tensor-core kernel's chunk holds every query head (O and max / sum pairs), the
+    // warp-level kernel's item the G heads of one KV head
+    const size_t heads = m->decode_tc ? (size_t)m->dims.nq : (size_t)(m->dims.nq / m->dims.nkv);
+    m->part_o = dalloc<float>(m, (size_t)cap * heads * m->dims.d);
+    m->part_lse = dalloc<float>(m, (size_t)cap * heads * 2);
     m->item_tab = dalloc<int4>(m, (size_t)cap);
     if (!m->part_o || !m->part_lse || !m->item_tab) { m->part_capacity = 0; return NF_ERR_OUT_OF_MEMORY; }
     m->part_capacity = cap;
@@ -389,6 +399,8 @@ nf::DecodeArgs decode_args(const nf_model* m, const nf_iter_io* io, const void* 
     a.split_pages = nf::kDecodeSplitPages;
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m->dims.d));
     a.merge_cnt = m->merge_cnt;
+    a.chunk_off = m->chunk_off;
+    a.part_ml = m->part_lse;
     a.status = m->status;
     if (m->trace_on) { a.trace_ctr = m->trace_ctr; a.trace = m->trace; a.trace_cap = m->trace_cap; }
     return a;
@@ -440,7 +452,9 @@ struct OpTimer {
 cudaError_t decode_prologue(nf_model* m, const nf_iter_io* io, int R, cudaStream_t s) {
     if (R <= 0) return cudaSuccess;
     const nf::ModelDims& d = m->dims;
-    if (m->decode_tc) return nf::launch_decode_schedule(io->ctx_len, R, 1, 1, m->item_off, s);
+    if (m->decode_tc)
+        return nf::launch_decode_tc_schedule(io->ctx_len, R, nf::kDecodeSplitPages, m->item_off, m->chunk_off,
+                                             m->status, s);
     cudaError_t e = nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, s);
     if (e != cudaSuccess) return e;
     return nf::launch_decode_items(io->ctx_len, io->page_indptr, R, d.nkv, nf::kDecodeSplitPages, m->item_off,
@@ -466,7 +480,7 @@ cudaError_t launch_prefill(nf_model* m, const nf_iter_io* io, const CUtensorMap&
 }
 
 nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::Op& op, int grid,
-                 cudaStream_t s) {
+                 cudaStream_t s, int* tile_ctr) {
     const nf::ModelDims& d = m->dims;
     const int j = op.nano, l = op.layer;
     const int t0 = p->tok_begin[j], t1 = p->tok_end[j], M = t1 - t0;
@@ -476,6 +490,7 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
     GemmArgs a = base_args(m);
     a.a_row0 = t0;
     a.tok0 = t0;
+    a.tile_ctr = tile_ctr;
     switch (op.kind) {
         case nf::OP_QKV: {
             set_tiles(a, M, d.qkv, d.H);
@@ -644,6 +659,8 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
         if ((st = check_pool(m, l, io)) != NF_OK) return st;
 
     const int S = p->sm_total;
+    // one zeroed work counter per op that claims its GEMM tiles dynamically (elastic ops)
+    NF_CUDA_TRY(cudaMemsetAsync(m->tile_ctr, 0, nf::kMaxCountedOps * sizeof(int), sg));
     NF_CUDA_TRY(cudaEventRecord(m->ev_fork, sg));
     NF_CUDA_TRY(cudaStreamWaitEvent(sa, m->ev_fork, 0));
     if (m->trace_on) NF_CUDA_TRY(cudaMemsetAsync(m->trace_ctr, 0, sizeof(int), sg));
@@ -685,7 +702,8 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
         const int grid = nf::op_grid(*p, op);
         OpTimer tm{m};
         NF_CUDA_TRY(tm.begin(s));
-        if ((st = run_op(m, p, io, op, grid, s)) != NF_OK) return st;
+        int* ctr = (op.elastic && i < (size_t)nf::kMaxCountedOps) ? m->tile_ctr + i : nullptr;
+        if ((st = run_op(m, p, io, op, op.elastic && !ctr ? p->sm_gemm : grid, s, ctr)) != NF_OK) return st;
         NF_CUDA_TRY(tm.end(s, kTimingKind[op.kind], op.nano, op.layer, op.stream, grid));
         if (io->layer_hidden_out && (op.kind == nf::OP_D || op.kind == nf::OP_MOE)) {
             // the nano-batch's rows have finished this layer: copy them out before any later op
@@ -891,7 +909,7 @@ extern "C" nf_status nf_op_gemm_bf16(const void* A, const void* B, float* C, int
     if (st != NF_OK) return st;
     CUtensorMap ta, tb;
     if (!nf::make_tmap_bf16_2d(&ta, A, (uint64_t)M, (uint64_t)K, nf::kGemmBM) ||
-        !nf::make_tmap_bf16_2d(&tb, B, (uint64_t)N, (uint64_t)K, nf::kGemmBN))
+        !nf::make_tmap_bf16_2d(&tb, B, (uint64_t)N, (uint64_t)K, nf::kGemmBBoxRows))
         return NF_ERR_INVALID_ARGUMENT;
     GemmArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -920,11 +938,17 @@ extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* ou
     cudaStream_t s = (cudaStream_t)stream;
     nf_status st = check_pool(m, layer, io);
     if (st != NF_OK) return st;
-    if (!m->decode_tc) {
-        NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, req_end, m->dims.nkv, nf::kDecodeSplitPages, m->item_off,
-                                               s));
+    {  // work items of these requests (the device holds ctx_len): size the split-KV partials
         int items = 0;
-        NF_CUDA_TRY(cudaMemcpyAsync(&items, m->item_off + req_end, sizeof(int), cudaMemcpyDeviceToHost, s));
+        if (m->decode_tc) {
+            NF_CUDA_TRY(nf::launch_decode_tc_schedule(io->ctx_len, req_end, nf::kDecodeSplitPages, m->item_off,
+                                                      m->chunk_off, m->status, s));
+            NF_CUDA_TRY(cudaMemcpyAsync(&items, m->chunk_off + req_end, sizeof(int), cudaMemcpyDeviceToHost, s));
+        } else {
+            NF_CUDA_TRY(nf::launch_decode_schedule(io->ctx_len, req_end, m->dims.nkv, nf::kDecodeSplitPages,
+                                                   m->item_off, s));
+            NF_CUDA_TRY(cudaMemcpyAsync(&items, m->item_off + req_end, sizeof(int), cudaMemcpyDeviceToHost, s));
+        }
         NF_CUDA_TRY(cudaStreamSynchronize(s));
         if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
     }
@@ -959,6 +983,43 @@ extern "C" nf_status nf_op_prefill_attention(nf_model* m, const void* q, void* o
                                                       m->dims.d, 128))
         return NF_ERR_INVALID_ARGUMENT;
     NF_CUDA_TRY(launch_prefill(m, io, tmq3, q, out, layer, num_decode, prefill_len, grid, (cudaStream_t)stream));
+    return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
+}
+
+extern "C" nf_status nf_offload_kv(nf_model* m, void* const* kv_pools, int32_t num_pool_pages, const int32_t* pages_host,
+                                   int32_t n_pages, int32_t layer_begin, int32_t layer_end, void* host_dst,
+                                   void* stream) try {
+    if (!m || !kv_pools || !pages_host || !host_dst || n_pages <= 0 || num_pool_pages <= 0) return NF_ERR_INVALID_ARGUMENT;
+    if (layer_begin < 0 || layer_end > m->dims.L || layer_end <= layer_begin) return NF_ERR_INVALID_ARGUMENT;
+    for (int i = 0; i < n_pages; ++i)
+        if (pages_host[i] < 0 || pages_host[i] >= num_pool_pages) return NF_ERR_INVALID_ARGUMENT;
+    for (int l = layer_begin; l < layer_end; ++l)
+        if (!kv_pools[l] || (reinterpret_cast<uintptr_t>(kv_pools[l]) & 15u) != 0) return NF_ERR_INVALID_ARGUMENT;
+    const size_t page_bytes = (size_t)2 * m->dims.nkv * 16 * m->dims.d * 2;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (n_pages > m->offload_cap) {
+        // grow the staging (earlier offloads on other streams may still read the old buffers)
+        NF_CUDA_TRY(cudaDeviceSynchronize());
+        dfree(m, m->offload_stage);
+        dfree(m, m->offload_ids);
+        m->offload_stage = dalloc<uint8_t>(m, 2 * (size_t)n_pages * page_bytes);
+        m->offload_ids = dalloc<int>(m, (size_t)n_pages);
+        if (!m->offload_stage || !m->offload_ids) { m->offload_cap = 0; return NF_ERR_OUT_OF_MEMORY; }
+        m->offload_cap = n_pages;
+    }
+    NF_CUDA_TRY(cudaMemcpyAsync(m->offload_ids, pages_host, sizeof(int) * n_pages, cudaMemcpyHostToDevice, s));
+    const size_t bytes = (size_t)n_pages * page_bytes;
+    for (int l = layer_begin; l < layer_end; ++l) {
+        uint8_t* stage = m->offload_stage + (size_t)((l - layer_begin) & 1) * m->offload_cap * page_bytes;
+        // a few CTAs: the gather only has to keep ahead of the copy engine
+        NF_CUDA_TRY(nf::launch_gather_pages(kv_pools[l], m->offload_ids, n_pages, page_bytes, stage, 8, s));
+        NF_CUDA_TRY(cudaMemcpyAsync(static_cast<uint8_t*>(host_dst) + (size_t)(l - layer_begin) * bytes, stage, bytes,
+                                    cudaMemcpyDeviceToHost, s));
+    }
     return NF_OK;
 } catch (const std::bad_alloc&) {
     return NF_ERR_OUT_OF_MEMORY;
@@ -1054,52 +1115,60 @@ extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_
     int64_t kv_bytes = 0;
     for (int r = 0; r < R; ++r) kv_bytes += (int64_t)((b->ctx_len[r] + 1 + 15) / 16) * 2 * 16 * d.d * 2 * d.nkv;
     if (R > 0) {
-        int64_t items = 0;
-        for (int r = 0; r < R; ++r) {
-            const int np = (b->ctx_len[r] + 1 + 15) / 16;
-            items += (int64_t)d.nkv * ((np + nf::kDecodeSplitPages - 1) / nf::kDecodeSplitPages);
-        }
-        if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
+        if ((st = ensure_part_capacity(m, nf::decode_work_items(d, b->ctx_len, R))) != NF_OK) return st;
         NF_CUDA_TRY(decode_prologue(m, io, R, sg));
         NF_CUDA_TRY(cudaMemsetAsync(m->q, 0, (size_t)R * d.nq * d.d * 2, sg));
         auto dec = [&](int grid, cudaStream_t s) -> nf_status {
             return launch_decode(m, io, m->tm_q, m->q, m->attn_o, 0, 0, R, grid, s) == cudaSuccess ? NF_OK
                                                                                                    : NF_ERR_CUDA;
         };
-        const int small = std::max(4, S / 8);
-        double t_small = 0, t_all = 0;
-        if ((st = time_us(sg, 3, [&] { return dec(small, sg); }, &t_small)) != NF_OK) return st;
-        if ((st = time_us(sg, 3, [&] { return dec(S, sg); }, &t_all)) != NF_OK) return st;
-        bw_small = kv_bytes / ((t_small - c.attn_launch_us) * 1e-6) / small;
-        bw_full = kv_bytes / ((t_all - c.attn_launch_us) * 1e-6);
+        // decode bandwidth on 1/8, 1/4, 1/2, 3/4 and all of the SMs
+        static const double shares[5] = {0.125, 0.25, 0.5, 0.75, 1.0};
+        double t_at[5] = {0, 0, 0, 0, 0};
+        for (int i = 0; i < 5; ++i) {
+            const int g = std::max(4, (int)(S * shares[i]));
+            if ((st = time_us(sg, 3, [&] { return dec(g, sg); }, &t_at[i])) != NF_OK) return st;
+            c.attn_bw_at[i] = kv_bytes / (std::max(1.0, t_at[i] - c.attn_launch_us) * 1e-6);
+        }
+        bw_small = c.attn_bw_at[0] / std::max(4, (int)(S * shares[0]));
+        bw_full = c.attn_bw_at[4];
         c.attn_bw_per_sm = bw_small;
         c.hbm_bw = bw_full;
 
-        // (d) co-run: decode attention on a quarter of the SMs beside the GEMM on the rest
-        const int sa_n = std::max(8, S / 4), sg_n = S - sa_n;
-        double t_g = 0, t_a = 0;
-        if ((st = time_us(sg, 3, [&] { return gemm(sg_n, sg); }, &t_g)) != NF_OK) return st;
-        if ((st = time_us(sg, 2, [&] { return dec(sa_n, sg); }, &t_a)) != NF_OK) return st;
-        // run both, the attention stream repeating while the GEMMs run
-        cudaEvent_t e0, e1, e2, e3;
-        cudaEventCreate(&e0); cudaEventCreate(&e1); cudaEventCreate(&e2); cudaEventCreate(&e3);
-        NF_CUDA_TRY(cudaEventRecord(e0, sg));
-        NF_CUDA_TRY(cudaStreamWaitEvent(sa, e0, 0));
-        NF_CUDA_TRY(cudaEventRecord(e2, sa));
-        if ((st = dec(sa_n, sa)) != NF_OK) return st;
-        NF_CUDA_TRY(cudaEventRecord(e3, sa));
-        const int reps = std::max(1, (int)(t_a / std::max(1.0, t_g)));
-        for (int i = 0; i < reps && st == NF_OK; ++i) st = gemm(sg_n, sg);
-        NF_CUDA_TRY(cudaEventRecord(e1, sg));
-        NF_CUDA_TRY(cudaStreamWaitEvent(sg, e3, 0));
-        NF_CUDA_TRY(cudaStreamSynchronize(sg));
-        float ms_g = 0, ms_a = 0;
-        cudaEventElapsedTime(&ms_g, e0, e1);
-        cudaEventElapsedTime(&ms_a, e2, e3);
-        cudaEventDestroy(e0); cudaEventDestroy(e1); cudaEventDestroy(e2); cudaEventDestroy(e3);
-        if (st != NF_OK) return st;
-        const double slow_g = ms_g * 1000.0 / (reps * t_g), slow_a = ms_a * 1000.0 / t_a;
-        c.interference = std::max(0.0, std::min(1.0, 0.5 * (slow_g + slow_a) - 1.0));
+        // (d) co-run: decode attention on 1/4, 1/2 and 3/4 of the SMs beside the GEMM on the rest; the
+        // GEMM repeats while the attention runs, and each is compared with its time alone on its share
+        static const double co[3] = {0.25, 0.5, 0.75};
+        double sum = 0;
+        for (int i = 0; i < 3; ++i) {
+            const int sa_n = std::max(8, (int)(S * co[i])), sg_n = S - sa_n;
+            double t_g = 0, t_a = 0;
+            if ((st = time_us(sg, 3, [&] { return gemm(sg_n, sg); }, &t_g)) != NF_OK) return st;
+            if ((st = time_us(sg, 2, [&] { return dec(sa_n, sg); }, &t_a)) != NF_OK) return st;
+            cudaEvent_t e0, e1, e2, e3;
+            NF_CUDA_TRY(cudaEventCreate(&e0));
+            NF_CUDA_TRY(cudaEventCreate(&e1));
+            NF_CUDA_TRY(cudaEventCreate(&e2));
+            NF_CUDA_TRY(cudaEventCreate(&e3));
+            NF_CUDA_TRY(cudaEventRecord(e0, sg));
+            NF_CUDA_TRY(cudaStreamWaitEvent(sa, e0, 0));
+            NF_CUDA_TRY(cudaEventRecord(e2, sa));
+            if ((st = dec(sa_n, sa)) != NF_OK) return st;
+            NF_CUDA_TRY(cudaEventRecord(e3, sa));
+            const int reps = std::max(1, (int)(t_a / std::max(1.0, t_g)));
+            for (int k = 0; k < reps && st == NF_OK; ++k) st = gemm(sg_n, sg);
+            NF_CUDA_TRY(cudaEventRecord(e1, sg));
+            NF_CUDA_TRY(cudaStreamWaitEvent(sg, e3, 0));
+            NF_CUDA_TRY(cudaStreamSynchronize(sg));
+            float ms_g = 0, ms_a = 0;
+            cudaEventElapsedTime(&ms_g, e0, e1);
+            cudaEventElapsedTime(&ms_a, e2, e3);
+            cudaEventDestroy(e0); cudaEventDestroy(e1); cudaEventDestroy(e2); cudaEventDestroy(e3);
+            if (st != NF_OK) return st;
+            c.interf_gemm[i] = std::max(1e-4, std::min(1.0, ms_g * 1000.0 / (reps * t_g) - 1.0));
+            c.interf_attn[i] = std::max(1e-4, std::min(1.0, ms_a * 1000.0 / t_a - 1.0));
+            sum += 0.5 * (c.interf_gemm[i] + c.interf_attn[i]);
+        }
+        c.interference = sum / 3.0;
     }
 
     // (c) prefill attention at a quarter of the SMs
@@ -1126,8 +1195,20 @@ extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_
 extern "C" nf_status nf_get_cost_model(const nf_model* m, nf_cost_model* out) try {
     if (m == nullptr || out == nullptr) return NF_ERR_INVALID_ARGUMENT;
     const nf::CostModel& c = m->cost;
-    *out = nf_cost_model{c.gemm_flops_per_sm, c.gemm_tile_us, c.gemm_launch_us, c.hbm_bw, c.attn_bw_per_sm,
-                         c.attn_launch_us, c.attn_flops_per_sm, c.interference, c.calibrated};
+    nf_cost_model r;
+    std::memset(&r, 0, sizeof(r));
+    r.gemm_flops_per_sm = c.gemm_flops_per_sm;
+    r.gemm_tile_us = c.gemm_tile_us;
+    r.gemm_launch_us = c.gemm_launch_us;
+    r.hbm_bw = c.hbm_bw;
+    r.attn_bw_per_sm = c.attn_bw_per_sm;
+    r.attn_launch_us = c.attn_launch_us;
+    r.attn_flops_per_sm = c.attn_flops_per_sm;
+    r.interference = c.interference;
+    r.calibrated = c.calibrated;
+    for (int i = 0; i < 5; ++i) r.attn_bw_at[i] = c.attn_bw_at[i];
+    for (int i = 0; i < 3; ++i) { r.interf_attn[i] = c.interf_attn[i]; r.interf_gemm[i] = c.interf_gemm[i]; }
+    *out = r;
     return NF_OK;
 } catch (const std::bad_alloc&) {
     return NF_ERR_OUT_OF_MEMORY;
@@ -1140,9 +1221,23 @@ extern "C" nf_status nf_set_cost_model(nf_model* m, const nf_cost_model* in) try
     if (!(in->gemm_flops_per_sm > 0) || !(in->hbm_bw > 0) || !(in->attn_bw_per_sm > 0) ||
         !(in->attn_flops_per_sm > 0) || in->interference < 0)
         return NF_ERR_INVALID_ARGUMENT;
-    m->cost = nf::CostModel{in->gemm_flops_per_sm, in->gemm_tile_us, in->gemm_launch_us, in->hbm_bw,
-                            in->attn_bw_per_sm, in->attn_launch_us, in->attn_flops_per_sm, in->interference,
-                            in->calibrated};
+    for (int i = 0; i < 5; ++i)
+        if (in->attn_bw_at[i] < 0) return NF_ERR_INVALID_ARGUMENT;
+    for (int i = 0; i < 3; ++i)
+        if (in->interf_attn[i] < 0 || in->interf_gemm[i] < 0) return NF_ERR_INVALID_ARGUMENT;
+    nf::CostModel c = nf::default_cost_model(m->sm_count);
+    c.gemm_flops_per_sm = in->gemm_flops_per_sm;
+    c.gemm_tile_us = in->gemm_tile_us;
+    c.gemm_launch_us = in->gemm_launch_us;
+    c.hbm_bw = in->hbm_bw;
+    c.attn_bw_per_sm = in->attn_bw_per_sm;
+    c.attn_launch_us = in->attn_launch_us;
+    c.attn_flops_per_sm = in->attn_flops_per_sm;
+    c.interference = in->interference;
+    c.calibrated = in->calibrated;
+    for (int i = 0; i < 5; ++i) c.attn_bw_at[i] = in->attn_bw_at[i];
+    for (int i = 0; i < 3; ++i) { c.interf_attn[i] = in->interf_attn[i]; c.interf_gemm[i] = in->interf_gemm[i]; }
+    m->cost = c;
     return NF_OK;
 } catch (const std::bad_alloc&) {
     return NF_ERR_OUT_OF_MEMORY;

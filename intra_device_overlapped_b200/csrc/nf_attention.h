@@ -11,6 +11,8 @@ namespace nf {
 // Decode keys are split into chunks of this many pages (512 keys); the split of a request
 // depends only on its ctx_len.
 constexpr int kDecodeSplitPages = 32;
+// split_pages value that keeps every request in one chunk (no partials, no merge pass)
+constexpr int kDecodeNoSplit = 1 << 30;
 
 struct DecodeArgs {
     const uint16_t* q;   // [rows x nq x d] bf16; decode request r is row r
@@ -29,6 +31,8 @@ struct DecodeArgs {
     int split_pages;
     float scale_log2;     // log2(e) / sqrt(d)
     int* merge_cnt;       // [R x nkv] split arrival counters (zeroed by decode_items_kernel)
+    const int* chunk_off; // tensor-core kernel: [R + 1] first partial slot of each request
+    float* part_ml;       // tensor-core kernel: [chunks x nq x 2] running maximum and row sum per query head
     int* status;
     int* trace_ctr;
     nf_trace_entry* trace;
@@ -67,6 +71,10 @@ cudaError_t launch_prefill_attention(const PrefillArgs& a, int head_dim, int gri
 // the per-request prefix of page counts (decode_schedule with nkv = 1, split_pages = 1); tmQ
 // maps q as [rows * nq x d] with boxes of nq rows.
 bool decode_tc_supported(int nq, int nkv, int head_dim);
+// item_off[r] = pages of requests [0, r), chunk_off[r] = chunks of requests [0, r) (nullable), for
+// requests [0, R] (one CTA; a negative ctx_len is recorded in *status and read as 0).
+cudaError_t launch_decode_tc_schedule(const int* ctx_len, int R, int split_pages, int* item_off, int* chunk_off,
+                                      int* status, cudaStream_t stream);
 cudaError_t launch_decode_attention_tc(const CUtensorMap& tmQ, const DecodeArgs& a, int grid, cudaStream_t stream);
 
 // Tensor-core (tcgen05) causal attention of the prefill chunk for head dim 128 (any G):

@@ -8,18 +8,25 @@
 // that one page of one layer -- K and V of all KV heads, 64 KB -- is a single contiguous
 // block whose bytes are already the shared-memory image the tensor cores read:
 //   [K|V][64-column half of d][KV head][16 tokens][8 chunks of 16 B, chunk c of row r at c ^ (r & 7)]
-// and one bulk copy moves a whole page into a ring stage.
+// and one bulk copy per half moves a page into a ring stage.
 //
-// Work item = one decode request with all of its heads; a stage is one page (16 keys x 8
-// KV heads = 128 rows). One thread issues
+// Split along KV. A request of n pages is cut into ceil(n / chunk_pages) chunks whose page counts
+// differ by at most one (chunk c = pages [c n / nch, (c + 1) n / nch)); the cut depends only on the
+// request's context length, never on the grid. A work item is one chunk with all heads. Items are dealt to the persistent CTAs in
+// contiguous ranges of equal page counts, so a CTA's share differs from the mean by less than
+// one chunk. A request of one chunk writes its output directly; the chunks of a longer request
+// each write their unnormalised partial (O, running maximum m, sum l per query head) and
+// decode_merge_kernel combines them in chunk order. Every rescale factor 2^(m_c - M) is an exact
+// power of two (the running maxima are integers), so the result is the same for every grid.
+//
+// Per page (16 keys x 8 KV heads = 128 rows) one thread issues
 //   S^T[128 rows x nq] = K_page Q^T       (A = K, K-major; B = the request's nq query rows)
 //   O^T[128 d x nq]   += V_page^T P^T     (A = V read MN-major; B = P, K-major)
 // with fp32 accumulators in TMEM. A row (KV head h, key k) of S^T only pairs with the G query
 // heads of head h, so P is block diagonal: each softmax thread owns one row, writes its G
 // probabilities and leaves the other entries at the zero they were set to once. Per query
 // head the running maximum moves only when a score exceeds it by more than 2^8 (O^T is then
-// rescaled in TMEM). Requests are dealt to persistent CTAs in contiguous ranges of equal
-// page counts; there is no split-KV merge.
+// rescaled in TMEM).
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -70,50 +77,73 @@ struct TcCfg {
 // warp 6 loads V halves of pages (bulk copies)
 constexpr int THREADS = 224;
 
-// Walks the CTA's requests whose first page index (in the page-prefix work space) is in [lo, hi).
-struct ReqIter {
-    int r, nkeys, npages;
-    long long w;
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Walks the CTA's work items: chunks whose first page (in the page prefix of the requests) lies
+// in [lo, hi). A request of npages pages has nch = ceil(npages / chunk_pages) chunks; chunk c holds
+// pages [c npages / nch, (c + 1) npages / nch).
+struct ItemIter {
+    int r, c;            // request, chunk
+    int nkeys, npages;   // of the request
+    int nch;
+    int pg0, pg1;        // the chunk's pages [pg0, pg1) within the request
+    long long start;     // prefix position of the chunk's first page
     bool valid;
 };
 
-__device__ __forceinline__ void req_load(ReqIter& it, const DecodeArgs& a) {
-    it.nkeys = a.ctx_len[it.r] + 1;
+__device__ __forceinline__ void item_req(ItemIter& it, const DecodeArgs& a) {
+    it.nkeys = max(a.ctx_len[it.r], 0) + 1;
     it.npages = (it.nkeys + 15) >> 4;
-    it.w = a.item_off[it.r];
+    it.nch = ceil_div(it.npages, a.split_pages);
 }
 
-__device__ __forceinline__ void req_init(ReqIter& it, const DecodeArgs& a, long long lo, long long hi) {
+__device__ __forceinline__ void item_chunk(ItemIter& it, const DecodeArgs& a, long long hi) {
+    it.pg0 = (int)((long long)it.c * it.npages / it.nch);
+    it.pg1 = (int)((long long)(it.c + 1) * it.npages / it.nch);
+    it.start = (long long)a.item_off[it.r] + it.pg0;
+    it.valid = it.r < a.req_end && it.start < hi;
+}
+
+__device__ __forceinline__ void item_init(ItemIter& it, const DecodeArgs& a, long long lo, long long hi) {
     int low = a.req_begin, high = a.req_end - 1;
-    while (low < high) {  // last request whose work starts at or before lo
+    while (low < high) {  // last request whose first page is at or before lo
         const int mid = (low + high + 1) >> 1;
         if ((long long)a.item_off[mid] <= lo) low = mid; else high = mid - 1;
     }
     it.r = low;
-    req_load(it, a);
-    if (it.w < lo) {  // starts before lo: belongs to the previous CTA
+    item_req(it, a);
+    const long long off = lo - (long long)a.item_off[it.r];
+    // first chunk starting at or after lo: c n / nch >= off  <=>  c >= off nch / n
+    it.c = off > 0 ? (int)((off * it.nch + it.npages - 1) / it.npages) : 0;
+    if (it.c >= it.nch) {
         it.r += 1;
-        if (it.r < a.req_end) req_load(it, a);
+        it.c = 0;
+        if (it.r < a.req_end) item_req(it, a);
     }
-    it.valid = it.r < a.req_end && it.w < hi;
+    if (it.r < a.req_end) item_chunk(it, a, hi); else it.valid = false;
 }
 
-__device__ __forceinline__ void req_next(ReqIter& it, const DecodeArgs& a, long long hi) {
-    if (++it.r < a.req_end) req_load(it, a);
-    it.valid = it.r < a.req_end && it.w < hi;
+__device__ __forceinline__ void item_next(ItemIter& it, const DecodeArgs& a, long long hi) {
+    if (++it.c == it.nch) {
+        it.c = 0;
+        if (++it.r >= a.req_end) { it.valid = false; return; }
+        item_req(it, a);
+    }
+    item_chunk(it, a, hi);
 }
 
-// Position in the CTA's page sequence: page j of request it.r, cs-th page overall, ni-th request.
+// Position in the CTA's page sequence: page j (within the request) of the current item, cs-th page
+// overall, ni-th item.
 struct PageCursor {
-    ReqIter it;
+    ItemIter it;
     int j;
     uint32_t cs, ni;
     bool valid;
 };
 
 __device__ __forceinline__ void cursor_init(PageCursor& x, const DecodeArgs& a, long long lo, long long hi) {
-    req_init(x.it, a, lo, hi);
-    x.j = 0;
+    item_init(x.it, a, lo, hi);
+    x.j = x.it.pg0;
     x.cs = 0;
     x.ni = 0;
     x.valid = x.it.valid;
@@ -121,9 +151,9 @@ __device__ __forceinline__ void cursor_init(PageCursor& x, const DecodeArgs& a, 
 
 __device__ __forceinline__ void cursor_next(PageCursor& x, const DecodeArgs& a, long long hi) {
     ++x.cs;
-    if (++x.j == x.it.npages) {
-        req_next(x.it, a, hi);
-        x.j = 0;
+    if (++x.j == x.it.pg1) {
+        item_next(x.it, a, hi);
+        x.j = x.it.pg0;
         ++x.ni;
         x.valid = x.it.valid;
     }
@@ -212,15 +242,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int nstage = is_k ? NSK : NSV;
         uint64_t* full = is_k ? k_full : v_full;
         uint8_t* ring = smem + (is_k ? 0u : C::OFF_V);
-        ReqIter it;
-        req_init(it, a, lo, hi);
+        ItemIter it;
+        item_init(it, a, lo, hi);
         uint32_t cs = 0, ni = 0;
         bool ok = true;
         const char* pool = reinterpret_cast<const char*>(a.kv_pool) + (is_k ? 0 : HALF_PAGE);
         // each page is read once per launch: stream it through L2 without displacing reused data
         const uint64_t stream_policy = l2_policy_evict_first();
-        for (; it.valid && ok; req_next(it, a, hi), ++ni) {
+        for (; it.valid && ok; item_next(it, a, hi), ++ni) {
             const int base = a.page_indptr[it.r];
+            const int rowlen = a.page_indptr[it.r + 1] - base;
             if (is_k) {
                 if (!wait_bcast(q_empty, (ni & 1u) ^ 1u, abort_flag, a.status, lane)) { ok = false; break; }
                 if (lane == 0) {
@@ -231,13 +262,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
             int ids = 0;
-            for (int j = 0; j < it.npages; ++j, ++cs) {
-                if ((j & 31) == 0) {
+            for (int j = it.pg0; j < it.pg1; ++j, ++cs) {
+                if (((j - it.pg0) & 31) == 0) {
+                    // one page id per lane; an index past the request's row of the page table, or a
+                    // page outside the pool, is recorded and page 0 read in its place
                     const int jj = j + lane;
-                    ids = jj < it.npages ? __ldg(a.page_indices + base + jj) : 0;
-                    if (ids < 0 || ids >= a.num_pages) { set_status(a.status, NF_ERR_DEVICE_BOUNDS); ids = 0; }
+                    ids = 0;
+                    if (jj < it.pg1) {
+                        if (jj < rowlen) ids = __ldg(a.page_indices + base + jj);
+                        if (jj >= rowlen || ids < 0 || ids >= a.num_pages) {
+                            set_status(a.status, NF_ERR_DEVICE_BOUNDS);
+                            ids = 0;
+                        }
+                    }
                 }
-                const int pg = __shfl_sync(0xffffffffu, ids, j & 31);
+                const int pg = __shfl_sync(0xffffffffu, ids, (j - it.pg0) & 31);
                 const int st = (int)(cs % nstage);
                 // the stage's previous page (cs - nstage) must be consumed: its S^T (K) or P V (V)
                 if (cs >= (uint32_t)nstage) {
@@ -277,7 +316,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint64_t pd0 = umma_desc_sw128(sbase + C::OFF_P);
         auto issue_s = [&](const PageCursor& x) -> bool {
             const uint32_t st = x.cs % NSK, sb = x.cs % NSB;
-            if (x.j == 0 && !wait_bcast(q_full, x.ni & 1u, abort_flag, a.status, lane)) return false;
+            if (x.j == x.it.pg0 && !wait_bcast(q_full, x.ni & 1u, abort_flag, a.status, lane)) return false;
             if (!wait_bcast(&k_full[st], (x.cs / NSK) & 1u, abort_flag, a.status, lane)) return false;
             if (!wait_bcast(&s_free[sb], ((x.cs / NSB) & 1u) ^ 1u, abort_flag, a.status, lane)) return false;
             tc_fence_after();
@@ -291,13 +330,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                     umma_bf16_c<true>(d, ad + (uint64_t)(((kk >> 2) * REGION + (kk & 3) * 32) >> 4),
                                       bd + (uint64_t)(((kk >> 2) * (NQ * 128) + (kk & 3) * 32) >> 4), C::IDESC_S);
                 umma_commit(&s_full[sb]);
-                if (x.j == x.it.npages - 1) umma_commit(q_empty);
+                if (x.j == x.it.pg1 - 1) umma_commit(q_empty);
             }
             return true;
         };
         auto issue_pv = [&](const PageCursor& x) -> bool {
             const uint32_t pb = x.cs % NPB, sv = x.cs % NSV;
-            const bool first = x.j == 0;
+            const bool first = x.j == x.it.pg0;
             if (!wait_bcast(&p_full[pb], (x.cs / NPB) & 1u, abort_flag, a.status, lane)) return false;
             if (!wait_bcast(&v_full[sv], (x.cs / NSV) & 1u, abort_flag, a.status, lane)) return false;
             if (first && !wait_bcast(o_free, (x.ni & 1u) ^ 1u, abort_flag, a.status, lane)) return false;
@@ -319,7 +358,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         while (ok && pc.valid) {
             while (ok && sc.valid && sc.cs <= pc.cs + (uint32_t)C::LOOK) {
                 // the first page of a later request waits for its Q only when P V has nothing to do
-                if (sc.j == 0 && sc.cs > pc.cs && !test_bcast(q_full, sc.ni & 1u, lane)) break;
+                if (sc.j == sc.it.pg0 && sc.cs > pc.cs && !test_bcast(q_full, sc.ni & 1u, lane)) break;
                 ok = issue_s(sc);
                 cursor_next(sc, a, hi);
             }
@@ -342,15 +381,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int h = t >> 4, k = t & 15;
         const int hsel = lane >> 4;           // which of the warp's two heads this lane's row belongs to
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-        ReqIter it;
-        req_init(it, a, lo, hi);
+        ItemIter it;
+        item_init(it, a, lo, hi);
         uint32_t cs = 0, ni = 0;
         bool ok = true;
-        for (; it.valid && ok; req_next(it, a, hi), ++ni) {
+        for (; it.valid && ok; item_next(it, a, hi), ++ni) {
             float m[G], lp[G];
 #pragma unroll
             for (int i = 0; i < G; ++i) { m[i] = -INFINITY; lp[i] = 0.f; }
-            for (int c = 0; c < it.npages; ++c, ++cs) {
+            for (int c = it.pg0; c < it.pg1; ++c, ++cs) {
                 const uint32_t sb = cs % NSB;
                 bool okc = wait_bcast(&s_full[sb], (cs / NSB) & 1u, abort_flag, a.status, lane);
                 float sw[2 * G];  // scores of the warp's two heads' query columns
@@ -395,7 +434,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         m[i] = nm;
                         lp[i] *= cf[i];
                     }
-                    if (c > 0) {
+                    if (c > it.pg0) {
                         if (k == 0) {
 #pragma unroll
                             for (int i = 0; i < G; ++i) cfs[h * G + i] = cf[i];
@@ -458,27 +497,41 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (bar_red_or(3, 128, !okc)) { ok = false; break; }
             }
             if (!ok) break;
-            // ---- request output: O^T (thread = one d) / l per query head
+            // ---- item output: row sums per query head, then O^T (thread = one d); a request of one
+            // chunk is normalised and written, a chunk of a longer request leaves its partial
+            const bool single = it.nch == 1;
+            const int slot = single ? 0 : a.chunk_off[it.r] + it.c;
 #pragma unroll
             for (int i = 0; i < G; ++i) {
                 float x = lp[i];
 #pragma unroll
                 for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-                if (k == 0) cfs[h * G + i] = x;
+                if (k == 0) {
+                    if (single) {
+                        cfs[h * G + i] = x;
+                    } else {
+                        a.part_ml[((size_t)slot * NQ + h * G + i) * 2] = m[i];
+                        a.part_ml[((size_t)slot * NQ + h * G + i) * 2 + 1] = x;
+                    }
+                }
             }
             bool okc = wait_bcast(&pv_done[(cs - 1) % NPB], ((cs - 1) / NPB) & 1u, abort_flag, a.status, lane);
             bar_sync_n(2, 128);
-            uint16_t* ob = a.out + (size_t)it.r * NQ * 128 + t;  // thread t writes d = t of every head
             if (okc) tc_fence_after();
 #pragma unroll
             for (int c16 = 0; c16 < NQ / 16; ++c16) {
                 float o[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) o[i] = 0.f;
                 if (okc) {
                     tmem_ld16(tmem + lane_addr + C::O_COL + c16 * 16, o);
+                    if (single) {
+                        uint16_t* ob = a.out + (size_t)it.r * NQ * 128 + t;  // thread t writes d = t of every head
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) ob[(size_t)(c16 * 16 + i) * 128] = f2bf(o[i] / cfs[c16 * 16 + i]);
+                        for (int i = 0; i < 16; ++i) ob[(size_t)(c16 * 16 + i) * 128] = f2bf(o[i] / cfs[c16 * 16 + i]);
+                    } else {
+                        float* po = a.part_o + (size_t)slot * NQ * 128 + t;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) po[(size_t)(c16 * 16 + i) * 128] = o[i];
+                    }
                 }
             }
             tc_fence_before();
@@ -504,6 +557,39 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
+// Requests cut into several chunks: out = bf16(sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c) per
+// query head, M the largest chunk maximum, both sums in chunk order (every factor is an exact power of
+// two). One CTA of 128 threads (one d each) per request at a time.
+template <int NQ>
+__global__ void __launch_bounds__(128) decode_merge_kernel(const __grid_constant__ DecodeArgs a) {
+    __shared__ float Ms[NQ], Ls[NQ];
+    const int t = threadIdx.x;
+    for (int r = a.req_begin + blockIdx.x; r < a.req_end; r += gridDim.x) {
+        const int npages = (max(a.ctx_len[r], 0) + 1 + 15) >> 4;
+        const int nch = ceil_div(npages, a.split_pages);
+        if (nch <= 1) continue;  // written by the attention kernel
+        const float* ml = a.part_ml + (size_t)a.chunk_off[r] * NQ * 2;
+        const float* po = a.part_o + (size_t)a.chunk_off[r] * NQ * 128;
+        __syncthreads();  // the previous request's Ms / Ls are no longer read
+        if (t < NQ) {
+            float M = -INFINITY;
+            for (int c = 0; c < nch; ++c) M = fmaxf(M, ml[(c * NQ + t) * 2]);
+            float L = 0.f;
+            for (int c = 0; c < nch; ++c) L += softmax_rescale(ml[(c * NQ + t) * 2], M) * ml[(c * NQ + t) * 2 + 1];
+            Ms[t] = M;
+            Ls[t] = L;
+        }
+        __syncthreads();
+        for (int qh = 0; qh < NQ; ++qh) {
+            const float M = Ms[qh];
+            float acc = 0.f;
+            for (int c = 0; c < nch; ++c)
+                acc += softmax_rescale(ml[(c * NQ + qh) * 2], M) * __ldcg(po + ((size_t)c * NQ + qh) * 128 + t);
+            a.out[((size_t)r * NQ + qh) * 128 + t] = f2bf(acc / Ls[qh]);
+        }
+    }
+}
+
 template <int NQ>
 cudaError_t launch_nq(const CUtensorMap& tmQ, const DecodeArgs& a, int grid, cudaStream_t stream) {
     static bool cfg = false;
@@ -514,13 +600,84 @@ cudaError_t launch_nq(const CUtensorMap& tmQ, const DecodeArgs& a, int grid, cud
         cfg = true;
     }
     decode_attention_tc_kernel<NQ><<<grid, THREADS, TcCfg<NQ>::SMEM, stream>>>(tmQ, a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || a.split_pages >= kDecodeNoSplit) return e;
+    decode_merge_kernel<NQ><<<grid, 128, 0, stream>>>(a);
     return cudaGetLastError();
+}
+
+// Page prefix (item_off) and chunk prefix (chunk_off, optional) of requests [0, R): request r has
+// ceil((ctx + 1) / 16) pages in ceil(pages / split_pages) chunks. A negative context length is
+// recorded as NF_ERR_DEVICE_BOUNDS and read as 0.
+__global__ void decode_tc_schedule_kernel(const int* ctx_len, int R, int split_pages, int* item_off, int* chunk_off,
+                                          int* status) {
+    __shared__ long long carry[2];
+    __shared__ int warp_sums[2][32];
+    if (threadIdx.x < 2) carry[threadIdx.x] = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int base = 0; base < R; base += blockDim.x) {
+        const int r = base + threadIdx.x;
+        int v[2] = {0, 0};
+        if (r < R) {
+            int c = ctx_len[r];
+            if (c < 0) { set_status(status, NF_ERR_DEVICE_BOUNDS); c = 0; }
+            v[0] = (c + 1 + 15) >> 4;
+            v[1] = ceil_div(v[0], split_pages);
+        }
+        int incl[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            int x = v[k];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (lane == 31) warp_sums[k][w] = x;
+            incl[k] = x;
+        }
+        __syncthreads();
+        if (w == 0) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                int s = lane < nw ? warp_sums[k][lane] : 0;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, s, o);
+                    if (lane >= o) s += y;
+                }
+                if (lane < nw) warp_sums[k][lane] = s;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < 2; ++k) incl[k] += (w > 0 ? warp_sums[k][w - 1] : 0);
+        if (r < R) {
+            item_off[r] = (int)(carry[0] + incl[0] - v[0]);
+            if (chunk_off) chunk_off[r] = (int)(carry[1] + incl[1] - v[1]);
+        }
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) { carry[0] += incl[0]; carry[1] += incl[1]; }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        item_off[R] = (int)carry[0];
+        if (chunk_off) chunk_off[R] = (int)carry[1];
+    }
 }
 
 }  // namespace
 
 bool decode_tc_supported(int nq, int nkv, int head_dim) {
     return head_dim == 128 && nkv == 8 && (nq == 32 || nq == 64);
+}
+
+cudaError_t launch_decode_tc_schedule(const int* ctx_len, int R, int split_pages, int* item_off, int* chunk_off,
+                                      int* status, cudaStream_t stream) {
+    if (R <= 0) return cudaSuccess;
+    decode_tc_schedule_kernel<<<1, 1024, 0, stream>>>(ctx_len, R, split_pages, item_off, chunk_off, status);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_decode_attention_tc(const CUtensorMap& tmQ, const DecodeArgs& a, int grid, cudaStream_t stream) {

@@ -17,6 +17,11 @@ constexpr int kGemmBarrierBytes = 256;
 constexpr int kGemmStagingBytes = 4 * 32 * 32 * 4;  // residual epilogue: 32 x 32 fp32 per epilogue warp
 constexpr int kGemmSmemBytes =
     kGemmStages * (kGemmBM + kGemmBN) * kGemmBK * 2 + 1024 + kGemmBarrierBytes + kGemmStagingBytes;
+// CTA-pair kernel: per CTA a stage holds 128 A rows and 128 B rows (its half of the 256-wide tile)
+constexpr int kGemm2Stages = 6;
+constexpr int kGemm2SmemBytes = kGemm2Stages * 256 * kGemmBK * 2 + 1024 + kGemmBarrierBytes + kGemmStagingBytes;
+// rows of the boxes of every B (weight) tensor map: both kernels load B in 128-row boxes
+constexpr int kGemmBBoxRows = 128;
 
 enum EpiKind : int {
     EPI_F32 = 0,     // out_f32 = acc (* rs if partials)
@@ -71,6 +76,10 @@ struct GemmArgs {
     // EPI_LMHEAD
     float* tile_max;  // [rows x n_tiles]
     int* tile_arg;
+    // Work order: nullptr = static (CTA b takes units b, b + grid, ...); else a zeroed counter from
+    // which CTAs claim units in increasing order, so that a launch whose CTAs start at different
+    // times (SMs freed by a kernel on another stream) still shares the units evenly.
+    int* tile_ctr;
     // diagnostics
     int* status;
     int* trace_ctr;
@@ -86,8 +95,13 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
 bool make_tmap_bf16_3d_heads(CUtensorMap* map, const void* base, uint64_t tokens, uint64_t heads, uint64_t head_dim,
                              uint32_t box_tokens);
 
+// Dense launches (not grouped) with a grid of at least 2 run on CTA pairs with 256 x 256 tiles; grouped
+// launches and single-CTA grids on single CTAs with 128 x 256 tiles.
 cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args, int grid,
                         cudaStream_t stream);
+bool gemm_uses_pairs(const GemmArgs& a);
+// work units (output tiles, times 2 with split K) of a launch on the kernel launch_gemm picks for grids >= 2
+int gemm_units(const GemmArgs& a);
 
 int device_sm_count();
 

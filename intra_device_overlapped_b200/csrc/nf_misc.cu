@@ -147,6 +147,17 @@ __global__ void widen_scaled_kernel(const uint16_t* __restrict__ src, float* __r
     }
 }
 
+// Page i of the list lands at dst + i * page_bytes; 16-byte loads that stream through L2 (the pages
+// are read once), one CTA per page at a time.
+__global__ void gather_pages_kernel(const uint4* __restrict__ pool, const int* __restrict__ ids, int n,
+                                    size_t page_vec, uint4* __restrict__ dst) {
+    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+        const uint4* src = pool + (size_t)ids[i] * page_vec;
+        uint4* out = dst + (size_t)i * page_vec;
+        for (size_t v = threadIdx.x; v < page_vec; v += blockDim.x) out[v] = __ldcs(src + v);
+    }
+}
+
 __global__ void wait_flag_kernel(volatile int* flag, uint64_t limit_ns, int* status) {
     const uint64_t t0 = globaltimer_ns();
     while (*flag == 0) {
@@ -223,4 +234,15 @@ cudaError_t launch_wait_flag(int* flag, uint64_t limit_ns, int* status, cudaStre
     return cudaGetLastError();
 }
 
+}  // namespace nf
+
+namespace nf {
+cudaError_t launch_gather_pages(const void* pool, const int* ids, int n, size_t page_bytes, void* dst, int max_blocks,
+                                cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    const int grid = n < max_blocks ? n : max_blocks;
+    gather_pages_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(pool), ids, n, page_bytes / 16,
+                                             static_cast<uint4*>(dst));
+    return cudaGetLastError();
+}
 }  // namespace nf

@@ -20,6 +20,9 @@ cudaError_t launch_pack_rows(const uint16_t* src, uint16_t* dst, int rows, int c
 cudaError_t launch_widen_scaled(const uint16_t* src, float* dst, int rows, int cols, const uint16_t* gamma,
                                 cudaStream_t s);
 cudaError_t launch_wait_flag(int* flag, uint64_t limit_ns, int* status, cudaStream_t s);
+// Pack pages ids[0..n) of a pool (page_bytes each, a multiple of 16) contiguously into dst.
+cudaError_t launch_gather_pages(const void* pool, const int* ids, int n, size_t page_bytes, void* dst, int max_blocks,
+                                cudaStream_t s);
 
 // --- mixture of experts (nf_moe.cu) ---
 struct MoeArgs {

@@ -12,6 +12,14 @@ namespace nf {
 
 constexpr int kDecodeSplitPagesHost = 32;  // must equal kDecodeSplitPages (nf_attention.h)
 
+// Decode attention work items of a batch (sizes the split-KV partials): chunks of at most
+// kDecodeSplitPagesHost pages, one per request chunk for the tensor-core kernel, one per KV head
+// and chunk for the warp-level kernel.
+int64_t decode_work_items(const ModelDims& d, const int32_t* ctx_len, int R);
+
+// ops of one forward that can have a work counter (later elastic ops run on the GEMM share statically)
+constexpr int kMaxCountedOps = 4096;
+
 struct LayerWeights {
     uint16_t* wqkv = nullptr;  // [(nq + 2 nkv) d x H], attn-norm gamma folded
     uint16_t* wo = nullptr;    // [H x nq d]
@@ -45,7 +53,13 @@ struct nf_model {
     uint16_t* act = nullptr;      // [T(*K) x F] SwiGLU output
     float* rope_cos = nullptr;    // [max_position x d/2]
     float* rope_sin = nullptr;
-    int* item_off = nullptr;      // [max_requests + 1]
+    int* item_off = nullptr;      // [max_requests + 1] page prefix (tensor-core decode) or item prefix
+    int* chunk_off = nullptr;     // [max_requests + 1] split-KV chunk prefix (tensor-core decode)
+    int* tile_ctr = nullptr;      // [kMaxCountedOps] work counters of elastic GEMM ops, zeroed per forward
+    // KV offload: two staging buffers of offload_cap pages and the device copy of the page list
+    uint8_t* offload_stage = nullptr;
+    int* offload_ids = nullptr;
+    int64_t offload_cap = 0;
     int* tok_feedback = nullptr;  // [T] token ids gathered from the previous iteration's next_token
     float* splitk_ws = nullptr;   // split-K partials of the residual GEMMs: [tiles x 128 x 256] fp32
     int* splitk_flags = nullptr;  // [tiles]: epoch of the last published first half

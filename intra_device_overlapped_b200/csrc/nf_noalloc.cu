@@ -5,9 +5,10 @@
 // handed all device memory to its own pool): they cannot create an nf_model, whose
 // workspace comes from cudaMalloc. This entry point runs the tensor-core decode attention of
 // the serving iteration from plain device pointers. Its only scratch -- the per-request
-// prefix of page counts that deals whole requests to the persistent CTAs, and a status word
-// -- lives in the file-scope array below, so the call makes no cudaMalloc, cudaFree or
-// allocating library call.
+// prefix of page counts that deals the requests to the persistent CTAs -- lives in the
+// file-scope array below, so the call makes no cudaMalloc, cudaFree or allocating library
+// call. Requests are not split along their keys here (split partials would need scratch
+// proportional to the batch), so each request is one work item.
 //
 // Every call on a device shares that one array: two calls that overlap on the GPU (on
 // different streams, or from different host threads) race on it and may produce wrong
@@ -27,10 +28,9 @@
 
 namespace {
 
-// Scratch layout: [0, 256) status word (int, zeroed by every call); [256, ...) item_off,
-// NF_NOALLOC_MAX_REQUESTS + 1 ints written in full by the schedule kernel before use.
-constexpr size_t kStatusBytes = 256;
-constexpr size_t kScratchBytes = kStatusBytes + 4 * (size_t)(NF_NOALLOC_MAX_REQUESTS + 64);
+// Scratch layout: item_off, NF_NOALLOC_MAX_REQUESTS + 1 ints, written in full by the schedule
+// kernel before the attention kernel reads them.
+constexpr size_t kScratchBytes = 4 * (size_t)(NF_NOALLOC_MAX_REQUESTS + 64);
 static_assert(kScratchBytes % 256 == 0, "scratch size");
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
@@ -39,7 +39,8 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once per device.
+// Device address of the scratch array on the current device, looked up once per device (and kept
+// for the life of the process: after cudaDeviceReset the cached address is stale).
 nf_status scratch_for_current_device(unsigned char** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NF_ERR_CUDA;
@@ -61,7 +62,8 @@ extern "C" nf_status nf_decode_attention_noalloc(const void* q, void* out, const
                                                  const int32_t* page_indices, int32_t num_requests,
                                                  int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                                                  int32_t sm_count, int32_t* status_device, void* stream) try {
-    if (!q || !out || !kv_pool || !ctx_len || !page_indptr || !page_indices) return NF_ERR_INVALID_ARGUMENT;
+    if (!q || !out || !kv_pool || !ctx_len || !page_indptr || !page_indices || !status_device)
+        return NF_ERR_INVALID_ARGUMENT;
     if (num_pages <= 0 || num_requests < 0 || sm_count < 0) return NF_ERR_INVALID_ARGUMENT;
     if (num_requests > NF_NOALLOC_MAX_REQUESTS) return NF_ERR_INVALID_ARGUMENT;  // scratch holds at most this many
     if (!nf::decode_tc_supported(n_q_heads, n_kv_heads, head_dim)) return NF_ERR_UNSUPPORTED;
@@ -70,8 +72,8 @@ extern "C" nf_status nf_decode_attention_noalloc(const void* q, void* out, const
     unsigned char* scratch = nullptr;
     nf_status st = scratch_for_current_device(&scratch);
     if (st != NF_OK) return st;
-    int* status = status_device ? status_device : reinterpret_cast<int*>(scratch);
-    int* item_off = reinterpret_cast<int*>(scratch + kStatusBytes);
+    int* status = status_device;
+    int* item_off = reinterpret_cast<int*>(scratch);
 
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -85,8 +87,9 @@ extern "C" nf_status nf_decode_attention_noalloc(const void* q, void* out, const
         return NF_ERR_INVALID_ARGUMENT;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (status_device == nullptr && cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return NF_ERR_CUDA;
-    if (nf::launch_decode_schedule(ctx_len, num_requests, 1, 1, item_off, s) != cudaSuccess) return NF_ERR_CUDA;
+    if (nf::launch_decode_tc_schedule(ctx_len, num_requests, nf::kDecodeNoSplit, item_off, nullptr, status, s) !=
+        cudaSuccess)
+        return NF_ERR_CUDA;
 
     nf::DecodeArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -103,7 +106,7 @@ extern "C" nf_status nf_decode_attention_noalloc(const void* q, void* out, const
     a.nkv = n_kv_heads;
     a.G = n_q_heads / n_kv_heads;
     a.num_pages = num_pages;
-    a.split_pages = 1;
+    a.split_pages = nf::kDecodeNoSplit;
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
     a.status = status;
     if (nf::launch_decode_attention_tc(tmq, a, grid, s) != cudaSuccess) return NF_ERR_CUDA;

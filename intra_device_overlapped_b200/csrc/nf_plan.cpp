@@ -19,10 +19,21 @@
 #include <cstring>
 #include <vector>
 
+#include "nf_attention.h"
 #include "nf_model.h"
 #include "nf_schedule.h"
 
 namespace nf {
+
+int64_t decode_work_items(const ModelDims& d, const int32_t* ctx_len, int R) {
+    const int per = decode_tc_supported(d.nq, d.nkv, d.d) ? 1 : d.nkv;
+    int64_t items = 0;
+    for (int r = 0; r < R; ++r) {
+        const int np = (std::max(ctx_len[r], 0) + 1 + 15) / 16;
+        items += (int64_t)per * ((np + kDecodeSplitPagesHost - 1) / kDecodeSplitPagesHost);
+    }
+    return items;
+}
 
 void nano_content(const nf_plan& p, bool* has_dec, bool* has_pre) {
     for (int j = 0; j < p.n_nano; ++j) {
@@ -31,11 +42,13 @@ void nano_content(const nf_plan& p, bool* has_dec, bool* has_pre) {
     }
 }
 
+void mark_elastic(std::vector<Op>& ops);
+
 std::vector<Op> build_ops(int tmpl, int n, const int* order, int L, bool moe, const bool* has_dec,
                           const bool* has_pre) {
     std::vector<Op> ops;
     auto push = [&](int kind, int stream, int j, int l) {
-        Op o{kind, stream, j, l, 0, -1, 0};
+        Op o{kind, stream, j, l, 0, 0, -1, 0};
         ops.push_back(o);
         return (int)ops.size() - 1;
     };
@@ -120,11 +133,77 @@ std::vector<Op> build_ops(int tmpl, int n, const int* order, int L, bool moe, co
     }
     for (size_t i = 0; i < ops.size(); ++i)
         if (ops[i].stream == STREAM_GEMM) ops[i].full_sm = covered[gpos[i]] ? 0 : 1;
+    mark_elastic(ops);
     return ops;
+}
+
+// A dense GEMM op inside an attention window may run elastically when that window holds exactly one
+// attention op A that is already resident when the GEMM starts: A's QKV is not the GEMM's immediate
+// predecessor on the GEMM stream (A is launched the moment that QKV completes), and the attention op
+// queued before A on its stream was consumed by a GEMM-stream op that completes before the GEMM's
+// predecessor does (so A started earlier). A GEMM holding every free SM then cannot delay any
+// attention kernel's start, since none starts while it runs.
+void mark_elastic(std::vector<Op>& ops) {
+    const int n = (int)ops.size();
+    std::vector<int> consumer(n, n), prev_attn(n, -1), prev_gemm(n, -1);
+    int last_a = -1, last_g = -1;
+    for (int i = 0; i < n; ++i) {
+        if (ops[i].wait >= 0) consumer[ops[i].wait] = std::min(consumer[ops[i].wait], i);
+        if (ops[i].stream == STREAM_ATTN) { prev_attn[i] = last_a; last_a = i; }
+        else { prev_gemm[i] = last_g; last_g = i; }
+    }
+    // consumer of an attention op: the first GEMM-stream op that waits for it
+    for (int g = 0; g < n; ++g) {
+        Op& o = ops[g];
+        if (o.stream != STREAM_GEMM || o.full_sm) continue;
+        if (!(o.kind == OP_QKV || o.kind == OP_O || o.kind == OP_GU || o.kind == OP_D)) continue;
+        int open = 0, a = -1;
+        for (int i = 0; i < g; ++i)
+            if (ops[i].stream == STREAM_ATTN && consumer[i] > g) { ++open; a = i; }
+        if (open != 1) continue;
+        const int trigger = ops[a].wait;  // the QKV that A waits for
+        if (prev_gemm[g] < 0 || prev_gemm[g] == trigger) continue;
+        const int pa = prev_attn[a];
+        if (pa >= 0 && !(consumer[pa] < prev_gemm[g])) continue;
+        o.elastic = 1;
+    }
+}
+
+namespace {
+// piecewise-linear interpolation of y at x over increasing knots xs (clamped at the ends)
+double interp(const double* xs, const double* ys, int n, double x) {
+    if (x <= xs[0]) return ys[0];
+    for (int i = 1; i < n; ++i)
+        if (x <= xs[i]) return ys[i - 1] + (ys[i] - ys[i - 1]) * (x - xs[i - 1]) / (xs[i] - xs[i - 1]);
+    return ys[n - 1];
+}
+constexpr double kBwShares[5] = {0.125, 0.25, 0.5, 0.75, 1.0};
+constexpr double kCoShares[3] = {0.25, 0.5, 0.75};
+}  // namespace
+
+double attn_bw(const CostModel& c, int grid, int sms) {
+    const double model = std::min(c.hbm_bw, grid * c.attn_bw_per_sm);
+    for (int i = 0; i < 5; ++i)
+        if (c.attn_bw_at[i] <= 0) return model;
+    const double x = (double)grid / std::max(1, sms);
+    if (x < kBwShares[0]) return c.attn_bw_at[0] * x / kBwShares[0];  // per-SM-bound below the table
+    return interp(kBwShares, c.attn_bw_at, 5, x);
+}
+
+double interf_attn(const CostModel& c, int sm_attn, int sms) {
+    if (c.interf_attn[0] <= 0 && c.interf_attn[1] <= 0 && c.interf_attn[2] <= 0) return c.interference;
+    return interp(kCoShares, c.interf_attn, 3, (double)sm_attn / std::max(1, sms));
+}
+
+double interf_gemm(const CostModel& c, int sm_attn, int sms) {
+    if (c.interf_gemm[0] <= 0 && c.interf_gemm[1] <= 0 && c.interf_gemm[2] <= 0) return c.interference;
+    return interp(kCoShares, c.interf_gemm, 3, (double)sm_attn / std::max(1, sms));
 }
 
 CostModel default_cost_model(int sms) {
     CostModel c;
+    for (int i = 0; i < 5; ++i) c.attn_bw_at[i] = 0;
+    for (int i = 0; i < 3; ++i) c.interf_attn[i] = c.interf_gemm[i] = 0;
     if (sms <= 0) sms = 148;
     c.gemm_flops_per_sm = 1.30e15 / 148.0;  // ~78% of the measured cuBLAS bf16 peak
     c.gemm_tile_us = 0.8;
@@ -142,7 +221,8 @@ namespace {
 
 double gemm_us(const CostModel& c, int M, int N, int K, int grid, int64_t weight_bytes) {
     if (M <= 0) return 0.0;
-    const int64_t tiles = (int64_t)((M + 127) / 128) * (N / 256);
+    // dense GEMMs run on CTA pairs with 256 x 256 tiles: two 128-row halves per pair tile
+    const int64_t tiles = (int64_t)2 * ((M + 255) / 256) * (N / 256);
     const int g = std::max(1, std::min<int>(grid, (int)tiles));
     const int64_t waves = (tiles + g - 1) / g;
     const double t_tile = 2.0 * 128 * 256 * (double)K / c.gemm_flops_per_sm * 1e6 + c.gemm_tile_us;
@@ -157,7 +237,7 @@ double gemm_us(const CostModel& c, int M, int N, int K, int grid, int64_t weight
 int op_grid(const nf_plan& p, const Op& o) {
     if (p.order_template == NF_TEMPLATE_SEQUENTIAL) return p.sm_total;
     if (o.stream == STREAM_ATTN) return p.sm_attn;
-    return o.full_sm ? p.sm_total : p.sm_gemm;
+    return (o.full_sm || o.elastic) ? p.sm_total : p.sm_gemm;
 }
 
 double op_time_us(int kind, int j, const nf_plan& p, const ModelDims& m, const BatchInfo& b, const CostModel& c,
@@ -183,8 +263,7 @@ double op_time_us(int kind, int j, const nf_plan& p, const ModelDims& m, const B
             const int r0 = std::min(t0, b.R), r1 = std::min(t1, b.R);
             const int64_t bytes = b.req_kv_prefix[r1] - b.req_kv_prefix[r0];
             if (bytes <= 0) return 0.0;
-            const double bw = std::min(c.hbm_bw, grid * c.attn_bw_per_sm);
-            return c.attn_launch_us + (double)bytes / bw * 1e6;
+            return c.attn_launch_us + (double)bytes / attn_bw(c, grid, p.sm_total) * 1e6;
         }
         case OP_PATT: {
             if (!(t1 > b.R && b.C > 0)) return 0.0;
@@ -206,23 +285,34 @@ double simulate_plan(const nf_plan& p, const ModelDims& m, const BatchInfo& b, c
     const bool pipelined = p.order_template != NF_TEMPLATE_SEQUENTIAL;
     std::vector<double> dur(ops.size()), beg(ops.size()), end(ops.size());
     double serial = 0.0;
+    std::vector<double> dur_gemm_share(ops.size(), 0.0);  // elastic ops: time on the GEMM share alone
     for (size_t i = 0; i < ops.size(); ++i) {
         const Op& o = ops[i];
         const int grid = op_grid(p, o);
         dur[i] = op_time_us(o.kind, o.nano, p, m, b, c, grid);
+        if (o.elastic) dur_gemm_share[i] = op_time_us(o.kind, o.nano, p, m, b, c, p.sm_gemm);
         serial += op_time_us(o.kind, o.nano, p, m, b, c, S);
     }
     if (serial_us) *serial_us = serial;
     double makespan = 0.0;
     for (int pass = 0; pass < 2; ++pass) {
         double free_t[2] = {0.0, 0.0};
+        double attn_end = 0.0;  // end of the latest attention op scheduled so far
         for (size_t i = 0; i < ops.size(); ++i) {
             const Op& o = ops[i];
             double st = free_t[o.stream];
             if (o.wait >= 0) st = std::max(st, end[o.wait]);
             beg[i] = st;
-            end[i] = st + dur[i];
+            double d = dur[i];
+            if (o.elastic && st < attn_end && dur_gemm_share[i] > 0) {
+                // on the GEMM share until the open attention op ends, then on every SM
+                const double full = dur[i], part = dur_gemm_share[i];
+                const double span = attn_end - st;
+                d = span >= part ? part : span + (1.0 - span / part) * full;
+            }
+            end[i] = st + d;
             free_t[o.stream] = end[i];
+            if (o.stream == STREAM_ATTN) attn_end = std::max(attn_end, end[i]);
         }
         makespan = std::max(free_t[0], free_t[1]);
         if (pass == 0 && pipelined) {
@@ -234,7 +324,11 @@ double simulate_plan(const nf_plan& p, const ModelDims& m, const BatchInfo& b, c
                 double ov = 0;
                 for (auto& iv : other[1 - ops[i].stream])
                     ov += std::max(0.0, std::min(end[i], iv.second) - std::max(beg[i], iv.first));
-                dur[i] *= 1.0 + c.interference * std::min(1.0, ov / dur[i]);
+                const double k = ops[i].stream == STREAM_ATTN ? interf_attn(c, p.sm_attn, p.sm_total)
+                                                              : interf_gemm(c, p.sm_attn, p.sm_total);
+                const double f = 1.0 + k * std::min(1.0, ov / dur[i]);
+                dur[i] *= f;
+                dur_gemm_share[i] *= f;
             }
         } else {
             break;
@@ -418,12 +512,7 @@ nf_status plan_impl(const nf_model* m, const nf_batch_desc* b, const nf_plan_opt
     for (int r = 0; r < R; ++r) pages += (b->ctx_len[r] + 1 + 15) / 16;
     pages += (C + 15) / 16;
     best.kv_pages_read = pages;
-    int64_t items = 0;
-    for (int r = 0; r < R; ++r) {
-        const int np = (b->ctx_len[r] + 1 + 15) / 16;
-        items += (int64_t)m->dims.nkv * ((np + nf::kDecodeSplitPagesHost - 1) / nf::kDecodeSplitPagesHost);
-    }
-    best.decode_items = items;
+    best.decode_items = nf::decode_work_items(m->dims, b->ctx_len, R);
     *out = best;
     return NF_OK;
 }

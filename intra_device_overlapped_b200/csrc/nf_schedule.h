@@ -17,6 +17,9 @@ struct Op {
     int nano;
     int layer;
     int full_sm;  // 1: no attention can co-run, the op may use every SM
+    int elastic;  // 1: a GEMM launched on every SM with work claimed from a counter: it runs on the SMs
+                  // the one attention kernel open beside it leaves free and grows onto the rest when
+                  // that kernel ends (never set where another attention kernel could start meanwhile)
     int wait;     // index (in issue order) of an op on the other stream to wait for, -1 = none
     int signal;   // 1: some later op waits for this one
 };
@@ -39,9 +42,18 @@ struct CostModel {
     double attn_bw_per_sm;      // bytes/s one attention SM can pull
     double attn_launch_us;
     double attn_flops_per_sm;   // prefill attention tensor FLOP/s per SM
-    double interference;        // fractional slow-down of two co-running kernels
+    double interference;        // fractional slow-down of two co-running kernels (fallback)
     int calibrated;
+    double attn_bw_at[5];       // decode bytes/s on 1/8, 1/4, 1/2, 3/4, 1 of the SMs (0 = not measured)
+    double interf_attn[3];      // decode slow-down beside GEMMs, attention on 1/4, 1/2, 3/4 of the SMs
+    double interf_gemm[3];      // GEMM slow-down beside decode attention, same shares
 };
+
+// Decode attention bytes/s on `grid` of `sms` SMs (measured table, else the per-SM / HBM model) and
+// the co-run slow-downs at attention share `sm_attn` / `sms`.
+double attn_bw(const CostModel& c, int grid, int sms);
+double interf_attn(const CostModel& c, int sm_attn, int sms);
+double interf_gemm(const CostModel& c, int sm_attn, int sms);
 
 CostModel default_cost_model(int sm_count);
 

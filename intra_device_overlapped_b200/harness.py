@@ -107,43 +107,52 @@ class DeviceWorkload:
 
     # -- set-up -----------------------------------------------------------------------------------
     def _load_weights(self):
+        for layer in range(self.shape.n_layers):
+            self.load_layer(layer)
+        if self.shape.vocab > 0:
+            self.load_globals()
+
+    def _seeded(self, specs: dict, edit=None) -> dict:
+        tens = {}
+        for name, spec in specs.items():
+            t = _empty_bf16(spec[1], self.device)
+            SW.gpu_fill(spec, t)
+            tens[name] = t
+        if edit is not None:  # tests: change the seeded tensors in place before they are handed over
+            edit(tens)
+        return tens
+
+    def load_layer(self, layer: int, edit=None) -> None:
+        """Seeded weights of one layer through nf_set_layer_weights; `edit(tensors)` may change them first."""
         s = self.shape
-        for layer in range(s.n_layers):
-            specs = SW.layer_specs(s, layer)
-            tens = {}
-            for name, spec in specs.items():
-                t = _empty_bf16(spec[1], self.device)
-                SW.gpu_fill(spec, t)
-                tens[name] = t
-            w = nf_layer_weights()
-            for f in ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm"):
-                setattr(w, f, tens[f].data_ptr())
-            keep = []
-            if s.n_experts == 0:
-                w.w_gate, w.w_up, w.w_down = (tens["w_gate"].data_ptr(), tens["w_up"].data_ptr(),
-                                              tens["w_down"].data_ptr())
-            else:
-                w.router, w.router_bias = tens["router"].data_ptr(), tens["router_bias"].data_ptr()
-                E = s.n_experts
-                g = (_vp * E)(*[tens[f"e{e}_gate"].data_ptr() for e in range(E)])
-                u = (_vp * E)(*[tens[f"e{e}_up"].data_ptr() for e in range(E)])
-                dn = (_vp * E)(*[tens[f"e{e}_down"].data_ptr() for e in range(E)])
-                keep = [g, u, dn]
-                w.expert_gate, w.expert_up, w.expert_down = g, u, dn
-            check(nf_set_layer_weights(self.model, layer, w, 0), f"nf_set_layer_weights({layer})")
-            torch.cuda.synchronize(self.device)
-            del tens, keep
-        if s.vocab > 0:
-            tens = {}
-            for name, spec in SW.global_specs(s).items():
-                t = _empty_bf16(spec[1], self.device)
-                SW.gpu_fill(spec, t)
-                tens[name] = t
-            g = nf_global_weights(embed=tens["embed"].data_ptr(), final_norm=tens["final_norm"].data_ptr(),
-                                  lm_head=tens["lm_head"].data_ptr())
-            check(nf_set_global_weights(self.model, g, 0), "nf_set_global_weights")
-            torch.cuda.synchronize(self.device)
-            del tens
+        tens = self._seeded(SW.layer_specs(s, layer), edit)
+        w = nf_layer_weights()
+        for f in ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm"):
+            setattr(w, f, tens[f].data_ptr())
+        keep = []
+        if s.n_experts == 0:
+            w.w_gate, w.w_up, w.w_down = (tens["w_gate"].data_ptr(), tens["w_up"].data_ptr(),
+                                          tens["w_down"].data_ptr())
+        else:
+            w.router, w.router_bias = tens["router"].data_ptr(), tens["router_bias"].data_ptr()
+            E = s.n_experts
+            g = (_vp * E)(*[tens[f"e{e}_gate"].data_ptr() for e in range(E)])
+            u = (_vp * E)(*[tens[f"e{e}_up"].data_ptr() for e in range(E)])
+            dn = (_vp * E)(*[tens[f"e{e}_down"].data_ptr() for e in range(E)])
+            keep = [g, u, dn]
+            w.expert_gate, w.expert_up, w.expert_down = g, u, dn
+        check(nf_set_layer_weights(self.model, layer, w, 0), f"nf_set_layer_weights({layer})")
+        torch.cuda.synchronize(self.device)
+        del tens, keep
+
+    def load_globals(self, edit=None) -> None:
+        """Seeded embedding, final norm and LM head through nf_set_global_weights (see load_layer)."""
+        tens = self._seeded(SW.global_specs(self.shape), edit)
+        g = nf_global_weights(embed=tens["embed"].data_ptr(), final_norm=tens["final_norm"].data_ptr(),
+                              lm_head=tens["lm_head"].data_ptr())
+        check(nf_set_global_weights(self.model, g, 0), "nf_set_global_weights")
+        torch.cuda.synchronize(self.device)
+        del tens
 
     def make_io(self, hidden_in: Optional[torch.Tensor] = None, hidden_out: Optional[torch.Tensor] = None,
                 next_token: Optional[torch.Tensor] = None) -> nf_iter_io:

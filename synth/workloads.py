@@ -94,6 +94,14 @@ def make_batch(w: Workload, seed: int = SEED_BATCH) -> Batch:
         ctx = np.clip(ctx, w.ctx_lo, w.ctx_hi).astype(np.int64)
     else:
         ctx = uniform_int(seed, B_CTX_UNIFORM, R, w.ctx_lo, w.ctx_hi)
+    return batch_for_contexts(s, ctx, C, seed)
+
+
+def batch_for_contexts(s: ModelShape, ctx, C: int, seed: int = SEED_BATCH) -> Batch:
+    """Batch of decode requests with the given context lengths plus a C-token prefill chunk, with the
+    seeded page permutation of ``make_batch`` (edge cases: empty contexts, page and chunk boundaries)."""
+    ctx = np.asarray(ctx, dtype=np.int64)
+    R, P = len(ctx), s.page_size
     # Pages: decode request r holds ctx+1 keys (its new token included); the prefill request C keys.
     counts = [pages_needed(c + 1, P) for c in ctx] + [pages_needed(C, P)]
     num_pages = int(sum(counts))

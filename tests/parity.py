@@ -20,3 +20,18 @@ def row_scaled_max_abs(gpu, ref):
     ref = np.asarray(ref, dtype=np.float64)
     rms = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True))
     return float(np.max(np.abs(gpu - ref) / np.maximum(rms, 1e-30)))
+
+
+def check_readings(got, refs, what, row_scaled=True):
+    """Assert the bars against each precision reading of the oracle in `refs` ({name: reference}).
+
+    Hidden states are compared with the row-scaled max-abs (each row divided by the oracle row's RMS);
+    logits with the raw max-abs. The raw max-abs and the relative L1 error are printed for every
+    reading, so the test output records the numbers behind each verdict.
+    """
+    for name, ref in refs.items():
+        raw, rel = errors(got, ref)
+        mx = row_scaled_max_abs(got, ref) if row_scaled else raw
+        print(f"{what} vs {name}: {'row-scaled ' if row_scaled else ''}max-abs {mx:.4g}, raw max-abs {raw:.4g}, "
+              f"relative L1 {rel:.4g}")
+        assert mx <= MAX_ABS and rel <= MEAN_REL, (what, name, mx, rel)

@@ -208,3 +208,13 @@ def test_planner_fuzz_returns_valid_plans_or_invalid_argument(nf):
         if p.order_template != nf.NF_TEMPLATE_SEQUENTIAL:
             assert 1 <= p.sm_attn and p.sm_attn + p.sm_gemm <= 148
     assert ok > 100
+
+
+def test_offload_rejects_bad_arguments_without_a_device(nf):
+    """nf_offload_kv validates on the host: a null model, empty page list or empty layer range is
+    rejected before anything is launched."""
+    import ctypes
+    pools = (ctypes.c_void_p * 1)(None)
+    buf = ctypes.create_string_buffer(16)
+    assert nf.nf_offload_kv(None, pools, 4, [0, 1], 0, 1, ctypes.addressof(buf), 0) == nf.NF_ERR_INVALID_ARGUMENT
+    assert nf.nf_offload_kv(None, pools, 4, [], 0, 1, ctypes.addressof(buf), 0) == nf.NF_ERR_INVALID_ARGUMENT

@@ -9,7 +9,7 @@ from synth.workloads import WORKLOADS, TEST_WORKLOADS
 from synth import weights as SW
 import synth
 
-from parity import MAX_ABS, MEAN_REL, errors
+from parity import MAX_ABS, MEAN_REL, errors, check_readings
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -39,6 +39,7 @@ def tiny():
     w = TEST_WORKLOADS["tiny_gamma"]
     dw = DeviceWorkload(w, DEV)
     b, res, kv = run_oracle(w, batch=dw.batch)
+    res["hidden_f64"] = run_oracle(w, batch=dw.batch, bf16_act=False)[1]["hidden"]
     yield dw, res, kv
     dw.close()
 
@@ -54,8 +55,8 @@ def test_tiny_iteration_matches_oracle(tiny, opts):
     _reset_kv(dw)
     plan = dw.plan(**opts)
     hid = _run(dw, plan)
-    mx, rel = errors(hid, res["hidden"])
-    assert mx <= MAX_ABS and rel <= MEAN_REL, (mx, rel, plan.describe())
+    check_readings(hid, {"bf16 model": res["hidden"], "float64 activations": res["hidden_f64"]},
+                   f"tiny layer, plan {plan.describe()}")
     # bf16 output copy is the rounded fp32 residual
     hb = dw.hidden_out.float().cpu().numpy()
     assert np.abs(hb - hid).max() <= np.abs(hid).max() * 2 ** -8
@@ -111,11 +112,11 @@ def test_degenerate_batches(name):
     dw = DeviceWorkload(w, DEV)
     try:
         _, res, _ = run_oracle(w, batch=dw.batch)
+        ref64 = run_oracle(w, batch=dw.batch, bf16_act=False)[1]["hidden"]
         for opts in (dict(nano=1, template=0), dict()):
             _reset_kv(dw)
             hid = _run(dw, dw.plan(**opts))
-            mx, rel = errors(hid, res["hidden"])
-            assert mx <= MAX_ABS and rel <= MEAN_REL, (mx, rel)
+            check_readings(hid, {"bf16 model": res["hidden"], "float64 activations": ref64}, f"{name} {opts}")
     finally:
         dw.close()
 
@@ -127,10 +128,12 @@ def test_tiny_lm_head_and_argmax():
     dw = DeviceWorkload(w, DEV)
     try:
         _, res, _ = run_oracle(w, batch=dw.batch)
+        res64 = run_oracle(w, batch=dw.batch, bf16_act=False)[1]
         _run(dw, dw.plan(nano=2, template=1, sm_attn=32))
         logits = dw.logits.float().cpu().numpy()
+        check_readings(logits, {"bf16 model": res["logits"], "float64 activations": res64["logits"]},
+                       "tiny LM logits", row_scaled=False)
         mx, rel = errors(logits, res["logits"])
-        assert mx <= MAX_ABS and rel <= MEAN_REL, (mx, rel)
         nxt = dw.next_token.cpu().numpy()
         ref = res["logits"]
         for r, tok in enumerate(nxt):
@@ -150,9 +153,9 @@ def test_tiny_moe_routing_and_output():
     dw = DeviceWorkload(w, DEV, moe_debug=True)
     try:
         _, res, _ = run_oracle(w, batch=dw.batch)
+        res64 = run_oracle(w, batch=dw.batch, bf16_act=False)[1]
         hid = _run(dw, dw.plan(nano=2, template=1, sm_attn=24))
-        mx, rel = errors(hid, res["hidden"])
-        assert mx <= MAX_ABS and rel <= MEAN_REL, (mx, rel)
+        check_readings(hid, {"bf16 model": res["hidden"], "float64 activations": res64["hidden"]}, "tiny MoE")
         for layer in range(w.shape.n_layers):
             z_gpu = dw.router_logits[layer].cpu().numpy().astype(np.float64)
             z_ref = res["layers"][layer]["router_logits"]
@@ -177,13 +180,13 @@ def test_gqa8_iteration_matches_oracle_and_is_invariant():
     dw = DeviceWorkload(w, DEV)
     try:
         _, res, _ = run_oracle(w, batch=dw.batch)
+        ref64 = run_oracle(w, batch=dw.batch, bf16_act=False)[1]["hidden"]
         outs = []
         for opts in (dict(nano=1, template=0), dict(nano=2, template=1, sm_attn=20),
                      dict(nano=3, template=2, sm_attn=36), dict()):
             _reset_kv(dw)
             hid = _run(dw, dw.plan(**opts))
-            mx, rel = errors(hid, res["hidden"])
-            assert mx <= MAX_ABS and rel <= MEAN_REL, (mx, rel, opts)
+            check_readings(hid, {"bf16 model": res["hidden"], "float64 activations": ref64}, f"small_gqa8 {opts}")
             outs.append(_bits(dw.hidden_out_f32))
         for o in outs[1:]:
             assert np.array_equal(o, outs[0])
@@ -205,5 +208,89 @@ def test_tuned_plan_is_bitwise_equal_to_sequential():
         _reset_kv(dw)
         _run(dw, plan)
         assert np.array_equal(_bits(dw.hidden_out_f32), ref)
+    finally:
+        dw.close()
+
+
+# --- bit-exact decisions: planted exact ties and the embedding gather -------------------------------
+
+def test_lm_head_exact_ties_pick_the_lower_index():
+    """LM head with every row zero except rows 5 and 900, which are equal: the fp32 logits of those two
+    columns are identical and every other logit is exactly 0. The greedy token must be 5 where that
+    shared logit is positive and 0 (the first of the zero logits) where it is negative: ties go to
+    the lower index, bit-exactly, across the tile-wise maximum and its reduction."""
+    from intra_device_overlapped_b200.harness import DeviceWorkload
+    w = TEST_WORKLOADS["tiny_lm"]
+    dw = DeviceWorkload(w, DEV)
+    try:
+        def edit(t):
+            head = t["lm_head"]
+            row = head[5].clone()
+            head.zero_()
+            head[5] = row
+            head[900] = row
+        dw.load_globals(edit)
+        _run(dw, dw.plan(nano=2, template=1, sm_attn=32))
+        logits = dw.logits.float().cpu().numpy()
+        nxt = dw.next_token.cpu().numpy()
+        assert np.array_equal(logits[:, 5], logits[:, 900])
+        others = np.delete(logits, [5, 900], axis=1)
+        assert np.all(others == 0.0)
+        expect = np.where(logits[:, 5] > 0, 5, 0)
+        assert np.any(expect == 5) and np.any(expect == 0)   # both tie kinds occur
+        assert np.array_equal(nxt, expect), (nxt, expect)
+    finally:
+        dw.close()
+
+
+@pytest.mark.parametrize("tie", ["all_equal", "pair"])
+def test_router_exact_ties_pick_the_lower_experts(tie):
+    """Router rows made equal: 'all_equal' gives every expert the same logit (top-2 must be experts
+    0 and 1 with weights 1/2 each); 'pair' gives experts 1 and 3 the same row and a bias above the
+    others (top-2 must be [1, 3]). Routing is compared bit-exactly on every token and layer."""
+    from intra_device_overlapped_b200.harness import DeviceWorkload
+    w = TEST_WORKLOADS["tiny_moe"]
+    dw = DeviceWorkload(w, DEV, moe_debug=True)
+    try:
+        def edit(t):
+            r, b = t["router"], t["router_bias"]
+            if tie == "all_equal":
+                r[:] = r[0].clone()
+                b[:] = b[0].clone()
+            else:
+                r[3] = r[1].clone()
+                b[:] = -8.0
+                b[1] = 8.0
+                b[3] = 8.0
+        for layer in range(w.shape.n_layers):
+            dw.load_layer(layer, edit)
+        _run(dw, dw.plan(nano=2, template=1, sm_attn=24))
+        want = [0, 1] if tie == "all_equal" else [1, 3]
+        for layer in range(w.shape.n_layers):
+            idx = dw.topk_idx[layer].cpu().numpy()
+            assert np.all(idx == np.array(want)[None, :]), (layer, idx[:4])
+            if tie == "all_equal":
+                assert np.all(dw.topk_w[layer].cpu().numpy() == 0.5)
+    finally:
+        dw.close()
+
+
+def test_embedding_gather_is_bit_exact():
+    """With the output and down projections zeroed, every layer adds exact zeros to the residual
+    stream, so the fp32 hidden state leaving the model is the gathered embedding row of each token:
+    compared bit for bit with the bf16 table widened to fp32."""
+    from intra_device_overlapped_b200.harness import DeviceWorkload
+    w = TEST_WORKLOADS["tiny_lm"]
+    dw = DeviceWorkload(w, DEV)
+    try:
+        def zero_out(t):
+            t["wo"].zero_()
+            t["w_down"].zero_()
+        for layer in range(w.shape.n_layers):
+            dw.load_layer(layer, zero_out)
+        _run(dw, dw.plan(nano=2, template=1, sm_attn=32))
+        got = dw.hidden_out_f32.cpu().numpy()
+        emb = synth.bf16_to_f64(SW.host_rows(SW.global_specs(w.shape)["embed"], np.asarray(dw.batch.tokens)))
+        assert np.array_equal(got.astype(np.float64), emb)
     finally:
         dw.close()
