@@ -439,6 +439,43 @@ def run_ours(args, work, dist):
                 "ops": {k: round(v / 1000, 4) for k, v in share.items()},
                 "sum_ms": round(sum(share.values()) / 1000, 4)}
 
+        # ---- KV offload beside the iteration: every step also copies the KV pages of two decode requests
+        # (every layer) to pinned host memory on a low-priority stream, as a serving loop does for the
+        # requests that finished; the timed region ends when both the iterations and the copies are done
+        s = work.shape
+        off_reqs = [0, 1] if R >= 2 else list(range(R))
+        if off_reqs:
+            pages = [int(pg) for r in off_reqs for pg in b.page_indices[b.page_indptr[r]:b.page_indptr[r + 1]]]
+            page_elems = dw.kv[0].shape[1]
+            host_kv = torch.empty((s.n_layers, len(pages), page_elems), dtype=torch.bfloat16).pin_memory()
+            side = torch.cuda.Stream(dev, priority=0)
+            side.wait_stream(stream)
+
+            def offload():
+                nf.check(nf.nf_offload_kv(dw.model, dw._kv_ptrs, b.num_pages, pages, 0, s.n_layers,
+                                          host_kv.data_ptr(), side.cuda_stream), "offload")
+            for _ in range(3):
+                offload()
+                dw.forward(plan, stream)
+            torch.cuda.synchronize(dev)
+            o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            o0.record(stream)
+            side.wait_stream(stream)
+            for _ in range(args.steps):
+                offload()
+                dw.forward(plan, stream)
+            stream.wait_stream(side)
+            o1.record(stream)
+            torch.cuda.synchronize(dev)
+            nf.check(dw.sync(), "offload steps")
+            off_ms = dist.max(o0.elapsed_time(o1)) / args.steps
+            extras["kv_offload"] = {
+                "requests_per_step": len(off_reqs), "pages_per_step": len(pages) * s.n_layers,
+                "bytes_per_step": int(host_kv.numel() * 2), "ms_per_step": round(off_ms, 4),
+                "slowdown": round(off_ms / ms_step - 1.0, 4),
+                "how": "nf_offload_kv on a low-priority stream beside every iteration (gather kernel + D2H copy "
+                       "per layer into pinned host memory)"}
+
         # ---- end to end through the C ABI with host buffers: every step copies its inputs from pinned
         # host memory to the device and reads its result back. As a serving loop does, the copies
         # of neighbouring steps overlap the compute of this one: two device input/output sets, the

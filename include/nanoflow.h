@@ -88,8 +88,12 @@ typedef struct {
     int32_t max_position; /* positions must be < max_position (RoPE table length) */
 } nf_model_config;
 
-/* Validate `cfg`, allocate the model's packed-weight buffers and workspace and
- * build the RoPE table (angles pos * theta^(-2i/d) in double, stored as fp32).
+/* A Llama-style model of the families the NanoFlow README benchmarks ("Feasibility": LLaMA-2-70B,
+ * LLaMA-3-8B, Mixtral 8x7B; dense SwiGLU or top-k mixture of experts, grouped-query attention).
+ * Validate `cfg`, allocate the model's packed-weight buffers and workspace and
+ * build the RoPE table (angles pos * theta^(-2i/d) in double, stored as fp32). The weights
+ * are handed over afterwards, layer by layer, with nf_set_layer_weights / nf_set_global_weights
+ * (a model of 34 GB of weights need not exist twice on the device at any moment).
  * On success *out owns device memory until nf_destroy_model. Requirements:
  * (nq + 2 nkv) d, nq d, H and 2F divisible by 256; H divisible by 64. */
 nf_status nf_init_model(const nf_model_config* cfg, nf_model** out);
@@ -227,8 +231,15 @@ typedef struct {
 } nf_iter_io;
 
 /* Run the iteration described by `plan` (made by nf_plan_iteration for the same
- * batch). GEMMs run on `stream`, attention on a model-owned second stream that
- * forks from and joins back into `stream`. Asynchronous. */
+ * batch): NanoFlow's nano-batched serving iteration (arXiv abstract of "NanoFlow: Towards Optimal
+ * Large Language Model Serving Throughput": the batch is split into nano-batches and each
+ * operation is duplicated per nano-batch so that operations bound by different resources overlap
+ * inside the device; README "Introduction": compute-bound GEMMs beside memory-bound attention).
+ * GEMMs run on `stream`, attention on a model-owned second stream (the higher-priority one) that
+ * forks from and joins back into `stream`; the result does not depend on the plan (bit for bit).
+ * Page ids of the device page table are checked on the device (an id outside the pool is recorded
+ * as NF_ERR_DEVICE_BOUNDS and the access skipped); nf_plan_iteration checks the host copy before
+ * anything runs. Asynchronous. */
 nf_status nf_forward_iteration(nf_model* m, const nf_plan* plan, const nf_iter_io* io, void* stream);
 
 /* Plan choice by measurement. For each template and nano-batch count the planner's best
@@ -373,7 +384,7 @@ nf_status nf_offload_kv(nf_model* m, void* const* kv_pools, int32_t num_pool_pag
  * attention step), with the same tensor-core kernel as nf_op_decode_attention. Each request is
  * one work item here (no split along the keys, whose partials would need scratch that grows
  * with the batch), so the result equals nf_op_decode_attention's bit for bit for requests of at
- * most 512 keys (which that entry point does not split either) and within rounding otherwise.
+ * most 2048 keys (which that entry point does not split either) and within rounding otherwise.
  *   q, out        device bf16 [num_requests x n_q_heads x head_dim], row r = request r.
  *   kv_pool       device bf16 pool of one layer, num_pages pages in the physical page layout
  *                 described for nf_iter_io.kv_pools.

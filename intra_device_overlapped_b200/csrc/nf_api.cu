@@ -396,7 +396,8 @@ nf::DecodeArgs decode_args(const nf_model* m, const nf_iter_io* io, const void* 
     a.nkv = m->dims.nkv;
     a.G = m->dims.nq / m->dims.nkv;
     a.num_pages = io->num_pages;
-    a.split_pages = nf::kDecodeSplitPages;
+    a.split_pages = m->decode_tc ? nf::kDecodeSplitPagesTc : nf::kDecodeSplitPages;
+    a.any_split = m->decode_any_split ? 1 : 0;
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m->dims.d));
     a.merge_cnt = m->merge_cnt;
     a.chunk_off = m->chunk_off;
@@ -453,7 +454,7 @@ cudaError_t decode_prologue(nf_model* m, const nf_iter_io* io, int R, cudaStream
     if (R <= 0) return cudaSuccess;
     const nf::ModelDims& d = m->dims;
     if (m->decode_tc)
-        return nf::launch_decode_tc_schedule(io->ctx_len, R, nf::kDecodeSplitPages, m->item_off, m->chunk_off,
+        return nf::launch_decode_tc_schedule(io->ctx_len, R, nf::kDecodeSplitPagesTc, m->item_off, m->chunk_off,
                                              m->status, s);
     cudaError_t e = nf::launch_decode_schedule(io->ctx_len, R, d.nkv, nf::kDecodeSplitPages, m->item_off, s);
     if (e != cudaSuccess) return e;
@@ -655,6 +656,7 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     cudaStream_t sg = (cudaStream_t)stream;
     cudaStream_t sa = m->s_attn;
     if ((st = ensure_part_capacity(m, std::max<int64_t>(p->decode_items, 1))) != NF_OK) return st;
+    m->decode_any_split = m->decode_tc ? p->decode_items > R : true;
     for (int l = 0; l < d.L; ++l)
         if ((st = check_pool(m, l, io)) != NF_OK) return st;
 
@@ -941,7 +943,7 @@ extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* ou
     {  // work items of these requests (the device holds ctx_len): size the split-KV partials
         int items = 0;
         if (m->decode_tc) {
-            NF_CUDA_TRY(nf::launch_decode_tc_schedule(io->ctx_len, req_end, nf::kDecodeSplitPages, m->item_off,
+            NF_CUDA_TRY(nf::launch_decode_tc_schedule(io->ctx_len, req_end, nf::kDecodeSplitPagesTc, m->item_off,
                                                       m->chunk_off, m->status, s));
             NF_CUDA_TRY(cudaMemcpyAsync(&items, m->chunk_off + req_end, sizeof(int), cudaMemcpyDeviceToHost, s));
         } else {
@@ -951,6 +953,7 @@ extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* ou
         }
         NF_CUDA_TRY(cudaStreamSynchronize(s));
         if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
+        m->decode_any_split = items > req_end;
     }
     NF_CUDA_TRY(decode_prologue(m, io, req_end, s));
     CUtensorMap tmq;
@@ -1115,7 +1118,9 @@ extern "C" nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_
     int64_t kv_bytes = 0;
     for (int r = 0; r < R; ++r) kv_bytes += (int64_t)((b->ctx_len[r] + 1 + 15) / 16) * 2 * 16 * d.d * 2 * d.nkv;
     if (R > 0) {
-        if ((st = ensure_part_capacity(m, nf::decode_work_items(d, b->ctx_len, R))) != NF_OK) return st;
+        const int64_t items = nf::decode_work_items(d, b->ctx_len, R);
+        if ((st = ensure_part_capacity(m, items)) != NF_OK) return st;
+        m->decode_any_split = m->decode_tc ? items > R : true;
         NF_CUDA_TRY(decode_prologue(m, io, R, sg));
         NF_CUDA_TRY(cudaMemsetAsync(m->q, 0, (size_t)R * d.nq * d.d * 2, sg));
         auto dec = [&](int grid, cudaStream_t s) -> nf_status {

@@ -8,9 +8,11 @@
 
 namespace nf {
 
-// Decode keys are split into chunks of this many pages (512 keys); the split of a request
-// depends only on its ctx_len.
+// Decode keys are split into chunks of at most this many pages; the split of a request depends only
+// on its ctx_len. The warp-level kernel splits every request longer than 512 keys; the tensor-core
+// kernel, whose chunks cost a hand-off and a merge, splits contexts longer than 2048 keys.
 constexpr int kDecodeSplitPages = 32;
+constexpr int kDecodeSplitPagesTc = 128;
 // split_pages value that keeps every request in one chunk (no partials, no merge pass)
 constexpr int kDecodeNoSplit = 1 << 30;
 
@@ -33,6 +35,7 @@ struct DecodeArgs {
     int* merge_cnt;       // [R x nkv] split arrival counters (zeroed by decode_items_kernel)
     const int* chunk_off; // tensor-core kernel: [R + 1] first partial slot of each request
     float* part_ml;       // tensor-core kernel: [chunks x nq x 2] running maximum and row sum per query head
+    int any_split;        // tensor-core kernel: 0 when no request of the launch has more than one chunk
     int* status;
     int* trace_ctr;
     nf_trace_entry* trace;

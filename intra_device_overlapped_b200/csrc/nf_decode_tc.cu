@@ -10,7 +10,8 @@
 //   [K|V][64-column half of d][KV head][16 tokens][8 chunks of 16 B, chunk c of row r at c ^ (r & 7)]
 // and one bulk copy per half moves a page into a ring stage.
 //
-// Split along KV. A request of n pages is cut into ceil(n / chunk_pages) chunks whose page counts
+// Split along KV. A request of n pages is cut into ceil(n / chunk_pages) chunks (chunk_pages = 128,
+// so contexts above 2048 keys are split) whose page counts
 // differ by at most one (chunk c = pages [c n / nch, (c + 1) n / nch)); the cut depends only on the
 // request's context length, never on the grid. A work item is one chunk with all heads. Items are dealt to the persistent CTAs in
 // contiguous ranges of equal page counts, so a CTA's share differs from the mean by less than
@@ -559,34 +560,48 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // Requests cut into several chunks: out = bf16(sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c) per
 // query head, M the largest chunk maximum, both sums in chunk order (every factor is an exact power of
-// two). One CTA of 128 threads (one d each) per request at a time.
+// two). CTA (x, y) of 128 threads (one d each) merges the 8 query heads of group y of requests
+// x, x + gridDim.x, ...; a thread's loads for its 8 heads are independent, so they overlap.
+constexpr int MERGE_HEADS = 8;
+
 template <int NQ>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const __grid_constant__ DecodeArgs a) {
-    __shared__ float Ms[NQ], Ls[NQ];
+    __shared__ float Ms[MERGE_HEADS], Ls[MERGE_HEADS];
     const int t = threadIdx.x;
+    const int h0 = blockIdx.y * MERGE_HEADS;
     for (int r = a.req_begin + blockIdx.x; r < a.req_end; r += gridDim.x) {
         const int npages = (max(a.ctx_len[r], 0) + 1 + 15) >> 4;
         const int nch = ceil_div(npages, a.split_pages);
         if (nch <= 1) continue;  // written by the attention kernel
-        const float* ml = a.part_ml + (size_t)a.chunk_off[r] * NQ * 2;
-        const float* po = a.part_o + (size_t)a.chunk_off[r] * NQ * 128;
+        const float* __restrict__ ml = a.part_ml + (size_t)a.chunk_off[r] * NQ * 2;
+        const float* __restrict__ po = a.part_o + (size_t)a.chunk_off[r] * NQ * 128;
         __syncthreads();  // the previous request's Ms / Ls are no longer read
-        if (t < NQ) {
+        if (t < MERGE_HEADS) {
+            const int qh = h0 + t;
             float M = -INFINITY;
-            for (int c = 0; c < nch; ++c) M = fmaxf(M, ml[(c * NQ + t) * 2]);
+            for (int c = 0; c < nch; ++c) M = fmaxf(M, ml[(c * NQ + qh) * 2]);
             float L = 0.f;
-            for (int c = 0; c < nch; ++c) L += softmax_rescale(ml[(c * NQ + t) * 2], M) * ml[(c * NQ + t) * 2 + 1];
+            for (int c = 0; c < nch; ++c) L += softmax_rescale(ml[(c * NQ + qh) * 2], M) * ml[(c * NQ + qh) * 2 + 1];
             Ms[t] = M;
             Ls[t] = L;
         }
         __syncthreads();
-        for (int qh = 0; qh < NQ; ++qh) {
-            const float M = Ms[qh];
-            float acc = 0.f;
-            for (int c = 0; c < nch; ++c)
-                acc += softmax_rescale(ml[(c * NQ + qh) * 2], M) * __ldcg(po + ((size_t)c * NQ + qh) * 128 + t);
-            a.out[((size_t)r * NQ + qh) * 128 + t] = f2bf(acc / Ls[qh]);
+        float acc[MERGE_HEADS];
+#pragma unroll
+        for (int i = 0; i < MERGE_HEADS; ++i) acc[i] = 0.f;
+        for (int c = 0; c < nch; ++c) {
+            float v[MERGE_HEADS], f[MERGE_HEADS];
+#pragma unroll
+            for (int i = 0; i < MERGE_HEADS; ++i) {
+                v[i] = __ldcg(po + ((size_t)c * NQ + h0 + i) * 128 + t);
+                f[i] = softmax_rescale(ml[(c * NQ + h0 + i) * 2], Ms[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < MERGE_HEADS; ++i) acc[i] += f[i] * v[i];
         }
+#pragma unroll
+        for (int i = 0; i < MERGE_HEADS; ++i)
+            a.out[((size_t)r * NQ + h0 + i) * 128 + t] = f2bf(acc[i] / Ls[i]);
     }
 }
 
@@ -601,8 +616,9 @@ cudaError_t launch_nq(const CUtensorMap& tmQ, const DecodeArgs& a, int grid, cud
     }
     decode_attention_tc_kernel<NQ><<<grid, THREADS, TcCfg<NQ>::SMEM, stream>>>(tmQ, a);
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess || a.split_pages >= kDecodeNoSplit) return e;
-    decode_merge_kernel<NQ><<<grid, 128, 0, stream>>>(a);
+    if (e != cudaSuccess || a.split_pages >= kDecodeNoSplit || !a.any_split) return e;
+    const int rows = a.req_end - a.req_begin;
+    decode_merge_kernel<NQ><<<dim3(rows < 1024 ? rows : 1024, NQ / MERGE_HEADS), 128, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

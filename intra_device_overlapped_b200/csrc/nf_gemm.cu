@@ -729,8 +729,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA producer of this CTA's A rows and B half
+            // A (activations) is re-read by every column block: keep it in L2; B (weights) is shared by
+            // the row blocks of a column block, which run at about the same time, under the default policy
             const uint64_t a_policy = l2_policy_evict_last();
-            const uint64_t b_policy = l2_policy_evict_first();
+            const uint64_t b_policy = l2_policy_evict_normal();
             uint32_t stage = 0, phase = 0;
             int pending[STAGES2];
             for (int s = 0; s < STAGES2; ++s) pending[s] = -1;

@@ -10,7 +10,8 @@
 
 namespace nf {
 
-constexpr int kDecodeSplitPagesHost = 32;  // must equal kDecodeSplitPages (nf_attention.h)
+constexpr int kDecodeSplitPagesHost = 32;     // must equal kDecodeSplitPages (nf_attention.h)
+constexpr int kDecodeSplitPagesTcHost = 128;  // must equal kDecodeSplitPagesTc (nf_attention.h)
 
 // Decode attention work items of a batch (sizes the split-KV partials): chunks of at most
 // kDecodeSplitPagesHost pages, one per request chunk for the tensor-core kernel, one per KV head
@@ -56,6 +57,7 @@ struct nf_model {
     int* item_off = nullptr;      // [max_requests + 1] page prefix (tensor-core decode) or item prefix
     int* chunk_off = nullptr;     // [max_requests + 1] split-KV chunk prefix (tensor-core decode)
     int* tile_ctr = nullptr;      // [kMaxCountedOps] work counters of elastic GEMM ops, zeroed per forward
+    bool decode_any_split = true; // some request of the current batch spans several decode chunks
     // KV offload: two staging buffers of offload_cap pages and the device copy of the page list
     uint8_t* offload_stage = nullptr;
     int* offload_ids = nullptr;

@@ -26,11 +26,13 @@
 namespace nf {
 
 int64_t decode_work_items(const ModelDims& d, const int32_t* ctx_len, int R) {
-    const int per = decode_tc_supported(d.nq, d.nkv, d.d) ? 1 : d.nkv;
+    const bool tc = decode_tc_supported(d.nq, d.nkv, d.d);
+    const int per = tc ? 1 : d.nkv;
+    const int split = tc ? kDecodeSplitPagesTcHost : kDecodeSplitPagesHost;
     int64_t items = 0;
     for (int r = 0; r < R; ++r) {
         const int np = (std::max(ctx_len[r], 0) + 1 + 15) / 16;
-        items += (int64_t)per * ((np + kDecodeSplitPagesHost - 1) / kDecodeSplitPagesHost);
+        items += (int64_t)per * ((np + split - 1) / split);
     }
     return items;
 }

@@ -119,6 +119,13 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
     return pol;
 }
 
+// The default L2 policy, as a cache-hint operand.
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // tma_load_2d with an L2 cache policy.
 __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
                                                  uint64_t policy) {

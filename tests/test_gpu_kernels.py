@@ -232,9 +232,9 @@ def test_tc64_decode_many_request_ends_per_cta_is_deterministic(nf):
 # --- decode attention edge cases: explicit context lengths ---------------------------------------------
 
 # Contexts of 0 keys cached (the new key alone), one page minus one / exactly / plus one, the split
-# boundaries of the tensor-core kernel (32 pages of 16 keys per chunk: 511 / 512 / 513 keys) and the
-# longest Mixtral context (4096 cached, 257 pages, 9 chunks).
-EDGE_CTX = [0, 15, 16, 17, 31, 510, 511, 512, 1023, 4096, 4095, 100, 1]
+# boundary of the tensor-core kernel (chunks of at most 128 pages of 16 keys: 2047 / 2048 / 2049 keys)
+# and the longest Mixtral context (4096 cached, 257 pages, 3 chunks).
+EDGE_CTX = [0, 15, 16, 17, 31, 510, 511, 2046, 2047, 2048, 4096, 4095, 100, 1]
 
 
 @pytest.mark.parametrize("nq", [32, 64])

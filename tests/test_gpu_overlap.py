@@ -41,7 +41,7 @@ def test_decode_and_gemm_ctas_split_the_sms_and_overlap():
         dw.trace(True)
         dw.forward(plan)
         assert dw.sync() == 0
-        entries = [(e.kernel, e.smid, e.t_start, e.t_end) for e in dw.get_trace()]
+        entries = list(dw.get_trace())   # (kernel, smid, t_start, t_end)
         dw.trace(False)
         assert torch.equal(dw.hidden_out_f32.view(torch.int32), ref.view(torch.int32)), plan.describe()
 
