@@ -244,8 +244,9 @@ nf_status nf_forward_iteration(nf_model* m, const nf_plan* plan, const nf_iter_i
 
 /* Plan choice by measurement. For each template and nano-batch count the planner's best
  * plan (the SM split chosen by the cost model) is run on this batch: one warm-up and `reps`
- * timed iterations (CUDA events on `stream`). The fastest plan is written to `out` and its
- * mean iteration time in microseconds to `best_us` (nullable). This is the search over
+ * timed iterations (CUDA events on `stream`). The four fastest are then timed again in turn over
+ * five rounds (so that clock drift under the power cap does not decide), and the one with the
+ * lowest median is written to `out` and that median, in microseconds, to `best_us` (nullable). This is the search over
  * measured costs that the arXiv abstract describes, with the final choice between templates
  * and counts made on the device, where the interference of co-running kernels is real.
  * Runs nf_forward_iteration with `io` repeatedly: the new tokens' K/V slots are rewritten
@@ -281,6 +282,11 @@ typedef struct {
     double attn_bw_at[5];
     double interf_attn[3];
     double interf_gemm[3];
+    /* Measured over predicted time of the sequential one-nano-batch plan on the calibration batch
+     * (1 = not measured). The kernel rates above are timed in bursts of a few launches; an iteration
+     * that runs for tens of milliseconds settles at the lower clock of the power cap, and this factor
+     * carries that into every prediction. */
+    double iter_scale;
 } nf_cost_model;
 
 nf_status nf_get_cost_model(const nf_model* m, nf_cost_model* out);
@@ -384,7 +390,7 @@ nf_status nf_offload_kv(nf_model* m, void* const* kv_pools, int32_t num_pool_pag
  * attention step), with the same tensor-core kernel as nf_op_decode_attention. Each request is
  * one work item here (no split along the keys, whose partials would need scratch that grows
  * with the batch), so the result equals nf_op_decode_attention's bit for bit for requests of at
- * most 2048 keys (which that entry point does not split either) and within rounding otherwise.
+ * most 1024 keys (which that entry point does not split either) and within rounding otherwise.
  *   q, out        device bf16 [num_requests x n_q_heads x head_dim], row r = request r.
  *   kv_pool       device bf16 pool of one layer, num_pages pages in the physical page layout
  *                 described for nf_iter_io.kv_pools.

@@ -10,9 +10,9 @@ namespace nf {
 
 // Decode keys are split into chunks of at most this many pages; the split of a request depends only
 // on its ctx_len. The warp-level kernel splits every request longer than 512 keys; the tensor-core
-// kernel, whose chunks cost a hand-off and a merge, splits contexts longer than 2048 keys.
+// kernel, whose chunks cost a hand-off and a merge, splits contexts longer than 1024 keys.
 constexpr int kDecodeSplitPages = 32;
-constexpr int kDecodeSplitPagesTc = 128;
+constexpr int kDecodeSplitPagesTc = 64;
 // split_pages value that keeps every request in one chunk (no partials, no merge pass)
 constexpr int kDecodeNoSplit = 1 << 30;
 

@@ -10,8 +10,8 @@
 //   [K|V][64-column half of d][KV head][16 tokens][8 chunks of 16 B, chunk c of row r at c ^ (r & 7)]
 // and one bulk copy per half moves a page into a ring stage.
 //
-// Split along KV. A request of n pages is cut into ceil(n / chunk_pages) chunks (chunk_pages = 128,
-// so contexts above 2048 keys are split) whose page counts
+// Split along KV. A request of n pages is cut into ceil(n / chunk_pages) chunks (chunk_pages = 64,
+// so contexts above 1024 keys are split) whose page counts
 // differ by at most one (chunk c = pages [c n / nch, (c + 1) n / nch)); the cut depends only on the
 // request's context length, never on the grid. A work item is one chunk with all heads. Items are dealt to the persistent CTAs in
 // contiguous ranges of equal page counts, so a CTA's share differs from the mean by less than
@@ -74,9 +74,10 @@ struct TcCfg {
                   "barrier slots (+1 for the TMEM slot and abort flag)");
 };
 
-// warp 0 loads Q (TMA) and K halves of pages, warp 1 issues MMAs and owns TMEM, warps 2..5 softmax,
-// warp 6 loads V halves of pages (bulk copies)
-constexpr int THREADS = 224;
+// warp 0 loads K halves of pages, warp 1 issues MMAs and owns TMEM, warps 2..5 softmax, warp 6 loads V
+// halves of pages (bulk copies), warp 7 loads each item's Q (TMA) once the previous item's scores are
+// done, so that the page rings keep streaming across item boundaries
+constexpr int THREADS = 256;
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
@@ -235,10 +236,30 @@ __global__ void __launch_bounds__(THREADS, 1)
     const long long lo = W0 + W * blockIdx.x / gridDim.x;
     const long long hi = W0 + W * (blockIdx.x + 1) / gridDim.x;
 
-    if (warp == 0 || warp == 6) {
-        // ---------------- loader warps: warp 0 streams Q of each request (TMA, two 64-column
-        // halves of NQ rows) and the K half of each page, warp 6 the V half; one 32 KB bulk copy
-        // per half page. Page ids are read 32 at a time (one per lane) and handed to lane 0.
+    if (warp == 7) {
+        // ---------------- Q loader: two 64-column halves of the item's NQ query rows (TMA)
+        ItemIter it;
+        item_init(it, a, lo, hi);
+        uint32_t ni = 0;
+        for (; it.valid; item_next(it, a, hi), ++ni) {
+            if (!wait_bcast(q_empty, (ni & 1u) ^ 1u, abort_flag, a.status, lane)) break;
+            if (lane == 0) {
+                uint8_t* qd = smem + C::OFF_Q;
+                mbar_arrive_expect_tx(q_full, C::QB);
+                tma_load_2d(qd, &tmQ, q_full, 0, it.r * NQ);
+                tma_load_2d(qd + NQ * 128, &tmQ, q_full, 64, it.r * NQ);
+            }
+            __syncwarp();
+        }
+        if (lane == 0 && ni > 0) {  // the last Q load lands before the CTA exits
+            volatile int quiet = 0;
+            mbar_wait(q_full, (ni - 1) & 1u, &quiet, nullptr);
+        }
+        __syncwarp();
+    } else if (warp == 0 || warp == 6) {
+        // ---------------- page loaders: warp 0 streams the K half of each page, warp 6 the V half;
+        // one 32 KB bulk copy per half page. Page ids are read 32 at a time (one per lane) and
+        // handed to lane 0.
         const bool is_k = warp == 0;
         const int nstage = is_k ? NSK : NSV;
         uint64_t* full = is_k ? k_full : v_full;
@@ -253,15 +274,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (; it.valid && ok; item_next(it, a, hi), ++ni) {
             const int base = a.page_indptr[it.r];
             const int rowlen = a.page_indptr[it.r + 1] - base;
-            if (is_k) {
-                if (!wait_bcast(q_empty, (ni & 1u) ^ 1u, abort_flag, a.status, lane)) { ok = false; break; }
-                if (lane == 0) {
-                    uint8_t* qd = smem + C::OFF_Q;
-                    mbar_arrive_expect_tx(q_full, C::QB);
-                    tma_load_2d(qd, &tmQ, q_full, 0, it.r * NQ);
-                    tma_load_2d(qd + NQ * 128, &tmQ, q_full, 64, it.r * NQ);
-                }
-            }
             int ids = 0;
             for (int j = it.pg0; j < it.pg1; ++j, ++cs) {
                 if (((j - it.pg0) & 31) == 0) {
@@ -298,7 +310,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             volatile int quiet = 0;
             for (uint32_t x = cs > (uint32_t)nstage ? cs - nstage : 0u; x < cs; ++x)
                 mbar_wait(&full[x % nstage], (x / nstage) & 1u, &quiet, nullptr);
-            if (is_k && ni > 0) mbar_wait(q_full, (ni - 1) & 1u, &quiet, nullptr);
         }
         __syncwarp();
     } else if (warp == 1) {

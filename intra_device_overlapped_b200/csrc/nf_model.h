@@ -11,7 +11,7 @@
 namespace nf {
 
 constexpr int kDecodeSplitPagesHost = 32;     // must equal kDecodeSplitPages (nf_attention.h)
-constexpr int kDecodeSplitPagesTcHost = 128;  // must equal kDecodeSplitPagesTc (nf_attention.h)
+constexpr int kDecodeSplitPagesTcHost = 64;  // must equal kDecodeSplitPagesTc (nf_attention.h)
 
 // Decode attention work items of a batch (sizes the split-KV partials): chunks of at most
 // kDecodeSplitPagesHost pages, one per request chunk for the tensor-core kernel, one per KV head

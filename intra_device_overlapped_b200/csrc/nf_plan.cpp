@@ -216,6 +216,7 @@ CostModel default_cost_model(int sms) {
     c.attn_flops_per_sm = 2.0e12;
     c.interference = 0.08;
     c.calibrated = 0;
+    c.iter_scale = 1.0;
     return c;
 }
 
@@ -295,7 +296,8 @@ double simulate_plan(const nf_plan& p, const ModelDims& m, const BatchInfo& b, c
         if (o.elastic) dur_gemm_share[i] = op_time_us(o.kind, o.nano, p, m, b, c, p.sm_gemm);
         serial += op_time_us(o.kind, o.nano, p, m, b, c, S);
     }
-    if (serial_us) *serial_us = serial;
+    const double scale = c.iter_scale > 0 ? c.iter_scale : 1.0;
+    if (serial_us) *serial_us = serial * scale;
     double makespan = 0.0;
     for (int pass = 0; pass < 2; ++pass) {
         double free_t[2] = {0.0, 0.0};
@@ -336,7 +338,7 @@ double simulate_plan(const nf_plan& p, const ModelDims& m, const BatchInfo& b, c
             break;
         }
     }
-    return makespan;
+    return makespan * scale;
 }
 
 }  // namespace nf

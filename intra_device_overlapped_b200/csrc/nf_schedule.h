@@ -47,6 +47,7 @@ struct CostModel {
     double attn_bw_at[5];       // decode bytes/s on 1/8, 1/4, 1/2, 3/4, 1 of the SMs (0 = not measured)
     double interf_attn[3];      // decode slow-down beside GEMMs, attention on 1/4, 1/2, 3/4 of the SMs
     double interf_gemm[3];      // GEMM slow-down beside decode attention, same shares
+    double iter_scale;          // measured / predicted sequential iteration (sustained clock), 1 = none
 };
 
 // Decode attention bytes/s on `grid` of `sms` SMs (measured table, else the per-SM / HBM model) and

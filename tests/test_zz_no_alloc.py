@@ -6,7 +6,7 @@ belongs to their own pool), so they cannot create a model. This entry point runs
 tensor-core decode attention from plain device pointers, with its scratch in a static device array.
 
 Checked here: two calls in a row (the scratch is reused, not cleared, between them) each give the
-bits of the model-based entry point nf_op_decode_attention (every request here has at most 2048 keys,
+bits of the model-based entry point nf_op_decode_attention (every request here has at most 1024 keys,
 which neither entry point splits) and match the oracle within the parity bar; a request whose page
 row is too short, or whose context length is negative, is reported through the status word with a
 finite output; the size limit, a missing status word and unsupported shapes are rejected. This file
