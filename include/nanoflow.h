@@ -242,9 +242,10 @@ typedef struct {
  * anything runs. Asynchronous. */
 nf_status nf_forward_iteration(nf_model* m, const nf_plan* plan, const nf_iter_io* io, void* stream);
 
-/* Plan choice by measurement. For each template and nano-batch count the planner's best
- * plan (the SM split chosen by the cost model) is run on this batch: one warm-up and `reps`
- * timed iterations (CUDA events on `stream`). The four fastest are then timed again in turn over
+/* Plan choice by measurement. After about 0.3 s of sequential iterations (the clock a power-capped
+ * GPU holds under load is lower than its first burst), for each template and nano-batch count the
+ * planner's best plan (the SM split chosen by the cost model) is run on this batch: one warm-up and
+ * `reps` timed iterations (CUDA events on `stream`). The four fastest are then timed again in turn over
  * five rounds (so that clock drift under the power cap does not decide), and the one with the
  * lowest median is written to `out` and that median, in microseconds, to `best_us` (nullable). This is the search over
  * measured costs that the arXiv abstract describes, with the final choice between templates

@@ -778,6 +778,30 @@ extern "C" nf_status nf_tune_plan(nf_model* m, const nf_batch_desc* b, const nf_
         *us = 1000.f * ms / (float)reps;
         return NF_OK;
     };
+    // A GPU under its power cap runs faster for the first fraction of a second of load: bring it to the
+    // clock it holds in steady state before anything is timed (about 0.3 s of sequential iterations).
+    {
+        nf_plan_opts o;
+        std::memset(&o, 0, sizeof(o));
+        o.force_nano = 1;
+        o.force_template = NF_TEMPLATE_SEQUENTIAL;
+        nf_plan p;
+        float us = 0.f;
+        nf_status st0 = nf_plan_iteration(m, b, &o, &p);
+        if (st0 == NF_OK) st0 = time_plan(p, &us);
+        if (st0 != NF_OK) {
+            cudaEventDestroy(e0);
+            cudaEventDestroy(e1);
+            return st0;
+        }
+        const int n_warm = us > 0.f ? std::min(20000, (int)(300000.f / us)) : 0;
+        for (int i = 0; i < n_warm && st0 == NF_OK; ++i) st0 = nf_forward_iteration(m, &p, io, stream);
+        if (st0 != NF_OK) {
+            cudaEventDestroy(e0);
+            cudaEventDestroy(e1);
+            return st0;
+        }
+    }
     std::vector<std::pair<float, nf_plan>> cands;
     auto try_plan = [&](const nf_plan& p) -> nf_status {
         float us = 0.f;

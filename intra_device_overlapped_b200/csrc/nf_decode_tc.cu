@@ -2,13 +2,14 @@
 //
 // Decode attention is the memory-bound operation NanoFlow overlaps with the GEMMs of
 // another nano-batch (README "Introduction"; arXiv abstract). For the overlap to pay, the
-// attention kernel must pull HBM bandwidth from a minority of the SMs, and on B200 one SM's
-// DRAM throughput grows with the size of each transfer (about 45 GB/s per SM with 2 KB
-// transfers, about 190 GB/s with 64 KB ones). The paged KV cache is therefore laid out so
-// that one page of one layer -- K and V of all KV heads, 64 KB -- is a single contiguous
-// block whose bytes are already the shared-memory image the tensor cores read:
+// attention kernel must pull HBM bandwidth from a minority of the SMs. On B200 an SM completes
+// bulk copies at a nearly fixed number per second whatever their size (measured on 16 SMs with a
+// ring of copies in flight: 23 GB/s per SM with 8 KB copies, 91 GB/s with 32 KB, 175 GB/s with
+// 64 KB). The paged KV cache is therefore laid out so that one page of one layer -- K and V of all
+// KV heads, 64 KB -- is a single contiguous block whose bytes are already the shared-memory image
+// the tensor cores read:
 //   [K|V][64-column half of d][KV head][16 tokens][8 chunks of 16 B, chunk c of row r at c ^ (r & 7)]
-// and one bulk copy per half moves a page into a ring stage.
+// and one bulk copy moves a page into a stage of the page ring.
 //
 // Split along KV. A request of n pages is cut into ceil(n / chunk_pages) chunks (chunk_pages = 64,
 // so contexts above 1024 keys are split) whose page counts
@@ -44,19 +45,19 @@ constexpr uint32_t PAGE_BYTES = 65536;      // K and V of all heads of one page
 constexpr uint32_t HALF_PAGE = 32768;       // K (or V) of all heads of one page
 constexpr uint32_t REGION = 16384;          // one 64-column half of K or V: 128 rows x 128 B
 constexpr float LAZY = 8.0f;
+constexpr int kPrefetchPages = 4;           // L2 prefetch distance of the page loader
 
 template <int NQ>
 struct TcCfg {
-    static constexpr int NSK = 3;                         // K stages (released after Q K^T)
-    static constexpr int NSV = NQ <= 32 ? 3 : 2;          // V stages (released after P V)
+    static constexpr int NSP = 3;                         // page stages (K and V, released after P V)
     static constexpr int NSB = 3;                         // S^T buffers in TMEM
-    static constexpr int LOOK = NSB - 1;                  // S is issued this many pages ahead of P V
-    static constexpr int NPB = 3;                         // P buffers: the softmax of page c reuses the
-                                                          // buffer of page c - 3, whose P V precedes S(c)
+    static constexpr int LOOK = 2;                        // S may run this many pages ahead of P V
+    // P buffers: the softmax of page c writes buffer c % NPB once the P V of page c - NPB is done (one
+    // buffer with 64 query heads, where three would not fit beside three page stages)
+    static constexpr int NPB = NQ <= 32 ? 3 : 1;
     static constexpr uint32_t QB = NQ * 256;              // Q: two halves of NQ rows x 128 B
     static constexpr uint32_t PB = NQ * 256;              // P buffer: two key halves of NQ rows x 128 B
-    static constexpr uint32_t OFF_V = NSK * HALF_PAGE;
-    static constexpr uint32_t OFF_Q = OFF_V + NSV * HALF_PAGE;
+    static constexpr uint32_t OFF_Q = NSP * PAGE_BYTES;
     static constexpr uint32_t OFF_P = OFF_Q + QB;
     static constexpr uint32_t OFF_CF = OFF_P + NPB * PB;  // float[NQ] rescale factors / row sums
     static constexpr uint32_t OFF_BAR = OFF_CF + NQ * 4;
@@ -66,18 +67,18 @@ struct TcCfg {
     static constexpr uint32_t IDESC_S = umma_idesc_bf16_f32(128, NQ);
     static constexpr uint32_t IDESC_PV = umma_idesc_bf16_f32_amn(128, NQ);
     static_assert(SMEM <= 232448, "shared memory");
-    // a K stage is free once the S^T of its page completes (s_full), a V stage once its P V
-    // completes (pv_done): the loaders wait on those barriers directly
-    static_assert(NSK == NSB && NSV <= NPB, "stage / buffer counts");
+    // S(c + LOOK) reads a page that must be in the ring while P V(c) is pending, into an S^T buffer
+    // the softmax of page c + LOOK - NSB has released
+    static_assert(LOOK >= 1 && LOOK < NSP && LOOK < NSB, "stage / buffer counts");
     static_assert((NSB + 1) * NQ <= 256, "tensor memory");
-    static_assert(NSK + NSV + 2 + 2 * NSB + 2 * NPB + 2 + 1 <= 32,
+    static_assert(2 * NSP + 2 + 2 * NSB + 2 * NPB + 2 + 1 <= 32,
                   "barrier slots (+1 for the TMEM slot and abort flag)");
 };
 
-// warp 0 loads K halves of pages, warp 1 issues MMAs and owns TMEM, warps 2..5 softmax, warp 6 loads V
-// halves of pages (bulk copies), warp 7 loads each item's Q (TMA) once the previous item's scores are
-// done, so that the page rings keep streaming across item boundaries
-constexpr int THREADS = 256;
+// warp 0 loads whole pages (one bulk copy each), warp 1 issues MMAs and owns TMEM, warps 2..5 softmax,
+// warp 6 loads each item's Q (TMA) once the previous item's scores are done, so that the page ring
+// keeps streaming across item boundaries
+constexpr int THREADS = 224;
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
@@ -162,9 +163,11 @@ __device__ __forceinline__ void cursor_next(PageCursor& x, const DecodeArgs& a, 
 }
 
 // Non-blocking: has the phase of `bar` with this parity completed? (uniform across the warp)
+// (test_wait returns at once; try_wait may hold the thread for a while before it reports an
+// incomplete phase, which would keep the issuer from work that is ready elsewhere)
 __device__ __forceinline__ bool test_bcast(uint64_t* bar, uint32_t parity, int lane) {
     int ok = 0;
-    if (lane == 0) ok = mbar_try_wait(smem_u32(bar), parity) ? 1 : 0;
+    if (lane == 0) ok = mbar_test_wait(smem_u32(bar), parity) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -182,15 +185,15 @@ template <int NQ>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ DecodeArgs a) {
     using C = TcCfg<NQ>;
-    constexpr int NSK = C::NSK, NSV = C::NSV, NSB = C::NSB, NPB = C::NPB;
+    constexpr int NSP = C::NSP, NSB = C::NSB, NPB = C::NPB;
     constexpr int G = NQ / 8;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* cfs = reinterpret_cast<float*>(smem + C::OFF_CF);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    uint64_t* k_full = bars;                   // [NSK]
-    uint64_t* v_full = k_full + NSK;           // [NSV]
-    uint64_t* q_full = v_full + NSV;           // [1]
+    uint64_t* page_full = bars;                // [NSP] the page's bulk copy has landed
+    uint64_t* stage_free = page_full + NSP;    // [NSP] the P V of the stage's page has completed
+    uint64_t* q_full = stage_free + NSP;       // [1]
     uint64_t* q_empty = q_full + 1;            // [1]
     uint64_t* s_full = q_empty + 1;            // [NSB]
     uint64_t* s_free = s_full + NSB;           // [NSB]
@@ -208,8 +211,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         reinterpret_cast<uint4*>(smem + C::OFF_P)[i] = make_uint4(0u, 0u, 0u, 0u);
     if (threadIdx.x == 0) {
         t_start = globaltimer_ns();
-        for (int i = 0; i < NSK; ++i) mbar_init(&k_full[i], 1);
-        for (int i = 0; i < NSV; ++i) mbar_init(&v_full[i], 1);
+        for (int i = 0; i < NSP; ++i) { mbar_init(&page_full[i], 1); mbar_init(&stage_free[i], 1); }
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
         for (int i = 0; i < NPB; ++i) { mbar_init(&p_full[i], 4); mbar_init(&pv_done[i], 1); }
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const long long lo = W0 + W * blockIdx.x / gridDim.x;
     const long long hi = W0 + W * (blockIdx.x + 1) / gridDim.x;
 
-    if (warp == 7) {
+    if (warp == 6) {
         // ---------------- Q loader: two 64-column halves of the item's NQ query rows (TMA)
         ItemIter it;
         item_init(it, a, lo, hi);
@@ -256,83 +258,102 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_wait(q_full, (ni - 1) & 1u, &quiet, nullptr);
         }
         __syncwarp();
-    } else if (warp == 0 || warp == 6) {
-        // ---------------- page loaders: warp 0 streams the K half of each page, warp 6 the V half;
-        // one 32 KB bulk copy per half page. Page ids are read 32 at a time (one per lane) and
-        // handed to lane 0.
-        const bool is_k = warp == 0;
-        const int nstage = is_k ? NSK : NSV;
-        uint64_t* full = is_k ? k_full : v_full;
-        uint8_t* ring = smem + (is_k ? 0u : C::OFF_V);
+    } else if (warp == 0) {
+        // ---------------- page loader: one 64 KB bulk copy per page (K and V of all heads) into the
+        // page ring. An SM completes bulk copies at a rate that hardly depends on their size, so whole
+        // pages stream about twice as fast as separate K and V halves. Page ids are read 32 at a time
+        // (one per lane) and handed to lane 0.
+        uint64_t* full = page_full;
+        uint8_t* ring = smem;
         ItemIter it;
         item_init(it, a, lo, hi);
         uint32_t cs = 0, ni = 0;
         bool ok = true;
-        const char* pool = reinterpret_cast<const char*>(a.kv_pool) + (is_k ? 0 : HALF_PAGE);
+        const char* pool = reinterpret_cast<const char*>(a.kv_pool);
         // each page is read once per launch: stream it through L2 without displacing reused data
         const uint64_t stream_policy = l2_policy_evict_first();
+        // page ids of the current window of 32 pages (one per lane) and of the next one
+        auto load_id = [&](int jj, int base, int rowlen, int pg1) -> int {
+            // an index past the request's row of the page table, or a page outside the pool, is
+            // recorded and page 0 read in its place
+            int id = 0;
+            if (jj < pg1) {
+                if (jj < rowlen) id = __ldg(a.page_indices + base + jj);
+                if (jj >= rowlen || id < 0 || id >= a.num_pages) {
+                    set_status(a.status, NF_ERR_DEVICE_BOUNDS);
+                    id = 0;
+                }
+            }
+            return id;
+        };
         for (; it.valid && ok; item_next(it, a, hi), ++ni) {
             const int base = a.page_indptr[it.r];
             const int rowlen = a.page_indptr[it.r + 1] - base;
-            int ids = 0;
+            int ids = 0, ids_next = 0, w0 = it.pg0;
+            // id of page jj of the request, jj in [w0, w0 + 64) (warp-uniform jj)
+            auto id_of = [&](int jj) -> int {
+                const int x = __shfl_sync(0xffffffffu, ids, (jj - w0) & 31);
+                const int y = __shfl_sync(0xffffffffu, ids_next, (jj - w0) & 31);
+                return jj - w0 < 32 ? x : y;
+            };
             for (int j = it.pg0; j < it.pg1; ++j, ++cs) {
                 if (((j - it.pg0) & 31) == 0) {
-                    // one page id per lane; an index past the request's row of the page table, or a
-                    // page outside the pool, is recorded and page 0 read in its place
-                    const int jj = j + lane;
-                    ids = 0;
-                    if (jj < it.pg1) {
-                        if (jj < rowlen) ids = __ldg(a.page_indices + base + jj);
-                        if (jj >= rowlen || ids < 0 || ids >= a.num_pages) {
-                            set_status(a.status, NF_ERR_DEVICE_BOUNDS);
-                            ids = 0;
+                    w0 = j;
+                    ids = load_id(j + lane, base, rowlen, it.pg1);
+                    ids_next = load_id(j + 32 + lane, base, rowlen, it.pg1);
+                    if (j == it.pg0) {
+                        // the item's first pages, which no earlier copy prefetched
+                        for (int k = 1; k < kPrefetchPages && j + k < it.pg1; ++k) {
+                            const int pid = id_of(j + k);
+                            if (lane == 0) prefetch_l2_bulk(pool + (size_t)pid * PAGE_BYTES, PAGE_BYTES);
                         }
                     }
                 }
-                const int pg = __shfl_sync(0xffffffffu, ids, (j - it.pg0) & 31);
-                const int st = (int)(cs % nstage);
-                // the stage's previous page (cs - nstage) must be consumed: its S^T (K) or P V (V)
-                if (cs >= (uint32_t)nstage) {
-                    const uint32_t prev = cs - nstage;
-                    uint64_t* done = is_k ? &s_full[prev % NSB] : &pv_done[prev % NPB];
-                    const uint32_t par = is_k ? (prev / NSB) & 1u : (prev / NPB) & 1u;
-                    if (!wait_bcast(done, par, abort_flag, a.status, lane)) { ok = false; break; }
+                const int pg = id_of(j);
+                const int pf = j + kPrefetchPages < it.pg1 ? id_of(j + kPrefetchPages) : -1;
+                const int st = (int)(cs % NSP);
+                // the stage's previous page (cs - NSP) must be consumed: its P V has completed (and with
+                // it the S^T issued before it)
+                if (cs >= (uint32_t)NSP &&
+                    !wait_bcast(&stage_free[st], ((cs / NSP) - 1u) & 1u, abort_flag, a.status, lane)) {
+                    ok = false;
+                    break;
                 }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[st], HALF_PAGE);
-                    bulk_load_hint(ring + st * HALF_PAGE, pool + (size_t)pg * PAGE_BYTES, HALF_PAGE, &full[st],
+                    mbar_arrive_expect_tx(&full[st], PAGE_BYTES);
+                    bulk_load_hint(ring + st * PAGE_BYTES, pool + (size_t)pg * PAGE_BYTES, PAGE_BYTES, &full[st],
                                    stream_policy);
+                    // a stage is held from its copy to the P V of its page, about three times the copy's
+                    // own latency: a page bound for the ring kPrefetchPages pages later is fetched into L2
+                    // now, so that its copy finds it there
+                    if (pf >= 0) prefetch_l2_bulk(pool + (size_t)pf * PAGE_BYTES, PAGE_BYTES);
                 }
             }
         }
         if (lane == 0) {
             // let the copies still in flight land before the CTA exits
             volatile int quiet = 0;
-            for (uint32_t x = cs > (uint32_t)nstage ? cs - nstage : 0u; x < cs; ++x)
-                mbar_wait(&full[x % nstage], (x / nstage) & 1u, &quiet, nullptr);
+            for (uint32_t x = cs > (uint32_t)NSP ? cs - NSP : 0u; x < cs; ++x)
+                mbar_wait(&full[x % NSP], (x / NSP) & 1u, &quiet, nullptr);
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer. The whole warp follows the page cursors and one elected lane
-        // issues; descriptors are built once and offset by constants, so the issue loop holds little
-        // besides the MMAs (16 per page, whose issue rate bounds this kernel). The scores S^T of page
-        // cs + LOOK are issued before P V of page cs, so the tensor core has work while the softmax
-        // warps handle page cs.
+        // ---------------- MMA issuer. The whole warp follows two page cursors (the next S^T and the next
+        // P V) and one elected lane issues; descriptors are built once and offset by constants. Issue is
+        // driven by readiness rather than a fixed order: P V of page pc as soon as its probabilities are
+        // in (its commit frees the page's stage for the next load), else S^T of page sc (up to LOOK pages
+        // ahead) as soon as its page has landed, so that no MMA waits behind a load it does not need.
         PageCursor sc, pc;
         cursor_init(sc, a, lo, hi);
         cursor_init(pc, a, lo, hi);
-        bool ok = true;
         const uint64_t kd0 = umma_desc_sw128(sbase);
         const uint64_t qd0 = umma_desc_sw128(sbase + C::OFF_Q);
-        const uint64_t vd0 = umma_desc_sw128_mn(sbase + C::OFF_V, REGION, 1024);
+        const uint64_t vd0 = umma_desc_sw128_mn(sbase + HALF_PAGE, REGION, 1024);
         const uint64_t pd0 = umma_desc_sw128(sbase + C::OFF_P);
-        auto issue_s = [&](const PageCursor& x) -> bool {
-            const uint32_t st = x.cs % NSK, sb = x.cs % NSB;
-            if (x.j == x.it.pg0 && !wait_bcast(q_full, x.ni & 1u, abort_flag, a.status, lane)) return false;
-            if (!wait_bcast(&k_full[st], (x.cs / NSK) & 1u, abort_flag, a.status, lane)) return false;
-            if (!wait_bcast(&s_free[sb], ((x.cs / NSB) & 1u) ^ 1u, abort_flag, a.status, lane)) return false;
+        auto issue_s = [&](const PageCursor& x) {
+            const uint32_t st = x.cs % NSP, sb = x.cs % NSB;
             tc_fence_after();
-            const uint64_t ad = kd0 + ((st * HALF_PAGE) >> 4);
+            const uint64_t ad = kd0 + ((st * PAGE_BYTES) >> 4);
             const uint64_t bd = qd0;
             const uint32_t d = tmem + sb * NQ;
             if (elect_one()) {
@@ -344,16 +365,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 umma_commit(&s_full[sb]);
                 if (x.j == x.it.pg1 - 1) umma_commit(q_empty);
             }
-            return true;
+            __syncwarp();
         };
-        auto issue_pv = [&](const PageCursor& x) -> bool {
-            const uint32_t pb = x.cs % NPB, sv = x.cs % NSV;
+        auto issue_pv = [&](const PageCursor& x) {
+            const uint32_t pb = x.cs % NPB, sv = x.cs % NSP;
             const bool first = x.j == x.it.pg0;
-            if (!wait_bcast(&p_full[pb], (x.cs / NPB) & 1u, abort_flag, a.status, lane)) return false;
-            if (!wait_bcast(&v_full[sv], (x.cs / NSV) & 1u, abort_flag, a.status, lane)) return false;
-            if (first && !wait_bcast(o_free, (x.ni & 1u) ^ 1u, abort_flag, a.status, lane)) return false;
             tc_fence_after();
-            const uint64_t ad = vd0 + ((sv * HALF_PAGE) >> 4);
+            const uint64_t ad = vd0 + ((sv * PAGE_BYTES) >> 4);
             const uint64_t bd = pd0 + ((pb * C::PB) >> 4);
             const uint32_t d = tmem + C::O_COL;
             if (elect_one()) {
@@ -364,19 +382,58 @@ __global__ void __launch_bounds__(THREADS, 1)
                     umma_bf16_c<true>(d, ad + (uint64_t)((kk * 2048) >> 4),
                                       bd + (uint64_t)(((kk >> 2) * (NQ * 128) + (kk & 3) * 32) >> 4), C::IDESC_PV);
                 umma_commit(&pv_done[pb]);
+                umma_commit(&stage_free[sv]);
             }
-            return true;
+            __syncwarp();
         };
-        while (ok && pc.valid) {
-            while (ok && sc.valid && sc.cs <= pc.cs + (uint32_t)C::LOOK) {
-                // the first page of a later request waits for its Q only when P V has nothing to do
-                if (sc.j == sc.it.pg0 && sc.cs > pc.cs && !test_bcast(q_full, sc.ni & 1u, lane)) break;
-                ok = issue_s(sc);
-                cursor_next(sc, a, hi);
+        uint32_t idle = 0;      // polls since the last issue
+        uint64_t idle_t0 = 0;   // time of the 64th of them
+        while (pc.valid) {
+            bool issued = false;
+            // P V of page pc: its S^T was issued (the softmax waits for it), its probabilities are in, and
+            // on an item's first page the previous item's output has been read out of TMEM
+            if (sc.cs > pc.cs) {
+                const bool first = pc.j == pc.it.pg0;
+                if (test_bcast(&p_full[pc.cs % NPB], (pc.cs / NPB) & 1u, lane) &&
+                    (!first || test_bcast(o_free, (pc.ni & 1u) ^ 1u, lane))) {
+                    issue_pv(pc);
+                    cursor_next(pc, a, hi);
+                    issued = true;
+                }
             }
-            if (!ok) break;
-            ok = issue_pv(pc);
-            cursor_next(pc, a, hi);
+            // S^T of page sc: its Q (first page of an item), its page and a free S^T buffer
+            if (!issued && sc.valid && sc.cs <= pc.cs + (uint32_t)C::LOOK) {
+                const bool first = sc.j == sc.it.pg0;
+                if ((!first || test_bcast(q_full, sc.ni & 1u, lane)) &&
+                    test_bcast(&page_full[sc.cs % NSP], (sc.cs / NSP) & 1u, lane) &&
+                    test_bcast(&s_free[sc.cs % NSB], ((sc.cs / NSB) & 1u) ^ 1u, lane)) {
+                    issue_s(sc);
+                    cursor_next(sc, a, hi);
+                    issued = true;
+                }
+            }
+            if (issued) {
+                idle = 0;
+                continue;
+            }
+            // nothing ready: poll again, within the same time limit as every other wait (lane 0 decides
+            // for the warp)
+            if ((++idle & 63u) == 0) {
+                int stop = 0;
+                if (lane == 0) {
+                    const uint64_t now = globaltimer_ns();
+                    if (*abort_flag) {
+                        stop = 1;
+                    } else if (idle == 64) {
+                        idle_t0 = now;
+                    } else if (now - idle_t0 > NF_WAIT_LIMIT_NS) {
+                        *abort_flag = 1;
+                        set_status(a.status, NF_ERR_DEVICE_TIMEOUT);
+                        stop = 1;
+                    }
+                }
+                if (__shfl_sync(0xffffffffu, stop, 0)) break;
+            }
         }
         if (elect_one()) umma_commit(drain);
         __syncwarp();
@@ -484,17 +541,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                             __float2bfloat16_rn(p);
                     }
                     if ((it.nkeys & 15) != 0 && c == it.npages - 1) {  // CTA-uniform
-                        // V rows of keys past the request in the last page: zero them (once the
-                        // V half has landed) so that 0 * garbage cannot occur in P V. The stage's
-                        // previous page (cs - NSV) must have been consumed first: with fewer V stages
-                        // than P buffers nothing else orders it, and until then the parity test
-                        // below could see that page's load as this one's.
-                        if (cs >= (uint32_t)NSV)
-                            okc = okc && wait_bcast(&pv_done[(cs - NSV) % NPB], ((cs - NSV) / NPB) & 1u, abort_flag,
-                                                    a.status, lane);
-                        okc = okc && wait_bcast(&v_full[cs % NSV], (cs / NSV) & 1u, abort_flag, a.status, lane);
+                        // V rows of keys past the request in the last page: zero them so that
+                        // 0 * garbage cannot occur in P V. One copy brings K and V of the page, and
+                        // its S^T (which waited for that copy) has completed, so V has landed; the
+                        // stage is refilled only after this page's P V.
                         if (okc && c * 16 + k >= it.nkeys) {
-                            uint8_t* vrow = smem + C::OFF_V + (cs % NSV) * HALF_PAGE + t * 128;
+                            uint8_t* vrow = smem + (cs % NSP) * PAGE_BYTES + HALF_PAGE + t * 128;
 #pragma unroll
                             for (int b = 0; b < 2; ++b)
 #pragma unroll

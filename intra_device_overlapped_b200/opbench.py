@@ -42,6 +42,7 @@ def main(argv=None) -> dict:
     ap.add_argument("--template", type=int, default=0)
     ap.add_argument("--sm-attn", type=int, default=0)
     ap.add_argument("--workload", default="llama3_8b_layer")
+    ap.add_argument("--layers", type=int, default=0, help="build only this many layers of the workload (0: all)")
     ap.add_argument("--requests", type=int, default=0, help="decode requests (0 = all)")
     ap.add_argument("--sm", type=int, default=0)
     ap.add_argument("--reps", type=int, default=5)
@@ -68,6 +69,9 @@ def main(argv=None) -> dict:
         from synth.workloads import WORKLOADS
         from .harness import DeviceWorkload
         w = WORKLOADS[args.workload]
+        if args.layers > 0:
+            from dataclasses import replace
+            w = replace(w, shape=replace(w.shape, n_layers=min(args.layers, w.shape.n_layers)))
         dw = DeviceWorkload(w, dev, keep_logits=False)
         s, bt = w.shape, dw.batch
         q = torch.zeros((dw.T, s.n_q_heads, s.head_dim), dtype=torch.bfloat16, device=dev)
