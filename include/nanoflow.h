@@ -258,10 +258,12 @@ nf_status nf_tune_plan(nf_model* m, const nf_batch_desc* b, const nf_iter_io* io
 /* Wait for the model's streams and return (and clear) the latched device status. */
 nf_status nf_sync_status(nf_model* m);
 
-/* Time the model's own kernels at the sizes of `b` on several SM shares, and one
- * GEMM + decode-attention co-run, and store the fitted rates as the planner's cost
- * model (synchronous; a few tens of milliseconds). Reads the KV pools of `io`;
- * writes only the model's workspace. */
+/* Time the model's own kernels at the sizes of `b` on several SM shares and GEMM + decode-attention
+ * co-runs at three shares, then two whole plans in steady state (the sequential one for
+ * iter_scale, one overlapped plan for power_floor), and store the fitted rates as the planner's
+ * cost model (synchronous; about half a second, longer for deep models). Reads the KV pools of
+ * `io`; the whole-plan timings run nf_forward_iteration with `io` (the new tokens' K/V slots are
+ * rewritten with the same values, the outputs overwritten). */
 nf_status nf_calibrate(nf_model* m, const nf_batch_desc* b, const nf_iter_io* io, void* stream);
 
 /* The planner's per-kernel cost model (defaults until nf_calibrate has run). */
@@ -288,6 +290,12 @@ typedef struct {
      * that runs for tens of milliseconds settles at the lower clock of the power cap, and this factor
      * carries that into every prediction. */
     double iter_scale;
+    /* Power floor (0 = none): a plan's predicted time is at least power_floor x its serial time (the
+     * sum of its kernels' times on all SMs, scaled like every prediction). Under a power cap the GPU
+     * trades the idle SM time that overlap removes for a lower clock, so an overlapped plan cannot
+     * run much faster than its kernels' energy allows. nf_calibrate sets it from one overlapped plan
+     * timed in steady state (its measured time over its serial time). */
+    double power_floor;
 } nf_cost_model;
 
 nf_status nf_get_cost_model(const nf_model* m, nf_cost_model* out);

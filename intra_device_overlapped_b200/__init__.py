@@ -118,7 +118,8 @@ class nf_cost_model(ctypes.Structure):
                 ("attn_bw_per_sm", ctypes.c_double), ("attn_launch_us", ctypes.c_double),
                 ("attn_flops_per_sm", ctypes.c_double), ("interference", ctypes.c_double), ("calibrated", _i32),
                 ("attn_bw_at", ctypes.c_double * 5), ("interf_attn", ctypes.c_double * 3),
-                ("interf_gemm", ctypes.c_double * 3), ("iter_scale", ctypes.c_double)]
+                ("interf_gemm", ctypes.c_double * 3), ("iter_scale", ctypes.c_double),
+                ("power_floor", ctypes.c_double)]
 
     def as_dict(self) -> dict:
         out = {}

@@ -217,6 +217,7 @@ CostModel default_cost_model(int sms) {
     c.interference = 0.08;
     c.calibrated = 0;
     c.iter_scale = 1.0;
+    c.power_floor = 0.0;
     return c;
 }
 
@@ -338,6 +339,8 @@ double simulate_plan(const nf_plan& p, const ModelDims& m, const BatchInfo& b, c
             break;
         }
     }
+    // energy bound: under a power cap the plan runs no faster than its kernels' energy allows
+    if (c.power_floor > 0) makespan = std::max(makespan, c.power_floor * serial);
     return makespan * scale;
 }
 

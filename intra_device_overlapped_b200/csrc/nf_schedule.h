@@ -48,6 +48,7 @@ struct CostModel {
     double interf_attn[3];      // decode slow-down beside GEMMs, attention on 1/4, 1/2, 3/4 of the SMs
     double interf_gemm[3];      // GEMM slow-down beside decode attention, same shares
     double iter_scale;          // measured / predicted sequential iteration (sustained clock), 1 = none
+    double power_floor;         // predicted time >= power_floor x serial time (0 = none)
 };
 
 // Decode attention bytes/s on `grid` of `sms` SMs (measured table, else the per-SM / HBM model) and
