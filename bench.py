@@ -398,21 +398,31 @@ def run_ours(args, work, dist):
     extras = {}
     if not args.no_extras:
         # ---- the same work without overlap: sequential plan, one nano-batch, every SM
+        # timed exactly like the headline: the same warm-up (at least W steps and --min-warmup-s seconds of
+        # this plan, so that the power-capped clock has settled on it), then K steps without per-op events
         seq_plan = dw.plan(nano=1, template=0)
-        for _ in range(3):
-            dw.forward(seq_plan, stream)
-        nf.check(nf.nf_set_timing(dw.model, True), "timing")
-        torch.cuda.synchronize(dev)
+        t_warm = time.perf_counter()
+        nw = 0
+        while nw < max(args.warmup, 3) or time.perf_counter() - t_warm < args.min_warmup_s:
+            for _ in range(8):
+                dw.forward(seq_plan, stream)
+            nw += 8
+            torch.cuda.synchronize(dev)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record(stream)
-        nseq = max(3, args.steps // 2)
-        for _ in range(nseq):
+        for _ in range(args.steps):
             dw.forward(seq_plan, stream)
         s1.record(stream)
         torch.cuda.synchronize(dev)
+        seq_ms = s0.elapsed_time(s1) / args.steps
+        # then the same steps again with per-op events (each op's time on all SMs)
+        nf.check(nf.nf_set_timing(dw.model, True), "timing")
+        nseq = max(3, args.steps // 2)
+        for _ in range(nseq):
+            dw.forward(seq_plan, stream)
+        torch.cuda.synchronize(dev)
         st, seq_ops = nf.nf_get_op_times(dw.model, 1 << 20)
         nf.nf_set_timing(dw.model, False)
-        seq_ms = s0.elapsed_time(s1) / nseq
         iso = {}
         for (name, nano, layer, stream_id, grid, us) in seq_ops:
             iso[name] = iso.get(name, 0.0) + us / nseq

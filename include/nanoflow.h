@@ -245,11 +245,12 @@ nf_status nf_forward_iteration(nf_model* m, const nf_plan* plan, const nf_iter_i
 /* Plan choice by measurement. After about 0.3 s of sequential iterations (the clock a power-capped
  * GPU holds under load is lower than its first burst), for each template and nano-batch count the
  * planner's best plan (the SM split chosen by the cost model) is run on this batch: one warm-up and
- * `reps` timed iterations (CUDA events on `stream`). The four fastest are then timed again in turn over
- * three rounds, each run for about 40 ms and timed over the next 60 ms (a short run inherits the
- * clock its predecessors left under the power cap), and the one with the lowest median is written
- * to `out` and that median, in microseconds, to `best_us` (nullable). The sequential plan is always
- * among the four and is kept unless another beats it by more than 1%. This is the search over
+ * `reps` timed iterations (CUDA events on `stream`). The three fastest (the sequential plan always
+ * among them) are then each run alone for about 0.8 s and timed over the next 0.2 s (a short run
+ * inherits the clock its predecessors left under the power cap, and the GPU's power control settles
+ * over a large fraction of a second); the fastest is written to `out` and its time, in
+ * microseconds, to `best_us` (nullable). The sequential plan is kept unless another beats it by
+ * more than 1%. Takes a few seconds. This is the search over
  * measured costs that the arXiv abstract describes, with the final choice between templates
  * and counts made on the device, where the interference of co-running kernels is real.
  * Runs nf_forward_iteration with `io` repeatedly: the new tokens' K/V slots are rewritten

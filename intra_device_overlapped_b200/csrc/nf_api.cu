@@ -834,9 +834,9 @@ extern "C" nf_status nf_tune_plan(nf_model* m, const nf_batch_desc* b, const nf_
     }
     // The first pass times each candidate once over a few iterations. Under a power cap that favours
     // the plans that draw the most power: a short run inherits the clock its predecessors left, and
-    // the GPU lowers it only after some milliseconds. The fastest few are therefore timed again, in
-    // turn, each over about 60 ms after about 40 ms of running the same plan, in three rounds, and the
-    // one with the lowest median wins.
+    // the GPU's power control settles over a large fraction of a second. The three fastest (the
+    // sequential plan always among them) are therefore each run alone for about 0.8 s and timed over
+    // the next 0.2 s, in their own steady state.
     nf_status result = cands.empty() ? NF_ERR_INVALID_ARGUMENT : NF_OK;
     float best = 0.f;
     if (st == NF_OK && !cands.empty()) {
@@ -844,7 +844,7 @@ extern "C" nf_status nf_tune_plan(nf_model* m, const nf_batch_desc* b, const nf_
                          [](const std::pair<float, nf_plan>& x, const std::pair<float, nf_plan>& y) {
                              return x.first < y.first;
                          });
-        constexpr int kFinalists = 4, kRounds = 3;
+        constexpr int kFinalists = 3, kRounds = 1;
         // the sequential plan is always among the finalists (moved up to the last finalist place)
         for (size_t i = kFinalists; i < cands.size(); ++i)
             if (cands[i].second.order_template == NF_TEMPLATE_SEQUENTIAL) {
@@ -857,8 +857,8 @@ extern "C" nf_status nf_tune_plan(nf_model* m, const nf_batch_desc* b, const nf_
             for (int i = 0; i < nf_ && st == NF_OK; ++i) {
                 const nf_plan& p = cands[i].second;
                 const float est = std::max(cands[i].first, 1.f);
-                const int n_warm = std::max(reps, std::min(20000, (int)(40000.f / est)));
-                const int n_time = std::max(reps, std::min(20000, (int)(60000.f / est)));
+                const int n_warm = std::max(reps, std::min(20000, (int)(800000.f / est)));
+                const int n_time = std::max(reps, std::min(5000, (int)(200000.f / est)));
                 for (int w = 0; w < n_warm && st == NF_OK; ++w) st = nf_forward_iteration(m, &p, io, stream);
                 if (st != NF_OK) break;
                 if (cudaEventRecord(e0, s) != cudaSuccess) { st = NF_ERR_CUDA; break; }
