@@ -432,12 +432,17 @@ def run_ours(args, work, dist):
                                 "sum_isolated_gemm_ms": round(sum(v for k, v in iso.items() if k not in att) / 1000, 4),
                                 "sum_isolated_attention_ms": round(sum(iso.get(k, 0.0) for k in att) / 1000, 4)}
 
-        # ---- each op alone at the plan's SM shares: the same sequential iteration restricted to the
-        # attention share (decode attention's time) and to the GEMM share (every other op's time)
+        # ---- each op alone at the SM share the plan gave it: for every op, the grid it ran on in the
+        # tuned plan (the one holding most of its time), then that op of the sequential iteration run
+        # alone on that many SMs
         if plan.order_template != nf.NF_TEMPLATE_SEQUENTIAL:
+            grid_time = {}
+            for (name, nano, layer, stream_id, grid, us) in op_times:
+                grid_time.setdefault(name, {}).setdefault(grid, 0.0)
+                grid_time[name][grid] += us
+            op_grid = {k: max(v, key=v.get) for k, v in grid_time.items()}
             share = {}
-            for sms, keep in ((plan.sm_attn, lambda k: k == "decode_attention"),
-                              (plan.sm_gemm, lambda k: k != "decode_attention")):
+            for sms in sorted(set(op_grid.values())):
                 sp = dw.plan(nano=1, template=0, sm_total=sms)
                 for _ in range(2):
                     dw.forward(sp, stream)
@@ -449,10 +454,10 @@ def run_ours(args, work, dist):
                 st, sh_ops = nf.nf_get_op_times(dw.model, 1 << 20)
                 nf.nf_set_timing(dw.model, False)
                 for (name, nano, layer, stream_id, grid, us) in sh_ops:
-                    if keep(name):
+                    if op_grid.get(name) == sms:
                         share[name] = share.get(name, 0.0) + us / nrep
             extras["sequential"]["isolated_op_ms_at_plan_share"] = {
-                "sm_attn": plan.sm_attn, "sm_gemm": plan.sm_gemm,
+                "sm_attn": plan.sm_attn, "sm_gemm": plan.sm_gemm, "grid_per_op": op_grid,
                 "ops": {k: round(v / 1000, 4) for k, v in share.items()},
                 "sum_ms": round(sum(share.values()) / 1000, 4)}
 

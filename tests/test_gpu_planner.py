@@ -3,9 +3,12 @@
 NanoFlow searches the nano-batch configuration taking into account how concurrent operations slow
 one another (arXiv abstract). After nf_calibrate (per-kernel rates, decode bandwidth at five SM
 shares, co-run slow-downs at three attention shares), the planner's best plan for each template
-and nano-batch count is run on the batch and timed; the prediction error of each is printed, and
-the plan the model ranks first must be within a few percent of the fastest one measured.
+and nano-batch count is run on the batch and timed in steady state (each plan alone for half a second
+first); the prediction error of each is printed, and the plan the model ranks first must be within
+10% of the fastest one measured, every prediction within 30%.
 """
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -18,9 +21,13 @@ CANDIDATES = [dict(nano=1, template=0), dict(nano=1, template=2), dict(nano=2, t
 
 
 def _time_us(dw, plan, reps):
-    for _ in range(2):
-        dw.forward(plan)
-    torch.cuda.synchronize()
+    # steady state: the GPU runs at its power cap, and a short run would inherit the clock the previous
+    # plan left, so each plan runs alone for about half a second before it is timed
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < 0.5:
+        for _ in range(4):
+            dw.forward(plan)
+        torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(reps):
@@ -55,6 +62,6 @@ def test_predicted_and_measured_plan_times(name, reps):
         best_meas = min(rows, key=lambda r: r[2])
         # the model's first choice runs within 10% of the best measured candidate
         assert best_pred[2] <= 1.10 * best_meas[2], (best_pred, best_meas)
-        assert max(errs) < 0.5
+        assert max(errs) < 0.3
     finally:
         dw.close()
