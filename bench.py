@@ -183,6 +183,10 @@ def op_algorithmic(work, batch, plan, op, nano):
         return "tensor", 2.0 * M * 2 * F * H
     if op == "down":
         return "tensor", 2.0 * M * H * F
+    if op == "moe":
+        # router GEMM plus, for each of the top-k experts of every row, its gate/up and down GEMMs
+        k = max(int(s.top_k), 1)
+        return "tensor", 2.0 * M * H * s.n_experts + 2.0 * M * k * (2 * F * H + H * F)
     if op == "lm_head":
         return "tensor", 2.0 * (batch.num_decode + (1 if batch.prefill_len else 0)) * H * s.vocab
     if op == "decode_attention":
@@ -198,9 +202,10 @@ def op_algorithmic(work, batch, plan, op, nano):
     return None, 0.0
 
 
-def count_launches(work, plan):
+def count_launches(work, plan, ctx_lens):
     """Kernels this library launches per iteration (checked against the ncu launch list)."""
     s = work.shape
+    plan_ctx = list(ctx_lens)
     R = plan.num_decode
     tc = s.head_dim == 128 and s.n_kv_heads == 8 and s.n_q_heads in (32, 64)
     per_step = 1                          # residual set-up (or embedding)
@@ -209,8 +214,10 @@ def count_launches(work, plan):
     for j in range(plan.n_nano):
         t0, t1 = plan.tok_begin[j], plan.tok_end[j]
         dec = 1 if min(t1, R) > min(t0, R) else 0
-        # tensor-core decode: the attention kernel and its split-KV merge pass
-        att = dec * (2 if tc else 1) + (1 if t1 > R and plan.prefill_len else 0)
+        # tensor-core decode: the attention kernel, and its split-KV merge pass when a request of the
+        # nano-batch spans more than one chunk of 64 pages (1024 keys)
+        split = any(-(-(int(c) + 1) // 16) > 64 for c in plan_ctx[min(t0, R):min(t1, R)])
+        att = dec * ((2 if split else 1) if tc else 1) + (1 if t1 > R and plan.prefill_len else 0)
         ffn = 6 if s.n_experts else 2      # MoE: route+sort, gather, 2 grouped GEMMs, combine
         per_step += s.n_layers * (1 + att + 1 + ffn)
     if s.vocab:
@@ -589,7 +596,7 @@ def run_ours(args, work, dist):
             "all_tokens_per_s": dist.world * b.num_tokens * args.steps / (ms_total / 1000.0),
             "ops": op_summary, "cost_model": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in cost.items()},
             "roofline": roofline, "cpu_baseline": cpu, "clocks": clk,
-            "gpu_launches": count_launches(work, plan) * args.steps}
+            "gpu_launches": count_launches(work, plan, b.ctx_lens) * args.steps}
     line.update(extras)
     if "e2e" not in line:
         line["e2e"] = None
