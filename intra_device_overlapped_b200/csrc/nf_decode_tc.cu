@@ -51,7 +51,6 @@ template <int NQ>
 struct TcCfg {
     static constexpr int NSP = 3;                         // page stages (K and V, released after P V)
     static constexpr int NSB = 3;                         // S^T buffers in TMEM
-    static constexpr int LOOK = 2;                        // S may run this many pages ahead of P V
     // P buffers: the softmax of page c writes buffer c % NPB once the P V of page c - NPB is done (one
     // buffer with 64 query heads, where three would not fit beside three page stages)
     static constexpr int NPB = NQ <= 32 ? 3 : 1;
@@ -67,18 +66,15 @@ struct TcCfg {
     static constexpr uint32_t IDESC_S = umma_idesc_bf16_f32(128, NQ);
     static constexpr uint32_t IDESC_PV = umma_idesc_bf16_f32_amn(128, NQ);
     static_assert(SMEM <= 232448, "shared memory");
-    // S(c + LOOK) reads a page that must be in the ring while P V(c) is pending, into an S^T buffer
-    // the softmax of page c + LOOK - NSB has released
-    static_assert(LOOK >= 1 && LOOK < NSP && LOOK < NSB, "stage / buffer counts");
     static_assert((NSB + 1) * NQ <= 256, "tensor memory");
     static_assert(2 * NSP + 2 + 2 * NSB + 2 * NPB + 2 + 1 <= 32,
                   "barrier slots (+1 for the TMEM slot and abort flag)");
 };
 
-// warp 0 loads whole pages (one bulk copy each), warp 1 issues MMAs and owns TMEM, warps 2..5 softmax,
-// warp 6 loads each item's Q (TMA) once the previous item's scores are done, so that the page ring
-// keeps streaming across item boundaries
-constexpr int THREADS = 224;
+// warp 0 loads whole pages (one bulk copy each), warp 1 issues the S^T MMAs and owns TMEM, warps 2..5
+// run the softmax, warp 6 loads each item's Q (TMA) once the previous item's scores are done, so that
+// the page ring keeps streaming across item boundaries, and warp 7 issues the P V MMAs
+constexpr int THREADS = 256;
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
@@ -217,7 +213,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < NPB; ++i) { mbar_init(&p_full[i], 4); mbar_init(&pv_done[i], 1); }
         for (int i = 0; i < NSB; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 4); }
         mbar_init(o_free, 4);
-        mbar_init(drain, 1);
+        mbar_init(drain, 2);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmQ);
@@ -337,21 +333,23 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_wait(&full[x % NSP], (x / NSP) & 1u, &quiet, nullptr);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ---------------- MMA issuer. The whole warp follows two page cursors (the next S^T and the next
-        // P V) and one elected lane issues; descriptors are built once and offset by constants. Issue is
-        // driven by readiness rather than a fixed order: P V of page pc as soon as its probabilities are
-        // in (its commit frees the page's stage for the next load), else S^T of page sc (up to LOOK pages
-        // ahead) as soon as its page has landed, so that no MMA waits behind a load it does not need.
-        PageCursor sc, pc;
-        cursor_init(sc, a, lo, hi);
-        cursor_init(pc, a, lo, hi);
+    } else if (warp == 1 || warp == 7) {
+        // ---------------- MMA issuers: warp 1 the scores S^T, warp 7 the products P V. Each follows the
+        // pages in order and one elected lane issues whatever is ready; descriptors are built once and
+        // offset by constants. Issuing the two kinds from different threads keeps a P V from waiting
+        // behind the issue of later pages' scores (its commit frees the page's stage for the next load);
+        // a commit tracks only the MMAs of the thread that issues it, so each warp's commits are its own.
+        // S^T of page c needs page c in the ring and a free S^T buffer, so it runs at most NSP pages
+        // ahead of the P V that frees the stage and NSB pages ahead of the softmax.
+        const bool is_s = warp == 1;
+        PageCursor x;
+        cursor_init(x, a, lo, hi);
         const uint64_t kd0 = umma_desc_sw128(sbase);
         const uint64_t qd0 = umma_desc_sw128(sbase + C::OFF_Q);
         const uint64_t vd0 = umma_desc_sw128_mn(sbase + HALF_PAGE, REGION, 1024);
         const uint64_t pd0 = umma_desc_sw128(sbase + C::OFF_P);
-        auto issue_s = [&](const PageCursor& x) {
-            const uint32_t st = x.cs % NSP, sb = x.cs % NSB;
+        auto issue_s = [&](const PageCursor& c) {
+            const uint32_t st = c.cs % NSP, sb = c.cs % NSB;
             tc_fence_after();
             const uint64_t ad = kd0 + ((st * PAGE_BYTES) >> 4);
             const uint64_t bd = qd0;
@@ -363,13 +361,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                     umma_bf16_c<true>(d, ad + (uint64_t)(((kk >> 2) * REGION + (kk & 3) * 32) >> 4),
                                       bd + (uint64_t)(((kk >> 2) * (NQ * 128) + (kk & 3) * 32) >> 4), C::IDESC_S);
                 umma_commit(&s_full[sb]);
-                if (x.j == x.it.pg1 - 1) umma_commit(q_empty);
+                if (c.j == c.it.pg1 - 1) umma_commit(q_empty);
             }
             __syncwarp();
         };
-        auto issue_pv = [&](const PageCursor& x) {
-            const uint32_t pb = x.cs % NPB, sv = x.cs % NSP;
-            const bool first = x.j == x.it.pg0;
+        auto issue_pv = [&](const PageCursor& c) {
+            const uint32_t pb = c.cs % NPB, sv = c.cs % NSP;
+            const bool first = c.j == c.it.pg0;
             tc_fence_after();
             const uint64_t ad = vd0 + ((sv * PAGE_BYTES) >> 4);
             const uint64_t bd = pd0 + ((pb * C::PB) >> 4);
@@ -388,31 +386,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         };
         uint32_t idle = 0;      // polls since the last issue
         uint64_t idle_t0 = 0;   // time of the 64th of them
-        while (pc.valid) {
-            bool issued = false;
-            // P V of page pc: its S^T was issued (the softmax waits for it), its probabilities are in, and
-            // on an item's first page the previous item's output has been read out of TMEM
-            if (sc.cs > pc.cs) {
-                const bool first = pc.j == pc.it.pg0;
-                if (test_bcast(&p_full[pc.cs % NPB], (pc.cs / NPB) & 1u, lane) &&
-                    (!first || test_bcast(o_free, (pc.ni & 1u) ^ 1u, lane))) {
-                    issue_pv(pc);
-                    cursor_next(pc, a, hi);
-                    issued = true;
-                }
+        while (x.valid) {
+            const bool first = x.j == x.it.pg0;
+            bool ready;
+            if (is_s) {
+                // its Q (first page of an item), its page and a free S^T buffer
+                ready = (!first || test_bcast(q_full, x.ni & 1u, lane)) &&
+                        test_bcast(&page_full[x.cs % NSP], (x.cs / NSP) & 1u, lane) &&
+                        test_bcast(&s_free[x.cs % NSB], ((x.cs / NSB) & 1u) ^ 1u, lane);
+            } else {
+                // its probabilities (written after its S^T completed), and on an item's first page the
+                // previous item's output read out of TMEM
+                ready = test_bcast(&p_full[x.cs % NPB], (x.cs / NPB) & 1u, lane) &&
+                        (!first || test_bcast(o_free, (x.ni & 1u) ^ 1u, lane));
             }
-            // S^T of page sc: its Q (first page of an item), its page and a free S^T buffer
-            if (!issued && sc.valid && sc.cs <= pc.cs + (uint32_t)C::LOOK) {
-                const bool first = sc.j == sc.it.pg0;
-                if ((!first || test_bcast(q_full, sc.ni & 1u, lane)) &&
-                    test_bcast(&page_full[sc.cs % NSP], (sc.cs / NSP) & 1u, lane) &&
-                    test_bcast(&s_free[sc.cs % NSB], ((sc.cs / NSB) & 1u) ^ 1u, lane)) {
-                    issue_s(sc);
-                    cursor_next(sc, a, hi);
-                    issued = true;
-                }
-            }
-            if (issued) {
+            if (ready) {
+                if (is_s) issue_s(x); else issue_pv(x);
+                cursor_next(x, a, hi);
                 idle = 0;
                 continue;
             }
@@ -435,6 +425,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (__shfl_sync(0xffffffffu, stop, 0)) break;
             }
         }
+        // both issuers' MMAs have completed before TMEM is released (drain counts the two commits)
         if (elect_one()) umma_commit(drain);
         __syncwarp();
         if (lane == 0) {
