@@ -209,6 +209,7 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) t
     ok &= (m->item_off = dalloc<int>(m, (size_t)cfg->max_requests + 1)) != nullptr;
     ok &= (m->chunk_off = dalloc<int>(m, (size_t)cfg->max_requests + 1)) != nullptr;
     ok &= (m->tile_ctr = dalloc<int>(m, nf::kMaxCountedOps)) != nullptr;
+    ok &= (m->op_claim = dalloc<int>(m, 1)) != nullptr;
     if (cfg->vocab > 0) ok &= (m->tok_feedback = dalloc<int>(m, T)) != nullptr;
     {  // split-K workspace of the residual GEMMs (O and down: N = hidden)
         // 128-row tiles, or two 128-row halves of each 256-row pair tile (at most one tile row more)
@@ -463,9 +464,10 @@ cudaError_t decode_prologue(nf_model* m, const nf_iter_io* io, int R, cudaStream
 }
 
 cudaError_t launch_decode(nf_model* m, const nf_iter_io* io, const CUtensorMap& tmq, const void* q, void* out,
-                          int layer, int rb, int re, int grid, cudaStream_t s) {
+                          int layer, int rb, int re, int grid, cudaStream_t s, int* claim_ctr = nullptr) {
     nf::DecodeArgs da = decode_args(m, io, q, out, rb, re);
     da.kv_pool = (const uint16_t*)io->kv_pools[layer];
+    da.claim_ctr = claim_ctr;
     if (m->decode_tc) return nf::launch_decode_attention_tc(tmq, da, grid, s);
     return nf::launch_decode_attention(da, m->dims.d, grid, s);
 }
@@ -514,7 +516,7 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
         }
         case nf::OP_DATT: {
             const int rb = std::min(t0, R), re = std::min(t1, R);
-            if (re > rb) NF_CUDA_TRY(launch_decode(m, io, m->tm_q, m->q, m->attn_o, l, rb, re, grid, s));
+            if (re > rb) NF_CUDA_TRY(launch_decode(m, io, m->tm_q, m->q, m->attn_o, l, rb, re, grid, s, tile_ctr));
             return NF_OK;
         }
         case nf::OP_PATT: {
@@ -704,7 +706,9 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
         const int grid = nf::op_grid(*p, op);
         OpTimer tm{m};
         NF_CUDA_TRY(tm.begin(s));
-        int* ctr = (op.elastic && i < (size_t)nf::kMaxCountedOps) ? m->tile_ctr + i : nullptr;
+        // work counters (zeroed above): elastic GEMMs claim their tiles, decode attention its work items
+        int* ctr = ((op.elastic || op.kind == nf::OP_DATT) && i < (size_t)nf::kMaxCountedOps) ? m->tile_ctr + i
+                                                                                               : nullptr;
         if ((st = run_op(m, p, io, op, op.elastic && !ctr ? p->sm_gemm : grid, s, ctr)) != NF_OK) return st;
         NF_CUDA_TRY(tm.end(s, kTimingKind[op.kind], op.nano, op.layer, op.stream, grid));
         if (io->layer_hidden_out && (op.kind == nf::OP_D || op.kind == nf::OP_MOE)) {
@@ -1049,7 +1053,8 @@ extern "C" nf_status nf_op_decode_attention(nf_model* m, const void* q, void* ou
         !nf::make_tmap_bf16_2d(&tmq, q, (uint64_t)req_end * m->dims.nq, m->dims.d, (uint32_t)m->dims.nq))
         return NF_ERR_INVALID_ARGUMENT;
     const int grid = sm_count > 0 ? std::min(sm_count, m->sm_count) : m->sm_count;
-    NF_CUDA_TRY(launch_decode(m, io, tmq, q, out, layer, req_begin, req_end, grid, s));
+    NF_CUDA_TRY(cudaMemsetAsync(m->op_claim, 0, sizeof(int), s));
+    NF_CUDA_TRY(launch_decode(m, io, tmq, q, out, layer, req_begin, req_end, grid, s, m->op_claim));
     return NF_OK;
 } catch (const std::bad_alloc&) {
     return NF_ERR_OUT_OF_MEMORY;

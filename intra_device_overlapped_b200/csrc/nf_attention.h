@@ -36,6 +36,8 @@ struct DecodeArgs {
     const int* chunk_off; // tensor-core kernel: [R + 1] first partial slot of each request
     float* part_ml;       // tensor-core kernel: [chunks x nq x 2] running maximum and row sum per query head
     int any_split;        // tensor-core kernel: 0 when no request of the launch has more than one chunk
+    int* claim_ctr;       // tensor-core kernel: zeroed counter from which the CTAs claim work items in
+                          // order (nullptr: each CTA takes an equal share of the page prefix)
     int* status;
     int* trace_ctr;
     nf_trace_entry* trace;

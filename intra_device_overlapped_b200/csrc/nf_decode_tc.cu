@@ -46,6 +46,8 @@ constexpr uint32_t HALF_PAGE = 32768;       // K (or V) of all heads of one page
 constexpr uint32_t REGION = 16384;          // one 64-column half of K or V: 128 rows x 128 B
 constexpr float LAZY = 8.0f;
 constexpr int kPrefetchPages = 4;           // L2 prefetch distance of the page loader
+constexpr int ITEM_SLOTS = 4;               // work-item ring between the page loader and the other roles
+constexpr int ITEM_READERS = 7;             // Q loader, two MMA issuers, four softmax warps
 
 template <int NQ>
 struct TcCfg {
@@ -60,14 +62,15 @@ struct TcCfg {
     static constexpr uint32_t OFF_P = OFF_Q + QB;
     static constexpr uint32_t OFF_CF = OFF_P + NPB * PB;  // float[NQ] rescale factors / row sums
     static constexpr uint32_t OFF_BAR = OFF_CF + NQ * 4;
-    static constexpr uint32_t SMEM = OFF_BAR + 32 * 8 + 1024;
+    static constexpr uint32_t OFF_RING = OFF_BAR + 40 * 8;   // int2[ITEM_SLOTS]: the CTA's work items
+    static constexpr uint32_t SMEM = OFF_RING + ITEM_SLOTS * 8 + 1024;
     static constexpr uint32_t O_COL = NSB * NQ;           // O^T accumulator after the S^T buffers
     static constexpr uint32_t TMEM_COLS = (NSB + 1) * NQ <= 128 ? 128 : 256;
     static constexpr uint32_t IDESC_S = umma_idesc_bf16_f32(128, NQ);
     static constexpr uint32_t IDESC_PV = umma_idesc_bf16_f32_amn(128, NQ);
     static_assert(SMEM <= 232448, "shared memory");
     static_assert((NSB + 1) * NQ <= 256, "tensor memory");
-    static_assert(2 * NSP + 2 + 2 * NSB + 2 * NPB + 2 + 1 <= 32,
+    static_assert(2 * NSP + 2 + 2 * NSB + 2 * NPB + 2 + 2 * ITEM_SLOTS + 1 <= 40,
                   "barrier slots (+1 for the TMEM slot and abort flag)");
 };
 
@@ -131,6 +134,57 @@ __device__ __forceinline__ void item_next(ItemIter& it, const DecodeArgs& a, lon
     item_chunk(it, a, hi);
 }
 
+// The item (request r, chunk c), all fields set.
+__device__ __forceinline__ void item_set(ItemIter& it, const DecodeArgs& a, int r, int c) {
+    it.r = r;
+    it.c = c;
+    item_req(it, a);
+    it.pg0 = (int)((long long)c * it.npages / it.nch);
+    it.pg1 = (int)((long long)(c + 1) * it.npages / it.nch);
+    it.start = (long long)a.item_off[r] + it.pg0;
+    it.valid = true;
+}
+
+// Global item k of the launch (items of requests [req_begin, req_end) in request order, chunks in
+// order) as (request, chunk).
+__device__ __forceinline__ int2 item_of(const DecodeArgs& a, long long k) {
+    if (a.chunk_off == nullptr) return make_int2((int)k, 0);   // one chunk per request
+    int low = a.req_begin, high = a.req_end - 1;
+    while (low < high) {  // last request whose first chunk is at or before k
+        const int mid = (low + high + 1) >> 1;
+        if ((long long)a.chunk_off[mid] <= k) low = mid; else high = mid - 1;
+    }
+    return make_int2(low, (int)(k - a.chunk_off[low]));
+}
+
+// The work items of a CTA pass from the page loader to the other roles through a ring of ITEM_SLOTS
+// (request, chunk) pairs ((-1, 0) ends the sequence): item_full[s] completes when the loader has
+// written slot s, item_empty[s] when all ITEM_READERS warps have read it.
+struct ItemRing {
+    int2* slot;
+    uint64_t* full;
+    uint64_t* empty;
+};
+
+// Reader side: the ni-th item of the CTA into `it` (valid = false at the end of the sequence).
+// Returns false if the wait gave up (the abort flag is then raised).
+__device__ __forceinline__ bool ring_get(const ItemRing& ring, const DecodeArgs& a, uint32_t ni, ItemIter& it,
+                                         volatile int* abort_flag, int lane) {
+    const uint32_t s = ni % ITEM_SLOTS;
+    const uint32_t par = (ni / ITEM_SLOTS) & 1u;
+    int ok = 1;
+    if (!__all_sync(0xffffffffu, mbar_test_wait(smem_u32(&ring.full[s]), par)))
+        if (lane == 0) ok = mbar_wait(&ring.full[s], par, abort_flag, a.status) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) { it.valid = false; return false; }
+    const volatile int* vs = reinterpret_cast<volatile int*>(&ring.slot[s]);
+    const int2 v = make_int2(vs[0], vs[1]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ring.empty[s]);
+    if (v.x < 0) it.valid = false; else item_set(it, a, v.x, v.y);
+    return true;
+}
+
 // Position in the CTA's page sequence: page j (within the request) of the current item, cs-th page
 // overall, ni-th item.
 struct PageCursor {
@@ -140,20 +194,22 @@ struct PageCursor {
     bool valid;
 };
 
-__device__ __forceinline__ void cursor_init(PageCursor& x, const DecodeArgs& a, long long lo, long long hi) {
-    item_init(x.it, a, lo, hi);
-    x.j = x.it.pg0;
+__device__ __forceinline__ void cursor_init(PageCursor& x, const DecodeArgs& a, const ItemRing& ring,
+                                            volatile int* abort_flag, int lane) {
     x.cs = 0;
     x.ni = 0;
+    ring_get(ring, a, 0, x.it, abort_flag, lane);
+    x.j = x.it.pg0;
     x.valid = x.it.valid;
 }
 
-__device__ __forceinline__ void cursor_next(PageCursor& x, const DecodeArgs& a, long long hi) {
+__device__ __forceinline__ void cursor_next(PageCursor& x, const DecodeArgs& a, const ItemRing& ring,
+                                            volatile int* abort_flag, int lane) {
     ++x.cs;
     if (++x.j == x.it.pg1) {
-        item_next(x.it, a, hi);
-        x.j = x.it.pg0;
         ++x.ni;
+        ring_get(ring, a, x.ni, x.it, abort_flag, lane);
+        x.j = x.it.pg0;
         x.valid = x.it.valid;
     }
 }
@@ -196,9 +252,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t* p_full = s_free + NSB;           // [NPB]
     uint64_t* pv_done = p_full + NPB;          // [NPB]
     uint64_t* o_free = pv_done + NPB;          // [1]
-    uint64_t* drain = o_free + 1;        // [1]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* drain = o_free + 1;              // [1]
+    uint64_t* item_full = drain + 1;           // [ITEM_SLOTS]
+    uint64_t* item_empty = item_full + ITEM_SLOTS;  // [ITEM_SLOTS]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_empty + ITEM_SLOTS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const ItemRing ring{reinterpret_cast<int2*>(smem + C::OFF_RING), item_full, item_empty};
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint64_t t_start = 0;
@@ -214,6 +273,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < NSB; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 4); }
         mbar_init(o_free, 4);
         mbar_init(drain, 2);
+        for (int i = 0; i < ITEM_SLOTS; ++i) { mbar_init(&item_full[i], 1); mbar_init(&item_empty[i], ITEM_READERS); }
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmQ);
@@ -237,9 +297,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 6) {
         // ---------------- Q loader: two 64-column halves of the item's NQ query rows (TMA)
         ItemIter it;
-        item_init(it, a, lo, hi);
         uint32_t ni = 0;
-        for (; it.valid; item_next(it, a, hi), ++ni) {
+        for (ring_get(ring, a, 0, it, abort_flag, lane); it.valid; ring_get(ring, a, ++ni, it, abort_flag, lane)) {
             if (!wait_bcast(q_empty, (ni & 1u) ^ 1u, abort_flag, a.status, lane)) break;
             if (lane == 0) {
                 uint8_t* qd = smem + C::OFF_Q;
@@ -259,12 +318,48 @@ __global__ void __launch_bounds__(THREADS, 1)
         // page ring. An SM completes bulk copies at a rate that hardly depends on their size, so whole
         // pages stream about twice as fast as separate K and V halves. Page ids are read 32 at a time
         // (one per lane) and handed to lane 0.
+        //
+        // The loader also chooses the CTA's work items and publishes them in the item ring just before
+        // it loads their pages: with a claim counter it takes the launch's next item from it, so that
+        // CTAs that run faster (SMs differ by more than 10% in the bandwidth they get) take more items
+        // and all finish together; without one it walks its share [lo, hi) of the page prefix.
         uint64_t* full = page_full;
-        uint8_t* ring = smem;
+        uint8_t* pring = smem;
+        ItemIter walk;
+        if (a.claim_ctr == nullptr) item_init(walk, a, lo, hi);
+        const long long k0 = a.chunk_off ? a.chunk_off[a.req_begin] : a.req_begin;
+        const long long k1 = a.chunk_off ? a.chunk_off[a.req_end] : a.req_end;
+        // the n-th item: chosen, published in the ring, and set in `it` (valid = false at the end)
+        auto produce = [&](uint32_t n, ItemIter& it) -> bool {
+            const uint32_t slot = n % ITEM_SLOTS;
+            if (n >= (uint32_t)ITEM_SLOTS &&
+                !wait_bcast(&item_empty[slot], ((n / ITEM_SLOTS) - 1u) & 1u, abort_flag, a.status, lane)) {
+                it.valid = false;
+                return false;
+            }
+            int2 v;
+            if (a.claim_ctr != nullptr) {
+                int kk = 0;
+                if (lane == 0) kk = atomicAdd(a.claim_ctr, 1);
+                const long long k = k0 + __shfl_sync(0xffffffffu, kk, 0);
+                v = k < k1 ? item_of(a, k) : make_int2(-1, 0);
+            } else {
+                v = walk.valid ? make_int2(walk.r, walk.c) : make_int2(-1, 0);
+                if (walk.valid) item_next(walk, a, hi);
+            }
+            if (lane == 0) {
+                volatile int* vd = reinterpret_cast<volatile int*>(&ring.slot[slot]);
+                vd[0] = v.x;
+                vd[1] = v.y;
+                mbar_arrive(&item_full[slot]);  // release: the slot's contents before the phase
+            }
+            __syncwarp();
+            if (v.x < 0) it.valid = false; else item_set(it, a, v.x, v.y);
+            return true;
+        };
         ItemIter it;
-        item_init(it, a, lo, hi);
         uint32_t cs = 0, ni = 0;
-        bool ok = true;
+        bool ok = produce(0, it);
         const char* pool = reinterpret_cast<const char*>(a.kv_pool);
         // each page is read once per launch: stream it through L2 without displacing reused data
         const uint64_t stream_policy = l2_policy_evict_first();
@@ -282,7 +377,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             return id;
         };
-        for (; it.valid && ok; item_next(it, a, hi), ++ni) {
+        for (; it.valid && ok; ok = ok && produce(++ni, it)) {
             const int base = a.page_indptr[it.r];
             const int rowlen = a.page_indptr[it.r + 1] - base;
             int ids = 0, ids_next = 0, w0 = it.pg0;
@@ -317,7 +412,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[st], PAGE_BYTES);
-                    bulk_load_hint(ring + st * PAGE_BYTES, pool + (size_t)pg * PAGE_BYTES, PAGE_BYTES, &full[st],
+                    bulk_load_hint(pring + st * PAGE_BYTES, pool + (size_t)pg * PAGE_BYTES, PAGE_BYTES, &full[st],
                                    stream_policy);
                     // a stage is held from its copy to the P V of its page, about three times the copy's
                     // own latency: a page bound for the ring kPrefetchPages pages later is fetched into L2
@@ -343,7 +438,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ahead of the P V that frees the stage and NSB pages ahead of the softmax.
         const bool is_s = warp == 1;
         PageCursor x;
-        cursor_init(x, a, lo, hi);
+        cursor_init(x, a, ring, abort_flag, lane);
         const uint64_t kd0 = umma_desc_sw128(sbase);
         const uint64_t qd0 = umma_desc_sw128(sbase + C::OFF_Q);
         const uint64_t vd0 = umma_desc_sw128_mn(sbase + HALF_PAGE, REGION, 1024);
@@ -402,7 +497,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             if (ready) {
                 if (is_s) issue_s(x); else issue_pv(x);
-                cursor_next(x, a, hi);
+                cursor_next(x, a, ring, abort_flag, lane);
                 idle = 0;
                 continue;
             }
@@ -442,10 +537,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int hsel = lane >> 4;           // which of the warp's two heads this lane's row belongs to
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
         ItemIter it;
-        item_init(it, a, lo, hi);
         uint32_t cs = 0, ni = 0;
         bool ok = true;
-        for (; it.valid && ok; item_next(it, a, hi), ++ni) {
+        // every softmax warp reads each item from the ring; the four agree on it before any named
+        // barrier inside the item (a read that gave up in one warp ends the item loop in all four)
+        auto next_item = [&](uint32_t n) {
+            const bool got = ring_get(ring, a, n, it, abort_flag, lane);
+            if (bar_red_or(4, 128, !got || !it.valid)) { it.valid = false; ok = ok && got; }
+        };
+        for (next_item(0); it.valid && ok; next_item(++ni)) {
             float m[G], lp[G];
 #pragma unroll
             for (int i = 0; i < G; ++i) { m[i] = -INFINITY; lp[i] = 0.f; }

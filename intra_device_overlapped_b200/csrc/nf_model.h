@@ -56,7 +56,8 @@ struct nf_model {
     float* rope_sin = nullptr;
     int* item_off = nullptr;      // [max_requests + 1] page prefix (tensor-core decode) or item prefix
     int* chunk_off = nullptr;     // [max_requests + 1] split-KV chunk prefix (tensor-core decode)
-    int* tile_ctr = nullptr;      // [kMaxCountedOps] work counters of elastic GEMM ops, zeroed per forward
+    int* tile_ctr = nullptr;      // [kMaxCountedOps] work counters of elastic GEMM and decode ops, zeroed per forward
+    int* op_claim = nullptr;      // work counter of the single-op decode attention entry point
     bool decode_any_split = true; // some request of the current batch spans several decode chunks
     // KV offload: two staging buffers of offload_cap pages and the device copy of the page list
     uint8_t* offload_stage = nullptr;

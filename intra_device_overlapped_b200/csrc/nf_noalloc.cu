@@ -29,7 +29,8 @@
 namespace {
 
 // Scratch layout: item_off, NF_NOALLOC_MAX_REQUESTS + 1 ints, written in full by the schedule
-// kernel before the attention kernel reads them.
+// kernel before the attention kernel reads them; then the work-item claim counter, zeroed before each
+// launch.
 constexpr size_t kScratchBytes = 4 * (size_t)(NF_NOALLOC_MAX_REQUESTS + 64);
 static_assert(kScratchBytes % 256 == 0, "scratch size");
 
@@ -74,6 +75,7 @@ extern "C" nf_status nf_decode_attention_noalloc(const void* q, void* out, const
     if (st != NF_OK) return st;
     int* status = status_device;
     int* item_off = reinterpret_cast<int*>(scratch);
+    int* claim = item_off + NF_NOALLOC_MAX_REQUESTS + 1;
 
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -90,6 +92,7 @@ extern "C" nf_status nf_decode_attention_noalloc(const void* q, void* out, const
     if (nf::launch_decode_tc_schedule(ctx_len, num_requests, nf::kDecodeNoSplit, item_off, nullptr, status, s) !=
         cudaSuccess)
         return NF_ERR_CUDA;
+    if (cudaMemsetAsync(claim, 0, sizeof(int), s) != cudaSuccess) return NF_ERR_CUDA;
 
     nf::DecodeArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -109,6 +112,7 @@ extern "C" nf_status nf_decode_attention_noalloc(const void* q, void* out, const
     a.split_pages = nf::kDecodeNoSplit;
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
     a.status = status;
+    a.claim_ctr = claim;
     if (nf::launch_decode_attention_tc(tmq, a, grid, s) != cudaSuccess) return NF_ERR_CUDA;
     return NF_OK;
 } catch (const std::bad_alloc&) {
