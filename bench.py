@@ -147,9 +147,9 @@ class ClockSampler:
 # kernel as it stands; the bench scales it to its own launches (traffic grows with the pages
 # read). Entries must be retaken whenever the kernel changes.
 TRAFFIC_PER_ALGO_BYTE = {
-    # all 512 requests of the Llama-3-8B layer on 148 SMs: 2,709,096,960 B read + 17,065,216 B written
+    # all 512 requests of the Llama-3-8B layer on 148 SMs: 2,704,816,640 B read + 17,256,192 B written
     # for 2,684,391,424 algorithmic bytes (the ncu capture summarised under profiles/)
-    "decode_attention": (1.0156, "ncu dram__bytes_read.sum + dram__bytes_write.sum, one full launch"),
+    "decode_attention": (1.0140, "ncu dram__bytes_read.sum + dram__bytes_write.sum, one full launch"),
 }
 
 def iteration_flops(work, batch):

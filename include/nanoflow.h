@@ -417,7 +417,8 @@ nf_status nf_offload_kv(nf_model* m, void* const* kv_pools, int32_t num_pool_pag
  *                 pipeline wait that passed its limit.
  * Supported shapes: head_dim 128, n_kv_heads 8, n_q_heads 32 or 64 (else NF_ERR_UNSUPPORTED).
  * num_requests > NF_NOALLOC_MAX_REQUESTS returns NF_ERR_INVALID_ARGUMENT.
- * Scratch: a static device array of 64 KB per device (the per-request page prefix), shared by
+ * Scratch: a static device array of 64 KB per device (the per-request page prefix and the work
+ * counter from which the CTAs claim requests), shared by
  * every call: calls that overlap on the GPU race on it and must be serialised. The first call
  * on each device looks up the array's address (cudaGetSymbolAddress) and keeps it for the life
  * of the process; make that first call before any stream capture, and do not call the entry
