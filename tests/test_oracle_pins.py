@@ -382,6 +382,18 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(F, "rmsnorm", lambda x, g, eps: x / np.sqrt(np.mean(x * x, axis=0, keepdims=True) + eps) * g)
     with pytest.raises(AssertionError):
         test_rmsnorm_constant_rows_closed_form()
+    monkeypatch.undo()
+
+    # the prefill chunk's token taken from its first row instead of its last breaks the cached-decode
+    # identity (the logits of a prompt's continuation)
+    def lm_rows_first_chunk_row(batch):
+        rows = list(range(batch.num_decode))
+        if batch.prefill_len > 0:
+            rows.append(batch.num_decode)
+        return np.array(rows, dtype=np.int64)
+    monkeypatch.setattr(F, "lm_rows", lm_rows_first_chunk_row)
+    with pytest.raises(AssertionError):
+        test_cached_decode_step_equals_full_sequence_recompute()
 
 
 def test_bf16_p_attention_definition():
