@@ -404,6 +404,31 @@ def run_ours(args, work, dist):
 
     extras = {}
     if not args.no_extras:
+        # ---- the same plan replayed as a CUDA graph (nf_graph_create / nf_graph_launch) on a side stream,
+        # timed like the headline
+        side = torch.cuda.Stream(dev)
+        torch.cuda.synchronize(dev)
+        g = dw.graph(plan, side)
+        t_warm = time.perf_counter()
+        nw = 0
+        while nw < max(args.warmup, 3) or time.perf_counter() - t_warm < args.min_warmup_s:
+            for _ in range(8):
+                nf.check(nf.nf_graph_launch(g, side.cuda_stream), "graph")
+            nw += 8
+            side.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(side)
+        for _ in range(args.steps):
+            nf.check(nf.nf_graph_launch(g, side.cuda_stream), "graph")
+        g1.record(side)
+        torch.cuda.synchronize(dev)
+        nf.check(dw.sync(), "graph steps")
+        g_ms = g0.elapsed_time(g1) / args.steps
+        extras["graph"] = {"ms_per_step": round(g_ms, 4),
+                           "value": round(dist.world * R * 1000.0 / g_ms, 1), "unit": "decode tokens/s",
+                           "how": "the tuned plan captured once as a CUDA graph (nf_graph_create) and replayed with "
+                                  "nf_graph_launch, same warm-up and K steps as the headline"}
+
         # ---- the same work without overlap: sequential plan, one nano-batch, every SM
         # timed exactly like the headline: the same warm-up (at least W steps and --min-warmup-s seconds of
         # this plan, so that the power-capped clock has settled on it), then K steps without per-op events

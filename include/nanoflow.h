@@ -242,6 +242,21 @@ typedef struct {
  * anything runs. Asynchronous. */
 nf_status nf_forward_iteration(nf_model* m, const nf_plan* plan, const nf_iter_io* io, void* stream);
 
+/* The iteration of one plan as a CUDA graph: every launch, copy and cross-stream dependency of
+ * nf_forward_iteration(m, plan, io) recorded once and replayed with one launch. nf_graph_create runs
+ * the iteration once normally on `stream` (so that workspaces are sized before the capture), then
+ * captures it on `stream` (a stream other than the legacy default stream; the model's attention
+ * stream joins the capture) and instantiates the graph. The graph holds the plan and the pointers of
+ * `io` (and their device contents are read at replay), so a caller reuses the same buffers from
+ * iteration to iteration; a new plan needs a new graph. nf_graph_launch replays it on `stream`,
+ * asynchronously, with the same results as nf_forward_iteration. NF_ERR_INVALID_ARGUMENT for null
+ * pointers, the default stream, or per-op timing switched on; the errors of nf_forward_iteration;
+ * NF_ERR_CUDA if the capture or instantiation fails. A graph must be destroyed before its model. */
+typedef struct nf_graph nf_graph; /* opaque */
+nf_status nf_graph_create(nf_model* m, const nf_plan* plan, const nf_iter_io* io, void* stream, nf_graph** out);
+nf_status nf_graph_launch(nf_graph* g, void* stream);
+void nf_graph_destroy(nf_graph* g);
+
 /* Plan choice by measurement. After about 0.3 s of sequential iterations (the clock a power-capped
  * GPU holds under load is lower than its first burst), for each template and nano-batch count the
  * planner's best plan (the SM split chosen by the cost model) is run on this batch: one warm-up and

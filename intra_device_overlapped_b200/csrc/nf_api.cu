@@ -755,6 +755,64 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     return NF_ERR_INVALID_ARGUMENT;
 }
 
+struct nf_graph {
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+};
+
+extern "C" nf_status nf_graph_create(nf_model* m, const nf_plan* p, const nf_iter_io* io, void* stream,
+                                     nf_graph** out) try {
+    if (!m || !p || !io || !out || stream == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    *out = nullptr;
+    if (m->timing_on) return NF_ERR_INVALID_ARGUMENT;  // per-op timing creates events on the fly
+    cudaStream_t s = (cudaStream_t)stream;
+    // one ordinary iteration: every workspace reaches its size for this plan before the capture
+    nf_status st = nf_forward_iteration(m, p, io, stream);
+    if (st != NF_OK) return st;
+    NF_CUDA_TRY(cudaStreamSynchronize(s));
+    NF_CUDA_TRY(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal));
+    st = nf_forward_iteration(m, p, io, stream);
+    cudaGraph_t g = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(s, &g);  // ends the capture whatever happened inside
+    if (st != NF_OK || e != cudaSuccess || g == nullptr) {
+        if (g) cudaGraphDestroy(g);
+        cudaGetLastError();
+        return st != NF_OK ? st : NF_ERR_CUDA;
+    }
+    cudaGraphExec_t ex = nullptr;
+    if (cudaGraphInstantiate(&ex, g, 0) != cudaSuccess) {
+        cudaGraphDestroy(g);
+        cudaGetLastError();
+        return NF_ERR_CUDA;
+    }
+    nf_graph* r = new (std::nothrow) nf_graph();
+    if (r == nullptr) {
+        cudaGraphExecDestroy(ex);
+        cudaGraphDestroy(g);
+        return NF_ERR_OUT_OF_MEMORY;
+    }
+    r->graph = g;
+    r->exec = ex;
+    *out = r;
+    return NF_OK;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
+}
+
+extern "C" nf_status nf_graph_launch(nf_graph* g, void* stream) {
+    if (g == nullptr || g->exec == nullptr) return NF_ERR_INVALID_ARGUMENT;
+    return cudaGraphLaunch(g->exec, (cudaStream_t)stream) == cudaSuccess ? NF_OK : NF_ERR_CUDA;
+}
+
+extern "C" void nf_graph_destroy(nf_graph* g) {
+    if (g == nullptr) return;
+    if (g->exec) cudaGraphExecDestroy(g->exec);
+    if (g->graph) cudaGraphDestroy(g->graph);
+    delete g;
+}
+
 // Search over measured costs: the planner's best plan for every (template, nano-batch count) is
 // run on this batch and timed; the fastest is returned. The simulated cost model ranks plans
 // within a template well but misjudges how much co-running kernels slow one another, so the

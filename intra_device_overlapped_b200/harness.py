@@ -19,7 +19,7 @@ from synth.workloads import Workload, make_batch
 
 from . import (NF_OK, check, nf_calibrate, nf_get_cost_model, nf_batch_desc, nf_destroy_model, nf_forward_iteration, nf_global_weights,
                nf_init_model, nf_iter_io, nf_layer_weights, nf_model_config, nf_plan_iteration, nf_plan_opts,
-               nf_tune_plan,
+               nf_tune_plan, nf_graph_create, nf_graph_destroy,
                nf_set_global_weights, nf_set_layer_weights, nf_sync_status, nf_set_trace, nf_get_trace)
 
 _vp = ctypes.c_void_p
@@ -194,6 +194,14 @@ class DeviceWorkload:
         s = stream.cuda_stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
         check(nf_forward_iteration(self.model, plan, io if io is not None else self.io, s), "nf_forward_iteration")
 
+    def graph(self, plan, stream: torch.cuda.Stream) -> int:
+        """The iteration of `plan` on this workload's buffers as a CUDA graph (nf_graph_create); the
+        handle is destroyed with the workload."""
+        st, g = nf_graph_create(self.model, plan, self.io, stream.cuda_stream)
+        check(st, "nf_graph_create")
+        self._graphs = getattr(self, "_graphs", []) + [g]
+        return g
+
     def calibrate(self, stream: Optional[torch.cuda.Stream] = None) -> dict:
         """Time the model's kernels on this batch and install the fitted cost model for planning."""
         s = stream.cuda_stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
@@ -214,6 +222,9 @@ class DeviceWorkload:
         return entries
 
     def close(self):
+        for g in getattr(self, "_graphs", []):
+            nf_graph_destroy(g)
+        self._graphs = []
         if getattr(self, "model", None):
             nf_destroy_model(self.model)
             self.model = None
