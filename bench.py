@@ -265,6 +265,16 @@ def cpu_oracle_sample(work, batch, n_requests: int, repeats: int = 1):
     return times, threads
 
 
+def workload_config(args, work, batch, world):
+    """The workload keys of `config`, the same in both arms."""
+    if work.ctx_lognormal_median > 0:
+        ctx = f"lognormal median {work.ctx_lognormal_median:g}, sigma {work.ctx_lognormal_sigma:g}"
+    else:
+        ctx = f"uniform [{work.ctx_lo},{work.ctx_hi}]"
+    return {"workload": args.workload, "decode_requests": batch.num_decode, "prefill_len": batch.prefill_len,
+            "tokens": batch.num_tokens, "ctx": ctx, "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args, work, dist):
     if dist.rank != 0:
         return
@@ -282,7 +292,7 @@ def run_reference(args, work, dist):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "decode tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "sample_decode_requests": n},
+            "config": workload_config(args, work, batch, dist.world),
             "cpu_baseline": {"value": value, "unit": "decode tokens/s", "cores": threads, "kind": "oracle",
                              "sample": f"{n} of {batch.num_decode} decode requests of {args.workload}, no prefill "
                                        "chunk, float64 numpy oracle, inputs pre-generated"},
@@ -610,9 +620,7 @@ def run_ours(args, work, dist):
             "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded random-init weights, seeded paged KV cache)",
-            "config": {"workload": args.workload, "decode_requests": R, "prefill_len": b.prefill_len,
-                       "tokens": b.num_tokens, "ctx": "uniform [1024,1536]" if args.workload.startswith("llama") else "",
-                       "parallelism": f"replicas x{dist.world}", "plan": plan.describe(),
+            "config": {**workload_config(args, work, b, dist.world), "plan": plan.describe(),
                        "plan_choice": "forced on the command line" if forced else
                        "planner candidates timed on this batch (nf_tune_plan), fastest kept",
                        "l2": "working set (KV cache + weights) > 126 MB L2 on every step; no flush"},
