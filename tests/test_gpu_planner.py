@@ -5,7 +5,7 @@ one another (arXiv abstract). After nf_calibrate (per-kernel rates, decode bandw
 shares, co-run slow-downs at three attention shares), the planner's best plan for each template
 and nano-batch count is run on the batch and timed in steady state (each plan alone for half a second
 first); the prediction error of each is printed, and the plan the model ranks first must be within
-10% of the fastest one measured, every prediction within 30%.
+10% of the fastest one measured, every prediction within 20%.
 """
 import time
 
@@ -62,6 +62,6 @@ def test_predicted_and_measured_plan_times(name, reps):
         best_meas = min(rows, key=lambda r: r[2])
         # the model's first choice runs within 10% of the best measured candidate
         assert best_pred[2] <= 1.10 * best_meas[2], (best_pred, best_meas)
-        assert max(errs) < 0.3
+        assert max(errs) < 0.2
     finally:
         dw.close()
