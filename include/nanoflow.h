@@ -242,6 +242,23 @@ typedef struct {
  * anything runs. Asynchronous. */
 nf_status nf_forward_iteration(nf_model* m, const nf_plan* plan, const nf_iter_io* io, void* stream);
 
+/* The same iteration with each layer run as ONE persistent kernel on `stream` instead of one launch
+ * per operation on two streams (NanoFlow's device-level pipeline, arXiv abstract: operations of
+ * different nano-batches run in parallel inside the device, here scheduled by the device itself).
+ * One CTA per SM (plan->sm_total of them) walks the layer's operations in the plan's issue order:
+ * attention-stream operations on the plan's sm_attn CTAs, GEMM-stream operations inside an attention
+ * window on the others, all other operations on every CTA. Before an operation a CTA waits until every
+ * CTA has finished each operation it depends on (completion counters in device memory, acquire/release,
+ * every wait bounded: NF_ERR_DEVICE_TIMEOUT on expiry); GEMM tiles and decode items are claimed from
+ * work counters, so a CTA that runs out of work in one operation moves on to the next at once. The
+ * GEMMs run on one-CTA 128 x 256 tiles (the stream executor pairs CTAs), so results equal those of
+ * nf_forward_iteration up to the rounding of the fp32 accumulation order in the tensor cores (in
+ * practice bit for bit). Same inputs, outputs and checks as nf_forward_iteration; NF_ERR_UNSUPPORTED
+ * for models whose attention does not run on the tensor-core kernels (head dim 128, 8 KV heads, 32 or
+ * 64 query heads) and for MoE models. Per-op timing (nf_set_timing) records nothing for the layers.
+ * Asynchronous. */
+nf_status nf_forward_iteration_persistent(nf_model* m, const nf_plan* plan, const nf_iter_io* io, void* stream);
+
 /* The iteration of one plan as a CUDA graph: every launch, copy and cross-stream dependency of
  * nf_forward_iteration(m, plan, io) recorded once and replayed with one launch. nf_graph_create runs
  * the iteration once normally on `stream` (so that workspaces are sized before the capture), then

@@ -151,6 +151,7 @@ def _load():
         "nf_plan_for_config": ([P(nf_model_config), _i32, P(nf_batch_desc), P(nf_plan_opts), P(nf_plan)],
                                ctypes.c_int),
         "nf_forward_iteration": ([_vp, P(nf_plan), P(nf_iter_io), _vp], ctypes.c_int),
+        "nf_forward_iteration_persistent": ([_vp, P(nf_plan), P(nf_iter_io), _vp], ctypes.c_int),
         "nf_graph_create": ([_vp, P(nf_plan), P(nf_iter_io), _vp, P(_vp)], ctypes.c_int),
         "nf_graph_launch": ([_vp, _vp], ctypes.c_int),
         "nf_graph_destroy": ([_vp], None),
@@ -187,7 +188,7 @@ def _load():
 
 _lib = _load()
 EXPORTED = ("nf_status_string", "nf_version", "nf_init_model", "nf_set_layer_weights", "nf_set_global_weights",
-            "nf_destroy_model", "nf_plan_iteration", "nf_plan_for_config", "nf_forward_iteration", "nf_tune_plan", "nf_sync_status", "nf_calibrate",
+            "nf_destroy_model", "nf_plan_iteration", "nf_plan_for_config", "nf_forward_iteration", "nf_forward_iteration_persistent", "nf_tune_plan", "nf_sync_status", "nf_calibrate",
             "nf_graph_create", "nf_graph_launch", "nf_graph_destroy",
             "nf_get_cost_model", "nf_set_cost_model",
             "nf_set_trace", "nf_get_trace", "nf_set_timing", "nf_get_op_times", "nf_op_gemm_bf16", "nf_op_decode_attention",
@@ -275,6 +276,10 @@ def nf_plan_for_config(cfg: nf_model_config, sm_count: int, batch: nf_batch_desc
 
 def nf_forward_iteration(model: int, plan: nf_plan, io: nf_iter_io, stream: int = 0) -> int:
     return _lib.nf_forward_iteration(model, ctypes.byref(plan), ctypes.byref(io), stream)
+
+
+def nf_forward_iteration_persistent(model: int, plan: nf_plan, io: nf_iter_io, stream: int = 0) -> int:
+    return _lib.nf_forward_iteration_persistent(model, ctypes.byref(plan), ctypes.byref(io), stream)
 
 
 def nf_graph_create(model: int, plan: nf_plan, io: nf_iter_io, stream: int):

@@ -14,6 +14,7 @@
 #include "nanoflow.h"
 #include "nf_attention.h"
 #include "nf_internal.h"
+#include "nf_mega.h"
 #include "nf_misc.h"
 #include "nf_model.h"
 #include "nf_schedule.h"
@@ -210,6 +211,7 @@ extern "C" nf_status nf_init_model(const nf_model_config* cfg, nf_model** out) t
     ok &= (m->chunk_off = dalloc<int>(m, (size_t)cfg->max_requests + 1)) != nullptr;
     ok &= (m->tile_ctr = dalloc<int>(m, nf::kMaxCountedOps)) != nullptr;
     ok &= (m->op_claim = dalloc<int>(m, 1)) != nullptr;
+    ok &= (m->mega_ctr = dalloc<int>(m, (size_t)d.L * nf::kMegaCountersPerLayer)) != nullptr;
     if (cfg->vocab > 0) ok &= (m->tok_feedback = dalloc<int>(m, T)) != nullptr;
     {  // split-K workspace of the residual GEMMs (O and down: N = hidden)
         // 128-row tiles, or two 128-row halves of each 256-row pair tile (at most one tile row more)
@@ -482,6 +484,58 @@ cudaError_t launch_prefill(nf_model* m, const nf_iter_io* io, const CUtensorMap&
     return nf::launch_prefill_attention(pa, m->dims.d, grid, s);
 }
 
+// Arguments of the dense GEMM of op kind `kind` (OP_QKV, OP_O, OP_GU or OP_D) of layer l over rows
+// [t0, t0 + M); the operand maps go to *tmA / *tmB and the epilogue to *epi.
+GemmArgs layer_gemm_args(nf_model* m, const nf_iter_io* io, int R, int kind, int l, int t0, int M, int* tile_ctr,
+                         const CUtensorMap** tmA, const CUtensorMap** tmB, int* epi) {
+    const nf::ModelDims& d = m->dims;
+    const nf::LayerWeights& W = m->layers[l];
+    GemmArgs a = base_args(m);
+    a.a_row0 = t0;
+    a.tok0 = t0;
+    a.tile_ctr = tile_ctr;
+    if (kind == nf::OP_QKV) {
+        set_tiles(a, M, d.qkv, d.H);
+        a.partials = m->partials;
+        a.positions = io->positions;
+        a.rope_cos = m->rope_cos;
+        a.rope_sin = m->rope_sin;
+        a.max_position = m->cfg.max_position;
+        a.q_out = m->q;
+        a.nq = d.nq;
+        a.nkv = d.nkv;
+        a.head_dim = d.d;
+        a.kv_pool = (uint16_t*)io->kv_pools[l];
+        a.num_pages = io->num_pages;
+        a.page_indptr = io->page_indptr;
+        a.page_indices = io->page_indices;
+        a.num_decode = R;
+        *tmA = &m->tm_xb;
+        *tmB = &W.tm_qkv;
+        *epi = nf::EPI_QKV;
+    } else if (kind == nf::OP_GU) {
+        set_tiles(a, M, 2 * d.F, d.H);
+        a.partials = m->partials;
+        a.out_bf16 = m->act;
+        a.ld_bf16 = d.F;
+        *tmA = &m->tm_xb;
+        *tmB = &W.tm_gu;
+        *epi = nf::EPI_SWIGLU;
+    } else {  // O or down: residual epilogue
+        const bool o = kind == nf::OP_O;
+        set_tiles(a, M, d.H, o ? d.nq * d.d : d.F);
+        a.resid = m->resid;
+        a.out_bf16 = m->xb;
+        a.ld_bf16 = d.H;
+        a.out_partials = m->partials;
+        set_splitk(m, a);
+        *tmA = o ? &m->tm_attn_o : &m->tm_act;
+        *tmB = o ? &W.tm_o : &W.tm_d;
+        *epi = nf::EPI_RESID;
+    }
+    return a;
+}
+
 nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::Op& op, int grid,
                  cudaStream_t s, int* tile_ctr) {
     const nf::ModelDims& d = m->dims;
@@ -490,28 +544,15 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
     const int R = p->num_decode, C = p->prefill_len, T = p->num_tokens;
     if (M <= 0) return NF_OK;
     nf::LayerWeights& W = m->layers[l];
-    GemmArgs a = base_args(m);
-    a.a_row0 = t0;
-    a.tok0 = t0;
-    a.tile_ctr = tile_ctr;
     switch (op.kind) {
-        case nf::OP_QKV: {
-            set_tiles(a, M, d.qkv, d.H);
-            a.partials = m->partials;
-            a.positions = io->positions;
-            a.rope_cos = m->rope_cos;
-            a.rope_sin = m->rope_sin;
-            a.max_position = m->cfg.max_position;
-            a.q_out = m->q;
-            a.nq = d.nq;
-            a.nkv = d.nkv;
-            a.head_dim = d.d;
-            a.kv_pool = (uint16_t*)io->kv_pools[l];
-            a.num_pages = io->num_pages;
-            a.page_indptr = io->page_indptr;
-            a.page_indices = io->page_indices;
-            a.num_decode = R;
-            NF_CUDA_TRY(nf::launch_gemm(nf::EPI_QKV, m->tm_xb, W.tm_qkv, a, gemm_grid(a, grid), s));
+        case nf::OP_QKV:
+        case nf::OP_O:
+        case nf::OP_GU:
+        case nf::OP_D: {
+            const CUtensorMap *tmA = nullptr, *tmB = nullptr;
+            int epi = 0;
+            const GemmArgs a = layer_gemm_args(m, io, R, op.kind, l, t0, M, tile_ctr, &tmA, &tmB, &epi);
+            NF_CUDA_TRY(nf::launch_gemm(epi, *tmA, *tmB, a, gemm_grid(a, grid), s));
             return NF_OK;
         }
         case nf::OP_DATT: {
@@ -521,34 +562,6 @@ nf_status run_op(nf_model* m, const nf_plan* p, const nf_iter_io* io, const nf::
         }
         case nf::OP_PATT: {
             if (t1 > R && C > 0) NF_CUDA_TRY(launch_prefill(m, io, m->tm_q3, m->q, m->attn_o, l, R, C, grid, s));
-            return NF_OK;
-        }
-        case nf::OP_O: {
-            set_tiles(a, M, d.H, d.nq * d.d);
-            a.resid = m->resid;
-            a.out_bf16 = m->xb;
-            a.ld_bf16 = d.H;
-            a.out_partials = m->partials;
-            set_splitk(m, a);
-            NF_CUDA_TRY(nf::launch_gemm(nf::EPI_RESID, m->tm_attn_o, W.tm_o, a, gemm_grid(a, grid), s));
-            return NF_OK;
-        }
-        case nf::OP_GU: {
-            set_tiles(a, M, 2 * d.F, d.H);
-            a.partials = m->partials;
-            a.out_bf16 = m->act;
-            a.ld_bf16 = d.F;
-            NF_CUDA_TRY(nf::launch_gemm(nf::EPI_SWIGLU, m->tm_xb, W.tm_gu, a, gemm_grid(a, grid), s));
-            return NF_OK;
-        }
-        case nf::OP_D: {
-            set_tiles(a, M, d.H, d.F);
-            a.resid = m->resid;
-            a.out_bf16 = m->xb;
-            a.ld_bf16 = d.H;
-            a.out_partials = m->partials;
-            set_splitk(m, a);
-            NF_CUDA_TRY(nf::launch_gemm(nf::EPI_RESID, m->tm_act, W.tm_d, a, gemm_grid(a, grid), s));
             return NF_OK;
         }
         case nf::OP_MOE: {
@@ -650,9 +663,119 @@ nf_status validate_forward(const nf_model* m, const nf_plan* p, const nf_iter_io
 
 }  // namespace
 
-extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const nf_iter_io* io, void* stream) try {
+namespace {
+
+// The layers of a forward as one persistent kernel launch each (nf_mega.h): the ops of `ops` of each
+// layer in issue order, attention-stream ops on the attention lane (the plan's sm_attn CTAs), GEMM-stream
+// ops inside an attention window on the others, every other op on all CTAs.
+nf_status run_layers_persistent(nf_model* m, const nf_plan* p, const nf_iter_io* io, const std::vector<nf::Op>& ops,
+                                cudaStream_t s) {
+    const nf::ModelDims& d = m->dims;
+    const int R = p->num_decode, C = p->prefill_len, T = p->num_tokens;
+    const bool lanes = p->order_template != NF_TEMPLATE_SEQUENTIAL;
+    NF_CUDA_TRY(cudaMemsetAsync(m->mega_ctr, 0, (size_t)d.L * nf::kMegaCountersPerLayer * sizeof(int), s));
+    std::unique_ptr<nf::MegaParams> P(new nf::MegaParams);
+    for (int l = 0; l < d.L; ++l) {
+        std::memset(P.get(), 0, sizeof(nf::MegaParams));
+        int* done = m->mega_ctr + (size_t)l * nf::kMegaCountersPerLayer;
+        int* claim = done + nf::kMegaMaxOps;
+        P->done = done;
+        P->n_attn = lanes ? p->sm_attn : 0;
+        P->status = m->status;
+        if (m->trace_on) {
+            P->trace_ctr = m->trace_ctr;
+            P->trace = m->trace;
+            P->trace_cap = m->trace_cap;
+        }
+        int last_qkv[NF_MAX_NANO], last_attn[NF_MAX_NANO][2], last_o[NF_MAX_NANO], last_gu[NF_MAX_NANO];
+        for (int j = 0; j < NF_MAX_NANO; ++j) last_qkv[j] = last_attn[j][0] = last_attn[j][1] = last_o[j] = last_gu[j] = -1;
+        int last_resid = -1;
+        auto add = [&](int kind, int lane, int d0, int d1, int d2) -> nf::MegaOp* {
+            if (P->n_ops >= nf::kMegaMaxOps) return nullptr;
+            nf::MegaOp* o = &P->ops[P->n_ops++];
+            o->kind = kind;
+            o->lane = lane;
+            o->dep[0] = d0;
+            o->dep[1] = d1;
+            o->dep[2] = d2;
+            return o;
+        };
+        for (const nf::Op& op : ops) {
+            if (op.layer != l) continue;
+            const int j = op.nano, t0 = p->tok_begin[j], t1 = p->tok_end[j], M = t1 - t0;
+            const int lane = (!lanes || op.full_sm || op.elastic) ? nf::LANE_ALL
+                             : op.stream == nf::STREAM_ATTN  ? nf::LANE_ATTN
+                                                             : nf::LANE_GEMM;
+            const int idx = P->n_ops;
+            if (op.kind == nf::OP_QKV || op.kind == nf::OP_O || op.kind == nf::OP_GU || op.kind == nf::OP_D) {
+                int kind = nf::MEGA_QKV, d0 = -1, d1 = -1, d2 = -1;
+                if (op.kind == nf::OP_O) {
+                    kind = nf::MEGA_RESID;
+                    d0 = last_attn[j][0];
+                    d1 = last_attn[j][1];
+                    d2 = last_resid;
+                } else if (op.kind == nf::OP_GU) {
+                    kind = nf::MEGA_SWIGLU;
+                    d0 = last_o[j];
+                } else if (op.kind == nf::OP_D) {
+                    kind = nf::MEGA_RESID;
+                    d0 = last_gu[j];
+                    d1 = last_resid;
+                }
+                nf::MegaOp* o = add(kind, lane, d0, d1, d2);
+                if (o == nullptr) return NF_ERR_UNSUPPORTED;
+                const CUtensorMap *tmA = nullptr, *tmB = nullptr;
+                int epi = 0;
+                o->g = layer_gemm_args(m, io, R, op.kind, l, t0, M, claim + idx, &tmA, &tmB, &epi);
+                o->g.trace = nullptr;  // the layer kernel traces per operation itself
+                o->tmA = *tmA;
+                o->tmB = *tmB;
+                if (op.kind == nf::OP_QKV) last_qkv[j] = idx;
+                if (op.kind == nf::OP_O) last_o[j] = idx;
+                if (op.kind == nf::OP_GU) last_gu[j] = idx;
+                if (kind == nf::MEGA_RESID) last_resid = idx;
+            } else if (op.kind == nf::OP_DATT) {
+                const int rb = std::min(t0, R), re = std::min(t1, R);
+                if (re <= rb) continue;
+                nf::MegaOp* o = add(nf::MEGA_DECODE, lane, last_qkv[j], -1, -1);
+                if (o == nullptr) return NF_ERR_UNSUPPORTED;
+                o->d = decode_args(m, io, m->q, m->attn_o, rb, re);
+                o->d.kv_pool = (const uint16_t*)io->kv_pools[l];
+                o->d.claim_ctr = claim + idx;
+                o->d.trace = nullptr;
+                o->tmA = m->tm_q;
+                last_attn[j][0] = idx;
+                if (o->d.split_pages < nf::kDecodeNoSplit && o->d.any_split) {
+                    nf::MegaOp* mg = add(nf::MEGA_MERGE, lane, idx, -1, -1);
+                    if (mg == nullptr) return NF_ERR_UNSUPPORTED;
+                    mg->d = P->ops[idx].d;
+                    last_attn[j][0] = idx + 1;
+                }
+            } else if (op.kind == nf::OP_PATT) {
+                if (!(t1 > R && C > 0)) continue;
+                nf::MegaOp* o = add(nf::MEGA_PREFILL, lane, last_qkv[j], -1, -1);
+                if (o == nullptr) return NF_ERR_UNSUPPORTED;
+                o->p = prefill_args(m, io, m->q, m->attn_o, R, C);
+                o->p.kv_pool = (const uint16_t*)io->kv_pools[l];
+                o->p.trace = nullptr;
+                o->tmA = m->tm_q3;
+                last_attn[j][1] = idx;
+            } else {
+                return NF_ERR_UNSUPPORTED;
+            }
+        }
+        NF_CUDA_TRY(nf::launch_mega(*P, d.nq, p->sm_total, s));
+        if (io->layer_hidden_out)
+            NF_CUDA_TRY(cudaMemcpyAsync(io->layer_hidden_out + (size_t)l * T * d.H, m->resid, (size_t)T * d.H * 4,
+                                        cudaMemcpyDeviceToDevice, s));
+    }
+    return NF_OK;
+}
+
+nf_status forward_impl(nf_model* m, const nf_plan* p, const nf_iter_io* io, void* stream, bool persistent) {
     nf_status st = validate_forward(m, p, io);
     if (st != NF_OK) return st;
+    if (persistent && (!m->decode_tc || !m->prefill_tc || m->dims.E > 0)) return NF_ERR_UNSUPPORTED;
     const nf::ModelDims& d = m->dims;
     const int R = p->num_decode, C = p->prefill_len, T = p->num_tokens;
     cudaStream_t sg = (cudaStream_t)stream;
@@ -663,10 +786,12 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
         if ((st = check_pool(m, l, io)) != NF_OK) return st;
 
     const int S = p->sm_total;
-    // one zeroed work counter per op that claims its GEMM tiles dynamically (elastic ops)
-    NF_CUDA_TRY(cudaMemsetAsync(m->tile_ctr, 0, nf::kMaxCountedOps * sizeof(int), sg));
-    NF_CUDA_TRY(cudaEventRecord(m->ev_fork, sg));
-    NF_CUDA_TRY(cudaStreamWaitEvent(sa, m->ev_fork, 0));
+    if (!persistent) {
+        // one zeroed work counter per op that claims its GEMM tiles dynamically (elastic ops)
+        NF_CUDA_TRY(cudaMemsetAsync(m->tile_ctr, 0, nf::kMaxCountedOps * sizeof(int), sg));
+        NF_CUDA_TRY(cudaEventRecord(m->ev_fork, sg));
+        NF_CUDA_TRY(cudaStreamWaitEvent(sa, m->ev_fork, 0));
+    }
     if (m->trace_on) NF_CUDA_TRY(cudaMemsetAsync(m->trace_ctr, 0, sizeof(int), sg));
 
     // prologue: decode work items, residual stream set-up
@@ -691,7 +816,8 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     nf::nano_content(*p, has_dec, has_pre);
     const std::vector<nf::Op> ops =
         nf::build_ops(p->order_template, p->n_nano, order, d.L, d.E > 0, has_dec, has_pre);
-    while (m->events.size() < ops.size()) {
+    if (persistent && (st = run_layers_persistent(m, p, io, ops, sg)) != NF_OK) return st;
+    while (!persistent && m->events.size() < ops.size()) {
         cudaEvent_t e;
         NF_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
         m->events.push_back(e);
@@ -699,7 +825,7 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     // timing entries accumulate over forwards until nf_set_timing is called again
     static const int kTimingKind[] = {NF_OP_QKV, NF_OP_DECODE_ATTN, NF_OP_O, NF_OP_GATE_UP, NF_OP_DOWN, NF_OP_MOE,
                                       NF_OP_PREFILL_ATTN};
-    for (size_t i = 0; i < ops.size(); ++i) {
+    for (size_t i = 0; i < (persistent ? 0 : ops.size()); ++i) {
         const nf::Op& op = ops[i];
         cudaStream_t s = op.stream == nf::STREAM_ATTN ? sa : sg;
         if (op.wait >= 0) NF_CUDA_TRY(cudaStreamWaitEvent(s, m->events[op.wait], 0));
@@ -722,8 +848,10 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
         }
         if (op.signal) NF_CUDA_TRY(cudaEventRecord(m->events[i], s));
     }
-    NF_CUDA_TRY(cudaEventRecord(m->ev_join, sa));
-    NF_CUDA_TRY(cudaStreamWaitEvent(sg, m->ev_join, 0));
+    if (!persistent) {
+        NF_CUDA_TRY(cudaEventRecord(m->ev_join, sa));
+        NF_CUDA_TRY(cudaStreamWaitEvent(sg, m->ev_join, 0));
+    }
 
     // final norm + LM head + greedy argmax over the decode rows and the chunk's last row
     if (m->cfg.vocab > 0 && (io->logits || io->next_token)) {
@@ -749,6 +877,21 @@ extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const n
     if (io->hidden_out_f32)
         NF_CUDA_TRY(cudaMemcpyAsync(io->hidden_out_f32, m->resid, (size_t)T * d.H * 4, cudaMemcpyDeviceToDevice, sg));
     return NF_OK;
+}
+
+}  // namespace
+
+extern "C" nf_status nf_forward_iteration(nf_model* m, const nf_plan* p, const nf_iter_io* io, void* stream) try {
+    return forward_impl(m, p, io, stream, false);
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
+}
+
+extern "C" nf_status nf_forward_iteration_persistent(nf_model* m, const nf_plan* p, const nf_iter_io* io,
+                                                     void* stream) try {
+    return forward_impl(m, p, io, stream, true);
 } catch (const std::bad_alloc&) {
     return NF_ERR_OUT_OF_MEMORY;
 } catch (...) {

@@ -58,6 +58,8 @@ struct nf_model {
     int* chunk_off = nullptr;     // [max_requests + 1] split-KV chunk prefix (tensor-core decode)
     int* tile_ctr = nullptr;      // [kMaxCountedOps] work counters of elastic GEMM and decode ops, zeroed per forward
     int* op_claim = nullptr;      // work counter of the single-op decode attention entry point
+    int* mega_ctr = nullptr;      // [n_layers x kMegaCountersPerLayer] completion and work counters of the
+                                  // persistent layer kernel, zeroed per forward
     bool decode_any_split = true; // some request of the current batch spans several decode chunks
     // KV offload: two staging buffers of offload_cap pages and the device copy of the page list
     uint8_t* offload_stage = nullptr;

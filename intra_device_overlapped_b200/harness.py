@@ -19,7 +19,7 @@ from synth.workloads import Workload, make_batch
 
 from . import (NF_OK, check, nf_calibrate, nf_get_cost_model, nf_batch_desc, nf_destroy_model, nf_forward_iteration, nf_global_weights,
                nf_init_model, nf_iter_io, nf_layer_weights, nf_model_config, nf_plan_iteration, nf_plan_opts,
-               nf_tune_plan, nf_graph_create, nf_graph_destroy,
+               nf_tune_plan, nf_graph_create, nf_graph_destroy, nf_forward_iteration_persistent,
                nf_set_global_weights, nf_set_layer_weights, nf_sync_status, nf_set_trace, nf_get_trace)
 
 _vp = ctypes.c_void_p
@@ -190,9 +190,13 @@ class DeviceWorkload:
         check(st, "nf_tune_plan")
         return plan, us
 
-    def forward(self, plan, stream: Optional[torch.cuda.Stream] = None, io: Optional[nf_iter_io] = None) -> None:
+    def forward(self, plan, stream: Optional[torch.cuda.Stream] = None, io: Optional[nf_iter_io] = None,
+                persistent: bool = False) -> None:
+        """One iteration of `plan`: one launch per operation on two streams (nf_forward_iteration), or
+        with persistent=True one persistent kernel per layer (nf_forward_iteration_persistent)."""
         s = stream.cuda_stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
-        check(nf_forward_iteration(self.model, plan, io if io is not None else self.io, s), "nf_forward_iteration")
+        fn = nf_forward_iteration_persistent if persistent else nf_forward_iteration
+        check(fn(self.model, plan, io if io is not None else self.io, s), fn.__name__)
 
     def graph(self, plan, stream: torch.cuda.Stream) -> int:
         """The iteration of `plan` on this workload's buffers as a CUDA graph (nf_graph_create); the

@@ -7,7 +7,8 @@ Ops: ``decode_attention`` (requests [0, --requests) of the workload's decode bat
 paged pool), ``prefill_attention`` (the workload's prefill chunk), ``gemm`` (--m x --n x --k bf16,
 random operands), ``iteration`` (whole serving iterations of the workload with a plan forced by
 --nano / --template / --sm-attn, the sequential one by default; one iteration of the Llama-3-8B
-layer launches the QKV, O, gate/up and down GEMMs in that order). ``--sm`` is the persistent grid (0 = every SM). The printed line holds the mean
+layer launches the QKV, O, gate/up and down GEMMs in that order; --persistent runs each layer as
+one persistent kernel instead). ``--sm`` is the persistent grid (0 = every SM). The printed line holds the mean
 launch time over --reps launches (CUDA events on the launching stream, after --warmup launches) and
 the algorithmic bytes or FLOPs of one launch, so that a profiler can target a small, known case.
 """
@@ -41,6 +42,8 @@ def main(argv=None) -> dict:
     ap.add_argument("--nano", type=int, default=1)
     ap.add_argument("--template", type=int, default=0)
     ap.add_argument("--sm-attn", type=int, default=0)
+    ap.add_argument("--persistent", action="store_true",
+                    help="iteration: one persistent kernel per layer (nf_forward_iteration_persistent)")
     ap.add_argument("--workload", default="llama3_8b_layer")
     ap.add_argument("--layers", type=int, default=0, help="build only this many layers of the workload (0: all)")
     ap.add_argument("--requests", type=int, default=0, help="decode requests (0 = all)")
@@ -78,8 +81,9 @@ def main(argv=None) -> dict:
         o = torch.zeros_like(q)
         if args.op == "iteration":
             plan = dw.plan(nano=args.nano, template=args.template, sm_attn=args.sm_attn)
-            us = _time(lambda: dw.forward(plan, stream), args.reps, args.warmup, stream)
-            out.update({"workload": args.workload, "plan": plan.describe(), "us": round(us, 2)})
+            us = _time(lambda: dw.forward(plan, stream, persistent=args.persistent), args.reps, args.warmup, stream)
+            out.update({"workload": args.workload, "plan": plan.describe(), "persistent": args.persistent,
+                        "us": round(us, 2)})
         elif args.op == "decode_attention":
             R = args.requests or bt.num_decode
             pages = sum(-(-(int(c) + 1) // s.page_size) for c in bt.ctx_lens[:R])
