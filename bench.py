@@ -439,6 +439,29 @@ def run_ours(args, work, dist):
                            "how": "the tuned plan captured once as a CUDA graph (nf_graph_create) and replayed with "
                                   "nf_graph_launch, same warm-up and K steps as the headline"}
 
+        # ---- the tuned plan with each layer as one persistent kernel (nf_forward_iteration_persistent):
+        # operations scheduled on the device by completion counters instead of launches and events
+        t_warm = time.perf_counter()
+        nw = 0
+        while nw < max(args.warmup, 3) or time.perf_counter() - t_warm < args.min_warmup_s:
+            for _ in range(8):
+                dw.forward(plan, stream, persistent=True)
+            nw += 8
+            torch.cuda.synchronize(dev)
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record(stream)
+        for _ in range(args.steps):
+            dw.forward(plan, stream, persistent=True)
+        p1.record(stream)
+        torch.cuda.synchronize(dev)
+        nf.check(dw.sync(), "persistent steps")
+        p_ms = p0.elapsed_time(p1) / args.steps
+        extras["persistent"] = {"ms_per_step": round(p_ms, 4),
+                                "value": round(dist.world * R * 1000.0 / p_ms, 1), "unit": "decode tokens/s",
+                                "how": "the tuned plan with each layer as one persistent kernel "
+                                       "(nf_forward_iteration_persistent: one-CTA GEMM tiles, device-side "
+                                       "completion counters), same warm-up and K steps as the headline"}
+
         # ---- the same work without overlap: sequential plan, one nano-batch, every SM
         # timed exactly like the headline: the same warm-up (at least W steps and --min-warmup-s seconds of
         # this plan, so that the power-capped clock has settled on it), then K steps without per-op events

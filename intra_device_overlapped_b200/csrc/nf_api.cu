@@ -690,6 +690,10 @@ nf_status run_layers_persistent(nf_model* m, const nf_plan* p, const nf_iter_io*
         int last_qkv[NF_MAX_NANO], last_attn[NF_MAX_NANO][2], last_o[NF_MAX_NANO], last_gu[NF_MAX_NANO];
         for (int j = 0; j < NF_MAX_NANO; ++j) last_qkv[j] = last_attn[j][0] = last_attn[j][1] = last_o[j] = last_gu[j] = -1;
         int last_resid = -1;
+        // the split-KV merge of nano-batch j's decode attention is placed after the attention ops of j
+        // that follow its decode (the prefill attention in the sequential and pipelined templates), so
+        // that CTAs which finish their decode items early run those while the others finish theirs
+        int pending_merge = -1, pending_nano = -1;
         auto add = [&](int kind, int lane, int d0, int d1, int d2) -> nf::MegaOp* {
             if (P->n_ops >= nf::kMegaMaxOps) return nullptr;
             nf::MegaOp* o = &P->ops[P->n_ops++];
@@ -700,8 +704,21 @@ nf_status run_layers_persistent(nf_model* m, const nf_plan* p, const nf_iter_io*
             o->dep[2] = d2;
             return o;
         };
+        auto flush_merge = [&]() -> bool {
+            if (pending_merge < 0) return true;
+            const nf::MegaOp& dec = P->ops[pending_merge];
+            nf::MegaOp* mg = add(nf::MEGA_MERGE, dec.lane, pending_merge, -1, -1);
+            if (mg == nullptr) return false;
+            mg->d = dec.d;
+            last_attn[pending_nano][0] = P->n_ops - 1;
+            pending_merge = -1;
+            return true;
+        };
         for (const nf::Op& op : ops) {
             if (op.layer != l) continue;
+            if (!(op.kind == nf::OP_PATT && op.nano == pending_nano && (op.stream == nf::STREAM_ATTN || !lanes)) &&
+                !flush_merge())
+                return NF_ERR_UNSUPPORTED;
             const int j = op.nano, t0 = p->tok_begin[j], t1 = p->tok_end[j], M = t1 - t0;
             const int lane = (!lanes || op.full_sm || op.elastic) ? nf::LANE_ALL
                              : op.stream == nf::STREAM_ATTN  ? nf::LANE_ATTN
@@ -746,10 +763,8 @@ nf_status run_layers_persistent(nf_model* m, const nf_plan* p, const nf_iter_io*
                 o->tmA = m->tm_q;
                 last_attn[j][0] = idx;
                 if (o->d.split_pages < nf::kDecodeNoSplit && o->d.any_split) {
-                    nf::MegaOp* mg = add(nf::MEGA_MERGE, lane, idx, -1, -1);
-                    if (mg == nullptr) return NF_ERR_UNSUPPORTED;
-                    mg->d = P->ops[idx].d;
-                    last_attn[j][0] = idx + 1;
+                    pending_merge = idx;
+                    pending_nano = j;
                 }
             } else if (op.kind == nf::OP_PATT) {
                 if (!(t1 > R && C > 0)) continue;
@@ -764,6 +779,7 @@ nf_status run_layers_persistent(nf_model* m, const nf_plan* p, const nf_iter_io*
                 return NF_ERR_UNSUPPORTED;
             }
         }
+        if (!flush_merge()) return NF_ERR_UNSUPPORTED;
         NF_CUDA_TRY(nf::launch_mega(*P, d.nq, p->sm_total, s));
         if (io->layer_hidden_out)
             NF_CUDA_TRY(cudaMemcpyAsync(io->layer_hidden_out + (size_t)l * T * d.H, m->resid, (size_t)T * d.H * 4,

@@ -672,45 +672,53 @@ __device__ __forceinline__ void decode_body(const CUtensorMap* tmQ, const Decode
 
 // Requests cut into several chunks: out = bf16(sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c) per
 // query head, M the largest chunk maximum, both sums in chunk order (every factor is an exact power of
-// two). One group of 128 threads (t = one d each, named barrier `bar`, scratch Ms / Ls of MERGE_HEADS
-// floats) merges query heads [h0, h0 + MERGE_HEADS) of request r; a thread's loads for its heads are
-// independent, so they overlap. A request of one chunk was written by the attention itself.
+// two). One warp merges query heads [h0, h0 + MERGE_HEADS) of request r: lane l owns d = 4 l .. 4 l + 3
+// (one 16-byte load per chunk and head), lane i < MERGE_HEADS finds M and the row sum of head h0 + i.
+// A request of one chunk was written by the attention itself.
 constexpr int MERGE_HEADS = 8;
 
 template <int NQ>
-__device__ __forceinline__ void merge_heads(const DecodeArgs& a, int r, int h0, int t, float* Ms, float* Ls, int bar) {
+__device__ __forceinline__ void merge_heads_warp(const DecodeArgs& a, int r, int h0, int lane) {
     const int npages = (max(a.ctx_len[r], 0) + 1 + 15) >> 4;
     const int nch = ceil_div(npages, a.split_pages);
     if (nch <= 1) return;
     const float* __restrict__ ml = a.part_ml + (size_t)a.chunk_off[r] * NQ * 2;
     const float* __restrict__ po = a.part_o + (size_t)a.chunk_off[r] * NQ * 128;
-    bar_sync_n(bar, 128);  // the group's previous request's Ms / Ls are no longer read
-    if (t < MERGE_HEADS) {
-        const int qh = h0 + t;
-        float M = -INFINITY;
+    float M = -INFINITY, L = 0.f;
+    if (lane < MERGE_HEADS) {
+        const int qh = h0 + lane;
         for (int c = 0; c < nch; ++c) M = fmaxf(M, ml[(c * NQ + qh) * 2]);
-        float L = 0.f;
         for (int c = 0; c < nch; ++c) L += softmax_rescale(ml[(c * NQ + qh) * 2], M) * ml[(c * NQ + qh) * 2 + 1];
-        Ms[t] = M;
-        Ls[t] = L;
     }
-    bar_sync_n(bar, 128);
-    float acc[MERGE_HEADS];
+    float Mh[MERGE_HEADS];
 #pragma unroll
-    for (int i = 0; i < MERGE_HEADS; ++i) acc[i] = 0.f;
+    for (int i = 0; i < MERGE_HEADS; ++i) Mh[i] = __shfl_sync(0xffffffffu, M, i);
+    float acc[MERGE_HEADS][4];
+#pragma unroll
+    for (int i = 0; i < MERGE_HEADS; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
     for (int c = 0; c < nch; ++c) {
-        float v[MERGE_HEADS], f[MERGE_HEADS];
+        float4 v[MERGE_HEADS];
+        float f[MERGE_HEADS];
 #pragma unroll
         for (int i = 0; i < MERGE_HEADS; ++i) {
-            v[i] = __ldcg(po + ((size_t)c * NQ + h0 + i) * 128 + t);
-            f[i] = softmax_rescale(ml[(c * NQ + h0 + i) * 2], Ms[i]);
+            v[i] = __ldcg(reinterpret_cast<const float4*>(po + ((size_t)c * NQ + h0 + i) * 128) + lane);
+            f[i] = softmax_rescale(ml[(c * NQ + h0 + i) * 2], Mh[i]);
         }
 #pragma unroll
-        for (int i = 0; i < MERGE_HEADS; ++i) acc[i] += f[i] * v[i];
+        for (int i = 0; i < MERGE_HEADS; ++i) {
+            acc[i][0] += f[i] * v[i].x;
+            acc[i][1] += f[i] * v[i].y;
+            acc[i][2] += f[i] * v[i].z;
+            acc[i][3] += f[i] * v[i].w;
+        }
     }
 #pragma unroll
-    for (int i = 0; i < MERGE_HEADS; ++i)
-        a.out[((size_t)r * NQ + h0 + i) * 128 + t] = f2bf(acc[i] / Ls[i]);
+    for (int i = 0; i < MERGE_HEADS; ++i) {
+        const float Li = __shfl_sync(0xffffffffu, L, i);
+        *reinterpret_cast<uint2*>(a.out + ((size_t)r * NQ + h0 + i) * 128 + 4 * lane) =
+            make_uint2((uint32_t)f2bf(acc[i][0] / Li) | ((uint32_t)f2bf(acc[i][1] / Li) << 16),
+                       (uint32_t)f2bf(acc[i][2] / Li) | ((uint32_t)f2bf(acc[i][3] / Li) << 16));
+    }
 }
 
 }  // namespace decode_impl

@@ -76,12 +76,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
-// CTA (x, y) of 128 threads merges query-head group y of requests x, x + gridDim.x, ...
+// Warp w of CTA b merges units (request, group of MERGE_HEADS query heads) 8 b + w, 8 (b + grid) + w, ...
+constexpr int MERGE_THREADS = 256;
+
 template <int NQ>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const __grid_constant__ DecodeArgs a) {
-    __shared__ float Ms[MERGE_HEADS], Ls[MERGE_HEADS];
-    for (int r = a.req_begin + blockIdx.x; r < a.req_end; r += gridDim.x)
-        merge_heads<NQ>(a, r, blockIdx.y * MERGE_HEADS, threadIdx.x, Ms, Ls, 1);
+__global__ void __launch_bounds__(MERGE_THREADS) decode_merge_kernel(const __grid_constant__ DecodeArgs a) {
+    constexpr int NG = NQ / MERGE_HEADS;
+    const int units = (a.req_end - a.req_begin) * NG;
+    const int wpc = MERGE_THREADS / 32;
+    for (int u = blockIdx.x * wpc + (threadIdx.x >> 5); u < units; u += gridDim.x * wpc)
+        merge_heads_warp<NQ>(a, a.req_begin + u / NG, (u % NG) * MERGE_HEADS, threadIdx.x & 31);
 }
 
 template <int NQ>
@@ -96,8 +100,9 @@ cudaError_t launch_nq(const CUtensorMap& tmQ, const DecodeArgs& a, int grid, cud
     decode_attention_tc_kernel<NQ><<<grid, THREADS, TcCfg<NQ>::SMEM, stream>>>(tmQ, a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || a.split_pages >= kDecodeNoSplit || !a.any_split) return e;
-    const int rows = a.req_end - a.req_begin;
-    decode_merge_kernel<NQ><<<dim3(rows < 1024 ? rows : 1024, NQ / MERGE_HEADS), 128, 0, stream>>>(a);
+    const int units = (a.req_end - a.req_begin) * (NQ / MERGE_HEADS);
+    const int blocks = (units + MERGE_THREADS / 32 - 1) / (MERGE_THREADS / 32);
+    decode_merge_kernel<NQ><<<blocks < 2048 ? blocks : 2048, MERGE_THREADS, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -297,7 +297,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 const int wslot = tile * 2 + (int)rank;
                 float* ws = p.splitk_ws + (size_t)wslot * BM * BN;
                 if (ks == 2 && unit < ntiles) {
-                    epilogue_resid(p, t, tacc, quarter * 32, lane, stg, nullptr, ws);
+                    epilogue_resid<2>(p, t, tacc, quarter * 32, lane, stg, nullptr, ws);
                     __threadfence();
                     bar_sync_n(1, 128);
                     if (warp == 2 && lane == 0) st_release_gpu(p.splitk_flags + wslot, p.splitk_epoch);
@@ -317,7 +317,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         }
                         bar_sync_n(1, 128);
                     }
-                    epilogue_resid(p, t, tacc, quarter * 32, lane, stg, ks == 2 ? ws : nullptr, nullptr);
+                    epilogue_resid<2>(p, t, tacc, quarter * 32, lane, stg, ks == 2 ? ws : nullptr, nullptr);
                 }
             } else {
                 epilogue_tile<EPI>(p, t, tacc, row, valid);

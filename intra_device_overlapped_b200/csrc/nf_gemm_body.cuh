@@ -219,6 +219,9 @@ __device__ __forceinline__ void resid_block(const ResidCtx& c, int j, const floa
 
 static_assert((BN / 32) % 2 == 0, "the residual epilogue walks column blocks in pairs");
 
+// AHEAD: column blocks whose global reads are in flight while a block is written (2: the next two,
+// double-buffered; 1: the next one, half the registers)
+template <int AHEAD = 2>
 __device__ __forceinline__ void epilogue_resid(const GemmArgs& p, const Tile& t, uint32_t tacc, int rbase, int lane,
                                                float* stg, const float* part, float* publish) {
     if (publish != nullptr) {
@@ -240,19 +243,34 @@ __device__ __forceinline__ void epilogue_resid(const GemmArgs& p, const Tile& t,
     }
     const ResidCtx c{&p, &t, tacc, rbase, lane, stg, part};
     float ss[8];
-    float4 ra[8], wa[8], rb[8], wb[8];
+    if constexpr (AHEAD == 2) {
+        float4 ra[8], wa[8], rb[8], wb[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        ss[i] = 0.f;
-        ra[i] = rb[i] = wa[i] = wb[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    resid_load(c, 0, ra, wa);
+        for (int i = 0; i < 8; ++i) {
+            ss[i] = 0.f;
+            ra[i] = rb[i] = wa[i] = wb[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        resid_load(c, 0, ra, wa);
 #pragma unroll 1
-    for (int j = 0; j < BN / 32; j += 2) {
-        resid_load(c, j + 1, rb, wb);
-        resid_block(c, j, ra, wa, ss);
-        if (j + 2 < BN / 32) resid_load(c, j + 2, ra, wa);
-        resid_block(c, j + 1, rb, wb, ss);
+        for (int j = 0; j < BN / 32; j += 2) {
+            resid_load(c, j + 1, rb, wb);
+            resid_block(c, j, ra, wa, ss);
+            if (j + 2 < BN / 32) resid_load(c, j + 2, ra, wa);
+            resid_block(c, j + 1, rb, wb, ss);
+        }
+    } else {
+        float4 ra[8], wa[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            ss[i] = 0.f;
+            ra[i] = wa[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        resid_load(c, 0, ra, wa);
+#pragma unroll 1
+        for (int j = 0; j < BN / 32; ++j) {
+            resid_block(c, j, ra, wa, ss);
+            if (j + 1 < BN / 32) resid_load(c, j + 1, ra, wa);
+        }
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -402,7 +420,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, 
 // work counter (p.tile_ctr == nullptr), CTA `cta` of `ncta` takes units cta, cta + ncta, ... . The
 // body starts and ends on a block-wide barrier and invalidates every mbarrier it initialised before
 // it returns, so that the caller may reuse all of the shared memory.
-template <int EPI>
+template <int EPI, int RESID_AHEAD = 2>
 __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensorMap* tmB, const GemmArgs& p,
                                           uint8_t* smem, uint32_t tmem_base, int cta, int ncta) {
     // barriers in the kGemmBarrierBytes after the ring, then the epilogue warps' staging blocks
@@ -542,6 +560,15 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             if (lane == 0 && okw) mbar_arrive(&unit_empty[slot]);
             if (bar_red_or(1, 128, !okw)) break;  // every epilogue warp read the same unit
             if (unit < 0) break;
+            if constexpr (EPI == EPI_RESID) {
+                // the residual row this lane will read and rewrite once the accumulator is ready (a
+                // main loop from now): start bringing it into L2 (a first half only publishes)
+                if (!(ks == 2 && unit < ntiles)) {
+                    const Tile tp = tile_at(p, unit % ntiles);
+                    const int r = tp.row_begin + row_in_tile;
+                    if (r < tp.row_end) prefetch_l2_bulk(p.resid + (size_t)(p.tok0 + r) * p.N + tp.n_blk * BN, BN * 4);
+                }
+            }
             const int acc = local & 1;
             const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
             int ok = 1;
@@ -560,7 +587,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
                 float* ws = p.splitk_ws + (size_t)tile * BM * BN;
                 if (ks == 2 && unit < ntiles) {
                     // first half of the k blocks: publish the fp32 partial for the second half
-                    epilogue_resid(p, t, tacc, quarter * 32, lane, stg, nullptr, ws);
+                    epilogue_resid<RESID_AHEAD>(p, t, tacc, quarter * 32, lane, stg, nullptr, ws);
                     __threadfence();
                     bar_sync_n(1, 128);
                     if (warp == 2 && lane == 0) st_release_gpu(p.splitk_flags + tile, p.splitk_epoch);
@@ -581,7 +608,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
                         }
                         bar_sync_n(1, 128);
                     }
-                    epilogue_resid(p, t, tacc, quarter * 32, lane, stg, ks == 2 ? ws : nullptr, nullptr);
+                    epilogue_resid<RESID_AHEAD>(p, t, tacc, quarter * 32, lane, stg, ks == 2 ? ws : nullptr, nullptr);
                 }
             } else {
                 epilogue_tile<EPI>(p, t, tacc, row, valid);

@@ -67,10 +67,13 @@ __device__ __forceinline__ int trace_kind(int kind) {
 
 // Each body is a separate (not inlined) function, so that its registers are allocated for it alone
 // rather than for the union of all bodies.
+// The residual epilogue keeps one column block of reads in flight instead of two: its arguments are
+// read through a pointer here (not from the kernel's constant bank), which costs the registers the
+// second buffer would take.
 template <int EPI>
 __device__ __noinline__ void run_gemm(const CUtensorMap* tmA, const CUtensorMap* tmB, const GemmArgs& g, uint8_t* smem,
                                       uint32_t tmem, int cta, int ncta) {
-    gemm_impl::gemm_body<EPI>(tmA, tmB, g, smem, tmem, cta, ncta);
+    gemm_impl::gemm_body<EPI, 1>(tmA, tmB, g, smem, tmem, cta, ncta);
 }
 
 template <int NQ>
@@ -90,7 +93,6 @@ __global__ void __launch_bounds__(kMegaThreads, 1) mega_layer_kernel(const __gri
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint32_t tmem_slot;
     __shared__ int s_stop;
-    __shared__ float merge_m[2][decode_impl::MERGE_HEADS], merge_l[2][decode_impl::MERGE_HEADS];
     const int warp = threadIdx.x >> 5;
     if (warp == 1) {
         tmem_alloc(&tmem_slot, kMegaTmemCols);
@@ -146,14 +148,14 @@ __global__ void __launch_bounds__(kMegaThreads, 1) mega_layer_kernel(const __gri
                     run_decode<NQ>(&op.tmA, op.d, smem, tmem, cta, ncta);
                     break;
                 case MEGA_MERGE: {
-                    // two groups of 128 threads per CTA, one (request, group of 8 query heads) each
+                    // one (request, group of 8 query heads) per warp
                     const DecodeArgs& a = op.d;
                     constexpr int NG = NQ / decode_impl::MERGE_HEADS;
-                    const int half = warp >> 2;
+                    constexpr int WPC = kMegaThreads / 32;
                     const int units = (a.req_end - a.req_begin) * NG;
-                    for (int u = 2 * cta + half; u < units; u += 2 * ncta)
-                        decode_impl::merge_heads<NQ>(a, a.req_begin + u / NG, (u % NG) * decode_impl::MERGE_HEADS,
-                                                     threadIdx.x & 127, merge_m[half], merge_l[half], 8 + half);
+                    for (int u = cta * WPC + warp; u < units; u += ncta * WPC)
+                        decode_impl::merge_heads_warp<NQ>(a, a.req_begin + u / NG,
+                                                          (u % NG) * decode_impl::MERGE_HEADS, threadIdx.x & 31);
                     break;
                 }
                 case MEGA_PREFILL:
