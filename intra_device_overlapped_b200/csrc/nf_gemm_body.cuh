@@ -157,38 +157,56 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volati
 // Residual epilogue of one warp's 32 rows (rows rbase .. rbase + 31 of the tile), through the
 // warp's staging block so that every global access is row-contiguous:
 //   publish != null (first k half of a split tile): the fp32 partial goes to the workspace;
-//   otherwise h = (part + acc) + resid, written back to resid (fp32), to out_bf16 and, if set,
-//   out_f32; the row's sum of squares over this column block goes to out_partials.
+//   otherwise h = (part + acc) + resid, written back to resid (fp32) and to out_bf16; the row's
+//   sum of squares over this column block goes to out_partials.
 // The global reads of a 32-column block (residual, first-half partial) are issued together one
 // block ahead of their use, so that their latency overlaps the previous block's work instead of
 // being paid once per row behind that row's stores.
+// The argument values the loops use are copied into the context once: the epilogue's global stores
+// could alias the argument block where it is read through a pointer (not from the kernel's constant
+// bank), which would make every store force a reload.
 struct ResidCtx {
-    const GemmArgs* p;
-    const Tile* t;
+    float* resid;       // row 0 of the launch, column n0 of the tile
+    uint16_t* out_bf16;
+    int N, ld_bf16;
+    int row_begin, row_end;
     uint32_t tacc;
     int rbase, lane;
     float* stg;
     const float* part;
 };
 
+__device__ __forceinline__ ResidCtx resid_ctx(const GemmArgs& p, const Tile& t, uint32_t tacc, int rbase, int lane,
+                                              float* stg, const float* part) {
+    const int n0 = t.n_blk * BN;
+    ResidCtx c;
+    c.resid = p.resid + (size_t)p.tok0 * p.N + n0;
+    c.out_bf16 = p.out_bf16 + (size_t)p.tok0 * p.ld_bf16 + n0;
+    c.N = p.N;
+    c.ld_bf16 = p.ld_bf16;
+    c.row_begin = t.row_begin;
+    c.row_end = t.row_end;
+    c.tacc = tacc;
+    c.rbase = rbase;
+    c.lane = lane;
+    c.stg = stg;
+    c.part = part;
+    return c;
+}
+
 __device__ __forceinline__ void resid_load(const ResidCtx& c, int j, float4 (&r)[8], float4 (&w)[8]) {
-    const GemmArgs& p = *c.p;
-    const int n0 = c.t->n_blk * BN;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int rt = c.rbase + 4 * i + (c.lane >> 3);
         const int col = 32 * j + 4 * (c.lane & 7);
         if (c.part != nullptr) w[i] = __ldcg(reinterpret_cast<const float4*>(c.part + (size_t)rt * BN + col));
-        const int row = c.t->row_begin + rt;
-        if (row < c.t->row_end)
-            r[i] = __ldcg(reinterpret_cast<const float4*>(p.resid + (size_t)(p.tok0 + row) * p.N + n0 + col));
+        const int row = c.row_begin + rt;
+        if (row < c.row_end) r[i] = __ldcg(reinterpret_cast<const float4*>(c.resid + (size_t)row * c.N + col));
     }
 }
 
 __device__ __forceinline__ void resid_block(const ResidCtx& c, int j, const float4 (&r)[8], const float4 (&w)[8],
                                             float (&ss)[8]) {
-    const GemmArgs& p = *c.p;
-    const int n0 = c.t->n_blk * BN;
     float v[32];
     tmem_ld32(c.tacc + 32 * j, v);
     stage_rows32(c.stg, c.lane, v);
@@ -200,18 +218,16 @@ __device__ __forceinline__ void resid_block(const ResidCtx& c, int j, const floa
         float4 x = staged_quad(c.stg, 4 * i + (c.lane >> 3), c.lane & 7);
         if (c.part != nullptr)  // split-K: first half's partial + this half, in that order
             x = make_float4(w[i].x + x.x, w[i].y + x.y, w[i].z + x.z, w[i].w + x.w);
-        const int row = c.t->row_begin + rt;
-        if (row < c.t->row_end) {
-            const size_t g = (size_t)(p.tok0 + row);
+        const int row = c.row_begin + rt;
+        if (row < c.row_end) {
             x = make_float4(x.x + r[i].x, x.y + r[i].y, x.z + r[i].z, x.w + r[i].w);
             ss[i] += x.x * x.x;
             ss[i] += x.y * x.y;
             ss[i] += x.z * x.z;
             ss[i] += x.w * x.w;
-            *reinterpret_cast<float4*>(p.resid + g * p.N + n0 + col) = x;
-            *reinterpret_cast<uint2*>(p.out_bf16 + g * p.ld_bf16 + n0 + col) =
+            *reinterpret_cast<float4*>(c.resid + (size_t)row * c.N + col) = x;
+            *reinterpret_cast<uint2*>(c.out_bf16 + (size_t)row * c.ld_bf16 + col) =
                 make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
-            if (p.out_f32) *reinterpret_cast<float4*>(p.out_f32 + g * p.ld_f32 + n0 + col) = x;
         }
     }
     __syncwarp();  // the next block overwrites the staging buffer
@@ -241,7 +257,9 @@ __device__ __forceinline__ void epilogue_resid(const GemmArgs& p, const Tile& t,
         }
         return;
     }
-    const ResidCtx c{&p, &t, tacc, rbase, lane, stg, part};
+    const ResidCtx c = resid_ctx(p, t, tacc, rbase, lane, stg, part);
+    float* const out_partials = p.out_partials;
+    const int tok0 = p.tok0, n_tiles = p.n_tiles;
     float ss[8];
     if constexpr (AHEAD == 2) {
         float4 ra[8], wa[8], rb[8], wb[8];
@@ -279,7 +297,7 @@ __device__ __forceinline__ void epilogue_resid(const GemmArgs& p, const Tile& t,
         x += __shfl_xor_sync(0xffffffffu, x, 2);
         x += __shfl_xor_sync(0xffffffffu, x, 4);
         const int row = t.row_begin + rbase + 4 * i + (lane >> 3);
-        if ((lane & 7) == 0 && row < t.row_end) p.out_partials[(size_t)(p.tok0 + row) * p.n_tiles + t.n_blk] = x;
+        if ((lane & 7) == 0 && row < t.row_end) out_partials[(size_t)(tok0 + row) * n_tiles + t.n_blk] = x;
     }
 }
 
@@ -367,13 +385,19 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, 
         const int slot = pos & 15;
         // the rotation angles depend on the position and the column pair only: each column
         // block's cos / sin row segment is loaded once (16-byte loads) for both heads of the tile
-        const bool any_rope = n0 / d < p.nq + p.nkv;
+        // argument values used in the loops, read once (see ResidCtx)
+        const int nq = p.nq, nkv = p.nkv;
+        uint16_t* const q_out = p.q_out;
+        uint16_t* const kv_pool = p.kv_pool;
+        const float* const rope_cos = p.rope_cos;
+        const float* const rope_sin = p.rope_sin;
+        const bool any_rope = n0 / d < nq + nkv;
         float x2[32], cs[32], sn[32];
 #pragma unroll 1
         for (int j = 0; j < half / 32; ++j) {
             if (ok && any_rope) {
-                const float4* c4 = reinterpret_cast<const float4*>(p.rope_cos + (size_t)pos * half + 32 * j);
-                const float4* s4 = reinterpret_cast<const float4*>(p.rope_sin + (size_t)pos * half + 32 * j);
+                const float4* c4 = reinterpret_cast<const float4*>(rope_cos + (size_t)pos * half + 32 * j);
+                const float4* s4 = reinterpret_cast<const float4*>(rope_sin + (size_t)pos * half + 32 * j);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const float4 c = __ldg(c4 + q), sv = __ldg(s4 + q);
@@ -384,8 +408,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, 
 #pragma unroll 1
             for (int hc = 0; hc < BN / d; ++hc) {
                 const int head = (n0 + hc * d) / d;
-                const int kind = head < p.nq ? 0 : (head < p.nq + p.nkv ? 1 : 2);
-                const int g = kind == 1 ? head - p.nq : head - p.nq - p.nkv;
+                const int kind = head < nq ? 0 : (head < nq + nkv ? 1 : 2);
+                const int g = kind == 1 ? head - nq : head - nq - nkv;
                 tmem_ld32(tacc + hc * d + 32 * j, v);
                 tmem_ld32(tacc + hc * d + half + 32 * j, x2);
                 if (!ok || (kind != 0 && page_base < 0)) continue;
@@ -401,12 +425,12 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const Tile& t, 
                     for (int e = 0; e < 32; ++e) { v[e] *= rs; x2[e] *= rs; }
                 }
                 if (kind == 0) {
-                    uint16_t* dst = p.q_out + ((size_t)tok * p.nq + head) * d;
+                    uint16_t* dst = q_out + ((size_t)tok * nq + head) * d;
                     store_bf16x32(dst + 32 * j, v);
                     store_bf16x32(dst + half + 32 * j, x2);
                 } else {
-                    store_kv_row32(p.kv_pool + page_base, kind - 1, g, p.nkv, d, slot, 32 * j, v);
-                    store_kv_row32(p.kv_pool + page_base, kind - 1, g, p.nkv, d, slot, half + 32 * j, x2);
+                    store_kv_row32(kv_pool + page_base, kind - 1, g, nkv, d, slot, 32 * j, v);
+                    store_kv_row32(kv_pool + page_base, kind - 1, g, nkv, d, slot, half + 32 * j, x2);
                 }
             }
         }
