@@ -584,15 +584,6 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             if (lane == 0 && okw) mbar_arrive(&unit_empty[slot]);
             if (bar_red_or(1, 128, !okw)) break;  // every epilogue warp read the same unit
             if (unit < 0) break;
-            if constexpr (EPI == EPI_RESID) {
-                // the residual row this lane will read and rewrite once the accumulator is ready (a
-                // main loop from now): start bringing it into L2 (a first half only publishes)
-                if (!(ks == 2 && unit < ntiles)) {
-                    const Tile tp = tile_at(p, unit % ntiles);
-                    const int r = tp.row_begin + row_in_tile;
-                    if (r < tp.row_end) prefetch_l2_bulk(p.resid + (size_t)(p.tok0 + r) * p.N + tp.n_blk * BN, BN * 4);
-                }
-            }
             const int acc = local & 1;
             const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
             int ok = 1;
