@@ -11,6 +11,8 @@ layer launches the QKV, O, gate/up and down GEMMs in that order; --persistent ru
 one persistent kernel instead). ``--sm`` is the persistent grid (0 = every SM). The printed line holds the mean
 launch time over --reps launches (CUDA events on the launching stream, after --warmup launches) and
 the algorithmic bytes or FLOPs of one launch, so that a profiler can target a small, known case.
+--power-s S adds the op's steady state under load: S seconds of back-to-back launches after 1 s,
+with the median SM clock and board power that nvidia-smi samples meanwhile.
 """
 from __future__ import annotations
 
@@ -21,6 +23,46 @@ import numpy as np
 import torch
 
 from . import check, nf_op_decode_attention, nf_op_gemm_bf16, nf_op_prefill_attention
+
+
+def _power(launch, seconds: float, stream) -> dict:
+    """Steady state of `launch` run back to back: 1 s of warm-up, then `seconds` of launches while
+    nvidia-smi samples the SM clock and the board power every 50 ms (medians reported)."""
+    import statistics
+    import subprocess
+    import threading
+    import time
+    smi = subprocess.Popen(["nvidia-smi", "--id=0", "--query-gpu=clocks.sm,power.draw,clocks_event_reasons.active",
+                            "--format=csv,noheader,nounits", "-lms", "50"], stdout=subprocess.PIPE, text=True)
+    lines = []
+    reader = threading.Thread(target=lambda: [lines.append(x.strip()) for x in smi.stdout], daemon=True)
+    reader.start()
+    try:
+        t0 = time.time()
+        while time.time() - t0 < 1.0:
+            for _ in range(8):
+                launch()
+            torch.cuda.synchronize()
+        mark = len(lines)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = 0
+        e0.record(stream)
+        t0 = time.time()
+        while time.time() - t0 < seconds:
+            for _ in range(8):
+                launch()
+            n += 8
+            torch.cuda.synchronize()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        rows = [x.split(",") for x in lines[mark:] if x.count(",") == 2]
+    finally:
+        smi.terminate()
+    sm = [float(r[0]) for r in rows if r[0].strip()]
+    pw = [float(r[1]) for r in rows if r[1].strip()]
+    return {"steady_us": round(e0.elapsed_time(e1) * 1000.0 / max(n, 1), 2),
+            "sm_mhz": statistics.median(sm) if sm else None, "power_w": statistics.median(pw) if pw else None,
+            "samples": len(sm), "reasons": sorted({r[2].strip() for r in rows})}
 
 
 def _time(launch, reps: int, warmup: int, stream) -> float:
@@ -53,6 +95,9 @@ def main(argv=None) -> dict:
     ap.add_argument("--m", type=int, default=1536)
     ap.add_argument("--n", type=int, default=4096)
     ap.add_argument("--k", type=int, default=4096)
+    ap.add_argument("--power-s", type=float, default=0.0,
+                    help="also run the op back to back for this many seconds (after 1 s) and report the median "
+                         "SM clock and board power sampled by nvidia-smi")
     args = ap.parse_args(argv)
     dev = "cuda:0"
     torch.cuda.set_device(dev)
@@ -65,9 +110,12 @@ def main(argv=None) -> dict:
         a = torch.randn((M, K), device=dev, generator=g).to(torch.bfloat16)
         b = (torch.randn((N, K), device=dev, generator=g) * 0.02).to(torch.bfloat16)
         c = torch.empty((M, N), dtype=torch.float32, device=dev)
-        us = _time(lambda: check(nf_op_gemm_bf16(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, args.sm,
-                                                 stream.cuda_stream), "gemm"), args.reps, args.warmup, stream)
+        launch = lambda: check(nf_op_gemm_bf16(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, args.sm,
+                                               stream.cuda_stream), "gemm")
+        us = _time(launch, args.reps, args.warmup, stream)
         out.update({"shape": [M, N, K], "us": round(us, 2), "tflops": round(2.0 * M * N * K / us / 1e6, 1)})
+        if args.power_s > 0:
+            out["power"] = _power(launch, args.power_s, stream)
     else:
         from synth.workloads import WORKLOADS
         from .harness import DeviceWorkload
@@ -81,26 +129,29 @@ def main(argv=None) -> dict:
         o = torch.zeros_like(q)
         if args.op == "iteration":
             plan = dw.plan(nano=args.nano, template=args.template, sm_attn=args.sm_attn)
-            us = _time(lambda: dw.forward(plan, stream, persistent=args.persistent), args.reps, args.warmup, stream)
+            launch = lambda: dw.forward(plan, stream, persistent=args.persistent)
+            us = _time(launch, args.reps, args.warmup, stream)
             out.update({"workload": args.workload, "plan": plan.describe(), "persistent": args.persistent,
                         "us": round(us, 2)})
         elif args.op == "decode_attention":
             R = args.requests or bt.num_decode
             pages = sum(-(-(int(c) + 1) // s.page_size) for c in bt.ctx_lens[:R])
             nbytes = pages * 2 * s.n_kv_heads * s.page_size * s.head_dim * 2
-            us = _time(lambda: check(nf_op_decode_attention(dw.model, q.data_ptr(), o.data_ptr(), dw.io, 0, 0, R,
-                                                            args.sm, stream.cuda_stream), "decode"),
-                       args.reps, args.warmup, stream)
+            launch = lambda: check(nf_op_decode_attention(dw.model, q.data_ptr(), o.data_ptr(), dw.io, 0, 0, R,
+                                                          args.sm, stream.cuda_stream), "decode")
+            us = _time(launch, args.reps, args.warmup, stream)
             out.update({"workload": args.workload, "requests": R, "kv_bytes": nbytes, "us": round(us, 2),
                         "gbs": round(nbytes / us / 1e3, 1)})
         else:
             R, C = bt.num_decode, bt.prefill_len
             flops = 4.0 * s.n_q_heads * s.head_dim * C * (C + 1) / 2
-            us = _time(lambda: check(nf_op_prefill_attention(dw.model, q.data_ptr(), o.data_ptr(), dw.io, 0, R, C,
-                                                             args.sm, stream.cuda_stream), "prefill"),
-                       args.reps, args.warmup, stream)
+            launch = lambda: check(nf_op_prefill_attention(dw.model, q.data_ptr(), o.data_ptr(), dw.io, 0, R, C,
+                                                           args.sm, stream.cuda_stream), "prefill")
+            us = _time(launch, args.reps, args.warmup, stream)
             out.update({"workload": args.workload, "chunk": C, "flops": flops, "us": round(us, 2),
                         "tflops": round(flops / us / 1e6, 2)})
+        if args.power_s > 0:
+            out["power"] = _power(launch, args.power_s, stream)
         check(dw.sync(), "status")
         dw.close()
     print(json.dumps(out), flush=True)
