@@ -47,8 +47,8 @@ def _release(dw):
     torch.cuda.empty_cache()
 
 
-def _forward(dw, plan):
-    dw.forward(plan)
+def _forward(dw, plan, persistent=False):
+    dw.forward(plan, persistent=persistent)
     st = dw.sync()
     assert st == 0, f"device status {st}"
 
@@ -146,19 +146,20 @@ def test_llama3_8b_layer_full_size_planner_plan():
 
 
 def test_llama2_70b_slice_full_size_nano_2_and_4():
-    """20 layers of the 70B shape at nano-batch counts 2 and 4: bitwise the same; every fourth layer
+    """20 layers of the 70B shape (64 query heads) at nano-batch counts 2 and 4, and the 2-nano-batch
+    plan again with each layer as one persistent kernel: bitwise the same; every fourth layer
     matches the oracle on sampled decode and chunk rows."""
     from synth import weights as SW
     name = "llama2_70b_slice"
     dw = _dw(name, keep_logits=False, layer_outputs=True)
     try:
         outs = []
-        for n in (2, 2, 4):
+        for n, persistent in ((2, False), (2, False), (4, False), (2, True)):
             for layer, pool in enumerate(dw.kv):   # fresh cache: the iteration writes its new K/V
                 SW.gpu_fill_kv_pool(dw.shape, layer, pool)
             plan = dw.plan(nano=n)
-            _forward(dw, plan)
-            outs.append((plan.describe(), dw.hidden_out_f32.cpu().numpy()))
+            _forward(dw, plan, persistent)
+            outs.append((str(plan.describe()) + (" persistent" if persistent else ""), dw.hidden_out_f32.cpu().numpy()))
         for desc, o in outs[1:]:
             if not np.array_equal(o, outs[0][1]):
                 bad = np.nonzero(np.any(o != outs[0][1], axis=1))[0]
