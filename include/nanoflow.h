@@ -401,6 +401,13 @@ nf_status nf_op_prefill_attention(nf_model* m, const void* q, void* out, const n
  * outcome) after the kernel has given up and exited, or NF_OK if the flag was set. */
 nf_status nf_op_wait_flag_test(int32_t* flag_device, uint64_t limit_ns, void* stream);
 
+/* Self test of the persistent layer kernel's dependency waits: the kernel is launched on a few CTAs
+ * with an operation list whose first operation depends on its second (which every CTA reaches only
+ * after the first), each wait limited to `limit_ns` (1 ns .. 10 s). Every CTA's wait must expire:
+ * returns NF_ERR_DEVICE_TIMEOUT (the expected outcome) once the kernel has exited, NF_OK if a wait
+ * did not expire, NF_ERR_CUDA on a launch or copy error. Blocks the host until done. */
+nf_status nf_op_persistent_wait_test(uint64_t limit_ns, void* stream);
+
 /* ------------------------------------------------------------------ KV offload
  *
  * Offload of a finished request's KV cache to host memory (hysenlabs review, "KV-cache offload to

@@ -168,6 +168,7 @@ def _load():
         "nf_op_decode_attention": ([_vp, _vp, _vp, P(nf_iter_io), _i32, _i32, _i32, _i32, _vp], ctypes.c_int),
         "nf_op_prefill_attention": ([_vp, _vp, _vp, P(nf_iter_io), _i32, _i32, _i32, _i32, _vp], ctypes.c_int),
         "nf_op_wait_flag_test": ([_vp, _u64, _vp], ctypes.c_int),
+        "nf_op_persistent_wait_test": ([_u64, _vp], ctypes.c_int),
         "nf_decode_attention_noalloc": ([_vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp],
                                         ctypes.c_int),
         "nf_offload_kv": ([_vp, P(_vp), _i32, P(_i32), _i32, _i32, _i32, _vp, _vp], ctypes.c_int),
@@ -193,7 +194,7 @@ EXPORTED = ("nf_status_string", "nf_version", "nf_init_model", "nf_set_layer_wei
             "nf_get_cost_model", "nf_set_cost_model",
             "nf_set_trace", "nf_get_trace", "nf_set_timing", "nf_get_op_times", "nf_op_gemm_bf16", "nf_op_decode_attention",
             "nf_offload_kv",
-            "nf_op_prefill_attention", "nf_op_wait_flag_test", "nf_decode_attention_noalloc",
+            "nf_op_prefill_attention", "nf_op_wait_flag_test", "nf_op_persistent_wait_test", "nf_decode_attention_noalloc",
             "nf_sched_create", "nf_sched_destroy", "nf_sched_add_request", "nf_sched_next", "nf_sched_complete",
             "nf_sched_request_tokens", "nf_sched_get_stats")
 
@@ -368,6 +369,10 @@ def nf_op_prefill_attention(model: int, q_ptr: int, out_ptr: int, io: nf_iter_io
 
 def nf_op_wait_flag_test(flag_ptr: int, limit_ns: int, stream: int = 0) -> int:
     return _lib.nf_op_wait_flag_test(flag_ptr, limit_ns, stream)
+
+
+def nf_op_persistent_wait_test(limit_ns: int, stream: int = 0) -> int:
+    return _lib.nf_op_persistent_wait_test(limit_ns, stream)
 
 
 def _i32_array(values) -> "ctypes.Array":

@@ -1339,6 +1339,41 @@ extern "C" nf_status nf_offload_kv(nf_model* m, void* const* kv_pools, int32_t n
     return NF_ERR_INVALID_ARGUMENT;
 }
 
+extern "C" nf_status nf_op_persistent_wait_test(uint64_t limit_ns, void* stream) try {
+    if (limit_ns == 0 || limit_ns > 10000000000ull) return NF_ERR_INVALID_ARGUMENT;
+    int* status = nullptr;
+    nf_status st = op_status_word(&status);
+    if (st != NF_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    int* done = nullptr;
+    NF_CUDA_TRY(cudaMalloc(&done, 2 * sizeof(int)));
+    std::unique_ptr<nf::MegaParams> P(new nf::MegaParams);
+    std::memset(P.get(), 0, sizeof(nf::MegaParams));
+    // operation 0 depends on operation 1, which every CTA reaches only after operation 0
+    P->n_ops = 2;
+    P->ops[0].kind = P->ops[1].kind = nf::MEGA_NOP;
+    P->ops[0].lane = P->ops[1].lane = nf::LANE_ALL;
+    P->ops[0].dep[0] = 1;
+    P->ops[0].dep[1] = P->ops[0].dep[2] = -1;
+    P->ops[1].dep[0] = P->ops[1].dep[1] = P->ops[1].dep[2] = -1;
+    P->done = done;
+    P->status = status;
+    P->wait_limit_ns = limit_ns;
+    int h = -1;
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(done, 0, 2 * sizeof(int), s);
+    if (e == cudaSuccess) e = nf::launch_mega(*P, 32, std::min(8, nf::device_sm_count()), s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&h, status, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    cudaFree(done);
+    if (e != cudaSuccess) return NF_ERR_CUDA;
+    return (nf_status)h;
+} catch (const std::bad_alloc&) {
+    return NF_ERR_OUT_OF_MEMORY;
+} catch (...) {
+    return NF_ERR_INVALID_ARGUMENT;
+}
+
 extern "C" nf_status nf_op_wait_flag_test(int32_t* flag_device, uint64_t limit_ns, void* stream) try {
     if (flag_device == nullptr || limit_ns == 0 || limit_ns > 10000000000ull) return NF_ERR_INVALID_ARGUMENT;
     int* status = nullptr;

@@ -42,12 +42,12 @@ __device__ __forceinline__ void red_release_add(int* p, int v) {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Waits until *ctr >= target (bounded). Returns false after NF_WAIT_LIMIT_NS.
-__device__ __forceinline__ bool wait_count(const int* ctr, int target, int* status) {
+// Waits until *ctr >= target (bounded). Returns false after limit_ns.
+__device__ __forceinline__ bool wait_count(const int* ctr, int target, int* status, uint64_t limit_ns) {
     if (ld_acquire(ctr) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
     while (ld_acquire(ctr) < target) {
-        if (globaltimer_ns() - t0 > NF_WAIT_LIMIT_NS) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             set_status(status, NF_ERR_DEVICE_TIMEOUT);
             return false;
         }
@@ -122,7 +122,9 @@ __global__ void __launch_bounds__(kMegaThreads, 1) mega_layer_kernel(const __gri
                 bool ok = true;
                 for (int k = 0; k < kMegaMaxDeps && ok; ++k) {
                     const int d = op.dep[k];
-                    if (d >= 0) ok = wait_count(P.done + d, lane_ctas(P.ops[d].lane, P.n_attn), P.status);
+                    if (d >= 0)
+                        ok = wait_count(P.done + d, lane_ctas(P.ops[d].lane, P.n_attn), P.status,
+                                        P.wait_limit_ns ? P.wait_limit_ns : NF_WAIT_LIMIT_NS);
                 }
                 if (ok && *reinterpret_cast<volatile int*>(P.status) == NF_ERR_DEVICE_TIMEOUT) ok = false;
                 s_stop = ok ? 0 : 1;

@@ -29,6 +29,7 @@ enum MegaKind : int {
     MEGA_DECODE = 3,   // tensor-core decode attention
     MEGA_MERGE = 4,    // split-KV merge of the decode chunks
     MEGA_PREFILL = 5,  // tensor-core causal attention of the prefill chunk
+    MEGA_NOP = 6,      // no work (self tests of the scheduling)
 };
 
 enum MegaLane : int { LANE_ALL = 0, LANE_GEMM = 1, LANE_ATTN = 2 };
@@ -58,6 +59,7 @@ struct MegaParams {
     int n_attn;     // CTAs [0, n_attn) form the attention lane (0: every operation is LANE_ALL)
     int* done;      // [n_ops], zeroed: CTAs of the operation's lane that have finished it
     int* status;
+    unsigned long long wait_limit_ns;  // limit of each dependency wait (0: NF_WAIT_LIMIT_NS)
     int* trace_ctr;  // per-CTA, per-operation trace (nullable)
     nf_trace_entry* trace;
     int trace_cap;

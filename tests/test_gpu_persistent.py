@@ -13,7 +13,10 @@ query heads):
   time on different SMs inside the one launch;
 - the full-size Llama-3-8B-shaped layer (512 decode requests, contexts U[1024, 1536], 1024-token
   chunk) matches the stream executor bit for bit;
-- models the kernel does not cover (head dim 64) are refused with NF_ERR_UNSUPPORTED.
+- models the kernel does not cover (head dim 64) are refused with NF_ERR_UNSUPPORTED;
+- a dependency wait that cannot be satisfied (an operation list whose first operation waits on its
+  second) expires with NF_ERR_DEVICE_TIMEOUT on every CTA, the kernel exits, and the context stays
+  usable.
 """
 import numpy as np
 import pytest
@@ -140,5 +143,20 @@ def test_persistent_refuses_uncovered_models():
         plan = dw.plan(nano=1, template=0)
         st = nf.nf_forward_iteration_persistent(dw.model, plan, dw.io, torch.cuda.current_stream().cuda_stream)
         assert st == nf.NF_ERR_UNSUPPORTED
+    finally:
+        dw.close()
+
+
+def test_persistent_dependency_wait_times_out_cleanly():
+    import intra_device_overlapped_b200 as nf
+    from intra_device_overlapped_b200.harness import DeviceWorkload
+    torch.cuda.set_device(DEV)
+    assert nf.nf_op_persistent_wait_test(10_000_000) == nf.NF_ERR_DEVICE_TIMEOUT
+    assert nf.nf_op_persistent_wait_test(0) == nf.NF_ERR_INVALID_ARGUMENT
+    # the context is usable afterwards: a persistent forward still equals the stream executor
+    dw = DeviceWorkload(TEST_WORKLOADS["small_gqa8"], DEV, layer_outputs=True)
+    try:
+        plan = dw.plan(nano=1, template=0)
+        _assert_same(_run(dw, plan, True), _run(dw, plan, False), "after the timeout test")
     finally:
         dw.close()
