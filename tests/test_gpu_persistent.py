@@ -5,8 +5,8 @@ wait on completion counters instead of kernel boundaries and events, and its GEM
 instead of CTA pairs. Checked here, on the tensor-core attention shapes (8 KV heads of 128, 32 and 64
 query heads):
 - the result equals the stream executor's bit for bit (fp32 residual stream after every layer, and
-  the KV slots written), for the sequential plan and for two-nano-batch plans of both overlapped
-  templates, including batches whose long requests are split along KV (merge operation);
+  the KV slots written), for the sequential plan and for plans of two to four nano-batches in both
+  overlapped templates, including batches whose long requests are split along KV (merge operation);
 - against the oracle, within the parity bars (so the bitwise equality above is not two equal
   mistakes);
 - the per-CTA trace of an overlapped plan shows GEMM and decode attention work running at the same
@@ -38,7 +38,9 @@ LONG = Workload(ModelShape("gqa8_long", 2, 1024, 32, 8, 128, 1024, rope_theta=50
 Q64 = Workload(ModelShape("gqa8_q64", 1, 2048, 64, 8, 128, 1024, rope_theta=10000.0, norm_sigma=0.1),
                16, 1, 1300, prefill_len=40)
 
-PLANS = [dict(nano=1, template=0), dict(nano=2, template=1, sm_attn=36), dict(nano=2, template=2, sm_attn=40)]
+# up to four nano-batches: 7 operations each fill the layer kernel's list of 28
+PLANS = [dict(nano=1, template=0), dict(nano=2, template=1, sm_attn=36), dict(nano=2, template=2, sm_attn=40),
+         dict(nano=3, template=1, sm_attn=48), dict(nano=4, template=2, sm_attn=64)]
 
 
 def _reset_kv(dw):
